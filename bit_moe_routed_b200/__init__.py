@@ -1,0 +1,244 @@
+"""bitmoe: routed-expert FFN of a DeepSeek-V4-Flash-style MoE layer on B200 (sm_100a).
+
+Thin Python binding of the C ABI in ``include/bitmoe.h`` (libbitmoe.so).  It only
+marshals arguments: torch provides device memory and the current CUDA stream, and
+every step of the layer runs in the library's CUDA kernels.  There is no fallback:
+if the library is missing or the device is not sm_100, calls raise.
+
+    idx, w = route_topk(scores, k)              # step 1: top-k + sigmoid gate weights
+    counts, offsets, perm, pos = dispatch(idx, E)  # step 2: stable grouping per expert
+    y, y_sh = expert_ffn(x, k, weights, offsets, perm)  # steps 3-7 (tcgen05 FFN)
+    out = combine(y, y_sh, w, pos)              # step 8
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SO = os.path.join(_HERE, "libbitmoe.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = -1
+MOE_ERR_WORKSPACE = -2
+MOE_ERR_CUDA = -3
+MOE_ERR_TIMEOUT = -4
+MOE_ERR_UNSUPPORTED = -5
+
+EXPORTS = (
+    "moe_route_topk", "moe_dispatch", "moe_act_quant", "moe_expert_ffn", "moe_ffn_prepare",
+    "moe_ffn_gate_up", "moe_ffn_down", "moe_combine", "moe_workspace_size", "moe_last_error",
+    "moe_set_wait_limit_ns", "moe_sync_status",
+)
+
+
+class MoeError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"bitmoe error {code}: {msg}")
+        self.code = code
+
+
+class _Weights(ctypes.Structure):
+    _fields_ = [
+        ("gate_codes", ctypes.c_void_p), ("gate_scales", ctypes.c_void_p),
+        ("up_codes", ctypes.c_void_p), ("up_scales", ctypes.c_void_p),
+        ("down_codes", ctypes.c_void_p), ("down_scales", ctypes.c_void_p),
+        ("E", ctypes.c_int), ("d", ctypes.c_int), ("f", ctypes.c_int),
+    ]
+
+
+_lib = None
+
+
+def lib():
+    """Load libbitmoe.so (built in-tree by build.py); raise if it is not there."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(SO):
+            raise RuntimeError(
+                f"{SO} is missing: build it with `python -m bit_moe_routed_b200.build` "
+                "(or __graft_entry__.build()); there is no fallback path")
+        L = ctypes.CDLL(SO)
+        P, I, Z, LL = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_longlong
+        W = ctypes.POINTER(_Weights)
+        sig = {
+            "moe_route_topk": [P, I, I, I, P, P, P],
+            "moe_dispatch": [P, I, I, I, P, P, P, P, P, Z, P],
+            "moe_act_quant": [P, I, I, P, P, P],
+            "moe_expert_ffn": [P, I, I, W, P, P, P, P, P, Z, P],
+            "moe_ffn_prepare": [P, I, I, W, P, P, P, Z, P],
+            "moe_ffn_gate_up": [I, I, W, P, Z, P],
+            "moe_ffn_down": [I, I, W, P, P, P, Z, P],
+            "moe_combine": [P, P, P, P, I, I, I, P, P],
+            "moe_workspace_size": [I, I, I, I, I],
+            "moe_last_error": [],
+            "moe_set_wait_limit_ns": [LL],
+            "moe_sync_status": [P],
+        }
+        for name, args in sig.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = ctypes.c_int
+        L.moe_workspace_size.restype = ctypes.c_size_t
+        L.moe_last_error.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def _check(rc: int) -> None:
+    if rc != MOE_OK:
+        raise MoeError(rc, lib().moe_last_error().decode(errors="replace"))
+
+
+def _stream(stream=None) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _p(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to bitmoe must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+@dataclass
+class LayerWeights:
+    """One layer's FP4 weights on the device, E+1 experts (index E = shared).
+
+    gate_codes/up_codes [E+1, f, d/2] uint8, gate_scales/up_scales [E+1, f, d/32] uint8,
+    down_codes [E+1, d, f/2] uint8, down_scales [E+1, d, f/32] uint8.
+    """
+    gate_codes: torch.Tensor
+    gate_scales: torch.Tensor
+    up_codes: torch.Tensor
+    up_scales: torch.Tensor
+    down_codes: torch.Tensor
+    down_scales: torch.Tensor
+
+    @property
+    def E(self) -> int:
+        return self.gate_codes.shape[0] - 1
+
+    @property
+    def f(self) -> int:
+        return self.gate_codes.shape[1]
+
+    @property
+    def d(self) -> int:
+        return self.gate_codes.shape[2] * 2
+
+    def struct(self) -> _Weights:
+        return _Weights(*(t.data_ptr() for t in (
+            self.gate_codes, self.gate_scales, self.up_codes, self.up_scales, self.down_codes,
+            self.down_scales)), self.E, self.d, self.f)
+
+    @staticmethod
+    def from_dict(d: dict) -> "LayerWeights":
+        return LayerWeights(**{k: d[k] for k in (
+            "gate_codes", "gate_scales", "up_codes", "up_scales", "down_codes", "down_scales")})
+
+
+def set_wait_limit_ns(n: int) -> None:
+    _check(lib().moe_set_wait_limit_ns(int(n)))
+
+
+def sync_status(stream=None) -> None:
+    _check(lib().moe_sync_status(_stream(stream)))
+
+
+def workspace_size(T: int, k: int, E: int, d: int, f: int) -> int:
+    return int(lib().moe_workspace_size(T, k, E, d, f))
+
+
+def alloc_workspace(T: int, k: int, E: int, d: int, f: int, device="cuda") -> torch.Tensor:
+    n = workspace_size(T, k, E, d, f)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def route_topk(scores: torch.Tensor, k: int, stream=None):
+    T, E = scores.shape
+    idx = torch.empty((T, k), dtype=torch.int32, device=scores.device)
+    w = torch.empty((T, k), dtype=torch.float32, device=scores.device)
+    _check(lib().moe_route_topk(_p(scores), T, E, k, _p(idx), _p(w), _stream(stream)))
+    return idx, w
+
+
+def dispatch(idx: torch.Tensor, E: int, stream=None):
+    T, k = idx.shape
+    dev = idx.device
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(max(T * k, 1), dtype=torch.int32, device=dev)
+    pos = torch.empty(max(T * k, 1), dtype=torch.int32, device=dev)
+    _check(lib().moe_dispatch(_p(idx), T, k, E, _p(counts), _p(offsets), _p(perm), _p(pos), None,
+                              0, _stream(stream)))
+    return counts, offsets, perm[:T * k], pos[:T * k]
+
+
+def act_quant(x: torch.Tensor, stream=None):
+    T, d = x.shape
+    qx = torch.empty((T, d), dtype=torch.uint8, device=x.device)
+    sx = torch.empty((T, d // 128), dtype=torch.float32, device=x.device)
+    _check(lib().moe_act_quant(_p(x), T, d, _p(qx), _p(sx), _stream(stream)))
+    return qx, sx
+
+
+def expert_ffn(x: torch.Tensor, k: int, w: LayerWeights, offsets: torch.Tensor,
+               perm: torch.Tensor, ws: torch.Tensor | None = None, out=None, stream=None):
+    T, d = x.shape
+    if ws is None:
+        ws = alloc_workspace(T, k, w.E, w.d, w.f, x.device)
+    if out is None:
+        y = torch.empty((max(T * k, 1), d), dtype=torch.float32, device=x.device)
+        ysh = torch.empty((max(T, 1), d), dtype=torch.float32, device=x.device)
+    else:
+        y, ysh = out
+    ws_struct = w.struct()
+    _check(lib().moe_expert_ffn(_p(x), T, k, ctypes.byref(ws_struct), _p(offsets), _p(perm),
+                                _p(y), _p(ysh), _p(ws), ws.numel(), _stream(stream)))
+    return y[:T * k], ysh[:T]
+
+
+def ffn_prepare(x, k, w: LayerWeights, offsets, perm, ws, stream=None):
+    T = x.shape[0]
+    st = w.struct()
+    _check(lib().moe_ffn_prepare(_p(x), T, k, ctypes.byref(st), _p(offsets), _p(perm), _p(ws),
+                                 ws.numel(), _stream(stream)))
+
+
+def ffn_gate_up(T, k, w: LayerWeights, ws, stream=None):
+    st = w.struct()
+    _check(lib().moe_ffn_gate_up(T, k, ctypes.byref(st), _p(ws), ws.numel(), _stream(stream)))
+
+
+def ffn_down(T, k, w: LayerWeights, y, ysh, ws, stream=None):
+    st = w.struct()
+    _check(lib().moe_ffn_down(T, k, ctypes.byref(st), _p(y), _p(ysh), _p(ws), ws.numel(),
+                              _stream(stream)))
+
+
+def combine(y_routed: torch.Tensor, y_shared: torch.Tensor, w: torch.Tensor, pos: torch.Tensor,
+            out: torch.Tensor | None = None, stream=None):
+    T, k = w.shape
+    d = y_shared.shape[1]
+    if out is None:
+        out = torch.empty((T, d), dtype=torch.float32, device=y_shared.device)
+    _check(lib().moe_combine(_p(y_routed), _p(y_shared), _p(w), _p(pos), T, k, d, _p(out),
+                             _stream(stream)))
+    return out
+
+
+def forward(x: torch.Tensor, scores: torch.Tensor, k: int, w: LayerWeights,
+            ws: torch.Tensor | None = None, stream=None):
+    """The whole layer through the four calls; returns a dict of every intermediate."""
+    idx, gw = route_topk(scores, k, stream)
+    counts, offsets, perm, pos = dispatch(idx, w.E, stream)
+    y, ysh = expert_ffn(x, k, w, offsets, perm, ws, stream=stream)
+    out = combine(y, ysh, gw, pos, stream=stream)
+    return dict(idx=idx, w=gw, counts=counts, offsets=offsets, perm=perm, pos=pos, y=y,
+                y_shared=ysh, out=out)

@@ -1,0 +1,352 @@
+// C ABI of libbitmoe.so: argument checks, workspace layout, error reporting, and the
+// launches of the routing, dispatch, quantisation, expert-FFN and combine kernels.
+// The calls follow the pages' statement of the problem: route (dpshk.com article,
+// "核心实现一"), group tokens per expert (same article, "核心实现三"), fused low-bit FFN
+// (same article, "核心实现四"; tcti.cn post, "补齐软件栈缺失"), weighted combine.
+#include "../../include/bitmoe.h"
+#include "internal.cuh"
+
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+namespace bitmoe {
+
+__device__ int g_status;  // device status word (kStatus* bits), one per device
+
+namespace {
+
+thread_local std::string t_err;
+std::atomic<long long> g_wait_ns{2000000000LL};
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_err = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(MOE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+struct DeviceInfo {
+  int sms = 0;
+  int status_ok = 0;
+  int* status = nullptr;
+};
+
+// Per-device facts, looked up once per device (SM count, sm_100 check, status address).
+int device_info(DeviceInfo& out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  static DeviceInfo cache[64];
+  static std::atomic<int> ready[64];
+  if (dev < 0 || dev >= 64) return fail(MOE_ERR_UNSUPPORTED, "device index %d", dev);
+  if (ready[dev].load(std::memory_order_acquire)) {
+    out = cache[dev];
+    return MOE_OK;
+  }
+  cudaDeviceProp prop;
+  e = cudaGetDeviceProperties(&prop, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDeviceProperties");
+  if (prop.major != 10 || prop.minor != 0)
+    return fail(MOE_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a", dev,
+                prop.major, prop.minor);
+  DeviceInfo d;
+  d.sms = prop.multiProcessorCount;
+  void* sp = nullptr;
+  e = cudaGetSymbolAddress(&sp, g_status);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status)");
+  d.status = static_cast<int*>(sp);
+  cache[dev] = d;
+  ready[dev].store(1, std::memory_order_release);
+  out = d;
+  return MOE_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+int check_weights(const moe_weights_t* w) {
+  if (w == nullptr) return fail(MOE_ERR_INVALID_ARG, "weights descriptor is NULL");
+  if (!w->gate_codes || !w->gate_scales || !w->up_codes || !w->up_scales || !w->down_codes ||
+      !w->down_scales)
+    return fail(MOE_ERR_INVALID_ARG, "a weight pointer is NULL");
+  if (w->E < 1 || w->E > 1024) return fail(MOE_ERR_INVALID_ARG, "E=%d outside [1, 1024]", w->E);
+  if (w->d < 128 || w->d % 128 || w->f < 128 || w->f % 128)
+    return fail(MOE_ERR_INVALID_ARG, "d=%d, f=%d must be positive multiples of 128", w->d, w->f);
+  if (w->d > 8192 || w->f > 8192)
+    return fail(MOE_ERR_INVALID_ARG, "d=%d, f=%d: at most 8192 supported", w->d, w->f);
+  if (!aligned(w->gate_codes, 32) || !aligned(w->up_codes, 32) || !aligned(w->down_codes, 32))
+    return fail(MOE_ERR_INVALID_ARG, "weight code arrays must be 32-byte aligned");
+  if (!aligned(w->gate_scales, 4) || !aligned(w->up_scales, 4) || !aligned(w->down_scales, 4))
+    return fail(MOE_ERR_INVALID_ARG, "weight scale arrays must be 4-byte aligned");
+  return MOE_OK;
+}
+
+}  // namespace
+
+WorkspaceLayout workspace_layout(int T, int k, int E, int d, int f) {
+  WorkspaceLayout L{};
+  const size_t R = (size_t)T * k + T;
+  size_t o = 0;
+  L.plan = o;
+  o = align256(o + 4 * ((size_t)E + 2 + 2 * plan_ntmax((int)R, E)));
+  L.qx = o;
+  o = align256(o + R * d);
+  L.sx = o;
+  o = align256(o + R * (d / 128) * 4);
+  L.qh = o;
+  o = align256(o + R * f);
+  L.sh = o;
+  o = align256(o + R * (f / 128) * 4);
+  L.total = o;
+  return L;
+}
+
+}  // namespace bitmoe
+
+using namespace bitmoe;
+
+extern "C" {
+
+const char* moe_last_error(void) { return t_err.c_str(); }
+
+int moe_set_wait_limit_ns(long long n) {
+  g_wait_ns.store(n > 0 ? n : 2000000000LL);
+  return MOE_OK;
+}
+
+size_t moe_workspace_size(int T, int k, int E, int d, int f) {
+  if (T < 0 || k < 1 || E < 1 || d < 128 || f < 128 || d % 128 || f % 128) return 0;
+  return workspace_layout(T, k, E, d, f).total;
+}
+
+int moe_sync_status(void* stream) {
+  DeviceInfo di;
+  int rc = device_info(di);
+  if (rc) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int host = 0;
+  e = cudaMemcpy(&host, di.status, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "read status");
+  if (host != 0) {
+    const int zero = 0;
+    e = cudaMemcpy(di.status, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "clear status");
+    if (host & kStatusTimeout)
+      return fail(MOE_ERR_TIMEOUT, "a device-side wait exceeded its limit (status 0x%x)", host);
+    return fail(MOE_ERR_INVALID_ARG, "an expert id or position was out of range (status 0x%x)",
+                host);
+  }
+  return MOE_OK;
+}
+
+int moe_route_topk(const float* scores, int T, int E, int k, int32_t* topk_idx, float* topk_w,
+                   void* stream) {
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T=%d < 0", T);
+  if (E < 1 || E > 1024) return fail(MOE_ERR_INVALID_ARG, "E=%d outside [1, 1024]", E);
+  if (k < 1 || k > E || k > 32) return fail(MOE_ERR_INVALID_ARG, "k=%d outside [1, min(E, 32)]", k);
+  if (T == 0) return MOE_OK;
+  if (!scores || !topk_idx || !topk_w) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(scores, 4) || !aligned(topk_idx, 4) || !aligned(topk_w, 4))
+    return fail(MOE_ERR_INVALID_ARG, "pointers must be 4-byte aligned");
+  DeviceInfo di;
+  int rc = device_info(di);
+  if (rc) return rc;
+  cudaError_t e =
+      launch_route_topk(scores, T, E, k, topk_idx, topk_w, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "route_topk launch");
+}
+
+int moe_dispatch(const int32_t* topk_idx, int T, int k, int E, int32_t* counts, int32_t* offsets,
+                 int32_t* perm, int32_t* pos, void* ws, size_t ws_bytes, void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T=%d < 0", T);
+  if (E < 1 || E > 1024) return fail(MOE_ERR_INVALID_ARG, "E=%d outside [1, 1024]", E);
+  if (k < 1 || k > E) return fail(MOE_ERR_INVALID_ARG, "k=%d outside [1, E]", k);
+  if ((long long)T * k > (1LL << 30)) return fail(MOE_ERR_INVALID_ARG, "T*k too large");
+  if (!counts || !offsets) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  if (T > 0 && (!topk_idx || !perm || !pos)) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  DeviceInfo di;
+  int rc = device_info(di);
+  if (rc) return rc;
+  // T == 0 still writes counts = 0 and offsets = 0 (the kernel handles P == 0)
+  cudaError_t e = launch_dispatch(topk_idx, T, k, E, counts, offsets, perm, pos, di.status,
+                                  static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "dispatch launch");
+}
+
+int moe_act_quant(const uint16_t* x_bf16, int T, int d, uint8_t* qx, float* sx, void* stream) {
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T=%d < 0", T);
+  if (d < 128 || d % 128 || d > 16384)
+    return fail(MOE_ERR_INVALID_ARG, "d=%d must be a multiple of 128 in [128, 16384]", d);
+  if (T == 0) return MOE_OK;
+  if (!x_bf16 || !qx || !sx) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(x_bf16, 16) || !aligned(qx, 16) || !aligned(sx, 4))
+    return fail(MOE_ERR_INVALID_ARG, "x and qx must be 16-byte aligned, sx 4-byte aligned");
+  DeviceInfo di;
+  int rc = device_info(di);
+  if (rc) return rc;
+  cudaError_t e = launch_quant_rows(x_bf16, T, 1, d, nullptr, 0, qx, sx, nullptr, 0, 0, nullptr,
+                                    di.status, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "act_quant launch");
+}
+
+namespace {
+
+struct FfnCtx {
+  DeviceInfo di;
+  WorkspaceLayout L;
+  int nmax;
+  uint8_t* ws;
+};
+
+int ffn_check(int T, int k, const moe_weights_t* w, void* ws, size_t ws_bytes, FfnCtx& c) {
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T=%d < 0", T);
+  int rc = check_weights(w);
+  if (rc) return rc;
+  if (k < 1 || k > w->E) return fail(MOE_ERR_INVALID_ARG, "k=%d outside [1, E]", k);
+  if ((long long)T * (k + 1) > (1LL << 28)) return fail(MOE_ERR_INVALID_ARG, "T too large");
+  rc = device_info(c.di);
+  if (rc) return rc;
+  c.L = workspace_layout(T, k, w->E, w->d, w->f);
+  if (T > 0) {
+    if (ws == nullptr || !aligned(ws, 256))
+      return fail(MOE_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned");
+    if (ws_bytes < c.L.total)
+      return fail(MOE_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, c.L.total);
+  }
+  c.nmax = nmax_for(T);
+  c.ws = static_cast<uint8_t*>(ws);
+  int max_smem = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  const size_t need = ffn_smem_bytes(1, c.nmax, w->d / 128, w->E) > ffn_smem_bytes(2, c.nmax, w->f / 128, w->E)
+                          ? ffn_smem_bytes(1, c.nmax, w->d / 128, w->E)
+                          : ffn_smem_bytes(2, c.nmax, w->f / 128, w->E);
+  if (need > (size_t)max_smem)
+    return fail(MOE_ERR_INVALID_ARG, "shape needs %zu bytes of shared memory (> %d)", need,
+                max_smem);
+  return MOE_OK;
+}
+
+FfnArgs ffn_args(int phase, int T, int k, const moe_weights_t* w, const FfnCtx& c) {
+  FfnArgs a{};
+  const int P = T * k;
+  a.E = w->E;
+  a.R = P + T;
+  a.P = P;
+  a.f = w->f;
+  a.d = w->d;
+  a.plan = reinterpret_cast<const int32_t*>(c.ws + c.L.plan);
+  a.wait_ns = g_wait_ns.load();
+  a.status = c.di.status;
+  if (phase == 1) {
+    a.a0_codes = w->gate_codes;
+    a.a0_scales = w->gate_scales;
+    a.a1_codes = w->up_codes;
+    a.a1_scales = w->up_scales;
+    a.b_codes = c.ws + c.L.qx;
+    a.b_scales = reinterpret_cast<const float*>(c.ws + c.L.sx);
+    a.K = w->d;
+    a.rows_per_expert = w->f;
+    a.qh = c.ws + c.L.qh;
+    a.sh = reinterpret_cast<float*>(c.ws + c.L.sh);
+  } else {
+    a.a0_codes = w->down_codes;
+    a.a0_scales = w->down_scales;
+    a.b_codes = c.ws + c.L.qh;
+    a.b_scales = reinterpret_cast<const float*>(c.ws + c.L.sh);
+    a.K = w->f;
+    a.rows_per_expert = w->d;
+  }
+  return a;
+}
+
+}  // namespace
+
+int moe_ffn_prepare(const uint16_t* x_bf16, int T, int k, const moe_weights_t* w,
+                    const int32_t* offsets, const int32_t* perm, void* ws, size_t ws_bytes,
+                    void* stream) {
+  FfnCtx c;
+  int rc = ffn_check(T, k, w, ws, ws_bytes, c);
+  if (rc) return rc;
+  if (T == 0) return MOE_OK;
+  if (!x_bf16 || !offsets || !perm) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(x_bf16, 16)) return fail(MOE_ERR_INVALID_ARG, "x must be 16-byte aligned");
+  cudaError_t e = launch_quant_rows(
+      x_bf16, T, k, w->d, perm, T * k, c.ws + c.L.qx, reinterpret_cast<float*>(c.ws + c.L.sx),
+      offsets, w->E, c.nmax, reinterpret_cast<int32_t*>(c.ws + c.L.plan), c.di.status,
+      static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "ffn prepare launch");
+}
+
+int moe_ffn_gate_up(int T, int k, const moe_weights_t* w, void* ws, size_t ws_bytes,
+                    void* stream) {
+  FfnCtx c;
+  int rc = ffn_check(T, k, w, ws, ws_bytes, c);
+  if (rc) return rc;
+  if (T == 0) return MOE_OK;
+  cudaError_t e = launch_ffn(1, c.nmax, ffn_args(1, T, k, w, c),
+                             static_cast<cudaStream_t>(stream), c.di.sms);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "ffn gate/up launch");
+}
+
+int moe_ffn_down(int T, int k, const moe_weights_t* w, float* y_routed, float* y_shared,
+                 void* ws, size_t ws_bytes, void* stream) {
+  FfnCtx c;
+  int rc = ffn_check(T, k, w, ws, ws_bytes, c);
+  if (rc) return rc;
+  if (T == 0) return MOE_OK;
+  if (!y_routed || !y_shared) return fail(MOE_ERR_INVALID_ARG, "NULL output pointer");
+  if (!aligned(y_routed, 16) || !aligned(y_shared, 16))
+    return fail(MOE_ERR_INVALID_ARG, "outputs must be 16-byte aligned");
+  FfnArgs a = ffn_args(2, T, k, w, c);
+  a.y_routed = y_routed;
+  a.y_shared = y_shared;
+  cudaError_t e = launch_ffn(2, c.nmax, a, static_cast<cudaStream_t>(stream), c.di.sms);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "ffn down launch");
+}
+
+int moe_expert_ffn(const uint16_t* x_bf16, int T, int k, const moe_weights_t* w,
+                   const int32_t* offsets, const int32_t* perm, float* y_routed, float* y_shared,
+                   void* ws, size_t ws_bytes, void* stream) {
+  int rc = moe_ffn_prepare(x_bf16, T, k, w, offsets, perm, ws, ws_bytes, stream);
+  if (rc) return rc;
+  rc = moe_ffn_gate_up(T, k, w, ws, ws_bytes, stream);
+  if (rc) return rc;
+  return moe_ffn_down(T, k, w, y_routed, y_shared, ws, ws_bytes, stream);
+}
+
+int moe_combine(const float* y_routed, const float* y_shared, const float* topk_w,
+                const int32_t* pos, int T, int k, int d, float* out, void* stream) {
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T=%d < 0", T);
+  if (k < 1 || k > 32) return fail(MOE_ERR_INVALID_ARG, "k=%d outside [1, 32]", k);
+  if (d < 4 || d % 4) return fail(MOE_ERR_INVALID_ARG, "d=%d must be a positive multiple of 4", d);
+  if (T == 0) return MOE_OK;
+  if (!y_routed || !y_shared || !topk_w || !pos || !out)
+    return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(y_routed, 16) || !aligned(y_shared, 16) || !aligned(out, 16))
+    return fail(MOE_ERR_INVALID_ARG, "y_routed, y_shared and out must be 16-byte aligned");
+  DeviceInfo di;
+  int rc = device_info(di);
+  if (rc) return rc;
+  cudaError_t e = launch_combine(y_routed, y_shared, topk_w, pos, T, k, d, out, di.status,
+                                 static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "combine launch");
+}
+
+}  // extern "C"

@@ -1,0 +1,505 @@
+// Expert FFN on the 5th-generation tensor cores: block-scaled FP4 (e2m1) weights x
+// FP8 (e4m3) activations, tcgen05.mma kind::mxf8f6f4 with fp32 accumulators in TMEM.
+//
+// Pages followed: tcti.cn post, "补齐软件栈缺失" (fp4_gemm: FP8-quantised activation x
+// FP4 packed weight; act_quant) and "DeepSeek-V4-Flash的可能性" (prefill compute-bound,
+// decode memory-bound); dpshk.com article, "核心实现三" (an expert's weights are read
+// once for every token routed to it) and "核心实现四" (FP4 dequantised inside the
+// product, gate and up on one quantised input).  Here the dequantisation happens in
+// the tensor core itself: TMA unpacks the FP4 codes into byte containers in shared
+// memory and the MMA applies the ue8m0 block scales from TMEM.
+//
+// Work decomposition ("swap-AB"): a tile is (expert e, 128-row block of the weight
+// matrix, token tile of n <= NMAX rows).  The weight rows are the MMA's M = 128; the
+// tokens are its N (n rounded up to 16), so ragged expert groups waste at most 15
+// columns.  Phase 1 multiplies the gate AND up rows of the same 128 h-rows with one
+// shared activation tile, then computes h = silu(g) * u and re-quantises it per
+// 128-block to e4m3; phase 2 is the down projection writing fp32 y.
+//
+// Activation scales are fp32 (amax/448), not ue8m0, so they cannot ride in the MMA:
+// B's hardware scale is 1.0 and every 128-wide K chunk is accumulated into a fresh
+// TMEM partial, which the epilogue warps fold into fp32 registers as acc += s * P.
+// Two TMEM partial buffers let the MMA run one chunk ahead of the epilogue.
+//
+// Warp roles (320 threads, one CTA per SM, persistent over tiles):
+//   warp 0   : TMA producer (weights, activations) + cp.async of the weight scales
+//   warp 1   : TMEM allocator; lane 0 issues tcgen05.cp / tcgen05.mma / commits
+//   warps 2-9: epilogue; warp w reads TMEM lanes 32*(w%4).., column half (w-2)/4
+// Every wait is bounded by a %globaltimer limit; on expiry the kernel records a
+// timeout in the status word, lets in-flight copies and MMAs land, frees TMEM and
+// returns.
+#include "internal.cuh"
+#include "ptx.cuh"
+
+#include <cstring>
+#include <mutex>
+
+namespace bitmoe {
+namespace {
+
+constexpr int kThreads = 320;
+constexpr int kEpiWarps = 8;
+constexpr int kLag = 2;                         // scale cp.async groups in flight
+constexpr long long kDrainNs = 500000000LL;     // bound on draining in-flight work
+
+struct FfnParams {
+  CUtensorMap tmA0;  // gate (phase 1) / down (phase 2) codes, all experts stacked
+  CUtensorMap tmA1;  // up codes (phase 1)
+  CUtensorMap tmB;   // activation rows [R][K] e4m3
+  const uint8_t* sfa0;
+  const uint8_t* sfa1;
+  const float* b_scales;  // [R][K/128]
+  const int32_t* plan;
+  int E, K, rows_per_expert, R, P, f, d;
+  uint8_t* qh;
+  float* sh;
+  float* y_routed;
+  float* y_shared;
+  long long wait_ns;
+  int* status;
+};
+
+template <int PHASE, int NMAX, int STAGES>
+struct Cfg {
+  static constexpr int kNumA = PHASE == 1 ? 2 : 1;
+  static constexpr int kATile = 128 * 128;  // 128 rows x 128 FP4 in byte containers
+  static constexpr int kBTile = NMAX * 128;
+  static constexpr int kSF = 512;
+  static constexpr int kStageRaw = kNumA * kATile + kBTile + kNumA * kSF;
+  static constexpr int kStage = (kStageRaw + 1023) / 1024 * 1024;
+  static constexpr int kHalf = NMAX / 2;
+  static constexpr int kAccCols = PHASE == 1 ? 2 * NMAX : NMAX;  // per TMEM buffer
+  static constexpr int kColSFA0 = 2 * kAccCols;
+  static constexpr int kColSFA1 = kColSFA0 + 4;
+  static constexpr int kColSFB = kColSFA0 + 4 * kNumA;
+  static_assert(kColSFB + 4 <= 512, "TMEM columns");
+  static_assert(NMAX % 16 == 0 && kHalf % 8 == 0, "tile width");
+  static_assert(kLag <= STAGES - 1, "scale lag must leave a stage to the consumer");
+  // shared memory after the stages
+  static constexpr int kOffSFB = STAGES * kStage;
+  static constexpr int kOffBars = kOffSFB + 512;
+  static constexpr int kNumBars = 2 * STAGES + 5;
+  static constexpr int kOffMisc = kOffBars + 8 * kNumBars;  // tmem slot, abort flag
+  static constexpr int kOffAmax = kOffMisc + 16;
+  static constexpr int kOffTT = kOffAmax + 2 * 4 * kHalf * 4;  // plan prefix, E+2 ints
+  __host__ __device__ static size_t off_sbs(int E) { return (size_t)kOffTT + ((size_t)(E + 2) * 4 + 15) / 16 * 16; }
+  __host__ __device__ static size_t smem_bytes(int nk, int E) {
+    return 1024 + off_sbs(E) + (size_t)nk * NMAX * 4;
+  }
+};
+
+__device__ __forceinline__ void bar_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// Bounded wait by one thread; false if the limit ran out or another role aborted.
+__device__ bool wait_one(uint32_t bar, uint32_t parity, long long limit, volatile int* abort_flag,
+                         int* status) {
+  if (*abort_flag) return false;
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer();
+  while (!*abort_flag) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if ((long long)(ptx::globaltimer() - t0) > limit) {
+      *abort_flag = 1;
+      atomicOr(status, kStatusTimeout);
+      return false;
+    }
+  }
+  return false;
+}
+// Same, decided by lane 0 and shared with the whole warp (keeps the warp converged).
+__device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, long long limit,
+                                          volatile int* abort_flag, int* status) {
+  int ok = 0;
+  if ((threadIdx.x & 31) == 0) ok = wait_one(bar, parity, limit, abort_flag, status) ? 1 : 0;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+// Wait for in-flight work to land during teardown (ignores the abort flag).
+__device__ void drain_wait(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = ptx::globaltimer();
+  while (!ptx::mbar_try_wait(bar, parity)) {
+    if ((long long)(ptx::globaltimer() - t0) > kDrainNs) break;
+  }
+}
+
+// Tile i -> (expert, 128-row block, first activation row, rows).  Tiles of one expert
+// are ordered (block, token tile) so CTAs working at the same time share weight rows.
+__device__ __forceinline__ void decode_tile(const int32_t* ttbase, const int32_t* tiles, int E,
+                                            int HB, int i, int& e, int& blk, int& row0, int& n) {
+  int lo = 0, hi = E;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (ttbase[mid] * HB <= i) lo = mid; else hi = mid - 1;
+  }
+  e = lo;
+  const int nt = ttbase[e + 1] - ttbase[e];
+  const int local = i - ttbase[e] * HB;
+  blk = local / nt;
+  const int tt = ttbase[e] + local % nt;
+  row0 = __ldg(tiles + 2 * tt);
+  n = __ldg(tiles + 2 * tt + 1);
+}
+
+template <int PHASE, int NMAX, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant__ FfnParams p) {
+  using C = Cfg<PHASE, NMAX, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  uint8_t* sfb = smem + C::kOffSFB;
+  const uint32_t bars = ptx::smem_u32(smem + C::kOffBars);
+  auto full = [&](int s) { return bars + 8u * s; };
+  auto empty = [&](int s) { return bars + 8u * (STAGES + s); };
+  auto tfull = [&](int b) { return bars + 8u * (2 * STAGES + b); };
+  auto tempty = [&](int b) { return bars + 8u * (2 * STAGES + 2 + b); };
+  const uint32_t drain = bars + 8u * (2 * STAGES + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+  float* amax_s = reinterpret_cast<float*>(smem + C::kOffAmax);
+  int32_t* s_ttbase = reinterpret_cast<int32_t*>(smem + C::kOffTT);
+  float* sbs = reinterpret_cast<float*>(smem + C::off_sbs(p.E));
+
+  const int nk = p.K / 128;
+  const int HB = p.rows_per_expert / 128;
+  const int32_t* g_tiles = p.plan + p.E + 2;
+  for (int e = threadIdx.x; e < p.E + 2; e += kThreads) s_ttbase[e] = __ldg(p.plan + e);
+  const int32_t* g_ttbase = s_ttbase;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      ptx::mbar_init(full(s), 2);   // TMA arrive.expect_tx + scale-factor arrive
+      ptx::mbar_init(empty(s), 1);  // tcgen05.commit
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(tfull(b), 1);
+      ptx::mbar_init(tempty(b), kEpiWarps);
+    }
+    ptx::mbar_init(drain, 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), 512);
+    ptx::tmem_relinquish();
+  }
+  if (threadIdx.x >= 64 && threadIdx.x < 64 + 128)  // B scale factors: all 1.0 (0x7F)
+    reinterpret_cast<uint32_t*>(sfb)[threadIdx.x - 64] = 0x7F7F7F7Fu;
+  ptx::fence_proxy_async_smem();
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int total = g_ttbase[p.E + 1] * HB;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      ptx::prefetch_tmap(&p.tmA0);
+      if (PHASE == 1) ptx::prefetch_tmap(&p.tmA1);
+      ptx::prefetch_tmap(&p.tmB);
+    }
+    const size_t ldsf = (size_t)(p.K / 32);
+    int it = 0;
+    bool ok = true;
+    for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
+      int e, blk, row0, n;
+      decode_tile(g_ttbase, g_tiles, p.E, HB, i, e, blk, row0, n);
+      const int rowA = e * p.rows_per_expert + blk * 128;
+      const int nB = (n + 15) / 16;
+      const uint32_t tx = (uint32_t)(C::kNumA * 8192 + nB * 2048);  // packed FP4 + e4m3 bytes
+      for (int kc = 0; kc < nk; ++kc) {
+        const int s = it % STAGES;
+        const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+        if (!wait_warp(empty(s), ph ^ 1u, p.wait_ns, abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        uint8_t* st = smem + s * C::kStage;
+        const uint32_t st_u = ptx::smem_u32(st);
+        if (lane == 0) {
+          ptx::mbar_arrive_expect_tx(full(s), tx);
+          ptx::tma_load_2d(st_u, &p.tmA0, kc * 128, rowA, full(s));
+          if (PHASE == 1) ptx::tma_load_2d(st_u + C::kATile, &p.tmA1, kc * 128, rowA, full(s));
+          for (int j = 0; j < nB; ++j)
+            ptx::tma_load_2d(st_u + C::kNumA * C::kATile + j * 2048, &p.tmB, kc * 128,
+                             row0 + 16 * j, full(s));
+        }
+        // weight scales of this 128-wide chunk: 4 bytes per row, laid out for
+        // tcgen05.cp 32x128b.warpx4 (row m at byte (m%32)*16 + (m/32)*4)
+        const uint32_t sf0 = st_u + C::kNumA * C::kATile + C::kBTile;
+#pragma unroll
+        for (int m1 = 0; m1 < 4; ++m1) {
+          const size_t r = (size_t)(rowA + m1 * 32 + lane);
+          ptx::cp_async_4(sf0 + lane * 16 + m1 * 4, p.sfa0 + r * ldsf + kc * 4);
+          if (PHASE == 1) ptx::cp_async_4(sf0 + 512 + lane * 16 + m1 * 4, p.sfa1 + r * ldsf + kc * 4);
+        }
+        ptx::cp_async_commit();
+        if (it >= kLag) {
+          ptx::cp_async_wait_group<kLag>();
+          ptx::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(full((it - kLag) % STAGES));
+        }
+        ++it;
+      }
+    }
+    ptx::cp_async_wait_all();
+    ptx::fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      for (int j = it - kLag < 0 ? 0 : it - kLag; j < it; ++j) ptx::mbar_arrive(full(j % STAGES));
+      if (!ok)  // let every issued TMA copy land before the CTA can exit
+        for (int j = it - STAGES < 0 ? 0 : it - STAGES; j < it; ++j)
+          drain_wait(full(j % STAGES), (uint32_t)(j / STAGES) & 1u);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      ptx::tc_cp_32x128b_x4(tmem + C::kColSFB, ptx::make_sdesc(ptx::smem_u32(sfb), 0, 128, 0));
+      int it = 0, ch = 0;
+      bool ok = true;
+      for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
+        int e, blk, row0, n;
+        decode_tile(g_ttbase, g_tiles, p.E, HB, i, e, blk, row0, n);
+        const uint32_t N = (uint32_t)((n + 15) & ~15);
+        // kind::mxf8f6f4 instruction descriptor: A = e2m1 (5), B = e4m3 (0), both K-major,
+        // ue8m0 scales, N >> 3 at bit 17, M >> 4 at bit 24; A scale id at bits 29-30.
+        const uint32_t idesc0 = (5u << 7) | (0u << 10) | ((N >> 3) << 17) | (1u << 23) |
+                                ((128u >> 4) << 24);
+        for (int kc = 0; kc < nk; ++kc) {
+          const int s = it % STAGES;
+          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+          const int b = ch & 1;
+          const uint32_t tph = (uint32_t)(ch >> 1) & 1u;
+          if (!wait_one(tempty(b), tph ^ 1u, p.wait_ns, abort_flag, p.status)) { ok = false; break; }
+          ptx::tc_fence_after();
+          if (!wait_one(full(s), ph, p.wait_ns, abort_flag, p.status)) { ok = false; break; }
+          ptx::tc_fence_after();
+          const uint32_t a0 = ptx::smem_u32(smem + s * C::kStage);
+          const uint32_t bb = a0 + C::kNumA * C::kATile;
+          const uint32_t sf0 = bb + C::kBTile;
+          ptx::tc_cp_32x128b_x4(tmem + C::kColSFA0, ptx::make_sdesc(sf0, 0, 128, 0));
+          if (PHASE == 1)
+            ptx::tc_cp_32x128b_x4(tmem + C::kColSFA1, ptx::make_sdesc(sf0 + 512, 0, 128, 0));
+          const uint64_t da0 = ptx::make_sdesc(a0, 16, 1024, 2);
+          const uint64_t da1 = ptx::make_sdesc(a0 + C::kATile, 16, 1024, 2);
+          const uint64_t db = ptx::make_sdesc(bb, 16, 1024, 2);
+          const uint32_t acc = tmem + (uint32_t)(b * C::kAccCols);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {  // four K = 32 steps through the 128-byte rows
+            // scale id kk selects byte kk of each SFA word: the scale of K-block kk
+            const uint32_t idesc = idesc0 | ((uint32_t)kk << 29);
+            ptx::tc_mma_mxf8f6f4(acc, da0 + 2 * kk, db + 2 * kk, idesc,
+                                 tmem + C::kColSFA0, tmem + C::kColSFB,
+                                 kk > 0 ? 1u : 0u);
+            if (PHASE == 1)
+              ptx::tc_mma_mxf8f6f4(acc + NMAX, da1 + 2 * kk, db + 2 * kk, idesc,
+                                   tmem + C::kColSFA1, tmem + C::kColSFB,
+                                   kk > 0 ? 1u : 0u);
+          }
+          ptx::tc_commit(empty(s));
+          ptx::tc_commit(tfull(b));
+          ++it;
+          ++ch;
+        }
+      }
+      ptx::tc_commit(drain);  // every MMA / copy of this thread done before teardown
+      drain_wait(drain, 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int ew = warp - 2;
+    const int q = warp & 3;
+    const int h = ew >> 2;
+    const int col0 = h * C::kHalf;
+    const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
+    int ch = 0;
+    bool ok = true;
+    for (int i = blockIdx.x; i < total; i += gridDim.x) {
+      int e, blk, row0, n;
+      decode_tile(g_ttbase, g_tiles, p.E, HB, i, e, blk, row0, n);
+      // this tile's activation scales, transposed to sbs[kc][column]
+      bar_sync(1, kEpiWarps * 32);
+      for (int x = ew * 32 + lane; x < n * nk; x += kEpiWarps * 32) {
+        const int c = x / nk, kc = x - c * nk;
+        sbs[kc * NMAX + c] = __ldg(p.b_scales + (size_t)(row0 + c) * nk + kc);
+      }
+      bar_sync(1, kEpiWarps * 32);
+      float acc0[C::kHalf], acc1[C::kHalf];
+#pragma unroll
+      for (int c = 0; c < C::kHalf; ++c) {
+        acc0[c] = 0.f;
+        acc1[c] = 0.f;
+      }
+      for (int kc = 0; kc < nk; ++kc) {
+        const int b = ch & 1;
+        const uint32_t tph = (uint32_t)(ch >> 1) & 1u;
+        ok = ok && wait_warp(tfull(b), tph, p.wait_ns, abort_flag, p.status);
+        ptx::tc_fence_after();
+        if (ok) {
+          const uint32_t base = tl + (uint32_t)(b * C::kAccCols + col0);
+          const float* sc = sbs + kc * NMAX + col0;
+#pragma unroll
+          for (int g = 0; g < C::kHalf / 8; ++g) {
+            if (col0 + 8 * g < n) {
+              float v0[8], v1[8];
+              ptx::tc_ld_32x32b_x8(base + 8 * g, v0);
+              if (PHASE == 1) ptx::tc_ld_32x32b_x8(base + NMAX + 8 * g, v1);
+              ptx::tc_wait_ld();
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                acc0[8 * g + j] = fmaf(sc[8 * g + j], v0[j], acc0[8 * g + j]);
+                if (PHASE == 1) acc1[8 * g + j] = fmaf(sc[8 * g + j], v1[j], acc1[8 * g + j]);
+              }
+            }
+          }
+        }
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(tempty(b));
+        ++ch;
+      }
+      if (PHASE == 1) {
+        // h = silu(g) * u, then per-column (token) e4m3 re-quantisation over the 128 rows
+        float* hv = acc0;  // h overwrites g in place
+        float* am = amax_s + (h * 4 + q) * C::kHalf;
+#pragma unroll
+        for (int c = 0; c < C::kHalf; ++c) {
+          const float g = acc0[c];
+          hv[c] = g / (1.0f + expf(-g)) * acc1[c];
+          const unsigned m = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(hv[c])));
+          if (lane == 0) am[c] = __uint_as_float(m);
+        }
+        bar_sync(2 + h, 128);
+#pragma unroll
+        for (int c = 0; c < C::kHalf; ++c) {
+          if (ok && col0 + c < n) {
+            float amax = amax_s[(h * 4 + 0) * C::kHalf + c];
+            amax = fmaxf(amax, amax_s[(h * 4 + 1) * C::kHalf + c]);
+            amax = fmaxf(amax, amax_s[(h * 4 + 2) * C::kHalf + c]);
+            amax = fmaxf(amax, amax_s[(h * 4 + 3) * C::kHalf + c]);
+            const float s = amax == 0.f ? 1.0f : __fdiv_rn(amax, 448.0f);
+            const int row = row0 + col0 + c;
+            const uint16_t code = ptx::cvt_e4m3x2(__fdiv_rn(hv[c], s), 0.f);
+            p.qh[(size_t)row * p.f + blk * 128 + q * 32 + lane] = (uint8_t)(code & 0xFF);
+            if (q == 0 && lane == 0) p.sh[(size_t)row * (p.f / 128) + blk] = s;
+          }
+        }
+        bar_sync(2 + h, 128);
+      } else {
+#pragma unroll
+        for (int c = 0; c < C::kHalf; ++c) {
+          if (ok && col0 + c < n) {
+            const int row = row0 + col0 + c;
+            float* dst = row < p.P ? p.y_routed + (size_t)row * p.d
+                                   : p.y_shared + (size_t)(row - p.P) * p.d;
+            dst[blk * 128 + q * 32 + lane] = acc0[c];
+          }
+        }
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// 2-D map over a row-major matrix [rows][K]; box = 128 elements of K x box_rows rows,
+// 128-byte swizzle (the layout the UMMA shared-memory descriptors expect).
+bool make_map(CUtensorMap* m, const void* base, bool fp4, int K, long long rows, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)(fp4 ? K / 2 : K)};
+  const cuuint32_t box[2] = {128u, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1u, 1u};
+  const CUresult r = fn(m, fp4 ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B : CU_TENSOR_MAP_DATA_TYPE_UINT8,
+                        2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int PHASE, int NMAX, int STAGES>
+cudaError_t launch_one(const FfnParams& prm, int nk, cudaStream_t s, int grid) {
+  using C = Cfg<PHASE, NMAX, STAGES>;
+  const size_t smem = C::smem_bytes(nk, prm.E);
+  cudaError_t err = cudaFuncSetAttribute(ffn_kernel<PHASE, NMAX, STAGES>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  ffn_kernel<PHASE, NMAX, STAGES><<<grid, kThreads, smem, s>>>(prm);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t ffn_smem_bytes(int phase, int nmax, int nk, int E) {
+  if (phase == 1)
+    return nmax == kNmaxSmall ? Cfg<1, kNmaxSmall, 5>::smem_bytes(nk, E)
+                              : Cfg<1, kNmaxLarge, 4>::smem_bytes(nk, E);
+  return nmax == kNmaxSmall ? Cfg<2, kNmaxSmall, 8>::smem_bytes(nk, E)
+                            : Cfg<2, kNmaxLarge, 6>::smem_bytes(nk, E);
+}
+
+cudaError_t launch_ffn(int phase, int nmax, const FfnArgs& a, cudaStream_t s, int num_sms) {
+  FfnParams prm;
+  memset(&prm, 0, sizeof(prm));
+  const long long rows_total = (long long)(a.E + 1) * a.rows_per_expert;
+  if (!make_map(&prm.tmA0, a.a0_codes, true, a.K, rows_total, 128)) return cudaErrorInvalidValue;
+  if (phase == 1 && !make_map(&prm.tmA1, a.a1_codes, true, a.K, rows_total, 128))
+    return cudaErrorInvalidValue;
+  if (!make_map(&prm.tmB, a.b_codes, false, a.K, a.R, 16)) return cudaErrorInvalidValue;
+  prm.sfa0 = a.a0_scales;
+  prm.sfa1 = a.a1_scales;
+  prm.b_scales = a.b_scales;
+  prm.plan = a.plan;
+  prm.E = a.E;
+  prm.K = a.K;
+  prm.rows_per_expert = a.rows_per_expert;
+  prm.R = a.R;
+  prm.P = a.P;
+  prm.f = a.f;
+  prm.d = a.d;
+  prm.qh = a.qh;
+  prm.sh = a.sh;
+  prm.y_routed = a.y_routed;
+  prm.y_shared = a.y_shared;
+  prm.wait_ns = a.wait_ns;
+  prm.status = a.status;
+  const int nk = a.K / 128;
+  if (phase == 1)
+    return nmax == kNmaxSmall ? launch_one<1, kNmaxSmall, 5>(prm, nk, s, num_sms)
+                              : launch_one<1, kNmaxLarge, 4>(prm, nk, s, num_sms);
+  return nmax == kNmaxSmall ? launch_one<2, kNmaxSmall, 8>(prm, nk, s, num_sms)
+                            : launch_one<2, kNmaxLarge, 6>(prm, nk, s, num_sms);
+}
+
+}  // namespace bitmoe

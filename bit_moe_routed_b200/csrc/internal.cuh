@@ -1,0 +1,68 @@
+// Internal declarations shared by the bitmoe CUDA sources (not part of the C ABI).
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace bitmoe {
+
+// Device-side status word (one per device): bit 0 = a bounded wait expired,
+// bit 1 = an expert id outside [0, E) reached the dispatch kernel.
+constexpr int kStatusTimeout = 1;
+constexpr int kStatusBadIndex = 2;
+
+// Token tiles of the expert FFN: every expert's rows (routed pairs in expert-sorted
+// order, then the T shared-expert rows) are cut into tiles of at most kNmax rows.
+constexpr int kNmaxLarge = 112;  // T > 32
+constexpr int kNmaxSmall = 32;   // T <= 32: every group fits one tile
+inline int nmax_for(int T) { return T <= kNmaxSmall ? kNmaxSmall : kNmaxLarge; }
+
+// Plan layout (int32 words in the workspace):
+//   [0, E+2)              ttbase: first token tile of expert e (e = 0..E), ttbase[E+1] = total
+//   [E+2, E+2 + 2*ntmax)  tiles: (row0, n) per token tile
+inline size_t plan_ntmax(int R, int E) { return (size_t)R / 16 + (size_t)E + 2; }
+
+struct WorkspaceLayout {
+  size_t plan, qx, sx, qh, sh, total;
+};
+WorkspaceLayout workspace_layout(int T, int k, int E, int d, int f);
+
+// Host launchers (each returns a cudaError_t of the launch)
+cudaError_t launch_route_topk(const float* scores, int T, int E, int k, int32_t* idx, float* w,
+                              cudaStream_t s);
+cudaError_t launch_dispatch(const int32_t* idx, int T, int k, int E, int32_t* counts,
+                            int32_t* offsets, int32_t* perm, int32_t* pos, int* status,
+                            cudaStream_t s);
+// rows r < P = T*k take token perm[r]/k, rows P <= r < P+T take token r-P; perm may be
+// NULL with P = 0 for a plain quantisation of T rows.  If plan != NULL, one extra block
+// writes the token-tile plan.
+cudaError_t launch_quant_rows(const uint16_t* x, int T, int k, int d, const int32_t* perm,
+                              int nrows_routed, uint8_t* q, float* s, const int32_t* offsets,
+                              int E, int nmax, int32_t* plan, int* status, cudaStream_t st);
+cudaError_t launch_combine(const float* y, const float* ysh, const float* w, const int32_t* pos,
+                           int T, int k, int d, float* out, int* status, cudaStream_t s);
+
+struct FfnArgs {
+  const uint8_t* a0_codes;   // gate (phase 1) or down (phase 2) codes, all experts
+  const uint8_t* a0_scales;
+  const uint8_t* a1_codes;   // up (phase 1 only)
+  const uint8_t* a1_scales;
+  const uint8_t* b_codes;    // qx (phase 1) or qh (phase 2) rows [R][K]
+  const float* b_scales;     // sx or sh [R][K/128]
+  const int32_t* plan;
+  int E, K, rows_per_expert, R, P;
+  uint8_t* qh;               // phase 1 outputs
+  float* sh;
+  int f;
+  float* y_routed;           // phase 2 outputs
+  float* y_shared;
+  int d;
+  long long wait_ns;
+  int* status;
+};
+cudaError_t launch_ffn(int phase, int nmax, const FfnArgs& a, cudaStream_t s, int num_sms);
+size_t ffn_smem_bytes(int phase, int nmax, int nk, int E);  // dynamic shared memory of a launch
+
+
+}  // namespace bitmoe

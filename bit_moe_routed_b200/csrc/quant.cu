@@ -1,0 +1,125 @@
+// Activation quantisation (tcti.cn post, "补齐软件栈缺失": act_quant feeds the FP8
+// activations of fp4_gemm) fused with the gather of the expert FFN's input rows, and
+// the token-tile plan of the FFN kernels.
+//
+// Row r of the output takes token perm[r] / k for r < P (routed pairs in expert-sorted
+// order) and token r - P for P <= r < P + T (shared expert), so every expert's input
+// rows are contiguous and the FFN reads them with plain 2-D TMA boxes.
+// Per 128-element block: s = amax / 448 (fp32, IEEE divide; 1 if amax == 0),
+// q = e4m3(x / s), round to nearest even, saturating.  8 threads share a block; each
+// holds 16 consecutive bf16 values (two 16-byte loads) and writes 16 code bytes.
+#include "internal.cuh"
+#include "ptx.cuh"
+
+namespace bitmoe {
+namespace {
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Token tiles: expert e (e < E: routed group offsets[e]..offsets[e+1]; e == E: the T
+// shared rows) is cut into ceil(n / nmax) tiles of roundup16(ceil(n / ntiles)) rows,
+// the last one shorter.  One warp computes the per-expert tile counts and their scan.
+__device__ void write_plan(const int32_t* __restrict__ offsets, int E, int T, int P, int nmax,
+                           int32_t* __restrict__ plan) {
+  const int lane = threadIdx.x & 31;
+  int32_t* ttbase = plan;
+  int32_t* tiles = plan + E + 2;
+  const int per = (E + 1 + 31) / 32;  // experts per lane, contiguous
+  const int e0 = lane * per;
+  int local = 0;
+  for (int e = e0; e < min(E + 1, e0 + per); ++e) {
+    const int n = e < E ? offsets[e + 1] - offsets[e] : T;
+    local += (n + nmax - 1) / nmax;
+  }
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  int base = incl - local;
+  for (int e = e0; e < min(E + 1, e0 + per); ++e) {
+    const int n = e < E ? offsets[e + 1] - offsets[e] : T;
+    const int row = e < E ? offsets[e] : P;
+    const int nt = (n + nmax - 1) / nmax;
+    ttbase[e] = base;
+    if (nt > 0) {
+      const int step = (((n + nt - 1) / nt) + 15) / 16 * 16;
+      for (int i = 0; i < nt; ++i) {
+        tiles[2 * (base + i)] = row + i * step;
+        tiles[2 * (base + i) + 1] = min(step, n - i * step);
+      }
+    }
+    base += nt;
+  }
+  if (lane == 31) ttbase[E + 1] = incl;
+}
+
+__global__ void __launch_bounds__(256) quant_rows_kernel(
+    const uint16_t* __restrict__ x, int T, int k, int d, const int32_t* __restrict__ perm, int P,
+    uint8_t* __restrict__ q, float* __restrict__ s, const int32_t* __restrict__ offsets, int E,
+    int nmax, int32_t* __restrict__ plan, int* __restrict__ status) {
+  const int R = P + T;
+  const int r = blockIdx.x;
+  if (r == R) {  // the plan block
+    if (threadIdx.x < 32) write_plan(offsets, E, T, P, nmax, plan);
+    return;
+  }
+  int t = r < P ? perm[r] / k : r - P;
+  bool ok = t >= 0 && t < T;
+  if (!ok && threadIdx.x == 0) atomicOr(status, kStatusBadIndex);
+  const uint16_t* xr = x + (size_t)(ok ? t : 0) * d;
+  // every lane of a warp runs the same number of iterations (full-mask shuffles);
+  // a group of 8 lanes (one 128-block) is either wholly inside the row or wholly past it
+  const int lane16 = (threadIdx.x & 31) * 16;
+  for (int c0 = threadIdx.x * 16; c0 - lane16 < d; c0 += blockDim.x * 16) {
+    const bool act = c0 < d;
+    uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
+    if (act && ok) {
+      a = *reinterpret_cast<const uint4*>(xr + c0);
+      b = *reinterpret_cast<const uint4*>(xr + c0 + 8);
+    }
+    const float v[16] = {bf16_lo(a.x), bf16_hi(a.x), bf16_lo(a.y), bf16_hi(a.y),
+                         bf16_lo(a.z), bf16_hi(a.z), bf16_lo(a.w), bf16_hi(a.w),
+                         bf16_lo(b.x), bf16_hi(b.x), bf16_lo(b.y), bf16_hi(b.y),
+                         bf16_lo(b.z), bf16_hi(b.z), bf16_lo(b.w), bf16_hi(b.w)};
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    // the 8 threads of one 128-block are lanes 8j..8j+7 of a warp
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+    const float sc = amax == 0.f ? 1.0f : __fdiv_rn(amax, 448.0f);
+    uint32_t packed[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint16_t lo = ptx::cvt_e4m3x2(__fdiv_rn(v[4 * i], sc), __fdiv_rn(v[4 * i + 1], sc));
+      const uint16_t hi =
+          ptx::cvt_e4m3x2(__fdiv_rn(v[4 * i + 2], sc), __fdiv_rn(v[4 * i + 3], sc));
+      packed[i] = (uint32_t)lo | ((uint32_t)hi << 16);
+    }
+    if (act) {
+      *reinterpret_cast<uint4*>(q + (size_t)r * d + c0) =
+          make_uint4(packed[0], packed[1], packed[2], packed[3]);
+      if ((threadIdx.x & 7) == 0) s[(size_t)r * (d / 128) + c0 / 128] = sc;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_quant_rows(const uint16_t* x, int T, int k, int d, const int32_t* perm,
+                              int nrows_routed, uint8_t* q, float* s, const int32_t* offsets,
+                              int E, int nmax, int32_t* plan, int* status, cudaStream_t st) {
+  const int R = nrows_routed + T;
+  const unsigned blocks = (unsigned)(R + (plan != nullptr ? 1 : 0));
+  int threads = (d / 16 + 31) / 32 * 32;  // whole warps
+  if (threads > 256) threads = 256;
+  quant_rows_kernel<<<blocks, threads, 0, st>>>(x, T, k, d, perm, nrows_routed, q, s, offsets, E,
+                                               nmax, plan, status);
+  return cudaGetLastError();
+}
+
+}  // namespace bitmoe

@@ -1,0 +1,156 @@
+/*
+ * bitmoe — routed-expert FFN of one DeepSeek-V4-Flash-style MoE layer on B200 (sm_100a).
+ *
+ * C ABI of libbitmoe.so.  The pages this library follows:
+ *  [P1] "DeepSeek-V4-Flash on 4x RTX 2080 Ti" forum post (tcti.cn):
+ *       section "DeepSeek-V4-Flash的可能性" — routed experts stored as FP4, top-6 of
+ *       256 routed experts per token, an always-on shared expert;
+ *       section "补齐软件栈缺失" — act_quant (activation quantisation for the FP8/FP4
+ *       linears) and fp4_gemm (FP8-quantised activation x FP4 packed weight);
+ *       prefill is compute-bound and decode memory-bound, so they need different
+ *       operators.
+ *  [P2] "deepseek-v4-flash-0731-in-c" article (dpshk.com):
+ *       section "核心实现一：MoE 专家流式读取" — the router picks each token's experts;
+ *       section "核心实现三：多 token 批处理" — an expert's weights are read once for
+ *       every token routed to it;
+ *       section "核心实现四：低比特融合算子" — FP4 is dequantised inside the GEMV, never
+ *       expanded to a float matrix; gate and up share one quantised input;
+ *       workspaces are preallocated and reused.
+ *
+ * Numeric contract (what the pages leave open, fixed here):
+ *   T tokens, E routed experts + 1 shared expert (index E), top-k routing,
+ *   hidden size d, expert width f (d, f multiples of 128).
+ *   Weights per expert: W_gate, W_up [f][d] and W_down [d][f], FP4 e2m1 codes packed
+ *   two per byte (low nibble = even element), one ue8m0 scale byte (2^(b-127)) per 32
+ *   consecutive elements along the reduction axis: codes [rows][K/2], scales [rows][K/32].
+ *   Activations: per token and 128-element block, s = amax/448 (fp32, 1 if amax = 0),
+ *   q = e4m3(x/s) rounded to nearest even, saturating at +-448.
+ *   g = W_gate x^, u = W_up x^, h = silu(g) * u (fp32), h re-quantised like x,
+ *   y = W_down h^.  Combine: out[t] = y_shared[t] + sum_j w[t,j] y[t,j] with
+ *   w[t,j] = sigmoid(s_j) / sum_j' sigmoid(s_j') over the k selected scores.
+ *
+ * Conventions for every call:
+ *   - All array pointers are DEVICE pointers owned by the caller; the library never
+ *     allocates or frees memory on these calls and never synchronises the stream.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream); work is enqueued on it.
+ *   - Return 0 (MOE_OK) or a negative MOE_ERR_* code; moe_last_error() gives a
+ *     thread-local message for the last failing call on the calling thread.
+ *   - T == 0 is a valid no-op.
+ *   - Errors found on the device (a bounded wait that expired) are recorded in a
+ *     device-side status word and returned by moe_sync_status().
+ */
+#ifndef BITMOE_H
+#define BITMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_OK 0
+#define MOE_ERR_INVALID_ARG (-1) /* null / misaligned pointer, bad size or shape */
+#define MOE_ERR_WORKSPACE (-2)   /* workspace smaller than moe_workspace_size() */
+#define MOE_ERR_CUDA (-3)        /* a CUDA launch or driver call failed */
+#define MOE_ERR_TIMEOUT (-4)     /* a bounded device-side wait expired */
+#define MOE_ERR_UNSUPPORTED (-5) /* the current device is not sm_100 */
+
+/* One layer's weights, E+1 experts (index E = shared expert), contiguous per matrix:
+ *   gate_codes, up_codes  [E+1][f][d/2]   gate_scales, up_scales  [E+1][f][d/32]
+ *   down_codes            [E+1][d][f/2]   down_scales             [E+1][d][f/32]
+ * Code arrays must be 32-byte aligned; scale arrays 4-byte aligned. */
+typedef struct {
+  const uint8_t* gate_codes;
+  const uint8_t* gate_scales;
+  const uint8_t* up_codes;
+  const uint8_t* up_scales;
+  const uint8_t* down_codes;
+  const uint8_t* down_scales;
+  int E;
+  int d;
+  int f;
+} moe_weights_t;
+
+/* Step 1 — routing ([P1] "DeepSeek-V4-Flash的可能性": top-6 of 256 per token;
+ * [P2] "核心实现一": the router decides each token's experts).
+ *   scores   [T][E] fp32, finite.
+ *   topk_idx [T][k] int32 out: the k largest scores, descending; equal scores go to
+ *            the lower expert index.
+ *   topk_w   [T][k] fp32 out: sigmoid(score) renormalised over the k selected.
+ * 1 <= k <= min(E, 32); 1 <= E <= 1024.  Scores must be 4-byte aligned. */
+int moe_route_topk(const float* scores, int T, int E, int k, int32_t* topk_idx,
+                   float* topk_w, void* stream);
+
+/* Step 2 — dispatch ([P2] "核心实现三": group tokens by expert so each expert's
+ * weights are read once for its whole group).  Stable counting sort of the T*k
+ * (token, slot) pairs, flat id p = t*k + j, by expert.
+ *   counts  [E]   int32 out: pairs per expert.
+ *   offsets [E+1] int32 out: exclusive prefix sum of counts (offsets[E] = T*k).
+ *   perm    [T*k] int32 out: perm[r] = flat id at sorted position r; pairs of one
+ *           expert keep ascending flat-id order.
+ *   pos     [T*k] int32 out: inverse of perm.
+ * topk_idx values must lie in [0, E).  ws/ws_bytes are unused (may be NULL/0). */
+int moe_dispatch(const int32_t* topk_idx, int T, int k, int E, int32_t* counts,
+                 int32_t* offsets, int32_t* perm, int32_t* pos, void* ws, size_t ws_bytes,
+                 void* stream);
+
+/* Step 3 — activation quantisation ([P1] "补齐软件栈缺失": act_quant).
+ *   x_bf16 [T][d] bf16 bit patterns (16-byte aligned rows); qx [T][d] e4m3 codes out;
+ *   sx [T][d/128] fp32 out.  d % 128 == 0, d <= 16384. */
+int moe_act_quant(const uint16_t* x_bf16, int T, int d, uint8_t* qx, float* sx,
+                  void* stream);
+
+/* Steps 3-7 — expert FFN for every routed pair and the shared expert
+ * ([P1] "补齐软件栈缺失": fp4_gemm; [P2] "核心实现四": fused FP4 dequantisation,
+ * gate and up on one quantised input).  Quantises x, then for each expert runs
+ * gate+up (block-scaled FP4 x FP8 tcgen05 MMA), SwiGLU and e4m3 re-quantisation of h,
+ * then the down projection, reading each active expert's weights once per token tile.
+ *   x_bf16   [T][d] bf16.   offsets [E+1], perm [T*k] from moe_dispatch.
+ *   y_routed [T*k][d] fp32 out, row r = pair perm[r] (expert-sorted order).
+ *   y_shared [T][d] fp32 out, the shared expert's output per token.
+ *   ws       workspace of at least moe_workspace_size(T, k, E, d, f) bytes, 256-byte
+ *            aligned; its contents need not be initialised.
+ * k >= 1; d, f multiples of 128; d/2 and f/2 multiples of 32 (TMA row pitch). */
+int moe_expert_ffn(const uint16_t* x_bf16, int T, int k, const moe_weights_t* w,
+                   const int32_t* offsets, const int32_t* perm, float* y_routed,
+                   float* y_shared, void* ws, size_t ws_bytes, void* stream);
+
+/* The three stages moe_expert_ffn enqueues, exposed so that each can be timed alone.
+ * Calling them in order with the same arguments is identical to moe_expert_ffn. */
+int moe_ffn_prepare(const uint16_t* x_bf16, int T, int k, const moe_weights_t* w,
+                    const int32_t* offsets, const int32_t* perm, void* ws, size_t ws_bytes,
+                    void* stream);
+int moe_ffn_gate_up(int T, int k, const moe_weights_t* w, void* ws, size_t ws_bytes,
+                    void* stream);
+int moe_ffn_down(int T, int k, const moe_weights_t* w, float* y_routed, float* y_shared,
+                 void* ws, size_t ws_bytes, void* stream);
+
+/* Step 8 — combine: out[t][m] = y_shared[t][m] + sum_{j<k} topk_w[t][j] *
+ * y_routed[pos[t*k+j]][m], summed in fixed j order in fp32.
+ *   y_routed [T*k][d], y_shared [T][d], topk_w [T][k], pos [T*k], out [T][d] fp32.
+ * d % 4 == 0; y_routed, y_shared and out 16-byte aligned. */
+int moe_combine(const float* y_routed, const float* y_shared, const float* topk_w,
+                const int32_t* pos, int T, int k, int d, float* out, void* stream);
+
+/* Bytes of workspace moe_expert_ffn needs (0 on invalid sizes). */
+size_t moe_workspace_size(int T, int k, int E, int d, int f);
+
+/* Thread-local message for the last error on this thread ("" if none). */
+const char* moe_last_error(void);
+
+/* Upper bound, in nanoseconds of the GPU's global timer, on every device-side wait
+ * (mbarrier / pipeline waits in the FFN kernels).  A wait that runs out makes the
+ * kernel record MOE_ERR_TIMEOUT, release what it holds and return.  Default 2e9
+ * (2 s).  n <= 0 restores the default.  Applies to launches made after the call. */
+int moe_set_wait_limit_ns(long long n);
+
+/* Synchronise `stream`, then return MOE_ERR_CUDA for a pending CUDA error,
+ * MOE_ERR_TIMEOUT if a device-side wait expired since the last call (clearing the
+ * record), else MOE_OK. */
+int moe_sync_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BITMOE_H */

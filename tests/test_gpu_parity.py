@@ -1,0 +1,215 @@
+"""GPU parity: the CUDA library (through the C ABI) against the oracle.
+
+Routing indices, the dispatch permutation, offsets and the quantised activation codes
+and scales must match bit-exactly; FFN outputs (y_routed, y_shared, out) must be within
+rel-L2 <= 1e-3 and max-abs <= 1e-2 * max|ref|.  Small shapes are compared in full;
+the full-size workloads on sampled tokens the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from helpers import assert_close, check_layer, device_weights, gpu_layer, host_experts
+
+pytestmark = pytest.mark.gpu
+
+bm = pytest.importorskip("bit_moe_routed_b200")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    bm.lib()
+    yield
+    torch.cuda.empty_cache()
+
+
+# ---------------------------------------------------------------- routing and dispatch
+@pytest.mark.parametrize("name", list(synth.WORKLOADS))
+def test_route_and_dispatch_bit_exact(name):
+    w_ = synth.WORKLOADS[name]
+    s = synth.gen_scores(w_, 0)
+    idx_o, w_o = oracle.route_topk(s.numpy(), w_.k)
+    idx, w = bm.route_topk(s.cuda(), w_.k)
+    counts, offsets, perm, pos = bm.dispatch(idx, w_.E)
+    torch.cuda.synchronize()
+    assert np.array_equal(idx.cpu().numpy(), idx_o)
+    assert np.allclose(w.cpu().numpy(), w_o, rtol=2e-6, atol=1e-7)
+    c_o, off_o, perm_o, pos_o = oracle.dispatch(idx_o, w_.E)
+    assert np.array_equal(counts.cpu().numpy(), c_o)
+    assert np.array_equal(offsets.cpu().numpy(), off_o)
+    assert np.array_equal(perm.cpu().numpy(), perm_o)
+    assert np.array_equal(pos.cpu().numpy(), pos_o)
+
+
+@pytest.mark.parametrize("T,E,k", [(1, 1, 1), (5, 3, 3), (37, 1024, 8), (300, 512, 32),
+                                   (2000, 64, 6)])
+def test_route_and_dispatch_odd_shapes(T, E, k):
+    s = synth.gen_scores_uniform(T, E, seed=T + E + k)
+    idx_o, _ = oracle.route_topk(s.numpy(), k)
+    idx, _ = bm.route_topk(s.cuda(), k)
+    assert np.array_equal(idx.cpu().numpy(), idx_o)
+    counts, offsets, perm, pos = bm.dispatch(idx, E)
+    c_o, off_o, perm_o, pos_o = oracle.dispatch(idx_o, E)
+    assert np.array_equal(offsets.cpu().numpy(), off_o)
+    assert np.array_equal(perm.cpu().numpy(), perm_o)
+
+
+def test_route_ties_go_to_lower_index():
+    s = torch.tensor([[0.5, 0.9, 0.9, 0.1, 0.9] + [0.0] * 27], dtype=torch.float32)
+    idx, _ = bm.route_topk(s.cuda(), 4)
+    assert idx.cpu().tolist() == [[1, 2, 4, 0]]
+
+
+def test_dispatch_one_expert_and_empty():
+    idx = torch.zeros((300, 1), dtype=torch.int32, device="cuda")
+    counts, offsets, perm, pos = bm.dispatch(idx, 4)
+    assert counts.cpu().tolist() == [300, 0, 0, 0]
+    assert offsets.cpu().tolist() == [0, 300, 300, 300, 300]
+    assert perm.cpu().tolist() == list(range(300))
+    counts, offsets, _, _ = bm.dispatch(torch.zeros((0, 2), dtype=torch.int32, device="cuda"), 4)
+    assert counts.cpu().tolist() == [0] * 4 and offsets.cpu().tolist() == [0] * 5
+
+
+# ---------------------------------------------------------------- activation quantisation
+@pytest.mark.parametrize("T,d", [(1, 128), (3, 256), (64, 4096), (17, 8192), (4096, 4096)])
+def test_act_quant_bit_exact(T, d):
+    x = synth.gen_x(T, d, seed=T * 7 + d)
+    q_o, s_o = oracle.act_quant(x)
+    q, s = bm.act_quant(x.cuda())
+    assert np.array_equal(s.cpu().numpy(), s_o)
+    assert np.array_equal(q.cpu().numpy(), q_o)
+
+
+def test_act_quant_special_rows():
+    d = 512
+    rows = [torch.zeros(d), torch.full((d,), 448.0), torch.full((d,), -1e30),
+            torch.tensor([1e-30, -1e-30] * (d // 2)), torch.linspace(-3, 3, d)]
+    x = torch.stack(rows)
+    x[3, 0] = 1.0  # tiny values next to a large one round to +-0
+    x = x.to(torch.bfloat16)
+    q_o, s_o = oracle.act_quant(x)
+    q, s = bm.act_quant(x.cuda())
+    assert np.array_equal(s.cpu().numpy(), s_o)
+    assert np.array_equal(q.cpu().numpy(), q_o)
+
+
+# ---------------------------------------------------------------- whole layer, small shapes
+def _small_layer(T, E, k, d, f, routing="uniform", seed=5, zero_rows=()):
+    x = synth.gen_x(T, d, seed=seed)
+    for r in zero_rows:
+        x[r] = 0
+    s = synth.gen_scores_uniform(T, E, seed + 1) if routing == "uniform" else \
+        synth.gen_scores_zipf(T, E, 1.2, seed + 1)
+    W = device_weights(seed, 0, E, d, f)
+    g = gpu_layer(x, s, k, W)
+    check_layer(g, x, s, k, E, d, f, seed, 0, list(range(T)), f"T={T} E={E} k={k} d={d} f={f}")
+
+
+def test_layer_tiny_workload():
+    w_ = synth.WORKLOADS["tiny"]
+    x, s = synth.gen_layer_inputs(w_)
+    W = device_weights(w_.seed(), 0, w_.E, w_.d, w_.f)
+    g = gpu_layer(x, s, w_.k, W)
+    check_layer(g, x, s, w_.k, w_.E, w_.d, w_.f, w_.seed(), 0, list(range(w_.T)), "tiny")
+
+
+@pytest.mark.parametrize("T,E,k,d,f,routing", [
+    (1, 4, 1, 128, 128, "uniform"),
+    (3, 8, 2, 256, 128, "uniform"),
+    (33, 16, 4, 512, 256, "zipf"),      # crosses the small/large tile switch
+    (130, 8, 3, 256, 384, "zipf"),      # groups larger than one 112-row tile
+    (250, 32, 6, 384, 256, "uniform"),
+])
+def test_layer_ragged_shapes(T, E, k, d, f, routing):
+    _small_layer(T, E, k, d, f, routing, seed=T + E)
+
+
+def test_layer_zero_activations():
+    _small_layer(6, 8, 2, 256, 128, seed=77, zero_rows=(0, 3))
+
+
+def test_layer_all_tokens_one_expert():
+    T, E, k, d, f = 240, 8, 1, 256, 256
+    x = synth.gen_x(T, d, seed=90)
+    s = synth.gen_scores_uniform(T, E, seed=91)
+    s[:, 3] += 10.0  # every token picks expert 3: three token tiles of one expert
+    W = device_weights(92, 0, E, d, f)
+    g = gpu_layer(x, s, k, W)
+    assert g["counts"].tolist()[3] == T
+    check_layer(g, x, s, k, E, d, f, 92, 0, list(range(0, T, 7)), "one expert")
+
+
+def test_layer_extreme_weights():
+    """All codes +-6 with the largest scale used (2^-3), all codes 0, and mixed."""
+    T, E, k, d, f = 5, 4, 2, 256, 128
+    rng = np.random.default_rng(3)
+
+    def mk(which):
+        r, K = synth.matrix_shape(which, d, f)
+        codes = np.full((E + 1, r, K // 2), 0x77, np.uint8)  # +6, +6
+        codes[1] = 0xFF                                       # -6, -6
+        codes[2] = 0x00                                       # zeros
+        codes[3] = rng.integers(0, 256, codes[3].shape, dtype=np.uint8)
+        scales = np.full((E + 1, r, K // 32), 124, np.uint8)
+        scales[3] = rng.integers(121, 125, scales[3].shape, dtype=np.uint8)
+        return codes, scales
+
+    arrs = {}
+    for name, which in (("gate", synth.GATE), ("up", synth.UP), ("down", synth.DOWN)):
+        c, s_ = mk(which)
+        arrs[f"{name}_codes"], arrs[f"{name}_scales"] = c, s_
+    W = bm.LayerWeights.from_dict({kk: torch.from_numpy(v).cuda() for kk, v in arrs.items()})
+    x = synth.gen_x(T, d, seed=11)
+    s = synth.gen_scores_uniform(T, E, seed=12)
+    g = gpu_layer(x, s, k, W)
+    idx, w = oracle.route_topk(s.numpy(), k)
+    ex = {e: synth.HostExpert(*(arrs[n][e] for n in (
+        "gate_codes", "gate_scales", "up_codes", "up_scales", "down_codes", "down_scales")))
+        for e in range(E + 1)}
+    y_pair, y_sh, out = oracle.moe_layer(x, E, k, d, f, ex, idx, w)
+    assert np.array_equal(g["idx"].numpy(), idx)
+    assert_close(g["out"].numpy(), out, "extreme weights: out")
+    assert_close(g["y_shared"].numpy(), y_sh, "extreme weights: y_shared")
+
+
+def test_device_generator_matches_host_generator():
+    seed, layer, E, d, f = 1234, 3, 8, 256, 128
+    dev = synth.device_layer_weights(seed, layer, E, d, f)
+    host = synth.host_layer_weights(seed, layer, E, d, f)
+    for kk in host:
+        assert np.array_equal(dev[kk].cpu().numpy(), host[kk]), kk
+
+
+# ---------------------------------------------------------------- full-size workloads
+def _full_workload(name, tokens):
+    w_ = synth.WORKLOADS[name]
+    x, s = synth.gen_layer_inputs(w_, 0)
+    W = device_weights(w_.seed(), 0, w_.E, w_.d, w_.f)
+    oracle.set_threads(8)
+    g = gpu_layer(x, s, w_.k, W)
+    del W
+    torch.cuda.empty_cache()
+    check_layer(g, x, s, w_.k, w_.E, w_.d, w_.f, w_.seed(), 0, tokens, name)
+    return g
+
+
+def test_decode_t1_full():
+    _full_workload("decode_t1", [0])
+
+
+def test_decode_t64_zipf_sampled():
+    g = _full_workload("decode_t64_zipf", [0, 9, 31, 63])
+    assert int(g["counts"].max()) > 16  # a hot expert serves many tokens
+
+
+@pytest.mark.parametrize("name", ["prefill_t4096_uniform", "prefill_t4096_zipf"])
+def test_prefill_t4096_sampled(name):
+    g = _full_workload(name, [0, 1, 1777, 4095])
+    w_ = synth.WORKLOADS[name]
+    assert int(g["counts"].sum()) == w_.T * w_.k
+    # every output row finite
+    assert torch.isfinite(g["out"]).all() and torch.isfinite(g["y"]).all()

@@ -1,0 +1,35 @@
+"""Failure detection without a GPU fault: the FFN kernels bound every wait by a
+%globaltimer limit.  A 1 ns limit makes the first wait that is not already satisfied run
+out; the kernel must record MOE_ERR_TIMEOUT, release TMEM, drain its copies and return,
+leaving the context usable for the next (normal) call."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from helpers import check_layer, device_weights, gpu_layer
+
+pytestmark = pytest.mark.gpu
+
+bm = pytest.importorskip("bit_moe_routed_b200")
+
+
+def test_wait_limit_expiry_is_reported_and_recoverable():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    T, E, k, d, f = 8, 16, 2, 512, 256
+    x = synth.gen_x(T, d, seed=501)
+    s = synth.gen_scores_uniform(T, E, seed=502)
+    W = device_weights(503, 0, E, d, f)
+    bm.sync_status()  # clean start
+    bm.set_wait_limit_ns(1)
+    try:
+        bm.forward(x.cuda(), s.cuda(), k, W)
+        with pytest.raises(bm.MoeError) as ei:
+            bm.sync_status()
+        assert ei.value.code == bm.MOE_ERR_TIMEOUT
+    finally:
+        bm.set_wait_limit_ns(0)  # default limit
+    bm.sync_status()  # the status word was cleared by the report
+    g = gpu_layer(x, s, k, W)
+    check_layer(g, x, s, k, E, d, f, 503, 0, list(range(T)), "after timeout")
