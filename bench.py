@@ -136,6 +136,20 @@ def kernel_traffic(kernel_file: str, name: str, workload: str):
     return None
 
 
+def max_over_ranks(seconds: float, dist, device) -> float:
+    """Largest value over all ranks (the job's time is the slowest rank's time)."""
+    if dist is None:
+        return seconds
+    t = torch.tensor([seconds], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_seed(w, rank: int) -> int:
+    """Each rank of a multi-GPU run serves its own tokens (replicas, weak scaling)."""
+    return w.seed(0) + 100000 * rank
+
+
 # ------------------------------------------------------------------------ CPU oracle leg
 def oracle_sample(w, x, scores, seconds: float, layer_seed: int):
     """Time the oracle on whole tokens of this workload for about `seconds` seconds.
@@ -167,7 +181,8 @@ def run_reference(args, w):
     x, scores = synth.gen_layer_inputs(w, 0)
     import oracle
     oracle.build()
-    per_step = max(1.0, min(30.0, 60.0 / max(args.steps + args.warmup, 1)))
+    per_step = args.ref_seconds if args.ref_seconds else \
+        max(1.0, min(30.0, 60.0 / max(args.steps + args.warmup, 1)))
     for _ in range(args.warmup):
         oracle_sample(w, x, scores, 0.2, w.seed(0))
     times = []
@@ -209,7 +224,7 @@ def run_gpu(args, w):
     hbm_peak, bf16_peak, bf16_sus, peak_kind = load_peaks()
 
     # inputs: each rank its own tokens (replica); weights resident in HBM
-    seed = w.seed(0) + 100000 * rank
+    seed = replica_seed(w, rank)
     if rank == 0:
         x_cpu, s_cpu = synth.gen_layer_inputs(w, 0)
     else:
@@ -287,11 +302,8 @@ def run_gpu(args, w):
     clk = clocks.stop()
     step_ms = [starts[i].elapsed_time(ends[i]) for i in range(args.steps)]
     gu_ms = [gs[i].elapsed_time(ge[i]) for i in range(args.steps)]
-    total_s = sum(step_ms) / 1000.0
+    total_s = max_over_ranks(sum(step_ms) / 1000.0, dist, dev)
     if dist is not None:
-        t = torch.tensor([total_s], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_s = float(t.item())
         dist.barrier()
     value = world * T * args.steps / total_s
 
@@ -317,11 +329,7 @@ def run_gpu(args, w):
         b.synchronize()
         if i >= args.warmup:
             e2e_ms.append(a.elapsed_time(b))
-    e2e_s = sum(e2e_ms) / 1000.0
-    if dist is not None:
-        t = torch.tensor([e2e_s], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_s = float(t.item())
+    e2e_s = max_over_ranks(sum(e2e_ms) / 1000.0, dist, dev)
     e2e_value = world * T * args.steps / e2e_s
     bm.sync_status(stream)
 
@@ -391,6 +399,8 @@ def main():
     ap.add_argument("--impl", default="bitmoe", choices=["bitmoe", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-seconds", type=float, default=None,
+                    help="oracle seconds per step of the reference arm (default: fit ~1 min)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

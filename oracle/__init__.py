@@ -64,6 +64,7 @@ def lib():
         L.oracle_dispatch.argtypes = [P, I, I, I, P, P, P, P]
         L.oracle_fp4_gemv.argtypes = [P, P, I, I, P, P]
         L.oracle_expert_ffn.argtypes = [ctypes.POINTER(_Expert), I, I, P, P, I, P, P, P]
+        L.oracle_expert_ffn_h.argtypes = [ctypes.POINTER(_Expert), I, I, P, P, I, P, P, P, P]
         L.oracle_combine_token.argtypes = [P, P, P, I, I, P]
         L.oracle_moe_tokens.argtypes = [P, I, I, I, I, I, ctypes.POINTER(_Expert), P, P, P, I,
                                         P, P, P]
@@ -196,6 +197,21 @@ def expert_ffn(ex, d: int, f: int, qx: np.ndarray, sx: np.ndarray, want_h: bool 
                             hq.ctypes.data if want_h else None,
                             hs.ctypes.data if want_h else None)
     return (y, hq, hs) if want_h else y
+
+
+def expert_ffn_h(ex, d: int, f: int, qx: np.ndarray, sx: np.ndarray):
+    """(y [ntok, d], h codes [ntok, f], h scales [ntok, f/128], h fp32 before quantisation)."""
+    es = ExpertSet(1, {0: ex})
+    qx, pq = _c(qx, np.uint8)
+    sx, ps = _c(sx, np.float32)
+    ntok = qx.shape[0]
+    y = np.empty((ntok, d), np.float64)
+    hq = np.empty((ntok, f), np.uint8)
+    hs = np.empty((ntok, f // 128), np.float32)
+    hf = np.empty((ntok, f), np.float32)
+    lib().oracle_expert_ffn_h(es.arr, d, f, pq, ps, ntok, y.ctypes.data, hq.ctypes.data,
+                              hs.ctypes.data, hf.ctypes.data)
+    return y, hq, hs, hf
 
 
 def combine(y_sh: np.ndarray, y_pair: np.ndarray, w: np.ndarray) -> np.ndarray:

@@ -197,6 +197,12 @@ static void decode_row(const uint8_t* codes, const uint8_t* scales, int K, int r
  * Each weight row is decoded once and used for every token of the group. */
 void oracle_expert_ffn(const oracle_expert_t* w, int d, int f, const uint8_t* qx,
                        const float* sx, int ntok, double* y, uint8_t* h_q, float* h_s) {
+    oracle_expert_ffn_h(w, d, f, qx, sx, ntok, y, h_q, h_s, NULL);
+}
+
+void oracle_expert_ffn_h(const oracle_expert_t* w, int d, int f, const uint8_t* qx,
+                         const float* sx, int ntok, double* y, uint8_t* h_q, float* h_s,
+                         float* h_f32) {
     double* xhat = (double*)malloc(sizeof(double) * (size_t)ntok * d);
     double* g = (double*)malloc(sizeof(double) * (size_t)ntok * f);
     double* u = (double*)malloc(sizeof(double) * (size_t)ntok * f);
@@ -245,6 +251,7 @@ void oracle_expert_ffn(const oracle_expert_t* w, int d, int f, const uint8_t* qx
             hhat[(size_t)t * f + n] = oracle_e4m3_value(hq[(size_t)t * f + n]) *
                                       (double)hs[(size_t)t * (f / 128) + n / 128];
     }
+    if (h_f32) memcpy(h_f32, h, sizeof(float) * (size_t)ntok * f);
     if (h_q) memcpy(h_q, hq, (size_t)ntok * f);
     if (h_s) memcpy(h_s, hs, sizeof(float) * (size_t)ntok * (f / 128));
 

@@ -83,6 +83,11 @@ void oracle_fp4_gemv(const uint8_t* codes, const uint8_t* scales, int rows, int 
  * [ntok][f] codes and [ntok][f/128] scales. */
 void oracle_expert_ffn(const oracle_expert_t* w, int d, int f, const uint8_t* qx,
                        const float* sx, int ntok, double* y, uint8_t* h_q, float* h_s);
+/* Same, also returning the fp32 hidden state before re-quantisation (h_f32 [ntok][f],
+ * may be NULL). */
+void oracle_expert_ffn_h(const oracle_expert_t* w, int d, int f, const uint8_t* qx,
+                         const float* sx, int ntok, double* y, uint8_t* h_q, float* h_s,
+                         float* h_f32);
 
 /* Weighted combine for one token: out[m] = ysh[m] + sum_j w[j] * y[j][m]. */
 void oracle_combine_token(const double* ysh, const double* y, const double* w, int k, int d,
