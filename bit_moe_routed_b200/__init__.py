@@ -31,7 +31,7 @@ MOE_ERR_UNSUPPORTED = -5
 EXPORTS = (
     "moe_route_topk", "moe_dispatch", "moe_act_quant", "moe_expert_ffn", "moe_ffn_prepare",
     "moe_ffn_gate_up", "moe_ffn_down", "moe_combine", "moe_workspace_size", "moe_last_error",
-    "moe_set_wait_limit_ns", "moe_sync_status",
+    "moe_set_wait_limit_ns", "moe_sync_status", "moe_expert_ffn_noalloc",
 )
 
 
@@ -77,6 +77,7 @@ def lib():
             "moe_last_error": [],
             "moe_set_wait_limit_ns": [LL],
             "moe_sync_status": [P],
+            "moe_expert_ffn_noalloc": [P, I, I, W, P, P, P, P, P],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -201,6 +202,23 @@ def expert_ffn(x: torch.Tensor, k: int, w: LayerWeights, offsets: torch.Tensor,
     ws_struct = w.struct()
     _check(lib().moe_expert_ffn(_p(x), T, k, ctypes.byref(ws_struct), _p(offsets), _p(perm),
                                 _p(y), _p(ysh), _p(ws), ws.numel(), _stream(stream)))
+    return y[:T * k], ysh[:T]
+
+
+def expert_ffn_noalloc(x: torch.Tensor, k: int, w: LayerWeights, offsets: torch.Tensor,
+                       perm: torch.Tensor, out=None, stream=None):
+    """expert_ffn with the library's fixed device scratch instead of a workspace (for callers
+    that cannot allocate; at most MOE_NOALLOC_SCRATCH_BYTES of scratch, calls must not
+    overlap on the GPU)."""
+    T, d = x.shape
+    if out is None:
+        y = torch.empty((max(T * k, 1), d), dtype=torch.float32, device=x.device)
+        ysh = torch.empty((max(T, 1), d), dtype=torch.float32, device=x.device)
+    else:
+        y, ysh = out
+    st = w.struct()
+    _check(lib().moe_expert_ffn_noalloc(_p(x), T, k, ctypes.byref(st), _p(offsets), _p(perm),
+                                        _p(y), _p(ysh), _stream(stream)))
     return y[:T * k], ysh[:T]
 
 

@@ -94,6 +94,9 @@ int check_weights(const moe_weights_t* w) {
 
 }  // namespace
 
+// Sets the message moe_last_error returns, for the library's other translation units.
+int record_error(int code, const char* msg) { return fail(code, "%s", msg); }
+
 WorkspaceLayout workspace_layout(int T, int k, int E, int d, int f) {
   WorkspaceLayout L{};
   const size_t R = (size_t)T * k + T;

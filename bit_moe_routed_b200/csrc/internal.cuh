@@ -64,5 +64,8 @@ struct FfnArgs {
 cudaError_t launch_ffn(int phase, int nmax, const FfnArgs& a, cudaStream_t s, int num_sms);
 size_t ffn_smem_bytes(int phase, int nmax, int nk, int E);  // dynamic shared memory of a launch
 
+// Defined in abi.cu: sets the thread-local message that moe_last_error returns.
+int record_error(int code, const char* msg);
+
 
 }  // namespace bitmoe

@@ -126,6 +126,25 @@ int moe_ffn_gate_up(int T, int k, const moe_weights_t* w, void* ws, size_t ws_by
 int moe_ffn_down(int T, int k, const moe_weights_t* w, float* y_routed, float* y_shared,
                  void* ws, size_t ws_bytes, void* stream);
 
+/* moe_expert_ffn without a caller-owned workspace.  The pages have no counterpart of
+ * this call; it exists for callers that cannot allocate device memory when they run the
+ * layer (an engine plugin given no workspace, a serving loop that must not call
+ * cudaMalloc because it may synchronise the device).  Arguments and results are those of
+ * moe_expert_ffn minus ws/ws_bytes; the scratch is a fixed array of
+ * MOE_NOALLOC_SCRATCH_BYTES that the library keeps on every GPU that loads it, for the
+ * life of the process.
+ *   - Calls needing more scratch than that (moe_workspace_size > the maximum; for
+ *     d = 4096, f = 2048, k = 6, E = 256 that is T > 94) return MOE_ERR_WORKSPACE.
+ *   - Allocates nothing.  All calls share the one array per device: calls that overlap on
+ *     the GPU (other streams, other threads) race on it.  It keeps the previous call's
+ *     contents; nothing in it needs to start at zero.
+ *   - The first call on a device looks up the array's device address once; make that
+ *     first call before any stream capture. */
+#define MOE_NOALLOC_SCRATCH_BYTES (4u << 20)
+int moe_expert_ffn_noalloc(const uint16_t* x_bf16, int T, int k, const moe_weights_t* w,
+                           const int32_t* offsets, const int32_t* perm, float* y_routed,
+                           float* y_shared, void* stream);
+
 /* Step 8 — combine: out[t][m] = y_shared[t][m] + sum_{j<k} topk_w[t][j] *
  * y_routed[pos[t*k+j]][m], summed in fixed j order in fp32.
  *   y_routed [T*k][d], y_shared [T][d], topk_w [T][k], pos [T*k], out [T][d] fp32.
