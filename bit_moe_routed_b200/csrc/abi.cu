@@ -111,6 +111,12 @@ WorkspaceLayout workspace_layout(int T, int k, int E, int d, int f) {
   o = align256(o + R * f);
   L.sh = o;
   o = align256(o + R * (f / 128) * 4);
+  L.counters = o;
+  const size_t hb = (size_t)((d > f ? d : f) / 128);
+  L.n_counters = plan_ntmax((int)R, E) * hb;
+  o = align256(o + 4 * L.n_counters);
+  L.partials = o;
+  o = align256(o + (size_t)kMaxCtas * 2 * (size_t)ncap_for(T) * 2 * 128 * 4);
   L.total = o;
   return L;
 }
@@ -203,7 +209,7 @@ int moe_act_quant(const uint16_t* x_bf16, int T, int d, uint8_t* qx, float* sx, 
   int rc = device_info(di);
   if (rc) return rc;
   cudaError_t e = launch_quant_rows(x_bf16, T, 1, d, nullptr, 0, qx, sx, nullptr, 0, 0, nullptr,
-                                    di.status, static_cast<cudaStream_t>(stream));
+                                    nullptr, 0, di.status, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "act_quant launch");
 }
 
@@ -237,9 +243,9 @@ int ffn_check(int T, int k, const moe_weights_t* w, void* ws, size_t ws_bytes, F
   int dev = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-  const size_t need = ffn_smem_bytes(1, c.nmax, w->d / 128, w->E) > ffn_smem_bytes(2, c.nmax, w->f / 128, w->E)
-                          ? ffn_smem_bytes(1, c.nmax, w->d / 128, w->E)
-                          : ffn_smem_bytes(2, c.nmax, w->f / 128, w->E);
+  const size_t need1 = ffn_smem_bytes(1, c.nmax, w->d / 128, w->E, w->f);
+  const size_t need2 = ffn_smem_bytes(2, c.nmax, w->f / 128, w->E, w->d);
+  const size_t need = need1 > need2 ? need1 : need2;
   if (need > (size_t)max_smem)
     return fail(MOE_ERR_INVALID_ARG, "shape needs %zu bytes of shared memory (> %d)", need,
                 max_smem);
@@ -257,6 +263,10 @@ FfnArgs ffn_args(int phase, int T, int k, const moe_weights_t* w, const FfnCtx& 
   a.plan = reinterpret_cast<const int32_t*>(c.ws + c.L.plan);
   a.wait_ns = g_wait_ns.load();
   a.status = c.di.status;
+  a.counters = reinterpret_cast<int*>(c.ws + c.L.counters);
+  a.partials = reinterpret_cast<float*>(c.ws + c.L.partials);
+  a.ncap = ncap_for(T);
+  a.pf_dist = 0;
   if (phase == 1) {
     a.a0_codes = w->gate_codes;
     a.a0_scales = w->gate_scales;
@@ -292,7 +302,8 @@ int moe_ffn_prepare(const uint16_t* x_bf16, int T, int k, const moe_weights_t* w
   if (!aligned(x_bf16, 16)) return fail(MOE_ERR_INVALID_ARG, "x must be 16-byte aligned");
   cudaError_t e = launch_quant_rows(
       x_bf16, T, k, w->d, perm, T * k, c.ws + c.L.qx, reinterpret_cast<float*>(c.ws + c.L.sx),
-      offsets, w->E, c.nmax, reinterpret_cast<int32_t*>(c.ws + c.L.plan), c.di.status,
+      offsets, w->E, c.nmax, reinterpret_cast<int32_t*>(c.ws + c.L.plan),
+      reinterpret_cast<int*>(c.ws + c.L.counters), c.L.n_counters, c.di.status,
       static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "ffn prepare launch");
 }

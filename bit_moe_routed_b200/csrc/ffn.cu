@@ -9,22 +9,35 @@
 // the tensor core itself: TMA unpacks the FP4 codes into byte containers in shared
 // memory and the MMA applies the ue8m0 block scales from TMEM.
 //
-// Work decomposition ("swap-AB"): a tile is (expert e, 128-row block of the weight
-// matrix, token tile of n <= NMAX rows).  The weight rows are the MMA's M = 128; the
-// tokens are its N (n rounded up to 16), so ragged expert groups waste at most 15
-// columns.  Phase 1 multiplies the gate AND up rows of the same 128 h-rows with one
-// shared activation tile, then computes h = silu(g) * u and re-quantises it per
-// 128-block to e4m3; phase 2 is the down projection writing fp32 y.
+// Tiles ("swap-AB"): a tile is (expert e, 128-row block of the weight matrix, token
+// tile of n <= NMAX rows).  The weight rows are the MMA's M = 128; the tokens are its N
+// (n rounded up to 16), so ragged expert groups waste at most 15 columns.  Phase 1
+// multiplies the gate AND up rows of the same 128 h-rows with one shared activation
+// tile, then computes h = silu(g) * u and re-quantises it per 128-block to e4m3;
+// phase 2 is the down projection writing fp32 y.
+//
+// Work split ("stream-K"): the tiles' 128-wide K chunks form one sequence of W chunks;
+// CTA b of G takes chunks [bW/G, (b+1)W/G), so every SM gets the same number of weight
+// bytes whatever the number of tiles.  A tile cut between CTAs is finished by the CTA
+// that completes its last segment: each writes its fp32 partial to a slot, the last
+// one (an atomic count) adds the segments in fixed order, so results are deterministic.
 //
 // Activation scales are fp32 (amax/448), not ue8m0, so they cannot ride in the MMA:
-// B's hardware scale is 1.0 and every 128-wide K chunk is accumulated into a fresh
-// TMEM partial, which the epilogue warps fold into fp32 registers as acc += s * P.
-// Two TMEM partial buffers let the MMA run one chunk ahead of the epilogue.
+// B's hardware scale is 1.0 and every K chunk is accumulated into a fresh TMEM partial
+// that the epilogue warps fold into fp32 registers as acc += s * P.  A ring of NBUF
+// TMEM partials lets the MMA run NBUF chunks ahead of the epilogue.
 //
-// Warp roles (320 threads, one CTA per SM, persistent over tiles):
-//   warp 0   : TMA producer (weights, activations) + cp.async of the weight scales
+// Memory: the weights are row-major ([rows][K/2]) and a TMA box takes 64 bytes from each
+// of 128 rows, which DRAM serves poorly.  So the scale-loader warp first pulls each
+// segment's rows into L2 with line prefetches that run along each row (contiguous
+// runs), a few chunks ahead of the TMA loads, which then mostly hit L2.
+//
+// Warp roles (352 threads, one CTA per SM, persistent):
+//   warp 0   : TMA producer (weights, activations)
 //   warp 1   : TMEM allocator; lane 0 issues tcgen05.cp / tcgen05.mma / commits
 //   warps 2-9: epilogue; warp w reads TMEM lanes 32*(w%4).., column half (w-2)/4
+//   warp 10  : weight-scale loader (cp.async gather into the tcgen05.cp layout) and L2
+//              row prefetch
 // Every wait is bounded by a %globaltimer limit; on expiry the kernel records a
 // timeout in the status word, lets in-flight copies and MMAs land, frees TMEM and
 // returns.
@@ -37,15 +50,17 @@
 namespace bitmoe {
 namespace {
 
-constexpr int kThreads = 320;
 constexpr int kEpiWarps = 8;
-constexpr int kLag = 2;                         // scale cp.async groups in flight
+constexpr int kSfWarp = 2 + kEpiWarps;          // warp 10 loads the weight scales
+constexpr int kThreads = 32 * (kSfWarp + 1);
 constexpr long long kDrainNs = 500000000LL;     // bound on draining in-flight work
 
 struct FfnParams {
   CUtensorMap tmA0;  // gate (phase 1) / down (phase 2) codes, all experts stacked
   CUtensorMap tmA1;  // up codes (phase 1)
   CUtensorMap tmB;   // activation rows [R][K] e4m3
+  const uint8_t* a0_codes;  // the same codes as plain pointers (L2 prefetch)
+  const uint8_t* a1_codes;
   const uint8_t* sfa0;
   const uint8_t* sfa1;
   const float* b_scales;  // [R][K/128]
@@ -55,34 +70,43 @@ struct FfnParams {
   float* sh;
   float* y_routed;
   float* y_shared;
+  int* counters;          // per tile, zero on entry, left zero on exit
+  float* partials;        // [kMaxCtas][2][ncap][nmat][128]
+  int ncap;
+  int pf_dist;            // > 0: prefetch each segment's weight rows into L2
   long long wait_ns;
   int* status;
 };
 
-template <int PHASE, int NMAX, int STAGES>
+template <int PHASE, int NMAX, int STAGES, int NBUF, int MR>
 struct Cfg {
   static constexpr int kNumA = PHASE == 1 ? 2 : 1;
-  static constexpr int kATile = 128 * 128;  // 128 rows x 128 FP4 in byte containers
+  static constexpr int kRB = MR / 128;       // 128-row MMA blocks per weight tile
+  static constexpr int kATile = MR * 128;    // MR rows x 128 FP4 in byte containers
   static constexpr int kBTile = NMAX * 128;
-  static constexpr int kSF = 512;
+  static constexpr int kSF = 512 * kRB;      // per matrix: one 512-byte scale block per 128 rows
   static constexpr int kStageRaw = kNumA * kATile + kBTile + kNumA * kSF;
   static constexpr int kStage = (kStageRaw + 1023) / 1024 * 1024;
-  static constexpr int kHalf = NMAX / 2;
-  static constexpr int kAccCols = PHASE == 1 ? 2 * NMAX : NMAX;  // per TMEM buffer
-  static constexpr int kColSFA0 = 2 * kAccCols;
-  static constexpr int kColSFA1 = kColSFA0 + 4;
-  static constexpr int kColSFB = kColSFA0 + 4 * kNumA;
+  // epilogue: with two 128-row blocks each group of four warps owns one block and all
+  // columns; with one block the two groups split the columns
+  static constexpr int kCols = kRB == 2 ? NMAX : NMAX / 2;
+  static constexpr int kAccCols = kNumA * kRB * NMAX;  // per TMEM buffer
+  static constexpr int kColSFA0 = NBUF * kAccCols;
+  static constexpr int kColSFA1 = kColSFA0 + 4 * kRB;
+  static constexpr int kColSFB = kColSFA0 + 4 * kRB * kNumA;
+  static_assert(MR == 128 || MR == 256, "weight tile rows");
   static_assert(kColSFB + 4 <= 512, "TMEM columns");
-  static_assert(NMAX % 16 == 0 && kHalf % 8 == 0, "tile width");
-  static_assert(kLag <= STAGES - 1, "scale lag must leave a stage to the consumer");
+  static_assert(NMAX % 16 == 0 && kCols % 8 == 0, "tile width");
   // shared memory after the stages
   static constexpr int kOffSFB = STAGES * kStage;
   static constexpr int kOffBars = kOffSFB + 512;
-  static constexpr int kNumBars = 2 * STAGES + 5;
-  static constexpr int kOffMisc = kOffBars + 8 * kNumBars;  // tmem slot, abort flag
+  static constexpr int kNumBars = 3 * STAGES + 2 * NBUF + 1;
+  static constexpr int kOffMisc = kOffBars + 8 * kNumBars;  // tmem slot, abort, fix-up word
   static constexpr int kOffAmax = kOffMisc + 16;
-  static constexpr int kOffTT = kOffAmax + 2 * 4 * kHalf * 4;  // plan prefix, E+2 ints
-  __host__ __device__ static size_t off_sbs(int E) { return (size_t)kOffTT + ((size_t)(E + 2) * 4 + 15) / 16 * 16; }
+  static constexpr int kOffTT = kOffAmax + 2 * 4 * kCols * 4;  // plan prefix, E+2 ints
+  __host__ __device__ static size_t off_sbs(int E) {
+    return (size_t)kOffTT + ((size_t)(E + 2) * 4 + 15) / 16 * 16;
+  }
   __host__ __device__ static size_t smem_bytes(int nk, int E) {
     return 1024 + off_sbs(E) + (size_t)nk * NMAX * 4;
   }
@@ -91,7 +115,9 @@ struct Cfg {
 __device__ __forceinline__ void bar_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
-
+__device__ __forceinline__ void prefetch_line_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p) : "memory");
+}
 // Bounded wait by one thread; false if the limit ran out or another role aborted.
 __device__ bool wait_one(uint32_t bar, uint32_t parity, long long limit, volatile int* abort_flag,
                          int* status) {
@@ -124,7 +150,7 @@ __device__ void drain_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Tile i -> (expert, 128-row block, first activation row, rows).  Tiles of one expert
-// are ordered (block, token tile) so CTAs working at the same time share weight rows.
+// are ordered (block, token tile) so consecutive tiles share weight rows in L2.
 __device__ __forceinline__ void decode_tile(const int32_t* ttbase, const int32_t* tiles, int E,
                                             int HB, int i, int& e, int& blk, int& row0, int& n) {
   int lo = 0, hi = E;
@@ -141,9 +167,22 @@ __device__ __forceinline__ void decode_tile(const int32_t* ttbase, const int32_t
   n = __ldg(tiles + 2 * tt + 1);
 }
 
-template <int PHASE, int NMAX, int STAGES>
+// Stream-K partition of W chunks over G CTAs.
+struct Split {
+  unsigned long long W;
+  int G;
+  __device__ __forceinline__ unsigned long long begin(int b) const {
+    return (unsigned long long)b * W / (unsigned long long)G;
+  }
+  __device__ __forceinline__ int owner(unsigned long long c) const {  // CTA holding chunk c
+    return (int)(((c + 1) * (unsigned long long)G - 1) / W);
+  }
+};
+
+template <int PHASE, int NMAX, int STAGES, int NBUF, int MR>
 __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant__ FfnParams p) {
-  using C = Cfg<PHASE, NMAX, STAGES>;
+  using C = Cfg<PHASE, NMAX, STAGES, NBUF, MR>;
+  constexpr int kMat = PHASE == 1 ? 2 : 1;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -154,26 +193,29 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
   auto full = [&](int s) { return bars + 8u * s; };
   auto empty = [&](int s) { return bars + 8u * (STAGES + s); };
   auto tfull = [&](int b) { return bars + 8u * (2 * STAGES + b); };
-  auto tempty = [&](int b) { return bars + 8u * (2 * STAGES + 2 + b); };
-  const uint32_t drain = bars + 8u * (2 * STAGES + 4);
+  auto tempty = [&](int b) { return bars + 8u * (2 * STAGES + NBUF + b); };
+  const uint32_t drain = bars + 8u * (2 * STAGES + 2 * NBUF);
+  auto sf_full = [&](int s) { return bars + 8u * (2 * STAGES + 2 * NBUF + 1 + s); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+  volatile int* fix_word = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);
   float* amax_s = reinterpret_cast<float*>(smem + C::kOffAmax);
   int32_t* s_ttbase = reinterpret_cast<int32_t*>(smem + C::kOffTT);
   float* sbs = reinterpret_cast<float*>(smem + C::off_sbs(p.E));
 
   const int nk = p.K / 128;
-  const int HB = p.rows_per_expert / 128;
+  const int HB = p.rows_per_expert / MR;
   const int32_t* g_tiles = p.plan + p.E + 2;
   for (int e = threadIdx.x; e < p.E + 2; e += kThreads) s_ttbase[e] = __ldg(p.plan + e);
   const int32_t* g_ttbase = s_ttbase;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      ptx::mbar_init(full(s), 2);   // TMA arrive.expect_tx + scale-factor arrive
+      ptx::mbar_init(full(s), 1);      // TMA arrive.expect_tx (+ transaction bytes)
+      ptx::mbar_init(sf_full(s), 32);  // the 32 scale-loader lanes' cp.async arrivals
       ptx::mbar_init(empty(s), 1);  // tcgen05.commit
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NBUF; ++b) {
       ptx::mbar_init(tfull(b), 1);
       ptx::mbar_init(tempty(b), kEpiWarps);
     }
@@ -192,33 +234,36 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int total = g_ttbase[p.E + 1] * HB;
+  const int total_tiles = g_ttbase[p.E + 1] * HB;
+  const Split sp{(unsigned long long)total_tiles * (unsigned long long)nk, (int)gridDim.x};
+  const unsigned long long beg = sp.begin(blockIdx.x), end = sp.begin(blockIdx.x + 1);
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       ptx::prefetch_tmap(&p.tmA0);
       if (PHASE == 1) ptx::prefetch_tmap(&p.tmA1);
       ptx::prefetch_tmap(&p.tmB);
     }
-    const size_t ldsf = (size_t)(p.K / 32);
     int it = 0;
     bool ok = true;
-    for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
+    for (unsigned long long c = beg; c < end && ok;) {
+      const int ti = (int)(c / nk);
+      const int k0 = (int)(c % nk);
+      const int k1 = (int)min((unsigned long long)nk, (unsigned long long)k0 + (end - c));
       int e, blk, row0, n;
-      decode_tile(g_ttbase, g_tiles, p.E, HB, i, e, blk, row0, n);
-      const int rowA = e * p.rows_per_expert + blk * 128;
+      decode_tile(g_ttbase, g_tiles, p.E, HB, ti, e, blk, row0, n);
+      const int rowA = e * p.rows_per_expert + blk * MR;
       const int nB = (n + 15) / 16;
-      const uint32_t tx = (uint32_t)(C::kNumA * 8192 + nB * 2048);  // packed FP4 + e4m3 bytes
-      for (int kc = 0; kc < nk; ++kc) {
+      const uint32_t tx = (uint32_t)(C::kNumA * MR * 64 + nB * 2048);  // packed FP4 + e4m3 bytes
+      for (int kc = k0; kc < k1; ++kc) {
         const int s = it % STAGES;
         const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
         if (!wait_warp(empty(s), ph ^ 1u, p.wait_ns, abort_flag, p.status)) {
           ok = false;
           break;
         }
-        uint8_t* st = smem + s * C::kStage;
-        const uint32_t st_u = ptx::smem_u32(st);
+        const uint32_t st_u = ptx::smem_u32(smem + s * C::kStage);
         if (lane == 0) {
           ptx::mbar_arrive_expect_tx(full(s), tx);
           ptx::tma_load_2d(st_u, &p.tmA0, kc * 128, rowA, full(s));
@@ -227,128 +272,183 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
             ptx::tma_load_2d(st_u + C::kNumA * C::kATile + j * 2048, &p.tmB, kc * 128,
                              row0 + 16 * j, full(s));
         }
-        // weight scales of this 128-wide chunk: 4 bytes per row, laid out for
-        // tcgen05.cp 32x128b.warpx4 (row m at byte (m%32)*16 + (m/32)*4)
-        const uint32_t sf0 = st_u + C::kNumA * C::kATile + C::kBTile;
-#pragma unroll
-        for (int m1 = 0; m1 < 4; ++m1) {
-          const size_t r = (size_t)(rowA + m1 * 32 + lane);
-          ptx::cp_async_4(sf0 + lane * 16 + m1 * 4, p.sfa0 + r * ldsf + kc * 4);
-          if (PHASE == 1) ptx::cp_async_4(sf0 + 512 + lane * 16 + m1 * 4, p.sfa1 + r * ldsf + kc * 4);
-        }
-        ptx::cp_async_commit();
-        if (it >= kLag) {
-          ptx::cp_async_wait_group<kLag>();
-          ptx::fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(full((it - kLag) % STAGES));
-        }
         ++it;
       }
+      c += (unsigned long long)(k1 - k0);
     }
-    ptx::cp_async_wait_all();
-    ptx::fence_proxy_async_smem();
     __syncwarp();
-    if (lane == 0) {
-      for (int j = it - kLag < 0 ? 0 : it - kLag; j < it; ++j) ptx::mbar_arrive(full(j % STAGES));
-      if (!ok)  // let every issued TMA copy land before the CTA can exit
-        for (int j = it - STAGES < 0 ? 0 : it - STAGES; j < it; ++j)
-          drain_wait(full(j % STAGES), (uint32_t)(j / STAGES) & 1u);
+    if (lane == 0 && !ok)  // let every issued TMA copy land before the CTA can exit
+      for (int j = it - STAGES < 0 ? 0 : it - STAGES; j < it; ++j)
+        drain_wait(full(j % STAGES), (uint32_t)(j / STAGES) & 1u);
+  } else if (warp == kSfWarp) {
+    // ------------------------------------------------------------ weight-scale loader
+    // 4 bytes (4 K-blocks of 32) per weight row and chunk, gathered with cp.async into
+    // the tcgen05.cp 32x128b.warpx4 layout (row m at byte (m%32)*16 + (m/32)*4).  Each
+    // lane's copies arrive on the stage's full barrier by themselves when they land
+    // (cp.async.mbarrier.arrive.noinc), so this warp never waits for its own loads.
+    const size_t ldsf = (size_t)(p.K / 32);
+    int it = 0;
+    bool ok = true;
+    for (unsigned long long c = beg; c < end && ok;) {
+      const int ti = (int)(c / nk);
+      const int k0 = (int)(c % nk);
+      const int k1 = (int)min((unsigned long long)nk, (unsigned long long)k0 + (end - c));
+      int e, blk, row0, n;
+      decode_tile(g_ttbase, g_tiles, p.E, HB, ti, e, blk, row0, n);
+      const int rowA = e * p.rows_per_expert + blk * MR;
+      if (p.pf_dist > 0) {
+        // Pull this segment's weight bytes into L2 row by row ahead of the TMA loads:
+        // each row's K range is contiguous, so DRAM reads whole runs of a page instead of
+        // the 64-byte pieces the TMA boxes ask for one chunk at a time.
+        const size_t rb = (size_t)(p.K / 2);
+        const size_t lo = (size_t)k0 * 64, hi = (size_t)k1 * 64;
+        for (int r = lane; r < MR; r += 32) {
+          const uint8_t* g = p.a0_codes + (size_t)(rowA + r) * rb;
+          const uint8_t* u = p.a1_codes + (size_t)(rowA + r) * rb;
+          for (size_t o = lo & ~(size_t)127; o < hi; o += 128) {
+            prefetch_line_l2(g + o);
+            if (PHASE == 1) prefetch_line_l2(u + o);
+          }
+        }
+      }
+      for (int kc = k0; kc < k1; ++kc) {
+        const int s = it % STAGES;
+        const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+        if (!wait_warp(empty(s), ph ^ 1u, p.wait_ns, abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        const uint32_t sf0 = ptx::smem_u32(smem + s * C::kStage) + C::kNumA * C::kATile + C::kBTile;
+#pragma unroll
+        for (int rb = 0; rb < C::kRB; ++rb) {
+#pragma unroll
+          for (int m1 = 0; m1 < 4; ++m1) {
+            const size_t r = (size_t)(rowA + rb * 128 + m1 * 32 + lane);
+            const uint32_t off = rb * 512 + lane * 16 + m1 * 4;
+            ptx::cp_async_4(sf0 + off, p.sfa0 + r * ldsf + kc * 4);
+            if (PHASE == 1) ptx::cp_async_4(sf0 + C::kSF + off, p.sfa1 + r * ldsf + kc * 4);
+          }
+        }
+        ptx::cp_async_arrive_noinc(sf_full(s));
+        ++it;
+      }
+      c += (unsigned long long)(k1 - k0);
     }
+    ptx::cp_async_wait_all();  // no copy of this warp may still be in flight at exit
+    __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       ptx::tc_cp_32x128b_x4(tmem + C::kColSFB, ptx::make_sdesc(ptx::smem_u32(sfb), 0, 128, 0));
       int it = 0, ch = 0;
       bool ok = true;
-      for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
+      for (unsigned long long c = beg; c < end && ok;) {
+        const int ti = (int)(c / nk);
+        const int k0 = (int)(c % nk);
+        const int k1 = (int)min((unsigned long long)nk, (unsigned long long)k0 + (end - c));
         int e, blk, row0, n;
-        decode_tile(g_ttbase, g_tiles, p.E, HB, i, e, blk, row0, n);
+        decode_tile(g_ttbase, g_tiles, p.E, HB, ti, e, blk, row0, n);
         const uint32_t N = (uint32_t)((n + 15) & ~15);
         // kind::mxf8f6f4 instruction descriptor: A = e2m1 (5), B = e4m3 (0), both K-major,
         // ue8m0 scales, N >> 3 at bit 17, M >> 4 at bit 24; A scale id at bits 29-30.
         const uint32_t idesc0 = (5u << 7) | (0u << 10) | ((N >> 3) << 17) | (1u << 23) |
                                 ((128u >> 4) << 24);
-        for (int kc = 0; kc < nk; ++kc) {
+        for (int kc = k0; kc < k1; ++kc) {
           const int s = it % STAGES;
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-          const int b = ch & 1;
-          const uint32_t tph = (uint32_t)(ch >> 1) & 1u;
+          const int b = ch % NBUF;
+          const uint32_t tph = (uint32_t)(ch / NBUF) & 1u;
           if (!wait_one(tempty(b), tph ^ 1u, p.wait_ns, abort_flag, p.status)) { ok = false; break; }
           ptx::tc_fence_after();
           if (!wait_one(full(s), ph, p.wait_ns, abort_flag, p.status)) { ok = false; break; }
+          if (!wait_one(sf_full(s), ph, p.wait_ns, abort_flag, p.status)) { ok = false; break; }
           ptx::tc_fence_after();
+          ptx::fence_proxy_async_smem();  // scale bytes came through cp.async (generic proxy)
           const uint32_t a0 = ptx::smem_u32(smem + s * C::kStage);
           const uint32_t bb = a0 + C::kNumA * C::kATile;
           const uint32_t sf0 = bb + C::kBTile;
-          ptx::tc_cp_32x128b_x4(tmem + C::kColSFA0, ptx::make_sdesc(sf0, 0, 128, 0));
-          if (PHASE == 1)
-            ptx::tc_cp_32x128b_x4(tmem + C::kColSFA1, ptx::make_sdesc(sf0 + 512, 0, 128, 0));
-          const uint64_t da0 = ptx::make_sdesc(a0, 16, 1024, 2);
-          const uint64_t da1 = ptx::make_sdesc(a0 + C::kATile, 16, 1024, 2);
+#pragma unroll
+          for (int rb = 0; rb < C::kRB; ++rb) {
+            ptx::tc_cp_32x128b_x4(tmem + C::kColSFA0 + 4 * rb,
+                                  ptx::make_sdesc(sf0 + rb * 512, 0, 128, 0));
+            if (PHASE == 1)
+              ptx::tc_cp_32x128b_x4(tmem + C::kColSFA1 + 4 * rb,
+                                    ptx::make_sdesc(sf0 + C::kSF + rb * 512, 0, 128, 0));
+          }
           const uint64_t db = ptx::make_sdesc(bb, 16, 1024, 2);
           const uint32_t acc = tmem + (uint32_t)(b * C::kAccCols);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {  // four K = 32 steps through the 128-byte rows
             // scale id kk selects byte kk of each SFA word: the scale of K-block kk
             const uint32_t idesc = idesc0 | ((uint32_t)kk << 29);
-            ptx::tc_mma_mxf8f6f4(acc, da0 + 2 * kk, db + 2 * kk, idesc,
-                                 tmem + C::kColSFA0, tmem + C::kColSFB,
-                                 kk > 0 ? 1u : 0u);
-            if (PHASE == 1)
-              ptx::tc_mma_mxf8f6f4(acc + NMAX, da1 + 2 * kk, db + 2 * kk, idesc,
-                                   tmem + C::kColSFA1, tmem + C::kColSFB,
-                                   kk > 0 ? 1u : 0u);
+#pragma unroll
+            for (int m = 0; m < C::kNumA; ++m) {
+#pragma unroll
+              for (int rb = 0; rb < C::kRB; ++rb) {  // rows rb*128.. start 16 KB further in
+                const uint64_t da = ptx::make_sdesc(a0 + m * C::kATile + rb * 16384, 16, 1024, 2);
+                ptx::tc_mma_mxf8f6f4(acc + (uint32_t)((m * C::kRB + rb) * NMAX), da + 2 * kk,
+                                     db + 2 * kk, idesc,
+                                     tmem + (m == 0 ? C::kColSFA0 : C::kColSFA1) + 4 * rb,
+                                     tmem + C::kColSFB, kk > 0 ? 1u : 0u);
+              }
+            }
           }
           ptx::tc_commit(empty(s));
           ptx::tc_commit(tfull(b));
           ++it;
           ++ch;
         }
+        c += (unsigned long long)(k1 - k0);
       }
       ptx::tc_commit(drain);  // every MMA / copy of this thread done before teardown
       drain_wait(drain, 0);
     }
     __syncwarp();
-  } else {
+  } else if (warp < 2 + kEpiWarps) {
     // ------------------------------------------------------------ epilogue
     const int ew = warp - 2;
     const int q = warp & 3;
-    const int h = ew >> 2;
-    const int col0 = h * C::kHalf;
+    const int h = ew >> 2;                          // warp group 0/1
+    const int rb = C::kRB == 2 ? h : 0;             // 128-row block of the weight tile
+    const int col0 = C::kRB == 2 ? 0 : h * C::kCols;  // first column of this warp
     const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
+    const size_t slot_floats = (size_t)p.ncap * kMat * MR;
     int ch = 0;
     bool ok = true;
-    for (int i = blockIdx.x; i < total; i += gridDim.x) {
+    for (unsigned long long c = beg; c < end;) {
+      const int ti = (int)(c / nk);
+      const int k0 = (int)(c % nk);
+      const int k1 = (int)min((unsigned long long)nk, (unsigned long long)k0 + (end - c));
       int e, blk, row0, n;
-      decode_tile(g_ttbase, g_tiles, p.E, HB, i, e, blk, row0, n);
-      // this tile's activation scales, transposed to sbs[kc][column]
+      decode_tile(g_ttbase, g_tiles, p.E, HB, ti, e, blk, row0, n);
+      // this segment's activation scales, transposed to sbs[kc][column]
       bar_sync(1, kEpiWarps * 32);
-      for (int x = ew * 32 + lane; x < n * nk; x += kEpiWarps * 32) {
-        const int c = x / nk, kc = x - c * nk;
-        sbs[kc * NMAX + c] = __ldg(p.b_scales + (size_t)(row0 + c) * nk + kc);
+      const int nkk = k1 - k0;
+      for (int x = ew * 32 + lane; x < n * nkk; x += kEpiWarps * 32) {
+        const int cc = x / nkk, kc = k0 + (x - cc * nkk);
+        sbs[kc * NMAX + cc] = __ldg(p.b_scales + (size_t)(row0 + cc) * nk + kc);
       }
       bar_sync(1, kEpiWarps * 32);
-      float acc0[C::kHalf], acc1[C::kHalf];
+      float acc0[C::kCols], acc1[C::kCols];
 #pragma unroll
-      for (int c = 0; c < C::kHalf; ++c) {
-        acc0[c] = 0.f;
-        acc1[c] = 0.f;
+      for (int j = 0; j < C::kCols; ++j) {
+        acc0[j] = 0.f;
+        acc1[j] = 0.f;
       }
-      for (int kc = 0; kc < nk; ++kc) {
-        const int b = ch & 1;
-        const uint32_t tph = (uint32_t)(ch >> 1) & 1u;
+      for (int kc = k0; kc < k1; ++kc) {
+        const int b = ch % NBUF;
+        const uint32_t tph = (uint32_t)(ch / NBUF) & 1u;
         ok = ok && wait_warp(tfull(b), tph, p.wait_ns, abort_flag, p.status);
         ptx::tc_fence_after();
         if (ok) {
-          const uint32_t base = tl + (uint32_t)(b * C::kAccCols + col0);
+          const uint32_t base = tl + (uint32_t)(b * C::kAccCols + rb * NMAX + col0);
           const float* sc = sbs + kc * NMAX + col0;
 #pragma unroll
-          for (int g = 0; g < C::kHalf / 8; ++g) {
+          for (int g = 0; g < C::kCols / 8; ++g) {
             if (col0 + 8 * g < n) {
               float v0[8], v1[8];
               ptx::tc_ld_32x32b_x8(base + 8 * g, v0);
-              if (PHASE == 1) ptx::tc_ld_32x32b_x8(base + NMAX + 8 * g, v1);
+              if (PHASE == 1) ptx::tc_ld_32x32b_x8(base + C::kRB * NMAX + 8 * g, v1);
               ptx::tc_wait_ld();
 #pragma unroll
               for (int j = 0; j < 8; ++j) {
@@ -363,41 +463,102 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
         if (lane == 0) ptx::mbar_arrive(tempty(b));
         ++ch;
       }
+      c += (unsigned long long)nkk;
+
+      // ---- stream-K fix-up of a tile cut between CTAs.  The tile's segments belong to
+      // the CTAs owning its chunks (CTAs with empty ranges own none): walk them in order.
+      const unsigned long long t0c = (unsigned long long)ti * nk;
+      int nseg = 0;
+      for (unsigned long long cc = t0c; cc < t0c + nk;) {
+        ++nseg;
+        cc = sp.begin(sp.owner(cc) + 1);
+      }
+      bool finish = true;
+      if (nseg > 1) {
+        const int my_slot = 2 * blockIdx.x + ((int)(beg / nk) == ti ? 0 : 1);
+        float* mine = p.partials + (size_t)my_slot * slot_floats;
+        if (ok) {
+#pragma unroll
+          for (int j = 0; j < C::kCols; ++j) {
+            const int cc = col0 + j;
+            if (cc < n) {
+              mine[((size_t)cc * kMat + 0) * MR + rb * 128 + q * 32 + lane] = acc0[j];
+              if (PHASE == 1) mine[((size_t)cc * kMat + 1) * MR + rb * 128 + q * 32 + lane] = acc1[j];
+            }
+          }
+        }
+        __threadfence();
+        bar_sync(1, kEpiWarps * 32);
+        if (ew == 0 && lane == 0)
+          *fix_word = *abort_flag ? -1 : atomicAdd(p.counters + ti, 1);
+        bar_sync(1, kEpiWarps * 32);
+        const int arrived = *fix_word;
+        finish = arrived == nseg - 1;
+        if (finish) {
+          __threadfence();
+          // all segments, this CTA's included, from their slots in chunk order: the sum
+          // does not depend on which CTA finishes last
+          bool first_seg = true;
+          for (unsigned long long cs = t0c; cs < t0c + nk;) {
+            const int s = sp.owner(cs);
+            cs = sp.begin(s + 1);
+            const int slot = 2 * s + ((int)(sp.begin(s) / nk) == ti ? 0 : 1);
+            const float* src = p.partials + (size_t)slot * slot_floats;
+#pragma unroll
+            for (int j = 0; j < C::kCols; ++j) {
+              const int cc = col0 + j;
+              if (cc < n) {
+                const float v0 = __ldcg(src + ((size_t)cc * kMat + 0) * MR + rb * 128 + q * 32 + lane);
+                acc0[j] = first_seg ? v0 : acc0[j] + v0;
+                if (PHASE == 1) {
+                  const float v1 = __ldcg(src + ((size_t)cc * kMat + 1) * MR + rb * 128 + q * 32 + lane);
+                  acc1[j] = first_seg ? v1 : acc1[j] + v1;
+                }
+              }
+            }
+            first_seg = false;
+          }
+          if (ew == 0 && lane == 0) p.counters[ti] = 0;  // ready for the next launch
+        }
+      }
+      finish = finish && ok;
+
       if (PHASE == 1) {
         // h = silu(g) * u, then per-column (token) e4m3 re-quantisation over the 128 rows
         float* hv = acc0;  // h overwrites g in place
-        float* am = amax_s + (h * 4 + q) * C::kHalf;
+        float* am = amax_s + (h * 4 + q) * C::kCols;
 #pragma unroll
-        for (int c = 0; c < C::kHalf; ++c) {
-          const float g = acc0[c];
-          hv[c] = g / (1.0f + expf(-g)) * acc1[c];
-          const unsigned m = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(hv[c])));
-          if (lane == 0) am[c] = __uint_as_float(m);
+        for (int j = 0; j < C::kCols; ++j) {
+          const float g = acc0[j];
+          hv[j] = g / (1.0f + expf(-g)) * acc1[j];
+          const unsigned m = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(hv[j])));
+          if (lane == 0) am[j] = __uint_as_float(m);
         }
         bar_sync(2 + h, 128);
 #pragma unroll
-        for (int c = 0; c < C::kHalf; ++c) {
-          if (ok && col0 + c < n) {
-            float amax = amax_s[(h * 4 + 0) * C::kHalf + c];
-            amax = fmaxf(amax, amax_s[(h * 4 + 1) * C::kHalf + c]);
-            amax = fmaxf(amax, amax_s[(h * 4 + 2) * C::kHalf + c]);
-            amax = fmaxf(amax, amax_s[(h * 4 + 3) * C::kHalf + c]);
+        for (int j = 0; j < C::kCols; ++j) {
+          if (finish && col0 + j < n) {
+            float amax = amax_s[(h * 4 + 0) * C::kCols + j];
+            amax = fmaxf(amax, amax_s[(h * 4 + 1) * C::kCols + j]);
+            amax = fmaxf(amax, amax_s[(h * 4 + 2) * C::kCols + j]);
+            amax = fmaxf(amax, amax_s[(h * 4 + 3) * C::kCols + j]);
             const float s = amax == 0.f ? 1.0f : __fdiv_rn(amax, 448.0f);
-            const int row = row0 + col0 + c;
-            const uint16_t code = ptx::cvt_e4m3x2(__fdiv_rn(hv[c], s), 0.f);
-            p.qh[(size_t)row * p.f + blk * 128 + q * 32 + lane] = (uint8_t)(code & 0xFF);
-            if (q == 0 && lane == 0) p.sh[(size_t)row * (p.f / 128) + blk] = s;
+            const int row = row0 + col0 + j;
+            const uint16_t code = ptx::cvt_e4m3x2(__fdiv_rn(hv[j], s), 0.f);
+            const int hb = blk * C::kRB + rb;  // 128-wide block of h
+            p.qh[(size_t)row * p.f + hb * 128 + q * 32 + lane] = (uint8_t)(code & 0xFF);
+            if (q == 0 && lane == 0) p.sh[(size_t)row * (p.f / 128) + hb] = s;
           }
         }
         bar_sync(2 + h, 128);
       } else {
 #pragma unroll
-        for (int c = 0; c < C::kHalf; ++c) {
-          if (ok && col0 + c < n) {
-            const int row = row0 + col0 + c;
+        for (int j = 0; j < C::kCols; ++j) {
+          if (finish && col0 + j < n) {
+            const int row = row0 + col0 + j;
             float* dst = row < p.P ? p.y_routed + (size_t)row * p.d
                                    : p.y_shared + (size_t)(row - p.P) * p.d;
-            dst[blk * 128 + q * 32 + lane] = acc0[c];
+            dst[(blk * C::kRB + rb) * 128 + q * 32 + lane] = acc0[j];
           }
         }
       }
@@ -448,35 +609,54 @@ bool make_map(CUtensorMap* m, const void* base, bool fp4, int K, long long rows,
   return r == CUDA_SUCCESS;
 }
 
-template <int PHASE, int NMAX, int STAGES>
+template <int PHASE, int NMAX, int STAGES, int NBUF, int MR>
 cudaError_t launch_one(const FfnParams& prm, int nk, cudaStream_t s, int grid) {
-  using C = Cfg<PHASE, NMAX, STAGES>;
+  using C = Cfg<PHASE, NMAX, STAGES, NBUF, MR>;
   const size_t smem = C::smem_bytes(nk, prm.E);
-  cudaError_t err = cudaFuncSetAttribute(ffn_kernel<PHASE, NMAX, STAGES>,
+  cudaError_t err = cudaFuncSetAttribute(ffn_kernel<PHASE, NMAX, STAGES, NBUF, MR>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  ffn_kernel<PHASE, NMAX, STAGES><<<grid, kThreads, smem, s>>>(prm);
+  ffn_kernel<PHASE, NMAX, STAGES, NBUF, MR><<<grid, kThreads, smem, s>>>(prm);
   return cudaGetLastError();
+}
+
+// (PHASE, NMAX) -> pipeline stages, TMEM partial buffers, weight rows per tile.  Small
+// batches take 256-row tiles: one TMA box then moves 16 KB of FP4, which streams HBM far
+// better than 8 KB boxes; large batches keep 128-row tiles to leave TMEM for wide N.
+#define BITMOE_FFN_VARIANTS(X)                  \
+  X(1, kNmaxSmall, 3, 3, 256)                   \
+  X(1, kNmaxSmall, 5, 6, 128)                   \
+  X(1, kNmaxLarge, 4, 2, 128)                   \
+  X(2, kNmaxSmall, 5, 6, 256)                   \
+  X(2, kNmaxSmall, 8, 8, 128)                   \
+  X(2, kNmaxLarge, 6, 4, 128)
+
+int tile_rows(int nmax, int rows_per_expert) {
+  return nmax == kNmaxSmall && rows_per_expert % 256 == 0 ? 256 : 128;
 }
 
 }  // namespace
 
-size_t ffn_smem_bytes(int phase, int nmax, int nk, int E) {
-  if (phase == 1)
-    return nmax == kNmaxSmall ? Cfg<1, kNmaxSmall, 5>::smem_bytes(nk, E)
-                              : Cfg<1, kNmaxLarge, 4>::smem_bytes(nk, E);
-  return nmax == kNmaxSmall ? Cfg<2, kNmaxSmall, 8>::smem_bytes(nk, E)
-                            : Cfg<2, kNmaxLarge, 6>::smem_bytes(nk, E);
+size_t ffn_smem_bytes(int phase, int nmax, int nk, int E, int rows_per_expert) {
+  const int mr = tile_rows(nmax, rows_per_expert);
+#define X(P, N, S, B, M) \
+  if (phase == P && nmax == N && mr == M) return Cfg<P, N, S, B, M>::smem_bytes(nk, E);
+  BITMOE_FFN_VARIANTS(X)
+#undef X
+  return 0;
 }
 
 cudaError_t launch_ffn(int phase, int nmax, const FfnArgs& a, cudaStream_t s, int num_sms) {
   FfnParams prm;
   memset(&prm, 0, sizeof(prm));
   const long long rows_total = (long long)(a.E + 1) * a.rows_per_expert;
-  if (!make_map(&prm.tmA0, a.a0_codes, true, a.K, rows_total, 128)) return cudaErrorInvalidValue;
-  if (phase == 1 && !make_map(&prm.tmA1, a.a1_codes, true, a.K, rows_total, 128))
+  const int mr = tile_rows(nmax, a.rows_per_expert);
+  if (!make_map(&prm.tmA0, a.a0_codes, true, a.K, rows_total, mr)) return cudaErrorInvalidValue;
+  if (phase == 1 && !make_map(&prm.tmA1, a.a1_codes, true, a.K, rows_total, mr))
     return cudaErrorInvalidValue;
   if (!make_map(&prm.tmB, a.b_codes, false, a.K, a.R, 16)) return cudaErrorInvalidValue;
+  prm.a0_codes = a.a0_codes;
+  prm.a1_codes = a.a1_codes;
   prm.sfa0 = a.a0_scales;
   prm.sfa1 = a.a1_scales;
   prm.b_scales = a.b_scales;
@@ -494,12 +674,17 @@ cudaError_t launch_ffn(int phase, int nmax, const FfnArgs& a, cudaStream_t s, in
   prm.y_shared = a.y_shared;
   prm.wait_ns = a.wait_ns;
   prm.status = a.status;
+  prm.counters = a.counters;
+  prm.partials = a.partials;
+  prm.ncap = a.ncap;
+  prm.pf_dist = a.pf_dist;
   const int nk = a.K / 128;
-  if (phase == 1)
-    return nmax == kNmaxSmall ? launch_one<1, kNmaxSmall, 5>(prm, nk, s, num_sms)
-                              : launch_one<1, kNmaxLarge, 4>(prm, nk, s, num_sms);
-  return nmax == kNmaxSmall ? launch_one<2, kNmaxSmall, 8>(prm, nk, s, num_sms)
-                            : launch_one<2, kNmaxLarge, 6>(prm, nk, s, num_sms);
+  const int grid = num_sms < kMaxCtas ? num_sms : kMaxCtas;
+#define X(P, N, S, B, M) \
+  if (phase == P && nmax == N && mr == M) return launch_one<P, N, S, B, M>(prm, nk, s, grid);
+  BITMOE_FFN_VARIANTS(X)
+#undef X
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace bitmoe

@@ -17,6 +17,12 @@ constexpr int kStatusBadIndex = 2;
 constexpr int kNmaxLarge = 112;  // T > 32
 constexpr int kNmaxSmall = 32;   // T <= 32: every group fits one tile
 inline int nmax_for(int T) { return T <= kNmaxSmall ? kNmaxSmall : kNmaxLarge; }
+// Widest token tile a launch can see (a tile never holds more rows than T).
+inline int ncap_for(int T) { return T < nmax_for(T) ? T : nmax_for(T); }
+
+// The FFN kernels run at most this many CTAs (one per SM); the stream-K partial slots of
+// the workspace are sized for it.
+constexpr int kMaxCtas = 148;
 
 // Plan layout (int32 words in the workspace):
 //   [0, E+2)              ttbase: first token tile of expert e (e = 0..E), ttbase[E+1] = total
@@ -24,7 +30,8 @@ inline int nmax_for(int T) { return T <= kNmaxSmall ? kNmaxSmall : kNmaxLarge; }
 inline size_t plan_ntmax(int R, int E) { return (size_t)R / 16 + (size_t)E + 2; }
 
 struct WorkspaceLayout {
-  size_t plan, qx, sx, qh, sh, total;
+  size_t plan, qx, sx, qh, sh, counters, partials, total;
+  size_t n_counters;
 };
 WorkspaceLayout workspace_layout(int T, int k, int E, int d, int f);
 
@@ -39,7 +46,8 @@ cudaError_t launch_dispatch(const int32_t* idx, int T, int k, int E, int32_t* co
 // writes the token-tile plan.
 cudaError_t launch_quant_rows(const uint16_t* x, int T, int k, int d, const int32_t* perm,
                               int nrows_routed, uint8_t* q, float* s, const int32_t* offsets,
-                              int E, int nmax, int32_t* plan, int* status, cudaStream_t st);
+                              int E, int nmax, int32_t* plan, int* counters, size_t n_counters,
+                              int* status, cudaStream_t st);
 cudaError_t launch_combine(const float* y, const float* ysh, const float* w, const int32_t* pos,
                            int T, int k, int d, float* out, int* status, cudaStream_t s);
 
@@ -60,9 +68,14 @@ struct FfnArgs {
   int d;
   long long wait_ns;
   int* status;
+  int* counters;             // stream-K fix-up counters (zeroed by the prepare kernel)
+  float* partials;           // stream-K partial slots
+  int ncap;                  // widest token tile
+  int pf_dist;               // > 0: prefetch each segment's weight rows into L2
 };
 cudaError_t launch_ffn(int phase, int nmax, const FfnArgs& a, cudaStream_t s, int num_sms);
-size_t ffn_smem_bytes(int phase, int nmax, int nk, int E);  // dynamic shared memory of a launch
+// dynamic shared memory of a launch
+size_t ffn_smem_bytes(int phase, int nmax, int nk, int E, int rows_per_expert);
 
 // Defined in abi.cu: sets the thread-local message that moe_last_error returns.
 int record_error(int code, const char* msg);

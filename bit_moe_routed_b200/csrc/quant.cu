@@ -59,9 +59,14 @@ __device__ void write_plan(const int32_t* __restrict__ offsets, int E, int T, in
 __global__ void __launch_bounds__(256) quant_rows_kernel(
     const uint16_t* __restrict__ x, int T, int k, int d, const int32_t* __restrict__ perm, int P,
     uint8_t* __restrict__ q, float* __restrict__ s, const int32_t* __restrict__ offsets, int E,
-    int nmax, int32_t* __restrict__ plan, int* __restrict__ status) {
+    int nmax, int32_t* __restrict__ plan, int* __restrict__ counters, size_t n_counters,
+    int* __restrict__ status) {
   const int R = P + T;
   const int r = blockIdx.x;
+  // the FFN kernels' stream-K counters start every launch at zero
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_counters;
+       i += (size_t)gridDim.x * blockDim.x)
+    counters[i] = 0;
   if (r == R) {  // the plan block
     if (threadIdx.x < 32) write_plan(offsets, E, T, P, nmax, plan);
     return;
@@ -112,13 +117,14 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(
 
 cudaError_t launch_quant_rows(const uint16_t* x, int T, int k, int d, const int32_t* perm,
                               int nrows_routed, uint8_t* q, float* s, const int32_t* offsets,
-                              int E, int nmax, int32_t* plan, int* status, cudaStream_t st) {
+                              int E, int nmax, int32_t* plan, int* counters, size_t n_counters,
+                              int* status, cudaStream_t st) {
   const int R = nrows_routed + T;
   const unsigned blocks = (unsigned)(R + (plan != nullptr ? 1 : 0));
   int threads = (d / 16 + 31) / 32 * 32;  // whole warps
   if (threads > 256) threads = 256;
   quant_rows_kernel<<<blocks, threads, 0, st>>>(x, T, k, d, perm, nrows_routed, q, s, offsets, E,
-                                               nmax, plan, status);
+                                               nmax, plan, counters, n_counters, status);
   return cudaGetLastError();
 }
 
