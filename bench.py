@@ -6,8 +6,10 @@
 One step = one pass of the whole layer over one batch of synthetic tokens, with the
 layer's weights resident in HBM.  Default workload: one decode layer, T=1 token,
 256 routed experts + 1 shared, top-6, d=4096, f=2048 (FP4 e2m1 weights, e4m3
-activations).  The step is captured once in a CUDA graph and replayed; L2 is flushed
-(256 MiB write) between steps outside the timed events.  Multi-GPU runs are replicas
+activations).  Each step is one layer; the steps rotate over several resident layers,
+each with its own weights and tokens, so that a step never finds its weights in L2 from
+before (inputs larger than L2).  Each layer's step is captured once in a CUDA graph and
+replayed.  Multi-GPU runs are replicas
 (each rank its own tokens and weights, no collective on the data path) -> weak scaling.
 
 Prints one JSON line (rank 0).  `--impl reference` times the oracle (the plain CPU
@@ -223,56 +225,67 @@ def run_gpu(args, w):
     dev = torch.device("cuda", local)
     hbm_peak, bf16_peak, bf16_sus, peak_kind = load_peaks()
 
-    # inputs: each rank its own tokens (replica); weights resident in HBM
-    seed = replica_seed(w, rank)
-    if rank == 0:
-        x_cpu, s_cpu = synth.gen_layer_inputs(w, 0)
-    else:
-        x_cpu = synth.gen_x(w.T, w.d, seed)
-        s_cpu = synth.gen_scores_uniform(w.T, w.E, seed) if w.routing == "uniform" else \
-            synth.gen_scores_zipf(w.T, w.E, w.zipf_s, seed)
-    W = bm.LayerWeights.from_dict(synth.device_layer_weights(w.seed(0), 0, w.E, w.d, w.f))
-    x = x_cpu.to(dev)
-    scores = s_cpu.to(dev)
+    # Working set: L layers resident in HBM, each with its own weights and tokens; step i
+    # runs layer i % L.  L is chosen so the other L-1 layers' weights exceed four times
+    # the L2, so a step's weights are never still in L2 from its previous use (read-only
+    # weights: no dirty lines to write back, unlike a write-flush).
     T, k, E, d, f = w.T, w.k, w.E, w.d, w.f
+    per_expert = synth.expert_bytes(d, f)
+    est_active = min(E, T * k) + 1
+    step_bytes = est_active * per_expert
+    L2_BYTES = 126 * 2 ** 20
+    n_layers = max(2, min(args.max_layers, -(-4 * L2_BYTES // step_bytes) + 1))
+    layers = []
+    for l in range(n_layers):
+        seed = replica_seed(w, rank) + l
+        if rank == 0:
+            x_cpu, s_cpu = synth.gen_layer_inputs(w, l)
+        else:
+            x_cpu = synth.gen_x(T, d, seed)
+            s_cpu = synth.gen_scores_uniform(T, E, seed) if w.routing == "uniform" else \
+                synth.gen_scores_zipf(T, E, w.zipf_s, seed)
+        W = bm.LayerWeights.from_dict(synth.device_layer_weights(w.seed(l), l, E, d, f))
+        layers.append(dict(x_cpu=x_cpu, s_cpu=s_cpu, W=W, x=x_cpu.to(dev), scores=s_cpu.to(dev)))
     ws = bm.alloc_workspace(T, k, E, d, f, dev)
     y = torch.empty((T * k, d), dtype=torch.float32, device=dev)
     ysh = torch.empty((T, d), dtype=torch.float32, device=dev)
     out = torch.empty((T, d), dtype=torch.float32, device=dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.Stream(dev)
-    ev = {n: torch.cuda.Event(enable_timing=True) for n in ("a", "b", "c", "d", "e")}
 
-    def step(evs=None):
+    def step(L):
         # route -> dispatch -> FFN (prepare | gate/up | down) -> combine
-        idx, gw = bm.route_topk(scores, k, stream)
+        idx, gw = bm.route_topk(L["scores"], k, stream)
         counts, offsets, perm, pos = bm.dispatch(idx, E, stream)
-        bm.ffn_prepare(x, k, W, offsets, perm, ws, stream)
-        bm.ffn_gate_up(T, k, W, ws, stream)
-        bm.ffn_down(T, k, W, y, ysh, ws, stream)
+        bm.ffn_prepare(L["x"], k, L["W"], offsets, perm, ws, stream)
+        bm.ffn_gate_up(T, k, L["W"], ws, stream)
+        bm.ffn_down(T, k, L["W"], y, ysh, ws, stream)
         bm.combine(y, ysh, gw, pos, out, stream)
         return counts
 
-    # one eager pass (also checks the status word), then capture the step in a graph
-    with torch.cuda.stream(stream):
-        counts = step()
-    bm.sync_status(stream)
-    counts_np = counts.cpu().numpy()
-    work = layer_work(w, counts_np)
-
-    # graph of the whole step, and one of the gate/up kernel alone for its duration
-    g_step = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_step, stream=stream):
-        step()
-    g_gu = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_gu, stream=stream):
-        bm.ffn_gate_up(T, k, W, ws, stream)
+    # one eager pass per layer (checks the status word), then one graph per layer of the
+    # whole step, and one of the gate/up kernel alone (after its own prepare) per layer
+    works = []
+    for L in layers:
+        with torch.cuda.stream(stream):
+            counts = step(L)
+        bm.sync_status(stream)
+        works.append(layer_work(w, counts.cpu().numpy()))
+    work = works[0]
+    g_step, g_gu = [], []
+    for L in layers:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step(L)
+        g_step.append(g)
+        g2 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g2, stream=stream):
+            bm.ffn_gate_up(T, k, L["W"], ws, stream)
+        g_gu.append((g2, L))
     torch.cuda.synchronize()
 
-    for _ in range(args.warmup):
+    for i in range(args.warmup):
         with torch.cuda.stream(stream):
-            flush.zero_()
-            g_step.replay()
+            g_step[i % n_layers].replay()
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
@@ -281,22 +294,24 @@ def run_gpu(args, w):
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
-    step_ms, gu_ms = [], []
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     gs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ge = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     with torch.cuda.stream(stream):
         for i in range(args.steps):
-            flush.zero_()
             starts[i].record(stream)
-            g_step.replay()
+            g_step[i % n_layers].replay()
             ends[i].record(stream)
-        # the dominant kernel timed alone, same L2 treatment, same stream
+        # the dominant kernel timed alone: gate/up of layer i % L, after that layer's
+        # prepare (untimed) so its inputs are in place, same stream
         for i in range(args.steps):
-            flush.zero_()
+            gg, L = g_gu[i % n_layers]
+            idx, gw = bm.route_topk(L["scores"], k, stream)
+            _, offsets, perm, _ = bm.dispatch(idx, E, stream)
+            bm.ffn_prepare(L["x"], k, L["W"], offsets, perm, ws, stream)
             gs[i].record(stream)
-            g_gu.replay()
+            gg.replay()
             ge[i].record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
@@ -308,22 +323,22 @@ def run_gpu(args, w):
     value = world * T * args.steps / total_s
 
     # e2e through the public API with host buffers: pinned H2D of x and scores, the four
-    # calls, D2H of the layer output, every step
-    x_h = x_cpu.pin_memory()
-    s_h = s_cpu.pin_memory()
+    # calls, D2H of the layer output, every step (layer i % L)
+    for L in layers:
+        L["x_h"] = L["x_cpu"].pin_memory()
+        L["s_h"] = L["s_cpu"].pin_memory()
     out_h = torch.empty((T, d), dtype=torch.float32).pin_memory()
     e2e_ms = []
     for i in range(args.warmup + args.steps):
-        torch.cuda.synchronize()
-        flush.zero_()
+        L = layers[i % n_layers]
         torch.cuda.synchronize()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(stream):
             a.record(stream)
-            x.copy_(x_h, non_blocking=True)
-            scores.copy_(s_h, non_blocking=True)
-            r = bm.forward(x, scores, k, W, ws, stream)
+            L["x"].copy_(L["x_h"], non_blocking=True)
+            L["scores"].copy_(L["s_h"], non_blocking=True)
+            r = bm.forward(L["x"], L["scores"], k, L["W"], ws, stream)
             out_h.copy_(r["out"], non_blocking=True)
             b.record(stream)
         b.synchronize()
@@ -332,8 +347,13 @@ def run_gpu(args, w):
     e2e_s = max_over_ranks(sum(e2e_ms) / 1000.0, dist, dev)
     e2e_value = world * T * args.steps / e2e_s
     bm.sync_status(stream)
+    x_cpu, s_cpu = layers[0]["x_cpu"], layers[0]["s_cpu"]
 
     gu_avg_s = statistics.mean(gu_ms) / 1000.0
+    # per-launch algorithmic work averaged over the rotated layers
+    work = dict(work)
+    for key in ("gu_bytes", "dn_bytes", "flops_gu", "flops_dn", "weight_bytes", "active"):
+        work[key] = sum(wk[key] for wk in works) / len(works)
     is_prefill = T > 256
     kernel_file = os.path.join(ROOT, "bit_moe_routed_b200", "csrc", "ffn.cu")
     traffic = kernel_traffic(kernel_file, "gate_up", w.name)
@@ -369,9 +389,11 @@ def run_gpu(args, w):
             "dtype": "e2m1 x e4m3 -> f32", "data": "synthetic (seeded weights and tokens)",
             "config": {"workload": w.name, "T": T, "E": E, "k": k, "d": d, "f": f,
                        "routing": w.routing, "active_experts": work["active"],
-                       "l2": "flushed (256 MiB write) before every timed step",
+                       "l2": f"not flushed: step i runs layer i % {n_layers}, each with its own "
+                             f"weights ({n_layers * 257 * per_expert / 1e9:.1f} GB resident), so a "
+                             "step's weights were evicted by the other layers since their last use",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "launch": "CUDA graph of the 6 kernels"},
+                       "launch": "one CUDA graph of the 6 kernels per layer"},
             "layer": {"weight_gb_per_s": work["weight_bytes"] / layer_s / 1e9,
                       "weight_bytes": work["weight_bytes"],
                       "tflops": (work["flops_gu"] + work["flops_dn"]) / layer_s / 1e12},
@@ -399,6 +421,8 @@ def main():
     ap.add_argument("--impl", default="bitmoe", choices=["bitmoe", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--max-layers", type=int, default=8,
+                    help="most layers kept resident to rotate through (defeats L2 reuse)")
     ap.add_argument("--ref-seconds", type=float, default=None,
                     help="oracle seconds per step of the reference arm (default: fit ~1 min)")
     args = ap.parse_args()

@@ -108,7 +108,7 @@ struct Cfg {
     return (size_t)kOffTT + ((size_t)(E + 2) * 4 + 15) / 16 * 16;
   }
   __host__ __device__ static size_t smem_bytes(int nk, int E) {
-    return 1024 + off_sbs(E) + (size_t)nk * NMAX * 4;
+    return 1024 + off_sbs(E) + 2 * (size_t)nk * NMAX * 4;  // two scale buffers
   }
 };
 
@@ -413,22 +413,43 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
     const int col0 = C::kRB == 2 ? 0 : h * C::kCols;  // first column of this warp
     const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
     const size_t slot_floats = (size_t)p.ncap * kMat * MR;
-    int ch = 0;
+    // A segment's activation scales go to sbs[buf][kc][column] with cp.async, one commit
+    // group per segment, issued one segment ahead: when a segment starts, its scales have
+    // been in flight for the whole previous segment.
+    auto stage_scales = [&](unsigned long long cs, int buf) {
+      if (cs < end) {
+        const int ts = (int)(cs / nk);
+        const int s0 = (int)(cs % nk);
+        const int s1 = (int)min((unsigned long long)nk, (unsigned long long)s0 + (end - cs));
+        int e2, blk2, r2, n2;
+        decode_tile(g_ttbase, g_tiles, p.E, HB, ts, e2, blk2, r2, n2);
+        float* dstb = sbs + (size_t)buf * nk * NMAX;
+        const int ns = s1 - s0;
+        for (int x = ew * 32 + lane; x < n2 * ns; x += kEpiWarps * 32) {
+          const int cc = x / ns, kc = s0 + (x - cc * ns);
+          ptx::cp_async_4(ptx::smem_u32(dstb + kc * NMAX + cc),
+                          p.b_scales + (size_t)(r2 + cc) * nk + kc);
+        }
+      }
+      ptx::cp_async_commit();
+    };
+    int ch = 0, seg = 0;
     bool ok = true;
-    for (unsigned long long c = beg; c < end;) {
+    stage_scales(beg, 0);
+    for (unsigned long long c = beg; c < end; ++seg) {
       const int ti = (int)(c / nk);
       const int k0 = (int)(c % nk);
       const int k1 = (int)min((unsigned long long)nk, (unsigned long long)k0 + (end - c));
       int e, blk, row0, n;
       decode_tile(g_ttbase, g_tiles, p.E, HB, ti, e, blk, row0, n);
-      // this segment's activation scales, transposed to sbs[kc][column]
-      bar_sync(1, kEpiWarps * 32);
       const int nkk = k1 - k0;
-      for (int x = ew * 32 + lane; x < n * nkk; x += kEpiWarps * 32) {
-        const int cc = x / nkk, kc = k0 + (x - cc * nkk);
-        sbs[kc * NMAX + cc] = __ldg(p.b_scales + (size_t)(row0 + cc) * nk + kc);
-      }
+      // every warp is past the previous segment, so the other buffer is free: start the
+      // next segment's scales, then wait (normally not at all) for this segment's
       bar_sync(1, kEpiWarps * 32);
+      stage_scales(c + (unsigned long long)nkk, (seg + 1) & 1);
+      ptx::cp_async_wait_group<1>();
+      bar_sync(1, kEpiWarps * 32);
+      const float* sbs_cur = sbs + (size_t)(seg & 1) * nk * NMAX;
       float acc0[C::kCols], acc1[C::kCols];
 #pragma unroll
       for (int j = 0; j < C::kCols; ++j) {
@@ -442,7 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
         ptx::tc_fence_after();
         if (ok) {
           const uint32_t base = tl + (uint32_t)(b * C::kAccCols + rb * NMAX + col0);
-          const float* sc = sbs + kc * NMAX + col0;
+          const float* sc = sbs_cur + kc * NMAX + col0;
 #pragma unroll
           for (int g = 0; g < C::kCols / 8; ++g) {
             if (col0 + 8 * g < n) {
@@ -563,6 +584,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
         }
       }
     }
+    ptx::cp_async_wait_all();  // no scale copy may still be in flight at exit
   }
 
   ptx::tc_fence_before();
