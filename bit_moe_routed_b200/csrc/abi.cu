@@ -243,8 +243,8 @@ int ffn_check(int T, int k, const moe_weights_t* w, void* ws, size_t ws_bytes, F
   int dev = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-  const size_t need1 = ffn_smem_bytes(1, c.nmax, w->d / 128, w->E, w->f);
-  const size_t need2 = ffn_smem_bytes(2, c.nmax, w->f / 128, w->E, w->d);
+  const size_t need1 = ffn_smem_bytes(1, c.nmax, w->E, w->f);
+  const size_t need2 = ffn_smem_bytes(2, c.nmax, w->E, w->d);
   const size_t need = need1 > need2 ? need1 : need2;
   if (need > (size_t)max_smem)
     return fail(MOE_ERR_INVALID_ARG, "shape needs %zu bytes of shared memory (> %d)", need,
@@ -266,7 +266,7 @@ FfnArgs ffn_args(int phase, int T, int k, const moe_weights_t* w, const FfnCtx& 
   a.counters = reinterpret_cast<int*>(c.ws + c.L.counters);
   a.partials = reinterpret_cast<float*>(c.ws + c.L.partials);
   a.ncap = ncap_for(T);
-  a.pf_dist = 0;
+  a.l2_hints = 1;  // weight boxes evict-first
   if (phase == 1) {
     a.a0_codes = w->gate_codes;
     a.a0_scales = w->gate_scales;

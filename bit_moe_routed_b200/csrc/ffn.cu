@@ -16,28 +16,31 @@
 // tile, then computes h = silu(g) * u and re-quantises it per 128-block to e4m3;
 // phase 2 is the down projection writing fp32 y.
 //
-// Work split ("stream-K"): the tiles' 128-wide K chunks form one sequence of W chunks;
-// CTA b of G takes chunks [bW/G, (b+1)W/G), so every SM gets the same number of weight
-// bytes whatever the number of tiles.  A tile cut between CTAs is finished by the CTA
-// that completes its last segment: each writes its fp32 partial to a slot, the last
-// one (an atomic count) adds the segments in fixed order, so results are deterministic.
+// Work split: the tiles' 128-wide K chunks are the unit.  Whole tiles go out in rounds
+// (CTA b takes tiles b, b + G, b + 2G, ...), so the G CTAs always work on neighbouring
+// tiles and the weight blocks of one expert share each activation chunk through L2.  The
+// tiles left over after the last full round are cut into one run of chunks split evenly
+// over the CTAs ("stream-K"), so every SM gets the same number of weight bytes whatever
+// the number of tiles.  A tile cut between CTAs is finished by the CTA that completes its
+// last segment: each writes its fp32 partial to a slot, the last one (an atomic count)
+// adds the segments in fixed order, so results are deterministic.
 //
 // Activation scales are fp32 (amax/448), not ue8m0, so they cannot ride in the MMA:
 // B's hardware scale is 1.0 and every K chunk is accumulated into a fresh TMEM partial
 // that the epilogue warps fold into fp32 registers as acc += s * P.  A ring of NBUF
 // TMEM partials lets the MMA run NBUF chunks ahead of the epilogue.
 //
-// Memory: the weights are row-major ([rows][K/2]) and a TMA box takes 64 bytes from each
-// of 128 rows, which DRAM serves poorly.  So the scale-loader warp first pulls each
-// segment's rows into L2 with line prefetches that run along each row (contiguous
-// runs), a few chunks ahead of the TMA loads, which then mostly hit L2.
+// L2: a layer's weights stream through once; the TMA loads mark them evict-first so the
+// activation rows, which every weight block of an expert reads again, stay in L2.
 //
-// Warp roles (352 threads, one CTA per SM, persistent):
+// Warp roles (384 threads, one CTA per SM, persistent):
 //   warp 0   : TMA producer (weights, activations)
-//   warp 1   : TMEM allocator; lane 0 issues tcgen05.cp / tcgen05.mma / commits
+//   warp 1   : TMEM allocator; lane 0 issues tcgen05.cp / tcgen05.mma / commits for the
+//              gate (phase 1) or down (phase 2) matrix
 //   warps 2-9: epilogue; warp w reads TMEM lanes 32*(w%4).., column half (w-2)/4
-//   warp 10  : weight-scale loader (cp.async gather into the tcgen05.cp layout) and L2
-//              row prefetch
+//   warp 10  : scale loader: the weights' ue8m0 bytes (cp.async gather into the
+//              tcgen05.cp layout) and the tokens' fp32 activation scales of each chunk
+//   warp 11  : lane 0 issues the up matrix's tcgen05.cp / tcgen05.mma (phase 1)
 // Every wait is bounded by a %globaltimer limit; on expiry the kernel records a
 // timeout in the status word, lets in-flight copies and MMAs land, frees TMEM and
 // returns.
@@ -51,16 +54,15 @@ namespace bitmoe {
 namespace {
 
 constexpr int kEpiWarps = 8;
-constexpr int kSfWarp = 2 + kEpiWarps;          // warp 10 loads the weight scales
-constexpr int kThreads = 32 * (kSfWarp + 1);
+constexpr int kSfWarp = 2 + kEpiWarps;          // warp 10 loads the scales
+constexpr int kMma1Warp = kSfWarp + 1;          // warp 11 issues the up MMAs (phase 1)
+constexpr int kThreads = 32 * (kMma1Warp + 1);
 constexpr long long kDrainNs = 500000000LL;     // bound on draining in-flight work
 
 struct FfnParams {
   CUtensorMap tmA0;  // gate (phase 1) / down (phase 2) codes, all experts stacked
   CUtensorMap tmA1;  // up codes (phase 1)
   CUtensorMap tmB;   // activation rows [R][K] e4m3
-  const uint8_t* a0_codes;  // the same codes as plain pointers (L2 prefetch)
-  const uint8_t* a1_codes;
   const uint8_t* sfa0;
   const uint8_t* sfa1;
   const float* b_scales;  // [R][K/128]
@@ -73,7 +75,7 @@ struct FfnParams {
   int* counters;          // per tile, zero on entry, left zero on exit
   float* partials;        // [kMaxCtas][2][ncap][nmat][128]
   int ncap;
-  int pf_dist;            // > 0: prefetch each segment's weight rows into L2
+  int l2_hints;           // bit 0: weight boxes evict-first; bit 1: activation boxes evict-last
   long long wait_ns;
   int* status;
 };
@@ -90,6 +92,7 @@ struct Cfg {
   // epilogue: with two 128-row blocks each group of four warps owns one block and all
   // columns; with one block the two groups split the columns
   static constexpr int kCols = kRB == 2 ? NMAX : NMAX / 2;
+  static constexpr int kGroups = kCols / 8;            // 8-column TMEM loads per matrix
   static constexpr int kAccCols = kNumA * kRB * NMAX;  // per TMEM buffer
   static constexpr int kColSFA0 = NBUF * kAccCols;
   static constexpr int kColSFA1 = kColSFA0 + 4 * kRB;
@@ -100,23 +103,26 @@ struct Cfg {
   // shared memory after the stages
   static constexpr int kOffSFB = STAGES * kStage;
   static constexpr int kOffBars = kOffSFB + 512;
-  static constexpr int kNumBars = 3 * STAGES + 2 * NBUF + 1;
-  static constexpr int kOffMisc = kOffBars + 8 * kNumBars;  // tmem slot, abort, fix-up word
-  static constexpr int kOffAmax = kOffMisc + 16;
-  static constexpr int kOffTT = kOffAmax + 2 * 4 * kCols * 4;  // plan prefix, E+2 ints
-  __host__ __device__ static size_t off_sbs(int E) {
-    return (size_t)kOffTT + ((size_t)(E + 2) * 4 + 15) / 16 * 16;
-  }
-  __host__ __device__ static size_t smem_bytes(int nk, int E) {
-    return 1024 + off_sbs(E) + 2 * (size_t)nk * NMAX * 4;  // two scale buffers
+  static constexpr int kNumBars = 3 * STAGES + 3 * NBUF + 3;
+  static constexpr int kOffMisc = (kOffBars + 8 * kNumBars + 15) / 16 * 16;  // tmem slot, abort, fix-up word
+  static constexpr int kOffAmax = kOffMisc + 16;               // [2 groups][4 warps][kCols] column maxima
+  static constexpr int kOffInv = kOffAmax + 2 * 4 * kCols * 4;  // [2 groups][kCols] 1/s
+  static constexpr int kOffSx = kOffInv + 2 * kCols * 4;        // [NBUF][NMAX] activation scales
+  static constexpr int kOffTT = kOffSx + NBUF * NMAX * 4;       // plan prefix, E+2 ints
+  __host__ __device__ static size_t smem_bytes(int E) {
+    return 1024 + (size_t)kOffTT + (size_t)(E + 2) * 4;
   }
 };
 
 __device__ __forceinline__ void bar_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
-__device__ __forceinline__ void prefetch_line_l2(const void* p) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(p) : "memory");
+// Ties the values of a tcgen05.ld to this point, so that no use of them is scheduled
+// before the tcgen05.wait::ld that precedes it.
+template <int N>
+__device__ __forceinline__ void reg_fence(float (&v)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+f"(v[i]));
 }
 // Bounded wait by one thread; false if the limit ran out or another role aborted.
 __device__ bool wait_one(uint32_t bar, uint32_t parity, long long limit, volatile int* abort_flag,
@@ -167,7 +173,7 @@ __device__ __forceinline__ void decode_tile(const int32_t* ttbase, const int32_t
   n = __ldg(tiles + 2 * tt + 1);
 }
 
-// Stream-K partition of W chunks over G CTAs.
+// Even partition of W chunks over G CTAs: CTA b takes [bW/G, (b+1)W/G).
 struct Split {
   unsigned long long W;
   int G;
@@ -176,6 +182,50 @@ struct Split {
   }
   __device__ __forceinline__ int owner(unsigned long long c) const {  // CTA holding chunk c
     return (int)(((c + 1) * (unsigned long long)G - 1) / W);
+  }
+};
+
+// Work split of T tiles over G CTAs.  The first Q*G tiles (Q = T / G) go out whole, round
+// j giving tile b + j*G to CTA b: the G CTAs always work on G consecutive tiles, so the
+// weight blocks of one expert, which read the same activation chunks, run side by side and
+// share them through L2.  The last T - Q*G tiles (the tail) form one sequence of chunks
+// split evenly over the G CTAs (stream-K); a tail tile cut between CTAs is finished by
+// the last of them to complete its segment.
+struct Sched {
+  int Q, G, b, nk, base;          // base = Q*G, the first tail tile
+  Split tail;                     // over the tail's chunks
+  unsigned long long tbeg, tend;  // this CTA's tail chunks
+  __device__ Sched(int total_tiles, int nk_, int G_, int b_) {
+    G = G_;
+    b = b_;
+    nk = nk_;
+    Q = total_tiles / G;
+    base = Q * G;
+    tail = Split{(unsigned long long)(total_tiles - base) * (unsigned long long)nk, G};
+    tbeg = tail.begin(b);
+    tend = tail.begin(b + 1);
+  }
+};
+// Walks one CTA's segments in order: (tile, first chunk, end chunk) of each.
+struct Cursor {
+  int j;
+  unsigned long long c;
+  __device__ bool next(const Sched& s, int& tile, int& k0, int& k1) {
+    if (j < s.Q) {
+      tile = s.b + j * s.G;
+      k0 = 0;
+      k1 = s.nk;
+      ++j;
+      return true;
+    }
+    if (c < s.tend) {
+      tile = s.base + (int)(c / s.nk);
+      k0 = (int)(c % s.nk);
+      k1 = (int)min((unsigned long long)s.nk, (unsigned long long)k0 + (s.tend - c));
+      c += (unsigned long long)(k1 - k0);
+      return true;
+    }
+    return false;
   }
 };
 
@@ -192,16 +242,20 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
   const uint32_t bars = ptx::smem_u32(smem + C::kOffBars);
   auto full = [&](int s) { return bars + 8u * s; };
   auto empty = [&](int s) { return bars + 8u * (STAGES + s); };
-  auto tfull = [&](int b) { return bars + 8u * (2 * STAGES + b); };
-  auto tempty = [&](int b) { return bars + 8u * (2 * STAGES + NBUF + b); };
-  const uint32_t drain = bars + 8u * (2 * STAGES + 2 * NBUF);
-  auto sf_full = [&](int s) { return bars + 8u * (2 * STAGES + 2 * NBUF + 1 + s); };
+  auto sf_full = [&](int s) { return bars + 8u * (2 * STAGES + s); };
+  auto tfull = [&](int b) { return bars + 8u * (3 * STAGES + b); };
+  auto tempty = [&](int b) { return bars + 8u * (3 * STAGES + NBUF + b); };
+  auto sx_full = [&](int b) { return bars + 8u * (3 * STAGES + 2 * NBUF + b); };
+  // one drain barrier per MMA issuer; setup: the B scale copy has landed
+  auto drain = [&](int m) { return bars + 8u * (3 * STAGES + 3 * NBUF + m); };
+  const uint32_t setup = bars + 8u * (3 * STAGES + 3 * NBUF + 2);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   volatile int* fix_word = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);
   float* amax_s = reinterpret_cast<float*>(smem + C::kOffAmax);
+  float* inv_s = reinterpret_cast<float*>(smem + C::kOffInv);
+  float* sxb = reinterpret_cast<float*>(smem + C::kOffSx);
   int32_t* s_ttbase = reinterpret_cast<int32_t*>(smem + C::kOffTT);
-  float* sbs = reinterpret_cast<float*>(smem + C::off_sbs(p.E));
 
   const int nk = p.K / 128;
   const int HB = p.rows_per_expert / MR;
@@ -213,13 +267,16 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
     for (int s = 0; s < STAGES; ++s) {
       ptx::mbar_init(full(s), 1);      // TMA arrive.expect_tx (+ transaction bytes)
       ptx::mbar_init(sf_full(s), 32);  // the 32 scale-loader lanes' cp.async arrivals
-      ptx::mbar_init(empty(s), 1);  // tcgen05.commit
+      ptx::mbar_init(empty(s), C::kNumA);  // tcgen05.commit of each MMA issuer
     }
     for (int b = 0; b < NBUF; ++b) {
-      ptx::mbar_init(tfull(b), 1);
+      ptx::mbar_init(tfull(b), C::kNumA);
       ptx::mbar_init(tempty(b), kEpiWarps);
+      ptx::mbar_init(sx_full(b), 32);
     }
-    ptx::mbar_init(drain, 1);
+    ptx::mbar_init(drain(0), 1);
+    ptx::mbar_init(drain(1), 1);
+    ptx::mbar_init(setup, 1);
     *abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -234,9 +291,12 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (warp == 1 && lane == 0) {  // B scale factors into TMEM once; both issuers read them
+    ptx::tc_cp_32x128b_x4(tmem + C::kColSFB, ptx::make_sdesc(ptx::smem_u32(sfb), 0, 128, 0));
+    ptx::tc_commit(setup);
+  }
   const int total_tiles = g_ttbase[p.E + 1] * HB;
-  const Split sp{(unsigned long long)total_tiles * (unsigned long long)nk, (int)gridDim.x};
-  const unsigned long long beg = sp.begin(blockIdx.x), end = sp.begin(blockIdx.x + 1);
+  const Sched sch(total_tiles, nk, (int)gridDim.x, (int)blockIdx.x);
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -245,12 +305,15 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
       if (PHASE == 1) ptx::prefetch_tmap(&p.tmA1);
       ptx::prefetch_tmap(&p.tmB);
     }
+    // Weights are read once per layer and activations once per weight block: the weight
+    // stream should not push the activation rows out of L2 between their reuses.
+    const uint64_t pol_a = (p.l2_hints & 1) ? ptx::make_policy_evict_first() : ptx::make_policy_evict_normal();
+    const uint64_t pol_b = (p.l2_hints & 2) ? ptx::make_policy_evict_last() : ptx::make_policy_evict_normal();
     int it = 0;
     bool ok = true;
-    for (unsigned long long c = beg; c < end && ok;) {
-      const int ti = (int)(c / nk);
-      const int k0 = (int)(c % nk);
-      const int k1 = (int)min((unsigned long long)nk, (unsigned long long)k0 + (end - c));
+    Cursor cur{0, sch.tbeg};
+    int ti, k0, k1;
+    while (ok && cur.next(sch, ti, k0, k1)) {
       int e, blk, row0, n;
       decode_tile(g_ttbase, g_tiles, p.E, HB, ti, e, blk, row0, n);
       const int rowA = e * p.rows_per_expert + blk * MR;
@@ -266,51 +329,37 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
         const uint32_t st_u = ptx::smem_u32(smem + s * C::kStage);
         if (lane == 0) {
           ptx::mbar_arrive_expect_tx(full(s), tx);
-          ptx::tma_load_2d(st_u, &p.tmA0, kc * 128, rowA, full(s));
-          if (PHASE == 1) ptx::tma_load_2d(st_u + C::kATile, &p.tmA1, kc * 128, rowA, full(s));
+          ptx::tma_load_2d_hint(st_u, &p.tmA0, kc * 128, rowA, full(s), pol_a);
+          if (PHASE == 1)
+            ptx::tma_load_2d_hint(st_u + C::kATile, &p.tmA1, kc * 128, rowA, full(s), pol_a);
           for (int j = 0; j < nB; ++j)
-            ptx::tma_load_2d(st_u + C::kNumA * C::kATile + j * 2048, &p.tmB, kc * 128,
-                             row0 + 16 * j, full(s));
+            ptx::tma_load_2d_hint(st_u + C::kNumA * C::kATile + j * 2048, &p.tmB, kc * 128,
+                                  row0 + 16 * j, full(s), pol_b);
         }
         ++it;
       }
-      c += (unsigned long long)(k1 - k0);
     }
     __syncwarp();
     if (lane == 0 && !ok)  // let every issued TMA copy land before the CTA can exit
       for (int j = it - STAGES < 0 ? 0 : it - STAGES; j < it; ++j)
         drain_wait(full(j % STAGES), (uint32_t)(j / STAGES) & 1u);
   } else if (warp == kSfWarp) {
-    // ------------------------------------------------------------ weight-scale loader
-    // 4 bytes (4 K-blocks of 32) per weight row and chunk, gathered with cp.async into
-    // the tcgen05.cp 32x128b.warpx4 layout (row m at byte (m%32)*16 + (m/32)*4).  Each
-    // lane's copies arrive on the stage's full barrier by themselves when they land
+    // ------------------------------------------------------------ scale loader
+    // Per chunk: (1) the weights' ue8m0 bytes, 4 (4 K-blocks of 32) per weight row,
+    // gathered with cp.async into the stage in the tcgen05.cp 32x128b.warpx4 layout (row m
+    // at byte (m%32)*16 + (m/32)*4); (2) the tokens' fp32 activation scales of the chunk's
+    // 128-block, into the ring slot of the chunk's TMEM buffer, for the epilogue.  Each
+    // lane's copies arrive on the barrier by themselves when they land
     // (cp.async.mbarrier.arrive.noinc), so this warp never waits for its own loads.
     const size_t ldsf = (size_t)(p.K / 32);
-    int it = 0;
+    int it = 0, ch = 0;
     bool ok = true;
-    for (unsigned long long c = beg; c < end && ok;) {
-      const int ti = (int)(c / nk);
-      const int k0 = (int)(c % nk);
-      const int k1 = (int)min((unsigned long long)nk, (unsigned long long)k0 + (end - c));
+    Cursor cur{0, sch.tbeg};
+    int ti, k0, k1;
+    while (ok && cur.next(sch, ti, k0, k1)) {
       int e, blk, row0, n;
       decode_tile(g_ttbase, g_tiles, p.E, HB, ti, e, blk, row0, n);
       const int rowA = e * p.rows_per_expert + blk * MR;
-      if (p.pf_dist > 0) {
-        // Pull this segment's weight bytes into L2 row by row ahead of the TMA loads:
-        // each row's K range is contiguous, so DRAM reads whole runs of a page instead of
-        // the 64-byte pieces the TMA boxes ask for one chunk at a time.
-        const size_t rb = (size_t)(p.K / 2);
-        const size_t lo = (size_t)k0 * 64, hi = (size_t)k1 * 64;
-        for (int r = lane; r < MR; r += 32) {
-          const uint8_t* g = p.a0_codes + (size_t)(rowA + r) * rb;
-          const uint8_t* u = p.a1_codes + (size_t)(rowA + r) * rb;
-          for (size_t o = lo & ~(size_t)127; o < hi; o += 128) {
-            prefetch_line_l2(g + o);
-            if (PHASE == 1) prefetch_line_l2(u + o);
-          }
-        }
-      }
       for (int kc = k0; kc < k1; ++kc) {
         const int s = it % STAGES;
         const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
@@ -331,21 +380,39 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
         }
         ptx::cp_async_arrive_noinc(sf_full(s));
         ++it;
+        const int b = ch % NBUF;
+        const uint32_t tph = (uint32_t)(ch / NBUF) & 1u;
+        if (!wait_warp(tempty(b), tph ^ 1u, p.wait_ns, abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        const uint32_t dst = ptx::smem_u32(sxb + b * NMAX);
+        for (int cc = lane; cc < n; cc += 32)
+          ptx::cp_async_4(dst + 4u * cc, p.b_scales + (size_t)(row0 + cc) * nk + kc);
+        ptx::cp_async_arrive_noinc(sx_full(b));
+        ++ch;
       }
-      c += (unsigned long long)(k1 - k0);
     }
     ptx::cp_async_wait_all();  // no copy of this warp may still be in flight at exit
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || (PHASE == 1 && warp == kMma1Warp)) {
+    // ------------------------------------------------------------ MMA issuers
+    // One thread issues at most one tcgen05.mma per ~120 cycles whatever its N, so phase 1
+    // splits the issue by matrix: warp 1 the gate (m = 0), warp 11 the up (m = 1) MMAs.
+    // Both wait for the same stage and TMEM buffer and commit to both barriers, which
+    // count one arrival per issuer.
+    const int m = warp == 1 ? 0 : 1;
     if (lane == 0) {
-      ptx::tc_cp_32x128b_x4(tmem + C::kColSFB, ptx::make_sdesc(ptx::smem_u32(sfb), 0, 128, 0));
       int it = 0, ch = 0;
       bool ok = true;
-      for (unsigned long long c = beg; c < end && ok;) {
-        const int ti = (int)(c / nk);
-        const int k0 = (int)(c % nk);
-        const int k1 = (int)min((unsigned long long)nk, (unsigned long long)k0 + (end - c));
+      if (m == 1) {  // the B scale copy was issued by warp 1
+        ok = wait_one(setup, 0, p.wait_ns, abort_flag, p.status);
+        ptx::tc_fence_after();
+      }
+      const uint32_t col_sfa = m == 0 ? C::kColSFA0 : C::kColSFA1;
+      Cursor cur{0, sch.tbeg};
+      int ti, k0, k1;
+      while (ok && cur.next(sch, ti, k0, k1)) {
         int e, blk, row0, n;
         decode_tile(g_ttbase, g_tiles, p.E, HB, ti, e, blk, row0, n);
         const uint32_t N = (uint32_t)((n + 15) & ~15);
@@ -364,33 +431,23 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
           if (!wait_one(sf_full(s), ph, p.wait_ns, abort_flag, p.status)) { ok = false; break; }
           ptx::tc_fence_after();
           ptx::fence_proxy_async_smem();  // scale bytes came through cp.async (generic proxy)
-          const uint32_t a0 = ptx::smem_u32(smem + s * C::kStage);
-          const uint32_t bb = a0 + C::kNumA * C::kATile;
-          const uint32_t sf0 = bb + C::kBTile;
+          const uint32_t a0 = ptx::smem_u32(smem + s * C::kStage) + m * C::kATile;
+          const uint32_t bb = ptx::smem_u32(smem + s * C::kStage) + C::kNumA * C::kATile;
+          const uint32_t sf0 = bb + C::kBTile + m * C::kSF;
 #pragma unroll
-          for (int rb = 0; rb < C::kRB; ++rb) {
-            ptx::tc_cp_32x128b_x4(tmem + C::kColSFA0 + 4 * rb,
-                                  ptx::make_sdesc(sf0 + rb * 512, 0, 128, 0));
-            if (PHASE == 1)
-              ptx::tc_cp_32x128b_x4(tmem + C::kColSFA1 + 4 * rb,
-                                    ptx::make_sdesc(sf0 + C::kSF + rb * 512, 0, 128, 0));
-          }
+          for (int rb = 0; rb < C::kRB; ++rb)
+            ptx::tc_cp_32x128b_x4(tmem + col_sfa + 4 * rb, ptx::make_sdesc(sf0 + rb * 512, 0, 128, 0));
           const uint64_t db = ptx::make_sdesc(bb, 16, 1024, 2);
-          const uint32_t acc = tmem + (uint32_t)(b * C::kAccCols);
+          const uint32_t acc = tmem + (uint32_t)(b * C::kAccCols + m * C::kRB * NMAX);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {  // four K = 32 steps through the 128-byte rows
             // scale id kk selects byte kk of each SFA word: the scale of K-block kk
             const uint32_t idesc = idesc0 | ((uint32_t)kk << 29);
 #pragma unroll
-            for (int m = 0; m < C::kNumA; ++m) {
-#pragma unroll
-              for (int rb = 0; rb < C::kRB; ++rb) {  // rows rb*128.. start 16 KB further in
-                const uint64_t da = ptx::make_sdesc(a0 + m * C::kATile + rb * 16384, 16, 1024, 2);
-                ptx::tc_mma_mxf8f6f4(acc + (uint32_t)((m * C::kRB + rb) * NMAX), da + 2 * kk,
-                                     db + 2 * kk, idesc,
-                                     tmem + (m == 0 ? C::kColSFA0 : C::kColSFA1) + 4 * rb,
-                                     tmem + C::kColSFB, kk > 0 ? 1u : 0u);
-              }
+            for (int rb = 0; rb < C::kRB; ++rb) {  // rows rb*128.. start 16 KB further in
+              const uint64_t da = ptx::make_sdesc(a0 + rb * 16384, 16, 1024, 2);
+              ptx::tc_mma_mxf8f6f4(acc + (uint32_t)(rb * NMAX), da + 2 * kk, db + 2 * kk, idesc,
+                                   tmem + col_sfa + 4 * rb, tmem + C::kColSFB, kk > 0 ? 1u : 0u);
             }
           }
           ptx::tc_commit(empty(s));
@@ -398,10 +455,9 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
           ++it;
           ++ch;
         }
-        c += (unsigned long long)(k1 - k0);
       }
-      ptx::tc_commit(drain);  // every MMA / copy of this thread done before teardown
-      drain_wait(drain, 0);
+      ptx::tc_commit(drain(m));  // every MMA / copy of this thread done before teardown
+      drain_wait(drain(m), 0);
     }
     __syncwarp();
   } else if (warp < 2 + kEpiWarps) {
@@ -413,43 +469,15 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
     const int col0 = C::kRB == 2 ? 0 : h * C::kCols;  // first column of this warp
     const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
     const size_t slot_floats = (size_t)p.ncap * kMat * MR;
-    // A segment's activation scales go to sbs[buf][kc][column] with cp.async, one commit
-    // group per segment, issued one segment ahead: when a segment starts, its scales have
-    // been in flight for the whole previous segment.
-    auto stage_scales = [&](unsigned long long cs, int buf) {
-      if (cs < end) {
-        const int ts = (int)(cs / nk);
-        const int s0 = (int)(cs % nk);
-        const int s1 = (int)min((unsigned long long)nk, (unsigned long long)s0 + (end - cs));
-        int e2, blk2, r2, n2;
-        decode_tile(g_ttbase, g_tiles, p.E, HB, ts, e2, blk2, r2, n2);
-        float* dstb = sbs + (size_t)buf * nk * NMAX;
-        const int ns = s1 - s0;
-        for (int x = ew * 32 + lane; x < n2 * ns; x += kEpiWarps * 32) {
-          const int cc = x / ns, kc = s0 + (x - cc * ns);
-          ptx::cp_async_4(ptx::smem_u32(dstb + kc * NMAX + cc),
-                          p.b_scales + (size_t)(r2 + cc) * nk + kc);
-        }
-      }
-      ptx::cp_async_commit();
-    };
-    int ch = 0, seg = 0;
+    int ch = 0;
     bool ok = true;
-    stage_scales(beg, 0);
-    for (unsigned long long c = beg; c < end; ++seg) {
-      const int ti = (int)(c / nk);
-      const int k0 = (int)(c % nk);
-      const int k1 = (int)min((unsigned long long)nk, (unsigned long long)k0 + (end - c));
+    Cursor cur{0, sch.tbeg};
+    int ti, k0, k1;
+    while (cur.next(sch, ti, k0, k1)) {
       int e, blk, row0, n;
       decode_tile(g_ttbase, g_tiles, p.E, HB, ti, e, blk, row0, n);
-      const int nkk = k1 - k0;
-      // every warp is past the previous segment, so the other buffer is free: start the
-      // next segment's scales, then wait (normally not at all) for this segment's
-      bar_sync(1, kEpiWarps * 32);
-      stage_scales(c + (unsigned long long)nkk, (seg + 1) & 1);
-      ptx::cp_async_wait_group<1>();
-      bar_sync(1, kEpiWarps * 32);
-      const float* sbs_cur = sbs + (size_t)(seg & 1) * nk * NMAX;
+      // columns of this warp that hold tokens; the others are computed but never stored
+      const int jn = n - col0 < 0 ? 0 : (n - col0 < C::kCols ? n - col0 : C::kCols);
       float acc0[C::kCols], acc1[C::kCols];
 #pragma unroll
       for (int j = 0; j < C::kCols; ++j) {
@@ -460,22 +488,26 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
         const int b = ch % NBUF;
         const uint32_t tph = (uint32_t)(ch / NBUF) & 1u;
         ok = ok && wait_warp(tfull(b), tph, p.wait_ns, abort_flag, p.status);
+        ok = ok && wait_warp(sx_full(b), tph, p.wait_ns, abort_flag, p.status);
         ptx::tc_fence_after();
-        if (ok) {
+        if (ok && jn > 0) {
+          // acc += s * P, 8 columns of each matrix per TMEM round trip
           const uint32_t base = tl + (uint32_t)(b * C::kAccCols + rb * NMAX + col0);
-          const float* sc = sbs_cur + kc * NMAX + col0;
+          const float4* sc4 = reinterpret_cast<const float4*>(sxb + b * NMAX + col0);
 #pragma unroll
-          for (int g = 0; g < C::kCols / 8; ++g) {
-            if (col0 + 8 * g < n) {
-              float v0[8], v1[8];
-              ptx::tc_ld_32x32b_x8(base + 8 * g, v0);
-              if (PHASE == 1) ptx::tc_ld_32x32b_x8(base + C::kRB * NMAX + 8 * g, v1);
-              ptx::tc_wait_ld();
+          for (int g = 0; g < C::kGroups; ++g) {
+            float v0[8], v1[8];
+            ptx::tc_ld_32x32b_x8(base + 8 * g, v0);
+            if (PHASE == 1) ptx::tc_ld_32x32b_x8(base + C::kRB * NMAX + 8 * g, v1);
+            const float4 sa = sc4[2 * g], sb = sc4[2 * g + 1];
+            ptx::tc_wait_ld();
+            reg_fence(v0);
+            if (PHASE == 1) reg_fence(v1);
+            const float sv[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
 #pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                acc0[8 * g + j] = fmaf(sc[8 * g + j], v0[j], acc0[8 * g + j]);
-                if (PHASE == 1) acc1[8 * g + j] = fmaf(sc[8 * g + j], v1[j], acc1[8 * g + j]);
-              }
+            for (int j = 0; j < 8; ++j) {
+              acc0[8 * g + j] = fmaf(sv[j], v0[j], acc0[8 * g + j]);
+              if (PHASE == 1) acc1[8 * g + j] = fmaf(sv[j], v1[j], acc1[8 * g + j]);
             }
           }
         }
@@ -484,27 +516,30 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
         if (lane == 0) ptx::mbar_arrive(tempty(b));
         ++ch;
       }
-      c += (unsigned long long)nkk;
 
-      // ---- stream-K fix-up of a tile cut between CTAs.  The tile's segments belong to
-      // the CTAs owning its chunks (CTAs with empty ranges own none): walk them in order.
-      const unsigned long long t0c = (unsigned long long)ti * nk;
+      // ---- stream-K fix-up of a tail tile cut between CTAs.  The tile's segments belong
+      // to the CTAs owning its chunks (CTAs with empty ranges own none): walk them in order.
+      const Split& sp = sch.tail;
+      const int tt = ti - sch.base;  // index among the tail tiles (< 0: a whole tile)
+      const unsigned long long t0c = (unsigned long long)(tt < 0 ? 0 : tt) * nk;
       int nseg = 0;
-      for (unsigned long long cc = t0c; cc < t0c + nk;) {
-        ++nseg;
-        cc = sp.begin(sp.owner(cc) + 1);
-      }
+      if (tt >= 0)
+        for (unsigned long long cc = t0c; cc < t0c + nk;) {
+          ++nseg;
+          cc = sp.begin(sp.owner(cc) + 1);
+        }
       bool finish = true;
+      const size_t lane_off = (size_t)rb * 128 + q * 32 + lane;
       if (nseg > 1) {
-        const int my_slot = 2 * blockIdx.x + ((int)(beg / nk) == ti ? 0 : 1);
+        const int my_slot = 2 * blockIdx.x + ((int)(sch.tbeg / nk) == tt ? 0 : 1);
         float* mine = p.partials + (size_t)my_slot * slot_floats;
         if (ok) {
 #pragma unroll
           for (int j = 0; j < C::kCols; ++j) {
-            const int cc = col0 + j;
-            if (cc < n) {
-              mine[((size_t)cc * kMat + 0) * MR + rb * 128 + q * 32 + lane] = acc0[j];
-              if (PHASE == 1) mine[((size_t)cc * kMat + 1) * MR + rb * 128 + q * 32 + lane] = acc1[j];
+            if (j < jn) {
+              const size_t o = (size_t)(col0 + j) * kMat * MR + lane_off;
+              mine[o] = acc0[j];
+              if (PHASE == 1) mine[o + MR] = acc1[j];
             }
           }
         }
@@ -523,16 +558,16 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
           for (unsigned long long cs = t0c; cs < t0c + nk;) {
             const int s = sp.owner(cs);
             cs = sp.begin(s + 1);
-            const int slot = 2 * s + ((int)(sp.begin(s) / nk) == ti ? 0 : 1);
+            const int slot = 2 * s + ((int)(sp.begin(s) / nk) == tt ? 0 : 1);
             const float* src = p.partials + (size_t)slot * slot_floats;
 #pragma unroll
             for (int j = 0; j < C::kCols; ++j) {
-              const int cc = col0 + j;
-              if (cc < n) {
-                const float v0 = __ldcg(src + ((size_t)cc * kMat + 0) * MR + rb * 128 + q * 32 + lane);
+              if (j < jn) {
+                const size_t o = (size_t)(col0 + j) * kMat * MR + lane_off;
+                const float v0 = __ldcg(src + o);
                 acc0[j] = first_seg ? v0 : acc0[j] + v0;
                 if (PHASE == 1) {
-                  const float v1 = __ldcg(src + ((size_t)cc * kMat + 1) * MR + rb * 128 + q * 32 + lane);
+                  const float v1 = __ldcg(src + o + MR);
                   acc1[j] = first_seg ? v1 : acc1[j] + v1;
                 }
               }
@@ -543,48 +578,59 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
         }
       }
       finish = finish && ok;
+      const int js = finish ? jn : 0;   // columns this warp stores
+      const int hb = blk * C::kRB + rb;  // 128-wide block of h (phase 1) / of y (phase 2)
 
       if (PHASE == 1) {
-        // h = silu(g) * u, then per-column (token) e4m3 re-quantisation over the 128 rows
-        float* hv = acc0;  // h overwrites g in place
-        float* am = amax_s + (h * 4 + q) * C::kCols;
+        // h = silu(g) * u in place of g, then per-column (token) e4m3 re-quantisation over
+        // the 128 rows: column maxima per warp, combined by one thread per column, which
+        // writes s and 1/s; every thread then encodes its 128-row slice of each column.
 #pragma unroll
         for (int j = 0; j < C::kCols; ++j) {
           const float g = acc0[j];
-          hv[j] = g / (1.0f + expf(-g)) * acc1[j];
-          const unsigned m = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(hv[j])));
+          acc0[j] = __fdividef(g, 1.0f + expf(-g)) * acc1[j];
+        }
+        float* am = amax_s + (h * 4 + q) * C::kCols;
+#pragma unroll
+        for (int j = 0; j < C::kCols; ++j) {
+          const unsigned m = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(acc0[j])));
           if (lane == 0) am[j] = __uint_as_float(m);
         }
         bar_sync(2 + h, 128);
-#pragma unroll
-        for (int j = 0; j < C::kCols; ++j) {
-          if (finish && col0 + j < n) {
-            float amax = amax_s[(h * 4 + 0) * C::kCols + j];
-            amax = fmaxf(amax, amax_s[(h * 4 + 1) * C::kCols + j]);
-            amax = fmaxf(amax, amax_s[(h * 4 + 2) * C::kCols + j]);
-            amax = fmaxf(amax, amax_s[(h * 4 + 3) * C::kCols + j]);
-            const float s = amax == 0.f ? 1.0f : __fdiv_rn(amax, 448.0f);
-            const int row = row0 + col0 + j;
-            const uint16_t code = ptx::cvt_e4m3x2(__fdiv_rn(hv[j], s), 0.f);
-            const int hb = blk * C::kRB + rb;  // 128-wide block of h
-            p.qh[(size_t)row * p.f + hb * 128 + q * 32 + lane] = (uint8_t)(code & 0xFF);
-            if (q == 0 && lane == 0) p.sh[(size_t)row * (p.f / 128) + hb] = s;
-          }
+        const int t = q * 32 + lane;
+        if (t < C::kCols) {
+          const float* a = amax_s + h * 4 * C::kCols + t;
+          const float amax =
+              fmaxf(fmaxf(a[0], a[C::kCols]), fmaxf(a[2 * C::kCols], a[3 * C::kCols]));
+          const float s = amax == 0.f ? 1.0f : __fdiv_rn(amax, 448.0f);
+          inv_s[h * C::kCols + t] = __frcp_rn(s);
+          if (t < js) p.sh[(size_t)(row0 + col0 + t) * (p.f / 128) + hb] = s;
         }
         bar_sync(2 + h, 128);
+        const float4* inv4 = reinterpret_cast<const float4*>(inv_s + h * C::kCols);
+        uint8_t* dst = p.qh + (size_t)(row0 + col0) * p.f + hb * 128 + q * 32 + lane;
+#pragma unroll
+        for (int j = 0; j < C::kCols; j += 4) {
+          const float4 r = inv4[j / 4];
+          const uint16_t c01 = ptx::cvt_e4m3x2(acc0[j] * r.x, acc0[j + 1] * r.y);
+          const uint16_t c23 = ptx::cvt_e4m3x2(acc0[j + 2] * r.z, acc0[j + 3] * r.w);
+          if (j < js) dst[(size_t)j * p.f] = (uint8_t)(c01 & 0xFF);
+          if (j + 1 < js) dst[(size_t)(j + 1) * p.f] = (uint8_t)(c01 >> 8);
+          if (j + 2 < js) dst[(size_t)(j + 2) * p.f] = (uint8_t)(c23 & 0xFF);
+          if (j + 3 < js) dst[(size_t)(j + 3) * p.f] = (uint8_t)(c23 >> 8);
+        }
       } else {
 #pragma unroll
         for (int j = 0; j < C::kCols; ++j) {
-          if (finish && col0 + j < n) {
+          if (j < js) {
             const int row = row0 + col0 + j;
             float* dst = row < p.P ? p.y_routed + (size_t)row * p.d
                                    : p.y_shared + (size_t)(row - p.P) * p.d;
-            dst[(blk * C::kRB + rb) * 128 + q * 32 + lane] = acc0[j];
+            dst[(size_t)hb * 128 + q * 32 + lane] = acc0[j];
           }
         }
       }
     }
-    ptx::cp_async_wait_all();  // no scale copy may still be in flight at exit
   }
 
   ptx::tc_fence_before();
@@ -632,9 +678,9 @@ bool make_map(CUtensorMap* m, const void* base, bool fp4, int K, long long rows,
 }
 
 template <int PHASE, int NMAX, int STAGES, int NBUF, int MR>
-cudaError_t launch_one(const FfnParams& prm, int nk, cudaStream_t s, int grid) {
+cudaError_t launch_one(const FfnParams& prm, cudaStream_t s, int grid) {
   using C = Cfg<PHASE, NMAX, STAGES, NBUF, MR>;
-  const size_t smem = C::smem_bytes(nk, prm.E);
+  const size_t smem = C::smem_bytes(prm.E);
   cudaError_t err = cudaFuncSetAttribute(ffn_kernel<PHASE, NMAX, STAGES, NBUF, MR>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
@@ -659,10 +705,10 @@ int tile_rows(int nmax, int rows_per_expert) {
 
 }  // namespace
 
-size_t ffn_smem_bytes(int phase, int nmax, int nk, int E, int rows_per_expert) {
+size_t ffn_smem_bytes(int phase, int nmax, int E, int rows_per_expert) {
   const int mr = tile_rows(nmax, rows_per_expert);
 #define X(P, N, S, B, M) \
-  if (phase == P && nmax == N && mr == M) return Cfg<P, N, S, B, M>::smem_bytes(nk, E);
+  if (phase == P && nmax == N && mr == M) return Cfg<P, N, S, B, M>::smem_bytes(E);
   BITMOE_FFN_VARIANTS(X)
 #undef X
   return 0;
@@ -677,8 +723,6 @@ cudaError_t launch_ffn(int phase, int nmax, const FfnArgs& a, cudaStream_t s, in
   if (phase == 1 && !make_map(&prm.tmA1, a.a1_codes, true, a.K, rows_total, mr))
     return cudaErrorInvalidValue;
   if (!make_map(&prm.tmB, a.b_codes, false, a.K, a.R, 16)) return cudaErrorInvalidValue;
-  prm.a0_codes = a.a0_codes;
-  prm.a1_codes = a.a1_codes;
   prm.sfa0 = a.a0_scales;
   prm.sfa1 = a.a1_scales;
   prm.b_scales = a.b_scales;
@@ -699,11 +743,10 @@ cudaError_t launch_ffn(int phase, int nmax, const FfnArgs& a, cudaStream_t s, in
   prm.counters = a.counters;
   prm.partials = a.partials;
   prm.ncap = a.ncap;
-  prm.pf_dist = a.pf_dist;
-  const int nk = a.K / 128;
+  prm.l2_hints = a.l2_hints;
   const int grid = num_sms < kMaxCtas ? num_sms : kMaxCtas;
 #define X(P, N, S, B, M) \
-  if (phase == P && nmax == N && mr == M) return launch_one<P, N, S, B, M>(prm, nk, s, grid);
+  if (phase == P && nmax == N && mr == M) return launch_one<P, N, S, B, M>(prm, s, grid);
   BITMOE_FFN_VARIANTS(X)
 #undef X
   return cudaErrorInvalidValue;

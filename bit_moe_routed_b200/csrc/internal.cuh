@@ -71,11 +71,11 @@ struct FfnArgs {
   int* counters;             // stream-K fix-up counters (zeroed by the prepare kernel)
   float* partials;           // stream-K partial slots
   int ncap;                  // widest token tile
-  int pf_dist;               // > 0: prefetch each segment's weight rows into L2
+  int l2_hints;              // bit 0: weight boxes evict-first; bit 1: activation boxes evict-last
 };
 cudaError_t launch_ffn(int phase, int nmax, const FfnArgs& a, cudaStream_t s, int num_sms);
 // dynamic shared memory of a launch
-size_t ffn_smem_bytes(int phase, int nmax, int nk, int E, int rows_per_expert);
+size_t ffn_smem_bytes(int phase, int nmax, int E, int rows_per_expert);
 
 // Defined in abi.cu: sets the thread-local message that moe_last_error returns.
 int record_error(int code, const char* msg);
