@@ -234,7 +234,7 @@ def run_gpu(args, w):
     est_active = min(E, T * k) + 1
     step_bytes = est_active * per_expert
     L2_BYTES = 126 * 2 ** 20
-    n_layers = max(2, min(args.max_layers, -(-4 * L2_BYTES // step_bytes) + 1))
+    n_layers = max(min(2, args.max_layers), min(args.max_layers, -(-4 * L2_BYTES // step_bytes) + 1))
     layers = []
     for l in range(n_layers):
         seed = replica_seed(w, rank) + l

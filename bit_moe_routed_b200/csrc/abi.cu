@@ -115,8 +115,11 @@ WorkspaceLayout workspace_layout(int T, int k, int E, int d, int f) {
   const size_t hb = (size_t)((d > f ? d : f) / 128);
   L.n_counters = plan_ntmax((int)R, E) * hb;
   o = align256(o + 4 * L.n_counters);
+  // stream-K partial slots: two per CTA, each [ncap columns][2 matrices][tile rows] fp32;
+  // small batches take tiles of up to 256 weight rows, large ones 128
   L.partials = o;
-  o = align256(o + (size_t)kMaxCtas * 2 * (size_t)ncap_for(T) * 2 * 128 * 4);
+  const size_t tile_rows_max = nmax_for(T) == kNmaxSmall ? 256 : 128;
+  o = align256(o + (size_t)kMaxCtas * 2 * (size_t)ncap_for(T) * 2 * tile_rows_max * 4);
   L.total = o;
   return L;
 }
@@ -252,6 +255,9 @@ int ffn_check(int T, int k, const moe_weights_t* w, void* ws, size_t ws_bytes, F
   return MOE_OK;
 }
 
+// Set while moe_expert_ffn issues its second and third kernels (see launch_pdl).
+thread_local bool t_overlap = false;
+
 FfnArgs ffn_args(int phase, int T, int k, const moe_weights_t* w, const FfnCtx& c) {
   FfnArgs a{};
   const int P = T * k;
@@ -267,6 +273,7 @@ FfnArgs ffn_args(int phase, int T, int k, const moe_weights_t* w, const FfnCtx& 
   a.partials = reinterpret_cast<float*>(c.ws + c.L.partials);
   a.ncap = ncap_for(T);
   a.l2_hints = 1;  // weight boxes evict-first
+  a.overlap = t_overlap;
   if (phase == 1) {
     a.a0_codes = w->gate_codes;
     a.a0_scales = w->gate_scales;
@@ -340,6 +347,12 @@ int moe_expert_ffn(const uint16_t* x_bf16, int T, int k, const moe_weights_t* w,
                    void* ws, size_t ws_bytes, void* stream) {
   int rc = moe_ffn_prepare(x_bf16, T, k, w, offsets, perm, ws, ws_bytes, stream);
   if (rc) return rc;
+  // gate/up and down follow a kernel of this call on the stream: they may start while it
+  // finishes (their prologue overlaps its tail)
+  struct Overlap {
+    Overlap() { t_overlap = true; }
+    ~Overlap() { t_overlap = false; }
+  } guard;
   rc = moe_ffn_gate_up(T, k, w, ws, ws_bytes, stream);
   if (rc) return rc;
   return moe_ffn_down(T, k, w, y_routed, y_shared, ws, ws_bytes, stream);

@@ -10,6 +10,7 @@
 //           among equal experts in its 32-pair group.
 // No atomics decide a position, so the permutation is deterministic.
 #include "internal.cuh"
+#include "ptx.cuh"
 
 namespace bitmoe {
 namespace {
@@ -22,6 +23,8 @@ __global__ void __launch_bounds__(1024, 1) dispatch_kernel(const int32_t* __rest
                                                            int32_t* __restrict__ perm,
                                                            int32_t* __restrict__ pos,
                                                            int* __restrict__ status) {
+  ptx::griddep_launch_dependents();
+  ptx::griddep_wait();  // idx comes from earlier work on the stream
   extern __shared__ int32_t sm[];
   int32_t* cnt = sm;                     // [kWarps][E]
   int32_t* off = sm + kWarps * E;        // [E+1]
@@ -122,8 +125,8 @@ cudaError_t launch_dispatch(const int32_t* idx, int T, int k, int E, int32_t* co
   cudaError_t err = cudaFuncSetAttribute(dispatch_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  dispatch_kernel<<<1, 1024, smem, s>>>(idx, T * k, E, counts, offsets, perm, pos, status);
-  return cudaGetLastError();
+  return launch_pdl(dispatch_kernel, dim3(1), dim3(1024), smem, s, false, idx, T * k, E, counts, offsets,
+                    perm, pos, status);
 }
 
 }  // namespace bitmoe

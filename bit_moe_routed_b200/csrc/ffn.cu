@@ -55,8 +55,11 @@ namespace {
 
 constexpr int kEpiWarps = 8;
 constexpr int kSfWarp = 2 + kEpiWarps;          // warp 10 loads the scales
-constexpr int kMma1Warp = kSfWarp + 1;          // warp 11 issues the up MMAs (phase 1)
-constexpr int kThreads = 32 * (kMma1Warp + 1);
+constexpr int kIssuerWarp1 = kSfWarp + 1;       // warps 11.. issue MMAs beside warp 1
+// One issuing thread per (matrix, 128-row block) of a tile: a thread issues at most one
+// tcgen05.mma per ~120 cycles whatever its N, so small-N tiles need several issuers.
+constexpr int ffn_issuers(int phase, int mr) { return (phase == 1 ? 2 : 1) * (mr / 128); }
+constexpr int ffn_threads(int phase, int mr) { return 32 * (kIssuerWarp1 + ffn_issuers(phase, mr) - 1); }
 constexpr long long kDrainNs = 500000000LL;     // bound on draining in-flight work
 
 struct FfnParams {
@@ -84,6 +87,8 @@ template <int PHASE, int NMAX, int STAGES, int NBUF, int MR>
 struct Cfg {
   static constexpr int kNumA = PHASE == 1 ? 2 : 1;
   static constexpr int kRB = MR / 128;       // 128-row MMA blocks per weight tile
+  static constexpr int kIssuers = ffn_issuers(PHASE, MR);
+  static constexpr int kThreads = ffn_threads(PHASE, MR);
   static constexpr int kATile = MR * 128;    // MR rows x 128 FP4 in byte containers
   static constexpr int kBTile = NMAX * 128;
   static constexpr int kSF = 512 * kRB;      // per matrix: one 512-byte scale block per 128 rows
@@ -103,7 +108,7 @@ struct Cfg {
   // shared memory after the stages
   static constexpr int kOffSFB = STAGES * kStage;
   static constexpr int kOffBars = kOffSFB + 512;
-  static constexpr int kNumBars = 3 * STAGES + 3 * NBUF + 3;
+  static constexpr int kNumBars = 3 * STAGES + 3 * NBUF + kIssuers + 1;
   static constexpr int kOffMisc = (kOffBars + 8 * kNumBars + 15) / 16 * 16;  // tmem slot, abort, fix-up word
   static constexpr int kOffAmax = kOffMisc + 16;               // [2 groups][4 warps][kCols] column maxima
   static constexpr int kOffInv = kOffAmax + 2 * 4 * kCols * 4;  // [2 groups][kCols] 1/s
@@ -117,6 +122,12 @@ struct Cfg {
 __device__ __forceinline__ void bar_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
+// atomic add at GPU scope with acquire-release ordering
+__device__ __forceinline__ int atom_add_acq_rel(int* ptr, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(ptr), "r"(v) : "memory");
+  return old;
+}
 // Ties the values of a tcgen05.ld to this point, so that no use of them is scheduled
 // before the tcgen05.wait::ld that precedes it.
 template <int N>
@@ -124,21 +135,26 @@ __device__ __forceinline__ void reg_fence(float (&v)[N]) {
 #pragma unroll
   for (int i = 0; i < N; ++i) asm volatile("" : "+f"(v[i]));
 }
-// Bounded wait by one thread; false if the limit ran out or another role aborted.
+// Bounded wait by one thread; false if the limit ran out or another role aborted.  The
+// loop is try_wait alone (which itself parks the thread for a short, hardware-chosen
+// time); the abort flag and the clock are read only every 64 tries, so waiting threads
+// add little shared-memory traffic.  (Limits under 100 us are checked on every try.)
 __device__ bool wait_one(uint32_t bar, uint32_t parity, long long limit, volatile int* abort_flag,
                          int* status) {
-  if (*abort_flag) return false;
   if (ptx::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = ptx::globaltimer();
-  while (!*abort_flag) {
+  const uint32_t every = limit < 100000 ? 0u : 63u;
+  for (uint32_t i = 1;; ++i) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
-    if ((long long)(ptx::globaltimer() - t0) > limit) {
-      *abort_flag = 1;
-      atomicOr(status, kStatusTimeout);
-      return false;
+    if ((i & every) == 0) {
+      if (*abort_flag) return false;
+      if ((long long)(ptx::globaltimer() - t0) > limit) {
+        *abort_flag = 1;
+        atomicOr(status, kStatusTimeout);
+        return false;
+      }
     }
   }
-  return false;
 }
 // Same, decided by lane 0 and shared with the whole warp (keeps the warp converged).
 __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, long long limit,
@@ -230,7 +246,7 @@ struct Cursor {
 };
 
 template <int PHASE, int NMAX, int STAGES, int NBUF, int MR>
-__global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant__ FfnParams p) {
+__global__ void __launch_bounds__(ffn_threads(PHASE, MR), 1) ffn_kernel(const __grid_constant__ FfnParams p) {
   using C = Cfg<PHASE, NMAX, STAGES, NBUF, MR>;
   constexpr int kMat = PHASE == 1 ? 2 : 1;
   extern __shared__ uint8_t smem_raw[];
@@ -247,8 +263,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
   auto tempty = [&](int b) { return bars + 8u * (3 * STAGES + NBUF + b); };
   auto sx_full = [&](int b) { return bars + 8u * (3 * STAGES + 2 * NBUF + b); };
   // one drain barrier per MMA issuer; setup: the B scale copy has landed
-  auto drain = [&](int m) { return bars + 8u * (3 * STAGES + 3 * NBUF + m); };
-  const uint32_t setup = bars + 8u * (3 * STAGES + 3 * NBUF + 2);
+  auto drain = [&](int i) { return bars + 8u * (3 * STAGES + 3 * NBUF + i); };
+  const uint32_t setup = bars + 8u * (3 * STAGES + 3 * NBUF + C::kIssuers);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   volatile int* fix_word = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);
@@ -260,22 +276,21 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
   const int nk = p.K / 128;
   const int HB = p.rows_per_expert / MR;
   const int32_t* g_tiles = p.plan + p.E + 2;
-  for (int e = threadIdx.x; e < p.E + 2; e += kThreads) s_ttbase[e] = __ldg(p.plan + e);
   const int32_t* g_ttbase = s_ttbase;
 
+  ptx::griddep_launch_dependents();
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       ptx::mbar_init(full(s), 1);      // TMA arrive.expect_tx (+ transaction bytes)
       ptx::mbar_init(sf_full(s), 32);  // the 32 scale-loader lanes' cp.async arrivals
-      ptx::mbar_init(empty(s), C::kNumA);  // tcgen05.commit of each MMA issuer
+      ptx::mbar_init(empty(s), C::kIssuers);  // tcgen05.commit of each MMA issuer
     }
     for (int b = 0; b < NBUF; ++b) {
-      ptx::mbar_init(tfull(b), C::kNumA);
+      ptx::mbar_init(tfull(b), C::kIssuers);
       ptx::mbar_init(tempty(b), kEpiWarps);
       ptx::mbar_init(sx_full(b), 32);
     }
-    ptx::mbar_init(drain(0), 1);
-    ptx::mbar_init(drain(1), 1);
+    for (int i = 0; i < C::kIssuers; ++i) ptx::mbar_init(drain(i), 1);
     ptx::mbar_init(setup, 1);
     *abort_flag = 0;
     ptx::fence_mbar_init();
@@ -286,6 +301,10 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
   }
   if (threadIdx.x >= 64 && threadIdx.x < 64 + 128)  // B scale factors: all 1.0 (0x7F)
     reinterpret_cast<uint32_t*>(sfb)[threadIdx.x - 64] = 0x7F7F7F7Fu;
+  // everything above overlaps the end of the previous launch on the stream; the plan,
+  // the activation rows and their scales are written by it
+  ptx::griddep_wait();
+  for (int e = threadIdx.x; e < p.E + 2; e += C::kThreads) s_ttbase[e] = __ldg(p.plan + e);
   ptx::fence_proxy_async_smem();
   ptx::tc_fence_before();
   __syncthreads();
@@ -395,21 +414,22 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
     }
     ptx::cp_async_wait_all();  // no copy of this warp may still be in flight at exit
     __syncwarp();
-  } else if (warp == 1 || (PHASE == 1 && warp == kMma1Warp)) {
+  } else if (warp == 1 || (warp >= kIssuerWarp1 && warp - kIssuerWarp1 + 1 < C::kIssuers)) {
     // ------------------------------------------------------------ MMA issuers
-    // One thread issues at most one tcgen05.mma per ~120 cycles whatever its N, so phase 1
-    // splits the issue by matrix: warp 1 the gate (m = 0), warp 11 the up (m = 1) MMAs.
-    // Both wait for the same stage and TMEM buffer and commit to both barriers, which
-    // count one arrival per issuer.
-    const int m = warp == 1 ? 0 : 1;
+    // Issuer i (warp 1 for i = 0, warp 10 + i otherwise) owns matrix m = i / kRB (gate or
+    // down 0, up 1) and 128-row block rb = i % kRB of every tile.  All wait for the same
+    // stage and TMEM buffer and commit to both barriers, which count one arrival each.
+    const int issuer = warp == 1 ? 0 : warp - kIssuerWarp1 + 1;
+    const int m = issuer / C::kRB;
+    const int rbi = issuer % C::kRB;
     if (lane == 0) {
       int it = 0, ch = 0;
       bool ok = true;
-      if (m == 1) {  // the B scale copy was issued by warp 1
+      if (issuer != 0) {  // the B scale copy was issued by warp 1
         ok = wait_one(setup, 0, p.wait_ns, abort_flag, p.status);
         ptx::tc_fence_after();
       }
-      const uint32_t col_sfa = m == 0 ? C::kColSFA0 : C::kColSFA1;
+      const uint32_t col_sfa = (m == 0 ? C::kColSFA0 : C::kColSFA1) + 4 * rbi;
       Cursor cur{0, sch.tbeg};
       int ti, k0, k1;
       while (ok && cur.next(sch, ti, k0, k1)) {
@@ -431,24 +451,19 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
           if (!wait_one(sf_full(s), ph, p.wait_ns, abort_flag, p.status)) { ok = false; break; }
           ptx::tc_fence_after();
           ptx::fence_proxy_async_smem();  // scale bytes came through cp.async (generic proxy)
-          const uint32_t a0 = ptx::smem_u32(smem + s * C::kStage) + m * C::kATile;
+          const uint32_t a0 = ptx::smem_u32(smem + s * C::kStage) + m * C::kATile + rbi * 16384;
           const uint32_t bb = ptx::smem_u32(smem + s * C::kStage) + C::kNumA * C::kATile;
-          const uint32_t sf0 = bb + C::kBTile + m * C::kSF;
-#pragma unroll
-          for (int rb = 0; rb < C::kRB; ++rb)
-            ptx::tc_cp_32x128b_x4(tmem + col_sfa + 4 * rb, ptx::make_sdesc(sf0 + rb * 512, 0, 128, 0));
+          const uint32_t sf0 = bb + C::kBTile + m * C::kSF + rbi * 512;
+          ptx::tc_cp_32x128b_x4(tmem + col_sfa, ptx::make_sdesc(sf0, 0, 128, 0));
           const uint64_t db = ptx::make_sdesc(bb, 16, 1024, 2);
-          const uint32_t acc = tmem + (uint32_t)(b * C::kAccCols + m * C::kRB * NMAX);
+          const uint64_t da = ptx::make_sdesc(a0, 16, 1024, 2);
+          const uint32_t acc = tmem + (uint32_t)(b * C::kAccCols + (m * C::kRB + rbi) * NMAX);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {  // four K = 32 steps through the 128-byte rows
             // scale id kk selects byte kk of each SFA word: the scale of K-block kk
             const uint32_t idesc = idesc0 | ((uint32_t)kk << 29);
-#pragma unroll
-            for (int rb = 0; rb < C::kRB; ++rb) {  // rows rb*128.. start 16 KB further in
-              const uint64_t da = ptx::make_sdesc(a0 + rb * 16384, 16, 1024, 2);
-              ptx::tc_mma_mxf8f6f4(acc + (uint32_t)(rb * NMAX), da + 2 * kk, db + 2 * kk, idesc,
-                                   tmem + col_sfa + 4 * rb, tmem + C::kColSFB, kk > 0 ? 1u : 0u);
-            }
+            ptx::tc_mma_mxf8f6f4(acc, da + 2 * kk, db + 2 * kk, idesc, tmem + col_sfa,
+                                 tmem + C::kColSFB, kk > 0 ? 1u : 0u);
           }
           ptx::tc_commit(empty(s));
           ptx::tc_commit(tfull(b));
@@ -456,8 +471,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
           ++ch;
         }
       }
-      ptx::tc_commit(drain(m));  // every MMA / copy of this thread done before teardown
-      drain_wait(drain(m), 0);
+      ptx::tc_commit(drain(issuer));  // every MMA / copy of this thread done before teardown
+      drain_wait(drain(issuer), 0);
     }
     __syncwarp();
   } else if (warp < 2 + kEpiWarps) {
@@ -487,15 +502,21 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
       for (int kc = k0; kc < k1; ++kc) {
         const int b = ch % NBUF;
         const uint32_t tph = (uint32_t)(ch / NBUF) & 1u;
-        ok = ok && wait_warp(tfull(b), tph, p.wait_ns, abort_flag, p.status);
-        ok = ok && wait_warp(sx_full(b), tph, p.wait_ns, abort_flag, p.status);
+        // one warp waits for the chunk's partial and scales, then releases the others
+        // through a named barrier (eight warps spinning on one mbarrier would compete
+        // with the TMA and the MMA for shared memory)
+        if (ew == 0 && ok) {
+          ok = wait_warp(tfull(b), tph, p.wait_ns, abort_flag, p.status);
+          ok = ok && wait_warp(sx_full(b), tph, p.wait_ns, abort_flag, p.status);
+        }
+        bar_sync(4, kEpiWarps * 32);
+        ok = ok && *abort_flag == 0;
         ptx::tc_fence_after();
         if (ok && jn > 0) {
           // acc += s * P, 8 columns of each matrix per TMEM round trip
           const uint32_t base = tl + (uint32_t)(b * C::kAccCols + rb * NMAX + col0);
           const float4* sc4 = reinterpret_cast<const float4*>(sxb + b * NMAX + col0);
-#pragma unroll
-          for (int g = 0; g < C::kGroups; ++g) {
+          auto group = [&](int g) {
             float v0[8], v1[8];
             ptx::tc_ld_32x32b_x8(base + 8 * g, v0);
             if (PHASE == 1) ptx::tc_ld_32x32b_x8(base + C::kRB * NMAX + 8 * g, v1);
@@ -508,6 +529,16 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
             for (int j = 0; j < 8; ++j) {
               acc0[8 * g + j] = fmaf(sv[j], v0[j], acc0[8 * g + j]);
               if (PHASE == 1) acc1[8 * g + j] = fmaf(sv[j], v1[j], acc1[8 * g + j]);
+            }
+          };
+          if (jn > C::kCols - 8) {  // every group holds tokens: straight-line code
+#pragma unroll
+            for (int g = 0; g < C::kGroups; ++g) group(g);
+          } else {  // few tokens (decode): only the groups that hold some
+#pragma unroll
+            for (int g = 0; g < C::kGroups; ++g) {
+              if (8 * g >= jn) break;
+              group(g);
             }
           }
         }
@@ -543,15 +574,50 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
             }
           }
         }
-        __threadfence();
+        // one acq_rel atomic (after the barrier) publishes every thread's partial and, for
+        // the last arrival, makes the other CTAs' partials visible to the whole CTA
         bar_sync(1, kEpiWarps * 32);
         if (ew == 0 && lane == 0)
-          *fix_word = *abort_flag ? -1 : atomicAdd(p.counters + ti, 1);
+          *fix_word = *abort_flag ? -1 : atom_add_acq_rel(p.counters + ti, 1);
         bar_sync(1, kEpiWarps * 32);
         const int arrived = *fix_word;
         finish = arrived == nseg - 1;
-        if (finish) {
-          __threadfence();
+        if (finish && jn <= 4 && nseg <= 4) {
+          // few columns (decode): every segment's loads in flight at once, then summed in
+          // chunk order
+          float v[4][4][kMat];
+          unsigned long long cs = t0c;
+#pragma unroll
+          for (int si = 0; si < 4; ++si) {
+            const bool have = si < nseg;
+            const int s = have ? sp.owner(cs) : 0;
+            const int slot = 2 * s + ((int)(sp.begin(s) / nk) == tt ? 0 : 1);
+            if (have) cs = sp.begin(s + 1);
+            const float* src = p.partials + (size_t)slot * slot_floats;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+              for (int m = 0; m < kMat; ++m)
+                v[si][j][m] = have && j < jn
+                                  ? __ldcg(src + (size_t)(col0 + j) * kMat * MR + lane_off + m * MR)
+                                  : 0.f;
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            float a0 = v[0][j][0], a1 = v[0][j][kMat - 1];
+#pragma unroll
+            for (int q2 = 1; q2 < 4; ++q2)
+              if (q2 < nseg) {
+                a0 += v[q2][j][0];
+                a1 += v[q2][j][kMat - 1];
+              }
+            if (j < C::kCols) {
+              acc0[j] = a0;
+              if (PHASE == 1) acc1[j] = a1;
+            }
+          }
+          if (ew == 0 && lane == 0) p.counters[ti] = 0;  // ready for the next launch
+        } else if (finish) {
           // all segments, this CTA's included, from their slots in chunk order: the sum
           // does not depend on which CTA finishes last
           bool first_seg = true;
@@ -598,19 +664,20 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
         }
         bar_sync(2 + h, 128);
         const int t = q * 32 + lane;
-        if (t < C::kCols) {
+        if (t < js) {
           const float* a = amax_s + h * 4 * C::kCols + t;
           const float amax =
               fmaxf(fmaxf(a[0], a[C::kCols]), fmaxf(a[2 * C::kCols], a[3 * C::kCols]));
           const float s = amax == 0.f ? 1.0f : __fdiv_rn(amax, 448.0f);
           inv_s[h * C::kCols + t] = __frcp_rn(s);
-          if (t < js) p.sh[(size_t)(row0 + col0 + t) * (p.f / 128) + hb] = s;
+          p.sh[(size_t)(row0 + col0 + t) * (p.f / 128) + hb] = s;
         }
         bar_sync(2 + h, 128);
         const float4* inv4 = reinterpret_cast<const float4*>(inv_s + h * C::kCols);
         uint8_t* dst = p.qh + (size_t)(row0 + col0) * p.f + hb * 128 + q * 32 + lane;
 #pragma unroll
         for (int j = 0; j < C::kCols; j += 4) {
+          if (j >= js) break;
           const float4 r = inv4[j / 4];
           const uint16_t c01 = ptx::cvt_e4m3x2(acc0[j] * r.x, acc0[j + 1] * r.y);
           const uint16_t c23 = ptx::cvt_e4m3x2(acc0[j + 2] * r.z, acc0[j + 3] * r.w);
@@ -678,14 +745,14 @@ bool make_map(CUtensorMap* m, const void* base, bool fp4, int K, long long rows,
 }
 
 template <int PHASE, int NMAX, int STAGES, int NBUF, int MR>
-cudaError_t launch_one(const FfnParams& prm, cudaStream_t s, int grid) {
+cudaError_t launch_one(const FfnParams& prm, cudaStream_t s, int grid, bool overlap) {
   using C = Cfg<PHASE, NMAX, STAGES, NBUF, MR>;
   const size_t smem = C::smem_bytes(prm.E);
   cudaError_t err = cudaFuncSetAttribute(ffn_kernel<PHASE, NMAX, STAGES, NBUF, MR>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  ffn_kernel<PHASE, NMAX, STAGES, NBUF, MR><<<grid, kThreads, smem, s>>>(prm);
-  return cudaGetLastError();
+  return launch_pdl(ffn_kernel<PHASE, NMAX, STAGES, NBUF, MR>, dim3(grid), dim3(C::kThreads), smem, s,
+                    overlap, prm);
 }
 
 // (PHASE, NMAX) -> pipeline stages, TMEM partial buffers, weight rows per tile.  Small
@@ -746,7 +813,7 @@ cudaError_t launch_ffn(int phase, int nmax, const FfnArgs& a, cudaStream_t s, in
   prm.l2_hints = a.l2_hints;
   const int grid = num_sms < kMaxCtas ? num_sms : kMaxCtas;
 #define X(P, N, S, B, M) \
-  if (phase == P && nmax == N && mr == M) return launch_one<P, N, S, B, M>(prm, s, grid);
+  if (phase == P && nmax == N && mr == M) return launch_one<P, N, S, B, M>(prm, s, grid, a.overlap);
   BITMOE_FFN_VARIANTS(X)
 #undef X
   return cudaErrorInvalidValue;

@@ -72,10 +72,32 @@ struct FfnArgs {
   float* partials;           // stream-K partial slots
   int ncap;                  // widest token tile
   int l2_hints;              // bit 0: weight boxes evict-first; bit 1: activation boxes evict-last
+  bool overlap;              // launch as a dependent of the previous kernel (see launch_pdl)
 };
 cudaError_t launch_ffn(int phase, int nmax, const FfnArgs& a, cudaStream_t s, int num_sms);
 // dynamic shared memory of a launch
 size_t ffn_smem_bytes(int phase, int nmax, int E, int rows_per_expert);
+
+// Launch, with `overlap`, as a programmatic dependent launch: the kernel may start while
+// the previous kernel on the stream finishes (every kernel of this library calls
+// griddep_wait() before it touches global memory, and griddep_launch_dependents() early).
+// Only valid when the previous operation on the stream is one of this library's kernels:
+// the wait covers prerequisite kernels, not copies or host work queued before them.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, bool overlap, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = overlap ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
 
 // Defined in abi.cu: sets the thread-local message that moe_last_error returns.
 int record_error(int code, const char* msg);

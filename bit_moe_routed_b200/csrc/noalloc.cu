@@ -8,7 +8,7 @@
 // tile plan live in `g_noalloc_scratch` below.
 //
 // Costs and rules of use:
-//  - Every GPU that loads this library holds MOE_NOALLOC_SCRATCH_BYTES (4 MiB) for this
+//  - Every GPU that loads this library holds MOE_NOALLOC_SCRATCH_BYTES (24 MiB) for this
 //    array until the process exits.
 //  - Calls whose workspace would exceed that size are rejected with MOE_ERR_WORKSPACE.
 //  - All calls share the one array per device.  Two calls that overlap on the GPU (on
@@ -16,8 +16,7 @@
 //  - The array keeps the last call's contents.  Nothing in it needs to start at zero:
 //    each call writes the tile plan and every quantised row before reading them.
 //  - The first call on each device looks up the array's device address
-//    (cudaGetSymbolAddress, with that device current) and caches it; make that first call
-//    before any stream capture.
+//    (cudaGetSymbolAddress, with that device current), checks the result and caches it.
 #include "../../include/bitmoe.h"
 #include "internal.cuh"
 

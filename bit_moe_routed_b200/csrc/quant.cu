@@ -61,6 +61,8 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(
     uint8_t* __restrict__ q, float* __restrict__ s, const int32_t* __restrict__ offsets, int E,
     int nmax, int32_t* __restrict__ plan, int* __restrict__ counters, size_t n_counters,
     int* __restrict__ status) {
+  ptx::griddep_launch_dependents();
+  ptx::griddep_wait();  // x, perm, offsets, and the counters the previous FFN launch used
   const int R = P + T;
   const int r = blockIdx.x;
   // the FFN kernels' stream-K counters start every launch at zero
@@ -123,9 +125,8 @@ cudaError_t launch_quant_rows(const uint16_t* x, int T, int k, int d, const int3
   const unsigned blocks = (unsigned)(R + (plan != nullptr ? 1 : 0));
   int threads = (d / 16 + 31) / 32 * 32;  // whole warps
   if (threads > 256) threads = 256;
-  quant_rows_kernel<<<blocks, threads, 0, st>>>(x, T, k, d, perm, nrows_routed, q, s, offsets, E,
-                                               nmax, plan, counters, n_counters, status);
-  return cudaGetLastError();
+  return launch_pdl(quant_rows_kernel, dim3(blocks), dim3(threads), 0, st, false, x, T, k, d, perm,
+                    nrows_routed, q, s, offsets, E, nmax, plan, counters, n_counters, status);
 }
 
 }  // namespace bitmoe

@@ -4,6 +4,7 @@
 // (equal scores: lower expert index first).  The combine weights are the sigmoids of
 // the selected scores renormalised to sum 1, computed in fp32.
 #include "internal.cuh"
+#include "ptx.cuh"
 
 namespace bitmoe {
 namespace {
@@ -12,6 +13,8 @@ template <int PER_LANE>
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ scores, int T, int E,
                                                    int k, int32_t* __restrict__ idx_out,
                                                    float* __restrict__ w_out) {
+  ptx::griddep_launch_dependents();
+  ptx::griddep_wait();  // scores come from earlier work on the stream
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= T) return;
@@ -72,12 +75,10 @@ cudaError_t launch_route_topk(const float* scores, int T, int E, int k, int32_t*
   const int warps_per_block = 8;
   const unsigned blocks = (unsigned)((T + warps_per_block - 1) / warps_per_block);
   if (E <= 256)
-    topk_kernel<8><<<blocks, 256, 0, s>>>(scores, T, E, k, idx, w);
-  else if (E <= 512)
-    topk_kernel<16><<<blocks, 256, 0, s>>>(scores, T, E, k, idx, w);
-  else
-    topk_kernel<32><<<blocks, 256, 0, s>>>(scores, T, E, k, idx, w);
-  return cudaGetLastError();
+    return launch_pdl(topk_kernel<8>, dim3(blocks), dim3(256), 0, s, false, scores, T, E, k, idx, w);
+  if (E <= 512)
+    return launch_pdl(topk_kernel<16>, dim3(blocks), dim3(256), 0, s, false, scores, T, E, k, idx, w);
+  return launch_pdl(topk_kernel<32>, dim3(blocks), dim3(256), 0, s, false, scores, T, E, k, idx, w);
 }
 
 }  // namespace bitmoe

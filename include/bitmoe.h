@@ -134,13 +134,13 @@ int moe_ffn_down(int T, int k, const moe_weights_t* w, float* y_routed, float* y
  * MOE_NOALLOC_SCRATCH_BYTES that the library keeps on every GPU that loads it, for the
  * life of the process.
  *   - Calls needing more scratch than that (moe_workspace_size > the maximum; for
- *     d = 4096, f = 2048, k = 6, E = 256 that is T > 40) return MOE_ERR_WORKSPACE.
+ *     d = 4096, f = 2048, k = 6, E = 256 that is T > 72) return MOE_ERR_WORKSPACE.
  *   - Allocates nothing.  All calls share the one array per device: calls that overlap on
  *     the GPU (other streams, other threads) race on it.  It keeps the previous call's
  *     contents; nothing in it needs to start at zero.
- *   - The first call on a device looks up the array's device address once; make that
- *     first call before any stream capture. */
-#define MOE_NOALLOC_SCRATCH_BYTES (16u << 20)
+ *   - The first call on a device looks up the array's device address once
+ *     (cudaGetSymbolAddress) and fails with MOE_ERR_CUDA if that lookup fails. */
+#define MOE_NOALLOC_SCRATCH_BYTES (24u << 20)
 int moe_expert_ffn_noalloc(const uint16_t* x_bf16, int T, int k, const moe_weights_t* w,
                            const int32_t* offsets, const int32_t* perm, float* y_routed,
                            float* y_shared, void* stream);
