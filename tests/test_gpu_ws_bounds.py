@@ -1,6 +1,6 @@
 """The FFN writes only inside the workspace it is given: a guard region placed right after
 a workspace of exactly moe_workspace_size bytes keeps its fill pattern through the whole
-layer, for batch sizes that take each tile shape (256-row tiles at T <= 32, 128-row tiles
+layer, for batch sizes that take each tile shape (256-row tiles at T <= 64, 128-row tiles
 above) and split tiles between CTAs."""
 import pytest
 import torch
@@ -15,7 +15,7 @@ bm = pytest.importorskip("bit_moe_routed_b200")
 GUARD = 4 << 20
 
 
-@pytest.mark.parametrize("T", [1, 5, 32, 33, 64])
+@pytest.mark.parametrize("T", [1, 5, 64, 65, 100])
 def test_ffn_stays_inside_workspace(T):
     if not torch.cuda.is_available():
         pytest.skip("no GPU")
