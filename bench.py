@@ -355,7 +355,11 @@ def run_gpu(args, w):
     for key in ("gu_bytes", "dn_bytes", "flops_gu", "flops_dn", "weight_bytes", "active"):
         work[key] = sum(wk[key] for wk in works) / len(works)
     is_prefill = T > 256
-    kernel_file = os.path.join(ROOT, "bit_moe_routed_b200", "csrc", "ffn.cu")
+    # single-token batches run the FP4 GEMV kernels (the library's default switch)
+    gemv = T == 1 and d % 512 == 0 and f % 512 == 0
+    kernel_file = os.path.join(ROOT, "bit_moe_routed_b200", "csrc", "gemv.cu" if gemv else "ffn.cu")
+    kernel_name = ("ffn gate/up (FP4 GEMV: bulk-copy stages, in-register e2m1 decode, "
+                   "mma.sync f16 -> fp32)") if gemv else "ffn gate/up (tcgen05 kind::mxf8f6f4)"
     traffic = kernel_traffic(kernel_file, "gate_up", w.name)
     if is_prefill:
         fp8_peak = bf16_peak * 2.0  # dense FP8 = 2x dense BF16 (nominal 4.5 / 2.25 PF)
@@ -368,7 +372,7 @@ def run_gpu(args, w):
         achieved = work["gu_bytes"] / gu_avg_s / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                 "frac": achieved / hbm_peak, "traffic": traffic,
-                "kernel": "ffn gate/up (tcgen05 kind::mxf8f6f4)",
+                "kernel": kernel_name,
                 "peak_source": f"{peak_kind} HBM copy"}
     roof["avg_launch_us"] = gu_avg_s * 1e6
     roof["algorithmic_per_launch"] = work["gu_bytes"] if not is_prefill else work["flops_gu"]

@@ -32,6 +32,7 @@ EXPORTS = (
     "moe_route_topk", "moe_dispatch", "moe_act_quant", "moe_expert_ffn", "moe_ffn_prepare",
     "moe_ffn_gate_up", "moe_ffn_down", "moe_combine", "moe_workspace_size", "moe_last_error",
     "moe_set_wait_limit_ns", "moe_sync_status", "moe_expert_ffn_noalloc",
+    "moe_set_gemv_max_tokens",
 )
 
 
@@ -78,6 +79,7 @@ def lib():
             "moe_set_wait_limit_ns": [LL],
             "moe_sync_status": [P],
             "moe_expert_ffn_noalloc": [P, I, I, W, P, P, P, P, P],
+            "moe_set_gemv_max_tokens": [I],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -146,6 +148,11 @@ class LayerWeights:
 
 def set_wait_limit_ns(n: int) -> None:
     _check(lib().moe_set_wait_limit_ns(int(n)))
+
+
+def set_gemv_max_tokens(t: int) -> None:
+    """Batches up to t tokens (0 or 1) take the single-token FP4 GEMV path."""
+    _check(lib().moe_set_gemv_max_tokens(int(t)))
 
 
 def sync_status(stream=None) -> None:

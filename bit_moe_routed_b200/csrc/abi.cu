@@ -10,6 +10,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 
 namespace bitmoe {
@@ -20,6 +21,7 @@ namespace {
 
 thread_local std::string t_err;
 std::atomic<long long> g_wait_ns{2000000000LL};
+std::atomic<int> g_gemv_max_t{kGemvMaxT};  // batches up to this size take the GEMV path
 
 int fail(int code, const char* fmt, ...) {
   char buf[512];
@@ -94,6 +96,20 @@ int check_weights(const moe_weights_t* w) {
 
 }  // namespace
 
+EncodeTiledFn tensor_map_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
 // Sets the message moe_last_error returns, for the library's other translation units.
 int record_error(int code, const char* msg) { return fail(code, "%s", msg); }
 
@@ -120,6 +136,9 @@ WorkspaceLayout workspace_layout(int T, int k, int E, int d, int f) {
   L.partials = o;
   const size_t tile_rows_max = nmax_for(T) == kNmaxSmall ? 256 : 128;
   o = align256(o + (size_t)kMaxCtas * 2 * (size_t)ncap_for(T) * 2 * tile_rows_max * 4);
+  // single-token path: h of every active expert, fp32
+  L.hbuf = o;
+  if (T <= kGemvMaxT) o = align256(o + R * f * 4);
   L.total = o;
   return L;
 }
@@ -134,6 +153,12 @@ const char* moe_last_error(void) { return t_err.c_str(); }
 
 int moe_set_wait_limit_ns(long long n) {
   g_wait_ns.store(n > 0 ? n : 2000000000LL);
+  return MOE_OK;
+}
+
+int moe_set_gemv_max_tokens(int t) {
+  if (t < 0) return fail(MOE_ERR_INVALID_ARG, "t=%d < 0", t);
+  g_gemv_max_t.store(t);
   return MOE_OK;
 }
 
@@ -218,12 +243,29 @@ int moe_act_quant(const uint16_t* x_bf16, int T, int d, uint8_t* qx, float* sx, 
 
 namespace {
 
+// Set while moe_expert_ffn issues its second and third kernels (see launch_pdl).
+thread_local bool t_overlap = false;
+
 struct FfnCtx {
   DeviceInfo di;
   WorkspaceLayout L;
   int nmax;
+  bool gemv;  // single-token GEMV path (gemv.cu) instead of the tcgen05 tiles (ffn.cu)
   uint8_t* ws;
 };
+
+// The GEMV path needs whole 512-element stages along d and f, 16-byte aligned scale
+// rows for its bulk copies, every active expert's range within two per CTA
+// (k + 1 <= CTAs), and its shared memory.
+bool use_gemv(int T, int k, const moe_weights_t* w, int sms, int max_smem) {
+  if (T < 1 || T > g_gemv_max_t.load() || T > kGemvMaxT) return false;
+  if (w->d % 512 || w->f % 512) return false;
+  if (!aligned(w->gate_scales, 16) || !aligned(w->up_scales, 16) || !aligned(w->down_scales, 16))
+    return false;
+  const int ctas = sms < kMaxCtas ? sms : kMaxCtas;
+  if (k + 1 > ctas) return false;
+  return gemv_smem_bytes(w->d) <= (size_t)max_smem && gemv_smem_bytes(w->f) <= (size_t)max_smem;
+}
 
 int ffn_check(int T, int k, const moe_weights_t* w, void* ws, size_t ws_bytes, FfnCtx& c) {
   if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T=%d < 0", T);
@@ -252,11 +294,25 @@ int ffn_check(int T, int k, const moe_weights_t* w, void* ws, size_t ws_bytes, F
   if (need > (size_t)max_smem)
     return fail(MOE_ERR_INVALID_ARG, "shape needs %zu bytes of shared memory (> %d)", need,
                 max_smem);
+  c.gemv = use_gemv(T, k, w, c.di.sms, max_smem);
   return MOE_OK;
 }
 
-// Set while moe_expert_ffn issues its second and third kernels (see launch_pdl).
-thread_local bool t_overlap = false;
+GemvLaunch gemv_args(int T, int k, const moe_weights_t* w, const FfnCtx& c) {
+  GemvLaunch a{};
+  a.plan = reinterpret_cast<const int32_t*>(c.ws + c.L.plan);
+  a.qx = c.ws + c.L.qx;
+  a.sx = reinterpret_cast<const float*>(c.ws + c.L.sx);
+  a.hbuf = reinterpret_cast<float*>(c.ws + c.L.hbuf);
+  a.E = w->E;
+  a.d = w->d;
+  a.f = w->f;
+  a.P = T * k;
+  a.wait_ns = g_wait_ns.load();
+  a.status = c.di.status;
+  a.overlap = t_overlap;
+  return a;
+}
 
 FfnArgs ffn_args(int phase, int T, int k, const moe_weights_t* w, const FfnCtx& c) {
   FfnArgs a{};
@@ -307,6 +363,13 @@ int moe_ffn_prepare(const uint16_t* x_bf16, int T, int k, const moe_weights_t* w
   if (T == 0) return MOE_OK;
   if (!x_bf16 || !offsets || !perm) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
   if (!aligned(x_bf16, 16)) return fail(MOE_ERR_INVALID_ARG, "x must be 16-byte aligned");
+  if (c.gemv) {  // the token's codes (row 0 of qx) and the list of active experts
+    cudaError_t e = launch_quant_rows(
+        x_bf16, T, k, w->d, nullptr, 0, c.ws + c.L.qx, reinterpret_cast<float*>(c.ws + c.L.sx),
+        offsets, w->E, c.nmax, reinterpret_cast<int32_t*>(c.ws + c.L.plan), nullptr, 0,
+        c.di.status, static_cast<cudaStream_t>(stream), 1);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "ffn prepare launch");
+  }
   cudaError_t e = launch_quant_rows(
       x_bf16, T, k, w->d, perm, T * k, c.ws + c.L.qx, reinterpret_cast<float*>(c.ws + c.L.sx),
       offsets, w->E, c.nmax, reinterpret_cast<int32_t*>(c.ws + c.L.plan),
@@ -321,6 +384,15 @@ int moe_ffn_gate_up(int T, int k, const moe_weights_t* w, void* ws, size_t ws_by
   int rc = ffn_check(T, k, w, ws, ws_bytes, c);
   if (rc) return rc;
   if (T == 0) return MOE_OK;
+  if (c.gemv) {
+    GemvLaunch a = gemv_args(T, k, w, c);
+    a.a0_codes = w->gate_codes;
+    a.a0_scales = w->gate_scales;
+    a.a1_codes = w->up_codes;
+    a.a1_scales = w->up_scales;
+    cudaError_t e = launch_gemv(1, a, static_cast<cudaStream_t>(stream), c.di.sms);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "ffn gate/up launch");
+  }
   cudaError_t e = launch_ffn(1, c.nmax, ffn_args(1, T, k, w, c),
                              static_cast<cudaStream_t>(stream), c.di.sms);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "ffn gate/up launch");
@@ -335,6 +407,15 @@ int moe_ffn_down(int T, int k, const moe_weights_t* w, float* y_routed, float* y
   if (!y_routed || !y_shared) return fail(MOE_ERR_INVALID_ARG, "NULL output pointer");
   if (!aligned(y_routed, 16) || !aligned(y_shared, 16))
     return fail(MOE_ERR_INVALID_ARG, "outputs must be 16-byte aligned");
+  if (c.gemv) {
+    GemvLaunch g = gemv_args(T, k, w, c);
+    g.a0_codes = w->down_codes;
+    g.a0_scales = w->down_scales;
+    g.y_routed = y_routed;
+    g.y_shared = y_shared;
+    cudaError_t e = launch_gemv(2, g, static_cast<cudaStream_t>(stream), c.di.sms);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "ffn down launch");
+  }
   FfnArgs a = ffn_args(2, T, k, w, c);
   a.y_routed = y_routed;
   a.y_shared = y_shared;

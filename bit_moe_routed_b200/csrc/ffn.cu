@@ -46,6 +46,7 @@
 // returns.
 #include "internal.cuh"
 #include "ptx.cuh"
+#include "waits.cuh"
 
 #include <cstring>
 #include <mutex>
@@ -60,7 +61,6 @@ constexpr int kIssuerWarp1 = kSfWarp + 1;       // warps 11.. issue MMAs beside 
 // tcgen05.mma per ~120 cycles whatever its N, so small-N tiles need several issuers.
 constexpr int ffn_issuers(int phase, int mr) { return (phase == 1 ? 2 : 1) * (mr / 128); }
 constexpr int ffn_threads(int phase, int mr) { return 32 * (kIssuerWarp1 + ffn_issuers(phase, mr) - 1); }
-constexpr long long kDrainNs = 500000000LL;     // bound on draining in-flight work
 
 struct FfnParams {
   CUtensorMap tmA0;  // gate (phase 1) / down (phase 2) codes, all experts stacked
@@ -135,42 +135,6 @@ __device__ __forceinline__ void reg_fence(float (&v)[N]) {
 #pragma unroll
   for (int i = 0; i < N; ++i) asm volatile("" : "+f"(v[i]));
 }
-// Bounded wait by one thread; false if the limit ran out or another role aborted.  The
-// loop is try_wait alone (which itself parks the thread for a short, hardware-chosen
-// time); the abort flag and the clock are read only every 64 tries, so waiting threads
-// add little shared-memory traffic.  (Limits under 100 us are checked on every try.)
-__device__ bool wait_one(uint32_t bar, uint32_t parity, long long limit, volatile int* abort_flag,
-                         int* status) {
-  if (ptx::mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = ptx::globaltimer();
-  const uint32_t every = limit < 100000 ? 0u : 63u;
-  for (uint32_t i = 1;; ++i) {
-    if (ptx::mbar_try_wait(bar, parity)) return true;
-    if ((i & every) == 0) {
-      if (*abort_flag) return false;
-      if ((long long)(ptx::globaltimer() - t0) > limit) {
-        *abort_flag = 1;
-        atomicOr(status, kStatusTimeout);
-        return false;
-      }
-    }
-  }
-}
-// Same, decided by lane 0 and shared with the whole warp (keeps the warp converged).
-__device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, long long limit,
-                                          volatile int* abort_flag, int* status) {
-  int ok = 0;
-  if ((threadIdx.x & 31) == 0) ok = wait_one(bar, parity, limit, abort_flag, status) ? 1 : 0;
-  return __shfl_sync(0xffffffffu, ok, 0) != 0;
-}
-// Wait for in-flight work to land during teardown (ignores the abort flag).
-__device__ void drain_wait(uint32_t bar, uint32_t parity) {
-  const uint64_t t0 = ptx::globaltimer();
-  while (!ptx::mbar_try_wait(bar, parity)) {
-    if ((long long)(ptx::globaltimer() - t0) > kDrainNs) break;
-  }
-}
-
 // Tile i -> (expert, 128-row block, first activation row, rows).  Tiles of one expert
 // are ordered (block, token tile) so consecutive tiles share weight rows in L2.
 __device__ __forceinline__ void decode_tile(const int32_t* ttbase, const int32_t* tiles, int E,
@@ -709,29 +673,10 @@ __global__ void __launch_bounds__(ffn_threads(PHASE, MR), 1) ffn_kernel(const __
 }
 
 // ---------------------------------------------------------------- host side
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
-                                         &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  });
-  return fn;
-}
-
 // 2-D map over a row-major matrix [rows][K]; box = 128 elements of K x box_rows rows,
 // 128-byte swizzle (the layout the UMMA shared-memory descriptors expect).
 bool make_map(CUtensorMap* m, const void* base, bool fp4, int K, long long rows, int box_rows) {
-  EncodeTiledFn fn = encode_fn();
+  EncodeTiledFn fn = tensor_map_encode_fn();
   if (fn == nullptr) return false;
   const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)(fp4 ? K / 2 : K)};

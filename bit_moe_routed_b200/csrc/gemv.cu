@@ -1,0 +1,356 @@
+// Single-token decode path of the expert FFN: memory-bound FP4 GEMVs.
+//
+// At T = 1 every expert group holds the one token, so gate/up (phase 1) and down
+// (phase 2) are matrix-vector products whose cost is reading each selected expert's FP4
+// codes and block scales once (dpshk.com article, "核心实现三" and "核心实现四": an
+// expert is read once for all its tokens, and FP4 is decoded inside the product, never
+// expanded to a float matrix in memory).  The tcgen05 tile path would spend a
+// 32-column MMA tile and a TMEM round trip per 128-K chunk on one useful column.
+//
+// Each warp streams 16 weight rows (phase 1: 8 gate rows and the same 8 up rows;
+// phase 2: 16 down rows) through its own ring of shared-memory stages, filled by 2-D
+// TMA boxes: per matrix, 128 code bytes x rows (128-byte swizzle, so that the lanes'
+// 4-byte reads of eight rows hit distinct banks) twice, and 16 scale bytes x rows.
+// A stage holds 512 K-elements, i.e. 16 blocks of 32 per row.
+//
+// Per 32-element block b the warp runs two mma.sync m16n8k16 (f16 in, fp32 accumulate)
+// into a fresh accumulator: lane (g, t) decodes bytes 4t..4t+3 of the block in rows g
+// and g+8 (cvt e2m1x2 -> f16x2, eight elements per row) and holds the activation's
+// elements 8t..8t+7 of the block in the B fragment.  The MMA's K order is thus a
+// permutation of the block, the same on both sides.  The fp32 block partial is then
+// multiplied by 2^(e-127) (the row's ue8m0 scale; exact in fp32) times the activation's
+// fp32 scale of its 128-block and added to the row's accumulator.
+//
+// Phase 1 ends with h = silu(g) * u per row (fp32, to a workspace buffer).  Phase 2
+// quantises the h of its experts in its prologue (amax / 448, IEEE divide, e4m3 round
+// to nearest even: the same rule as the activations) and writes fp32 y rows.
+//
+// Work split: the units (16-row blocks of every selected expert, in plan order) are cut
+// into one contiguous range per CTA (148 CTAs, one per SM); warp w of a CTA takes units
+// w, w+16, ... of its range.  A range spans at most two experts, whose activations the
+// CTA keeps in shared memory as f16 values.
+#include "internal.cuh"
+#include "ptx.cuh"
+#include "waits.cuh"
+
+#include <cstring>
+
+namespace bitmoe {
+namespace {
+
+constexpr int kGvWarps = 16;
+constexpr int kGvThreads = kGvWarps * 32;
+constexpr int kGvStages = 3;                          // ring depth per warp
+constexpr int kGvRows = 16;                           // weight rows per unit
+constexpr int kGvCodeBytes = kGvRows * 256;           // 256 code bytes (512 elements) per row
+constexpr int kGvScaleBytes = kGvRows * 16;           // 16 ue8m0 bytes per row
+constexpr int kGvStageBytes = kGvCodeBytes + kGvScaleBytes;
+constexpr int kGvMaxSlots = 2;                        // experts per CTA range
+
+struct GemvParams {
+  CUtensorMap tm_c0;         // gate (phase 1) or down (phase 2) codes [rows][K/2], experts stacked
+  CUtensorMap tm_s0;         // their scales [rows][K/32]
+  CUtensorMap tm_c1;         // up codes and scales (phase 1)
+  CUtensorMap tm_s1;
+  const int32_t* plan;       // [0] = active experts n, then n pairs (expert, output row)
+  const uint8_t* qx;         // phase 1: the token's e4m3 codes [K]
+  const float* sx;           // phase 1: its block scales [K/128]
+  float* hbuf;               // phase 1 out, phase 2 in: h [slot][f] fp32
+  float* y_routed;           // phase 2 out: y rows [T*k][d] (expert-sorted order)
+  float* y_shared;           // phase 2 out: the shared expert's row [d]
+  int E, K, rows_per_expert, f, d, P;
+  long long wait_ns;
+  int* status;
+};
+
+// Shared memory (from a 1024-byte aligned base): code rings [warp][stage] (each stage
+// 4 KB, 1024-aligned for the swizzled boxes), scale rings, activations, barriers.
+struct GvSmem {
+  static constexpr int kOffScales = kGvWarps * kGvStages * kGvCodeBytes;
+  static constexpr int kOffB = kOffScales + kGvWarps * kGvStages * kGvScaleBytes;
+  __host__ __device__ static int off_bs(int K) { return kOffB + kGvMaxSlots * K * 2; }
+  __host__ __device__ static int off_bars(int K) { return off_bs(K) + kGvMaxSlots * (K / 128) * 4; }
+  __host__ __device__ static int off_misc(int K) { return off_bars(K) + kGvWarps * kGvStages * 8; }
+  // misc: abort flag, then (expert, output row) of the range's slots
+  __host__ __device__ static size_t bytes(int K) { return (size_t)off_misc(K) + 32 + 1024; }
+};
+
+// 2^(e-127) in fp32 for a ue8m0 byte e (2^-127 is a subnormal)
+__device__ __forceinline__ float ue8m0_f32(uint32_t e) {
+  return __uint_as_float(e > 0 ? e << 23 : 0x00400000u);
+}
+
+// Byte offset, in a stage, of bytes 4t..4t+3 of block b (0..15) of stage row r.  Row r
+// lies in box (matrix, half b/8) at box row rb; the 128-byte swizzle XORs the 16-byte
+// chunk index with the row index mod 8.
+template <int PHASE>
+__device__ __forceinline__ uint32_t code_offset(int r, int b, int t) {
+  const int half = b >> 3, chunk = b & 7;
+  uint32_t box, rb;
+  if (PHASE == 1) {  // rows 0-7 gate, 8-15 up; boxes of 8 rows: [matrix][half]
+    box = (uint32_t)((r >> 3) * 2 + half) * 1024u;
+    rb = (uint32_t)(r & 7);
+  } else {           // boxes of 16 rows: [half]
+    box = (uint32_t)half * 2048u;
+    rb = (uint32_t)r;
+  }
+  return box + rb * 128u + ((uint32_t)(chunk ^ (r & 7)) << 4) + 4u * (uint32_t)t;
+}
+
+template <int PHASE>
+__global__ void __launch_bounds__(kGvThreads, 1) gemv_kernel(const __grid_constant__ GemvParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (ptx::smem_u32(smem_raw) & 1023)) & 1023);
+  const int K = p.K;
+  uint16_t* bx = reinterpret_cast<uint16_t*>(smem + GvSmem::kOffB);   // [slot][K] f16
+  float* bs = reinterpret_cast<float*>(smem + GvSmem::off_bs(K));      // [slot][K/128]
+  const uint32_t bars = ptx::smem_u32(smem + GvSmem::off_bars(K));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + GvSmem::off_misc(K));
+  int* slot_info = reinterpret_cast<int*>(smem + GvSmem::off_misc(K) + 16);  // [slot][2]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  auto full = [&](int s) { return bars + 8u * (uint32_t)(warp * kGvStages + s); };
+  auto codes_at = [&](int s) { return smem + (warp * kGvStages + s) * kGvCodeBytes; };
+  auto scales_at = [&](int s) {
+    return smem + GvSmem::kOffScales + (warp * kGvStages + s) * kGvScaleBytes;
+  };
+
+  if (lane == 0)
+    for (int s = 0; s < kGvStages; ++s) ptx::mbar_init(full(s), 1);
+  if (threadIdx.x == 0) *abort_flag = 0;
+  ptx::fence_mbar_init();
+
+  ptx::griddep_wait();  // the plan, the activations and (phase 2) h come from earlier kernels
+  ptx::griddep_launch_dependents();
+
+  const int n_act = p.plan[0];
+  const int rows_unit = PHASE == 1 ? kGvRows / 2 : kGvRows;
+  const int upe = p.rows_per_expert / rows_unit;  // units per expert
+  const int N = n_act * upe;
+  const int u_lo = (int)((long long)blockIdx.x * N / gridDim.x);
+  const int u_hi = (int)((long long)(blockIdx.x + 1) * N / gridDim.x);
+  const int S = K / 512;                           // stages per unit
+  const int my_units = u_lo + warp < u_hi ? (u_hi - u_lo - warp + kGvWarps - 1) / kGvWarps : 0;
+  const int total = my_units * S;
+  const int slot_lo = u_lo / upe;
+  const int n_slots = u_lo < u_hi ? (u_hi - 1) / upe - slot_lo + 1 : 0;
+  // a CTA range covers at most kGvMaxSlots experts whenever n_act <= gridDim.x (the host
+  // checks it); a plan that breaks it is flagged, and the CTA stops before any copy
+  if (n_act < 0 || n_act > p.P + 1 || n_slots > kGvMaxSlots) {
+    if (threadIdx.x == 0) atomicOr(p.status, kStatusBadIndex);
+    return;
+  }
+  if (threadIdx.x < n_slots) {
+    int e = p.plan[1 + 2 * (slot_lo + threadIdx.x)];
+    int orow = p.plan[2 + 2 * (slot_lo + threadIdx.x)];
+    if (e < 0 || e > p.E || orow >= p.P) {  // never produced by the prepare kernel
+      atomicOr(p.status, kStatusBadIndex);
+      e = 0;
+      orow = -2;  // nothing is stored for this slot
+    }
+    slot_info[2 * threadIdx.x] = e;
+    slot_info[2 * threadIdx.x + 1] = orow;
+  }
+  __syncthreads();
+
+  const uint64_t pol = ptx::make_policy_evict_first();
+  if (threadIdx.x == 0) {
+    ptx::prefetch_tmap(&p.tm_c0);
+    ptx::prefetch_tmap(&p.tm_s0);
+    if (PHASE == 1) {
+      ptx::prefetch_tmap(&p.tm_c1);
+      ptx::prefetch_tmap(&p.tm_s1);
+    }
+  }
+
+  // stage q of this warp: unit u_lo + warp + (q / S) * 16, K-chunk q % S; lane 0 issues
+  auto issue = [&](int q) {
+    const int u = u_lo + warp + (q / S) * kGvWarps;
+    const int c = q % S;
+    const int e = slot_info[2 * (u / upe - slot_lo)];
+    const int st = q % kGvStages;
+    const uint32_t dc = ptx::smem_u32(codes_at(st)), ds = ptx::smem_u32(scales_at(st));
+    ptx::mbar_arrive_expect_tx(full(st), kGvStageBytes);
+    const int x0 = c * 256, xs = c * 16;
+    if (PHASE == 1) {
+      const int row = e * p.rows_per_expert + (u % upe) * 8;
+      ptx::tma_load_2d_hint(dc, &p.tm_c0, x0, row, full(st), pol);
+      ptx::tma_load_2d_hint(dc + 1024, &p.tm_c0, x0 + 128, row, full(st), pol);
+      ptx::tma_load_2d_hint(dc + 2048, &p.tm_c1, x0, row, full(st), pol);
+      ptx::tma_load_2d_hint(dc + 3072, &p.tm_c1, x0 + 128, row, full(st), pol);
+      ptx::tma_load_2d_hint(ds, &p.tm_s0, xs, row, full(st), pol);
+      ptx::tma_load_2d_hint(ds + 128, &p.tm_s1, xs, row, full(st), pol);
+    } else {
+      const int row = e * p.rows_per_expert + (u % upe) * 16;
+      ptx::tma_load_2d_hint(dc, &p.tm_c0, x0, row, full(st), pol);
+      ptx::tma_load_2d_hint(dc + 2048, &p.tm_c0, x0 + 128, row, full(st), pol);
+      ptx::tma_load_2d_hint(ds, &p.tm_s0, xs, row, full(st), pol);
+    }
+  };
+
+  int issued = 0;
+  if (lane == 0)
+    for (; issued < kGvStages && issued < total; ++issued) issue(issued);
+  issued = __shfl_sync(0xffffffffu, issued, 0);
+
+  // activations of this CTA's experts -> f16 values and fp32 block scales
+  const int nb = K / 128;
+  if (PHASE == 1) {
+    for (int i = threadIdx.x; i < K / 2; i += kGvThreads) {
+      const uint16_t pr = reinterpret_cast<const uint16_t*>(p.qx)[i];
+      reinterpret_cast<uint32_t*>(bx)[i] = ptx::cvt_e4m3x2_f16x2(pr);
+    }
+    for (int i = threadIdx.x; i < nb; i += kGvThreads) bs[i] = p.sx[i];
+  } else {
+    // one warp per 128-block: 4 consecutive h values per lane
+    for (int w = warp; w < n_slots * nb; w += kGvWarps) {
+      const int sl = w / nb, j = w % nb;
+      const float4 h = *reinterpret_cast<const float4*>(p.hbuf + (size_t)(slot_lo + sl) * K +
+                                                        128 * j + 4 * lane);
+      float amax = fmaxf(fmaxf(fabsf(h.x), fabsf(h.y)), fmaxf(fabsf(h.z), fabsf(h.w)));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      const float sc = amax == 0.f ? 1.0f : __fdiv_rn(amax, 448.0f);
+      const uint16_t q01 = ptx::cvt_e4m3x2(__fdiv_rn(h.x, sc), __fdiv_rn(h.y, sc));
+      const uint16_t q23 = ptx::cvt_e4m3x2(__fdiv_rn(h.z, sc), __fdiv_rn(h.w, sc));
+      uint32_t* dst = reinterpret_cast<uint32_t*>(bx + (size_t)sl * K + 128 * j + 4 * lane);
+      dst[0] = ptx::cvt_e4m3x2_f16x2(q01);
+      dst[1] = ptx::cvt_e4m3x2_f16x2(q23);
+      if (lane == 0) bs[sl * nb + j] = sc;
+    }
+  }
+  __syncthreads();
+
+  const int r0 = g, r1 = g + 8;  // this lane's stage rows (phase 1: gate g, up g)
+  bool ok = true;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  int q = 0;
+  for (; q < total; ++q) {
+    const int st = q % kGvStages;
+    if (!wait_warp(full(st), (uint32_t)(q / kGvStages) & 1u, p.wait_ns, abort_flag, p.status)) {
+      ok = false;
+      break;
+    }
+    const int u = u_lo + warp + (q / S) * kGvWarps;
+    const int c = q % S;
+    const int sl = u / upe - slot_lo;
+    const uint8_t* cst = codes_at(st);
+    const uint8_t* sst = scales_at(st);
+    const uint16_t* xb = bx + (PHASE == 1 ? 0 : (size_t)sl * K);
+    const float* sxb = bs + (PHASE == 1 ? 0 : sl * nb);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {  // 128-element activation block j = 4c + i
+      const int j = 4 * c + i;
+      const uint32_t ea = *reinterpret_cast<const uint32_t*>(sst + r0 * 16 + 4 * i);
+      const uint32_t eb = *reinterpret_cast<const uint32_t*>(sst + r1 * 16 + 4 * i);
+      const float sxj = sxb[j];
+#pragma unroll
+      for (int bb = 0; bb < 4; ++bb) {
+        const int b = 4 * i + bb;  // block within the stage
+        const uint32_t wa = *reinterpret_cast<const uint32_t*>(cst + code_offset<PHASE>(r0, b, t));
+        const uint32_t wb = *reinterpret_cast<const uint32_t*>(cst + code_offset<PHASE>(r1, b, t));
+        uint32_t ha[4], hb[4];
+        ptx::cvt_e2m1x8_f16(wa, ha);
+        ptx::cvt_e2m1x8_f16(wb, hb);
+        const uint4 xv = *reinterpret_cast<const uint4*>(xb + 128 * j + 32 * bb + 8 * t);
+        float cb[4] = {0.f, 0.f, 0.f, 0.f};
+        ptx::mma_m16n8k16_f16(cb, ha[0], hb[0], ha[1], hb[1], xv.x, xv.y);
+        ptx::mma_m16n8k16_f16(cb, ha[2], hb[2], ha[3], hb[3], xv.z, xv.w);
+        const float sa = sxj * ue8m0_f32((ea >> (8 * bb)) & 0xffu);
+        const float sb = sxj * ue8m0_f32((eb >> (8 * bb)) & 0xffu);
+        acc[0] = fmaf(sa, cb[0], acc[0]);
+        acc[1] = fmaf(sa, cb[1], acc[1]);
+        acc[2] = fmaf(sb, cb[2], acc[2]);
+        acc[3] = fmaf(sb, cb[3], acc[3]);
+      }
+    }
+    // every value read from the stage has been consumed above, so once all lanes are
+    // past this point the next TMA copy may overwrite it
+    __syncwarp();
+    if (issued < total) {
+      if (lane == 0) issue(issued);
+      ++issued;
+    }
+    if (c == S - 1) {  // unit complete: column 0 (the token) sits in lanes t == 0
+      const int blk = u % upe;
+      if (t == 0) {
+        if (PHASE == 1) {
+          const float gg = acc[0];
+          const float h = __fdividef(gg, 1.0f + expf(-gg)) * acc[2];
+          p.hbuf[(size_t)(sl + slot_lo) * p.f + (size_t)blk * 8 + g] = h;
+        } else {
+          const int orow = slot_info[2 * sl + 1];
+          if (orow >= -1) {
+            float* y = orow >= 0 ? p.y_routed + (size_t)orow * p.d : p.y_shared;
+            y[(size_t)blk * 16 + g] = acc[0];
+            y[(size_t)blk * 16 + g + 8] = acc[2];
+          }
+        }
+      }
+      acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+    }
+  }
+  if (!ok) {  // let the copies still in flight land before the CTA exits
+    if (lane == 0)
+      for (int r = q; r < issued; ++r)
+        drain_wait(full(r % kGvStages), (uint32_t)(r / kGvStages) & 1u);
+    __syncwarp();
+  }
+}
+
+// 2-D map over a row-major byte matrix [rows][cols]: box = box_cols bytes x box_rows rows
+bool make_byte_map(CUtensorMap* m, const void* base, long long cols, long long rows, int box_cols,
+                   int box_rows, bool swizzle128) {
+  EncodeTiledFn fn = tensor_map_encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols};
+  const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE,
+            swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+size_t gemv_smem_bytes(int K) { return GvSmem::bytes(K); }
+
+cudaError_t launch_gemv(int phase, const GemvLaunch& a, cudaStream_t s, int num_sms) {
+  GemvParams p;
+  memset(&p, 0, sizeof(p));
+  const int K = phase == 1 ? a.d : a.f;
+  const int rpe = phase == 1 ? a.f : a.d;
+  const long long rows = (long long)(a.E + 1) * rpe;
+  const int box_rows = phase == 1 ? 8 : 16;
+  if (!make_byte_map(&p.tm_c0, a.a0_codes, K / 2, rows, 128, box_rows, true) ||
+      !make_byte_map(&p.tm_s0, a.a0_scales, K / 32, rows, 16, box_rows, false))
+    return cudaErrorInvalidValue;
+  if (phase == 1 && (!make_byte_map(&p.tm_c1, a.a1_codes, K / 2, rows, 128, box_rows, true) ||
+                     !make_byte_map(&p.tm_s1, a.a1_scales, K / 32, rows, 16, box_rows, false)))
+    return cudaErrorInvalidValue;
+  p.plan = a.plan;
+  p.qx = a.qx;
+  p.sx = a.sx;
+  p.hbuf = a.hbuf;
+  p.y_routed = a.y_routed;
+  p.y_shared = a.y_shared;
+  p.E = a.E;
+  p.K = K;
+  p.rows_per_expert = rpe;
+  p.f = a.f;
+  p.d = a.d;
+  p.P = a.P;
+  p.wait_ns = a.wait_ns;
+  p.status = a.status;
+  const size_t smem = GvSmem::bytes(p.K);
+  auto kern = phase == 1 ? gemv_kernel<1> : gemv_kernel<2>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int grid = num_sms < kMaxCtas ? num_sms : kMaxCtas;
+  return launch_pdl(kern, dim3(grid), dim3(kGvThreads), smem, s, a.overlap, p);
+}
+
+}  // namespace bitmoe

@@ -8,7 +8,8 @@
 namespace bitmoe {
 
 // Device-side status word (one per device): bit 0 = a bounded wait expired,
-// bit 1 = an expert id outside [0, E) reached the dispatch kernel.
+// bit 1 = an expert id outside [0, E) reached the dispatch kernel (or a plan entry was
+// out of range).
 constexpr int kStatusTimeout = 1;
 constexpr int kStatusBadIndex = 2;
 
@@ -33,8 +34,12 @@ constexpr int kMaxCtas = 148;
 //   [E+2, E+2 + 2*ntmax)  tiles: (row0, n) per token tile
 inline size_t plan_ntmax(int R, int E) { return (size_t)R / 16 + (size_t)E + 2; }
 
+// Single-token batches (T = 1) run the expert FFN as two FP4 GEMV kernels (gemv.cu)
+// when the shapes allow it; larger batches use the tcgen05 tile kernels (ffn.cu).
+constexpr int kGemvMaxT = 1;
+
 struct WorkspaceLayout {
-  size_t plan, qx, sx, qh, sh, counters, partials, total;
+  size_t plan, qx, sx, qh, sh, counters, partials, hbuf, total;
   size_t n_counters;
 };
 WorkspaceLayout workspace_layout(int T, int k, int E, int d, int f);
@@ -47,11 +52,12 @@ cudaError_t launch_dispatch(const int32_t* idx, int T, int k, int E, int32_t* co
                             cudaStream_t s);
 // rows r < P = T*k take token perm[r]/k, rows P <= r < P+T take token r-P; perm may be
 // NULL with P = 0 for a plain quantisation of T rows.  If plan != NULL, one extra block
-// writes the token-tile plan.
+// writes the token-tile plan (plan_mode 0) or the single-token path's list of active
+// experts (plan_mode 1).
 cudaError_t launch_quant_rows(const uint16_t* x, int T, int k, int d, const int32_t* perm,
                               int nrows_routed, uint8_t* q, float* s, const int32_t* offsets,
                               int E, int nmax, int32_t* plan, int* counters, size_t n_counters,
-                              int* status, cudaStream_t st);
+                              int* status, cudaStream_t st, int plan_mode = 0);
 cudaError_t launch_combine(const float* y, const float* ysh, const float* w, const int32_t* pos,
                            int T, int k, int d, float* out, int* status, cudaStream_t s);
 
@@ -82,6 +88,29 @@ cudaError_t launch_ffn(int phase, int nmax, const FfnArgs& a, cudaStream_t s, in
 // dynamic shared memory of a launch
 size_t ffn_smem_bytes(int phase, int nmax, int E, int rows_per_expert);
 
+// Single-token FP4 GEMV path (gemv.cu).  The plan holds the active experts (routed
+// ones with a token, in ascending id, then the shared expert E) as (expert, output row)
+// pairs after their count; the output row is the routed row in expert-sorted order, or
+// -1 for the shared expert.
+struct GemvLaunch {
+  const uint8_t* a0_codes;   // gate (phase 1) or down (phase 2)
+  const uint8_t* a0_scales;
+  const uint8_t* a1_codes;   // up (phase 1)
+  const uint8_t* a1_scales;
+  const int32_t* plan;
+  const uint8_t* qx;         // phase 1: the token's e4m3 codes [d] and block scales
+  const float* sx;
+  float* hbuf;               // h [active experts][f] fp32
+  float* y_routed;
+  float* y_shared;
+  int E, d, f, P;
+  long long wait_ns;
+  int* status;
+  bool overlap;
+};
+cudaError_t launch_gemv(int phase, const GemvLaunch& a, cudaStream_t s, int num_sms);
+size_t gemv_smem_bytes(int K);
+
 // Launch, with `overlap`, as a programmatic dependent launch: the kernel may start while
 // the previous kernel on the stream finishes (every kernel of this library calls
 // griddep_wait() before it touches global memory, and griddep_launch_dependents() early).
@@ -102,6 +131,13 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   cfg.numAttrs = overlap ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
+
+// The driver's cuTensorMapEncodeTiled (looked up once; NULL if the driver lacks it).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn tensor_map_encode_fn();
 
 // Defined in abi.cu: sets the thread-local message that moe_last_error returns.
 int record_error(int code, const char* msg);

@@ -1,7 +1,7 @@
-// Thin inline-PTX wrappers for sm_100a: mbarriers, TMA tensor loads, cp.async,
-// tcgen05 (TMEM allocation, block-scaled MMA, TMEM loads/copies), fences and
-// conversions used by the bitmoe kernels.  All wrappers are single instructions
-// (or a predicate set-up plus one instruction); nothing here allocates.
+// Thin inline-PTX wrappers for sm_100a: mbarriers, TMA tensor and bulk loads, cp.async,
+// tcgen05 (TMEM allocation, block-scaled MMA, TMEM loads/copies), mma.sync, fences and
+// conversions used by the bitmoe kernels.  Each wrapper is one instruction, or a few of
+// the same kind (the e2m1 word decode); nothing here allocates.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -94,6 +94,16 @@ __device__ __forceinline__ uint64_t make_policy_evict_normal() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
   return p;
+}
+// 1-D bulk copy global -> shared (sizes and both addresses multiples of 16 bytes),
+// completing as transaction bytes on an mbarrier, with an L2 eviction-priority policy
+__device__ __forceinline__ void bulk_load_hint(uint32_t dst, const void* src, uint32_t bytes,
+                                               uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar), "l"(policy)
+      : "memory");
 }
 __device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
@@ -189,6 +199,38 @@ __device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
   uint16_t r;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// four packed e2m1 pairs (the bytes of w, low nibble = even element) -> four f16x2
+__device__ __forceinline__ void cvt_e2m1x8_f16(uint32_t w, uint32_t* h) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+      : "r"(w));
+}
+// packed e4m3 pair (lo in bits 0-7) -> f16x2 (exact)
+__device__ __forceinline__ uint32_t cvt_e4m3x2_f16x2(uint16_t v) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
+  return r;
+}
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+// warp-level D(16x8, fp32) += A(16x16, f16, row) x B(16x8, f16, col)
+__device__ __forceinline__ void mma_m16n8k16_f16(float* c, uint32_t a0, uint32_t a1, uint32_t a2,
+                                                 uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3},"
+      " {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 }  // namespace ptx

@@ -56,11 +56,41 @@ __device__ void write_plan(const int32_t* __restrict__ offsets, int E, int T, in
   if (lane == 31) ttbase[E + 1] = incl;
 }
 
+// Active experts of a single token for the GEMV path: routed experts with a row, in
+// ascending id, then the shared expert.  plan[0] = count, then (expert, row) pairs.
+__device__ void write_gemv_plan(const int32_t* __restrict__ offsets, int E,
+                                int32_t* __restrict__ plan) {
+  const int lane = threadIdx.x & 31;
+  const int per = (E + 31) / 32;
+  const int e0 = lane * per, e1 = min(E, e0 + per);
+  int local = 0;
+  for (int e = e0; e < e1; ++e) local += offsets[e + 1] > offsets[e] ? 1 : 0;
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  int i = incl - local;
+  for (int e = e0; e < e1; ++e) {
+    if (offsets[e + 1] > offsets[e]) {
+      plan[1 + 2 * i] = e;
+      plan[2 + 2 * i] = offsets[e];
+      ++i;
+    }
+  }
+  if (lane == 31) {
+    plan[1 + 2 * incl] = E;
+    plan[2 + 2 * incl] = -1;
+    plan[0] = incl + 1;
+  }
+}
+
 __global__ void __launch_bounds__(256) quant_rows_kernel(
     const uint16_t* __restrict__ x, int T, int k, int d, const int32_t* __restrict__ perm, int P,
     uint8_t* __restrict__ q, float* __restrict__ s, const int32_t* __restrict__ offsets, int E,
     int nmax, int32_t* __restrict__ plan, int* __restrict__ counters, size_t n_counters,
-    int* __restrict__ status) {
+    int* __restrict__ status, int plan_mode) {
   ptx::griddep_launch_dependents();
   ptx::griddep_wait();  // x, perm, offsets, and the counters the previous FFN launch used
   const int R = P + T;
@@ -70,7 +100,10 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(
        i += (size_t)gridDim.x * blockDim.x)
     counters[i] = 0;
   if (r == R) {  // the plan block
-    if (threadIdx.x < 32) write_plan(offsets, E, T, P, nmax, plan);
+    if (threadIdx.x < 32) {
+      if (plan_mode == 1) write_gemv_plan(offsets, E, plan);
+      else write_plan(offsets, E, T, P, nmax, plan);
+    }
     return;
   }
   int t = r < P ? perm[r] / k : r - P;
@@ -120,13 +153,14 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(
 cudaError_t launch_quant_rows(const uint16_t* x, int T, int k, int d, const int32_t* perm,
                               int nrows_routed, uint8_t* q, float* s, const int32_t* offsets,
                               int E, int nmax, int32_t* plan, int* counters, size_t n_counters,
-                              int* status, cudaStream_t st) {
+                              int* status, cudaStream_t st, int plan_mode) {
   const int R = nrows_routed + T;
   const unsigned blocks = (unsigned)(R + (plan != nullptr ? 1 : 0));
   int threads = (d / 16 + 31) / 32 * 32;  // whole warps
   if (threads > 256) threads = 256;
   return launch_pdl(quant_rows_kernel, dim3(blocks), dim3(threads), 0, st, false, x, T, k, d, perm,
-                    nrows_routed, q, s, offsets, E, nmax, plan, counters, n_counters, status);
+                    nrows_routed, q, s, offsets, E, nmax, plan, counters, n_counters, status,
+                    plan_mode);
 }
 
 }  // namespace bitmoe

@@ -164,6 +164,15 @@ const char* moe_last_error(void);
  * (2 s).  n <= 0 restores the default.  Applies to launches made after the call. */
 int moe_set_wait_limit_ns(long long n);
 
+/* Largest batch T that runs the expert FFN as two FP4 GEMV kernels (the single-token
+ * decode path) instead of the tcgen05 tile kernels.  The pages have no counterpart: it
+ * is a switch between two implementations of the same calls.  0 sends every batch to
+ * the tile kernels; values above 1 act as 1 (the GEMV path takes T = 1 only).  The
+ * GEMV path also needs d and f multiples of 512, 16-byte aligned scale arrays and
+ * k + 1 <= the SM count; other shapes take the tile kernels.  Default 1.  Applies to
+ * calls made after it. */
+int moe_set_gemv_max_tokens(int t);
+
 /* Synchronise `stream`, then return MOE_ERR_CUDA for a pending CUDA error,
  * MOE_ERR_TIMEOUT if a device-side wait expired since the last call (clearing the
  * record), else MOE_OK. */

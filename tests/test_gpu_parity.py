@@ -176,6 +176,69 @@ def test_layer_extreme_weights():
     assert_close(g["y_shared"].numpy(), y_sh, "extreme weights: y_shared")
 
 
+# ---------------------------------------------------------------- single-token GEMV path
+@pytest.mark.parametrize("E,k,d,f", [
+    (8, 2, 512, 512),       # one stage per row along d and along f
+    (16, 4, 1024, 512),
+    (32, 6, 512, 1536),     # three stages per down row
+    (256, 6, 2048, 1024),   # CTA ranges that span two experts
+])
+def test_gemv_single_token_shapes(E, k, d, f):
+    _small_layer(1, E, k, d, f, "uniform", seed=E + d + f)
+
+
+def _custom_layer_check(T, E, k, d, f, arrs, seed, label):
+    W = bm.LayerWeights.from_dict({kk: torch.from_numpy(v).cuda() for kk, v in arrs.items()})
+    x = synth.gen_x(T, d, seed=seed)
+    s = synth.gen_scores_uniform(T, E, seed=seed + 1)
+    g = gpu_layer(x, s, k, W)
+    idx, w = oracle.route_topk(s.numpy(), k)
+    ex = {e: synth.HostExpert(*(arrs[n][e] for n in (
+        "gate_codes", "gate_scales", "up_codes", "up_scales", "down_codes", "down_scales")))
+        for e in range(E + 1)}
+    y_pair, y_sh, out = oracle.moe_layer(x, E, k, d, f, ex, idx, w)
+    assert np.array_equal(g["idx"].numpy(), idx)
+    assert_close(g["out"].numpy(), out, f"{label}: out")
+    assert_close(g["y_shared"].numpy(), y_sh, f"{label}: y_shared")
+
+
+@pytest.mark.parametrize("gemv", [1, 0], ids=["gemv", "tiles"])
+def test_wide_scale_range_single_token(gemv):
+    """Block scales spread over 2^-40 .. 2^9 for gate/up and 2^-30 .. 2^-1 for down: more
+    than the f16 range inside one 512-element span, and rows of very different size."""
+    E, k, d, f = 8, 3, 1024, 512
+    rng = np.random.default_rng(21)
+    arrs = {}
+    for name, which, lo, hi in (("gate", synth.GATE, 87, 137), ("up", synth.UP, 87, 137),
+                                ("down", synth.DOWN, 97, 127)):
+        r, K = synth.matrix_shape(which, d, f)
+        arrs[f"{name}_codes"] = rng.integers(0, 256, (E + 1, r, K // 2), dtype=np.uint8)
+        arrs[f"{name}_scales"] = rng.integers(lo, hi, (E + 1, r, K // 32), dtype=np.uint8)
+    bm.set_gemv_max_tokens(gemv)
+    try:
+        _custom_layer_check(1, E, k, d, f, arrs, 31, "wide scales")
+    finally:
+        bm.set_gemv_max_tokens(1)
+
+
+def test_extreme_weights_single_token():
+    """All codes +-6 at scale 2^-3, all zeros, and rows whose 16 scales are 0 (2^-127)."""
+    E, k, d, f = 4, 2, 512, 512
+    rng = np.random.default_rng(4)
+    arrs = {}
+    for name, which in (("gate", synth.GATE), ("up", synth.UP), ("down", synth.DOWN)):
+        r, K = synth.matrix_shape(which, d, f)
+        codes = np.full((E + 1, r, K // 2), 0x77, np.uint8)
+        codes[1] = 0xFF
+        codes[2] = 0x00
+        codes[3] = rng.integers(0, 256, codes[3].shape, dtype=np.uint8)
+        scales = np.full((E + 1, r, K // 32), 124, np.uint8)
+        scales[3] = rng.integers(121, 125, scales[3].shape, dtype=np.uint8)
+        scales[3, ::7] = 0
+        arrs[f"{name}_codes"], arrs[f"{name}_scales"] = codes, scales
+    _custom_layer_check(1, E, k, d, f, arrs, 41, "extreme weights, T=1")
+
+
 def test_device_generator_matches_host_generator():
     seed, layer, E, d, f = 1234, 3, 8, 256, 128
     dev = synth.device_layer_weights(seed, layer, E, d, f)
@@ -197,8 +260,13 @@ def _full_workload(name, tokens):
     return g
 
 
-def test_decode_t1_full():
-    _full_workload("decode_t1", [0])
+@pytest.mark.parametrize("gemv", [1, 0], ids=["gemv", "tiles"])
+def test_decode_t1_full(gemv):
+    bm.set_gemv_max_tokens(gemv)
+    try:
+        _full_workload("decode_t1", [0])
+    finally:
+        bm.set_gemv_max_tokens(1)
 
 
 def test_decode_t64_zipf_sampled():
