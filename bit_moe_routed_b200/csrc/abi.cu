@@ -255,16 +255,21 @@ struct FfnCtx {
 };
 
 // The GEMV path needs whole 512-element stages along d and f, 16-byte aligned scale
-// rows for its bulk copies, every active expert's range within two per CTA
-// (k + 1 <= CTAs), and its shared memory.
+// rows for its TMA boxes, every CTA's range of units within two experts and the
+// kernel's unit bound, and its shared memory.
 bool use_gemv(int T, int k, const moe_weights_t* w, int sms, int max_smem) {
   if (T < 1 || T > g_gemv_max_t.load() || T > kGemvMaxT) return false;
   if (w->d % 512 || w->f % 512) return false;
   if (!aligned(w->gate_scales, 16) || !aligned(w->up_scales, 16) || !aligned(w->down_scales, 16))
     return false;
-  const int ctas = sms < kMaxCtas ? sms : kMaxCtas;
-  if (k + 1 > ctas) return false;
-  return gemv_smem_bytes(w->d) <= (size_t)max_smem && gemv_smem_bytes(w->f) <= (size_t)max_smem;
+  const long long ctas = sms < kMaxCtas ? sms : kMaxCtas;
+  const long long experts = (long long)T * k + 1;  // at most this many active
+  if (experts > ctas) return false;
+  const long long units1 = experts * (w->f / 8), units2 = experts * (w->d / 16);
+  const long long cap = (long long)gemv_max_units_per_cta() * ctas;
+  if (units1 > cap || units2 > cap) return false;
+  return gemv_smem_bytes(1, w->d) <= (size_t)max_smem &&
+         gemv_smem_bytes(2, w->f) <= (size_t)max_smem;
 }
 
 int ffn_check(int T, int k, const moe_weights_t* w, void* ws, size_t ws_bytes, FfnCtx& c) {

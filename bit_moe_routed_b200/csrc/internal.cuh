@@ -109,7 +109,10 @@ struct GemvLaunch {
   bool overlap;
 };
 cudaError_t launch_gemv(int phase, const GemvLaunch& a, cudaStream_t s, int num_sms);
-size_t gemv_smem_bytes(int K);
+size_t gemv_smem_bytes(int phase, int K);
+// a launch's units (8 h-rows in phase 1, 16 down rows in phase 2, of every active
+// expert) are cut into one range per CTA of at most this many units
+int gemv_max_units_per_cta();
 
 // Launch, with `overlap`, as a programmatic dependent launch: the kernel may start while
 // the previous kernel on the stream finishes (every kernel of this library calls

@@ -79,6 +79,14 @@ __device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap
       "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(bar), "l"(policy)
       : "memory");
 }
+__device__ __forceinline__ void tma_load_3d_hint(uint32_t dst, const CUtensorMap* m, int c0, int c1,
+                                                 int c2, uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(c2), "r"(bar), "l"(policy)
+      : "memory");
+}
 // L2 cache policies covering every access they are given to
 __device__ __forceinline__ uint64_t make_policy_evict_first() {
   uint64_t p;
@@ -222,6 +230,17 @@ __device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
   uint32_t d;
   asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
   return d;
+}
+// warp-level D(16x8, fp32) = A(16x16, f16, row) x B(16x8, f16, col), from a zero accumulator
+__device__ __forceinline__ void mma_m16n8k16_f16_zero(float* d, uint32_t a0, uint32_t a1,
+                                                      uint32_t a2, uint32_t a3, uint32_t b0,
+                                                      uint32_t b1) {
+  const float z = 0.0f;
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3},"
+      " {%4, %5, %6, %7}, {%8, %9}, {%10, %10, %10, %10};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(z));
 }
 // warp-level D(16x8, fp32) += A(16x16, f16, row) x B(16x8, f16, col)
 __device__ __forceinline__ void mma_m16n8k16_f16(float* c, uint32_t a0, uint32_t a1, uint32_t a2,
