@@ -243,6 +243,9 @@ int moe_act_quant(const uint16_t* x_bf16, int T, int d, uint8_t* qx, float* sx, 
 
 namespace {
 
+// Set while moe_expert_ffn issues its second and third kernels (see launch_pdl).
+thread_local bool t_overlap = false;
+
 struct FfnCtx {
   DeviceInfo di;
   WorkspaceLayout L;
@@ -312,6 +315,7 @@ GemvLaunch gemv_args(int T, int k, const moe_weights_t* w, const FfnCtx& c) {
   a.P = T * k;
   a.wait_ns = g_wait_ns.load();
   a.status = c.di.status;
+  a.overlap = t_overlap;
   return a;
 }
 
@@ -330,6 +334,7 @@ FfnArgs ffn_args(int phase, int T, int k, const moe_weights_t* w, const FfnCtx& 
   a.partials = reinterpret_cast<float*>(c.ws + c.L.partials);
   a.ncap = ncap_for(T);
   a.l2_hints = 1;  // weight boxes evict-first
+  a.overlap = t_overlap;
   if (phase == 1) {
     a.a0_codes = w->gate_codes;
     a.a0_scales = w->gate_scales;
@@ -428,6 +433,12 @@ int moe_expert_ffn(const uint16_t* x_bf16, int T, int k, const moe_weights_t* w,
                    void* ws, size_t ws_bytes, void* stream) {
   int rc = moe_ffn_prepare(x_bf16, T, k, w, offsets, perm, ws, ws_bytes, stream);
   if (rc) return rc;
+  // gate/up and down follow a kernel of this call on the stream: they may start while it
+  // finishes (their prologue overlaps its tail)
+  struct Overlap {
+    Overlap() { t_overlap = true; }
+    ~Overlap() { t_overlap = false; }
+  } guard;
   rc = moe_ffn_gate_up(T, k, w, ws, ws_bytes, stream);
   if (rc) return rc;
   return moe_ffn_down(T, k, w, y_routed, y_shared, ws, ws_bytes, stream);

@@ -59,7 +59,7 @@ cudaError_t launch_combine(const float* y, const float* ysh, const float* w, con
   int threads = d / 4 < 256 ? d / 4 : 256;
   threads = (threads + 31) / 32 * 32;
   const unsigned slices = (unsigned)((d / 4 + threads - 1) / threads);
-  return launch_pdl(combine_kernel, dim3((unsigned)T, slices), dim3(threads), 0, s, y, ysh, w, pos,
+  return launch_pdl(combine_kernel, dim3((unsigned)T, slices), dim3(threads), 0, s, false, y, ysh, w, pos,
                     T, k, d, out, status);
 }
 

@@ -125,7 +125,7 @@ cudaError_t launch_dispatch(const int32_t* idx, int T, int k, int E, int32_t* co
   cudaError_t err = cudaFuncSetAttribute(dispatch_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  return launch_pdl(dispatch_kernel, dim3(1), dim3(1024), smem, s, idx, T * k, E, counts, offsets,
+  return launch_pdl(dispatch_kernel, dim3(1), dim3(1024), smem, s, false, idx, T * k, E, counts, offsets,
                     perm, pos, status);
 }
 

@@ -690,14 +690,14 @@ bool make_map(CUtensorMap* m, const void* base, bool fp4, int K, long long rows,
 }
 
 template <int PHASE, int NMAX, int STAGES, int NBUF, int MR>
-cudaError_t launch_one(const FfnParams& prm, cudaStream_t s, int grid) {
+cudaError_t launch_one(const FfnParams& prm, cudaStream_t s, int grid, bool overlap) {
   using C = Cfg<PHASE, NMAX, STAGES, NBUF, MR>;
   const size_t smem = C::smem_bytes(prm.E);
   cudaError_t err = cudaFuncSetAttribute(ffn_kernel<PHASE, NMAX, STAGES, NBUF, MR>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   return launch_pdl(ffn_kernel<PHASE, NMAX, STAGES, NBUF, MR>, dim3(grid), dim3(C::kThreads), smem, s,
-                    prm);
+                    overlap, prm);
 }
 
 // (PHASE, NMAX) -> pipeline stages, TMEM partial buffers, weight rows per tile.  Small
@@ -758,7 +758,7 @@ cudaError_t launch_ffn(int phase, int nmax, const FfnArgs& a, cudaStream_t s, in
   prm.l2_hints = a.l2_hints;
   const int grid = num_sms < kMaxCtas ? num_sms : kMaxCtas;
 #define X(P, N, S, B, M) \
-  if (phase == P && nmax == N && mr == M) return launch_one<P, N, S, B, M>(prm, s, grid);
+  if (phase == P && nmax == N && mr == M) return launch_one<P, N, S, B, M>(prm, s, grid, a.overlap);
   BITMOE_FFN_VARIANTS(X)
 #undef X
   return cudaErrorInvalidValue;

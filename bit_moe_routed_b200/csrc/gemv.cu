@@ -441,7 +441,7 @@ cudaError_t launch_gemv(int phase, const GemvLaunch& a, cudaStream_t s, int num_
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int grid = num_sms < kMaxCtas ? num_sms : kMaxCtas;
-  return launch_pdl(kern, dim3(grid), dim3(kGvThreads), smem, s, p);
+  return launch_pdl(kern, dim3(grid), dim3(kGvThreads), smem, s, a.overlap, p);
 }
 
 }  // namespace bitmoe

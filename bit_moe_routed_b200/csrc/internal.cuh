@@ -82,6 +82,7 @@ struct FfnArgs {
   float* partials;           // stream-K partial slots
   int ncap;                  // widest token tile
   int l2_hints;              // bit 0: weight boxes evict-first; bit 1: activation boxes evict-last
+  bool overlap;              // launch as a dependent of the previous kernel (see launch_pdl)
 };
 cudaError_t launch_ffn(int phase, int nmax, const FfnArgs& a, cudaStream_t s, int num_sms);
 // dynamic shared memory of a launch
@@ -105,6 +106,7 @@ struct GemvLaunch {
   int E, d, f, P;
   long long wait_ns;
   int* status;
+  bool overlap;
 };
 cudaError_t launch_gemv(int phase, const GemvLaunch& a, cudaStream_t s, int num_sms);
 size_t gemv_smem_bytes(int phase, int K);
@@ -112,15 +114,14 @@ size_t gemv_smem_bytes(int phase, int K);
 // expert) are cut into one range per CTA of at most this many units
 int gemv_max_units_per_cta();
 
-// Launch as a programmatic dependent launch: when the previous operation on the stream is
-// a kernel that triggers early (every kernel of this library calls
-// griddep_launch_dependents()), this kernel may start while that one finishes.  Every
-// kernel of this library calls griddep_wait() before it reads what earlier work wrote
-// and before it writes anything, so only its set-up overlaps.  After a copy, a host
-// callback or another library's kernel the launch is ordered as usual.
+// Launch, with `overlap`, as a programmatic dependent launch: the kernel may start while
+// the previous kernel on the stream finishes (every kernel of this library calls
+// griddep_wait() before it touches global memory, and griddep_launch_dependents() early).
+// Only valid when the previous operation on the stream is one of this library's kernels:
+// the wait covers prerequisite kernels, not copies or host work queued before them.
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                       cudaStream_t s, Args... args) {
+                       cudaStream_t s, bool overlap, Args... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -130,7 +131,7 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = overlap ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 

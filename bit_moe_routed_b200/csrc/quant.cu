@@ -158,7 +158,7 @@ cudaError_t launch_quant_rows(const uint16_t* x, int T, int k, int d, const int3
   const unsigned blocks = (unsigned)(R + (plan != nullptr ? 1 : 0));
   int threads = (d / 16 + 31) / 32 * 32;  // whole warps
   if (threads > 256) threads = 256;
-  return launch_pdl(quant_rows_kernel, dim3(blocks), dim3(threads), 0, st, x, T, k, d, perm,
+  return launch_pdl(quant_rows_kernel, dim3(blocks), dim3(threads), 0, st, false, x, T, k, d, perm,
                     nrows_routed, q, s, offsets, E, nmax, plan, counters, n_counters, status,
                     plan_mode);
 }
