@@ -1,7 +1,9 @@
 """Failure detection without a GPU fault: the FFN kernels bound every wait by a
 %globaltimer limit.  A 1 ns limit makes the first wait that is not already satisfied run
-out; the kernel must record MOE_ERR_TIMEOUT, release TMEM, drain its copies and return,
-leaving the context usable for the next (normal) call."""
+out; the kernel must record MOE_ERR_TIMEOUT, release TMEM (tile kernels), drain its
+copies and return, leaving the context usable for the next (normal) call.  Both FFN
+implementations are covered: the tile kernels (T = 8) and the single-token GEMV kernels
+(T = 1)."""
 import numpy as np
 import pytest
 import torch
@@ -14,10 +16,13 @@ pytestmark = pytest.mark.gpu
 bm = pytest.importorskip("bit_moe_routed_b200")
 
 
-def test_wait_limit_expiry_is_reported_and_recoverable():
+@pytest.mark.parametrize("T,E,k,d,f", [
+    (8, 16, 2, 512, 256),   # tcgen05 tile kernels
+    (1, 16, 2, 512, 512),   # single-token GEMV kernels
+])
+def test_wait_limit_expiry_is_reported_and_recoverable(T, E, k, d, f):
     if not torch.cuda.is_available():
         pytest.skip("no GPU")
-    T, E, k, d, f = 8, 16, 2, 512, 256
     x = synth.gen_x(T, d, seed=501)
     s = synth.gen_scores_uniform(T, E, seed=502)
     W = device_weights(503, 0, E, d, f)
