@@ -2,8 +2,11 @@
 %globaltimer limit.  A 1 ns limit makes the first wait that is not already satisfied run
 out; the kernel must record MOE_ERR_TIMEOUT, release TMEM (tile kernels), drain its
 copies and return, leaving the context usable for the next (normal) call.  Both FFN
-implementations are covered: the tile kernels (T = 8) and the single-token GEMV kernels
-(T = 1)."""
+implementations run with the tiny limit: the tile kernels (T = 8) and the single-token
+GEMV kernels (T = 1).  The GEMV kernels wait only on their own TMA stages, and one
+try_wait usually outlasts a stage's copy, so a tiny limit may or may not run out there:
+the GEMV test accepts either outcome, but a timeout must be reported and a clean run must
+be correct."""
 import numpy as np
 import pytest
 import torch
@@ -16,13 +19,10 @@ pytestmark = pytest.mark.gpu
 bm = pytest.importorskip("bit_moe_routed_b200")
 
 
-@pytest.mark.parametrize("T,E,k,d,f", [
-    (8, 16, 2, 512, 256),   # tcgen05 tile kernels
-    (1, 16, 2, 512, 512),   # single-token GEMV kernels
-])
-def test_wait_limit_expiry_is_reported_and_recoverable(T, E, k, d, f):
+def test_wait_limit_expiry_is_reported_and_recoverable():
     if not torch.cuda.is_available():
         pytest.skip("no GPU")
+    T, E, k, d, f = 8, 16, 2, 512, 256  # tcgen05 tile kernels
     x = synth.gen_x(T, d, seed=501)
     s = synth.gen_scores_uniform(T, E, seed=502)
     W = device_weights(503, 0, E, d, f)
@@ -38,3 +38,30 @@ def test_wait_limit_expiry_is_reported_and_recoverable(T, E, k, d, f):
     bm.sync_status()  # the status word was cleared by the report
     g = gpu_layer(x, s, k, W)
     check_layer(g, x, s, k, E, d, f, 503, 0, list(range(T)), "after timeout")
+
+
+def test_gemv_tiny_wait_limit_reports_or_completes():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    T, E, k, d, f = 1, 64, 6, 4096, 2048  # single-token GEMV kernels, decode-sized rows
+    x = synth.gen_x(T, d, seed=511)
+    s = synth.gen_scores_uniform(T, E, seed=512)
+    W = device_weights(513, 0, E, d, f)
+    bm.sync_status()
+    bm.set_wait_limit_ns(1)
+    try:
+        r = bm.forward(x.cuda(), s.cuda(), k, W)
+        try:
+            bm.sync_status()
+            timed_out = False
+        except bm.MoeError as e:
+            assert e.code == bm.MOE_ERR_TIMEOUT
+            timed_out = True
+        g = {kk: v.cpu() for kk, v in r.items()}
+    finally:
+        bm.set_wait_limit_ns(0)
+    if not timed_out:
+        check_layer(g, x, s, k, E, d, f, 513, 0, [0], "tiny limit, no timeout")
+    bm.sync_status()
+    g = gpu_layer(x, s, k, W)
+    check_layer(g, x, s, k, E, d, f, 513, 0, [0], "after the tiny limit")
