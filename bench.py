@@ -269,22 +269,29 @@ def run_gpu(args, w):
         bm.sync_status(stream)
         works.append(layer_work(w, counts.cpu().numpy()))
     work = works[0]
-    g_step, g_gu = [], []
+    g_step = []
     for L in layers:
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             step(L)
         g_step.append(g)
-        # event-record nodes inside the graph bracket the kernel itself, without the
-        # graph's launch latency
-        ev = (torch.cuda.Event(enable_timing=True, external=True),
-              torch.cuda.Event(enable_timing=True, external=True))
-        g2 = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g2, stream=stream):
-            ev[0].record(stream)
+
+    # The dominant kernel's own duration: graph A runs route, dispatch, prepare and gate/up
+    # for every layer in turn, graph B the same without gate/up; gate/up per launch is
+    # (A - B) / layers.  Launch latencies cancel, and every gate/up meets its weights cold.
+    def pre(L):
+        idx, _ = bm.route_topk(L["scores"], k, stream)
+        _, offsets, perm, _ = bm.dispatch(idx, E, stream)
+        bm.ffn_prepare(L["x"], k, L["W"], offsets, perm, ws, stream)
+
+    g_a, g_b = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_a, stream=stream):
+        for L in layers:
+            pre(L)
             bm.ffn_gate_up(T, k, L["W"], ws, stream)
-            ev[1].record(stream)
-        g_gu.append((g2, L, ev))
+    with torch.cuda.graph(g_b, stream=stream):
+        for L in layers:
+            pre(L)
     torch.cuda.synchronize()
 
     for i in range(args.warmup):
@@ -300,24 +307,28 @@ def run_gpu(args, w):
     time.sleep(0.3)
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    gu_ms = []
     with torch.cuda.stream(stream):
         for i in range(args.steps):
             starts[i].record(stream)
             g_step[i % n_layers].replay()
             ends[i].record(stream)
-        # the dominant kernel timed alone: gate/up of layer i % L, after that layer's
-        # prepare (untimed) so its inputs are in place, same stream
-        for i in range(args.steps):
-            gg, L, ev = g_gu[i % n_layers]
-            idx, gw = bm.route_topk(L["scores"], k, stream)
-            _, offsets, perm, _ = bm.dispatch(idx, E, stream)
-            bm.ffn_prepare(L["x"], k, L["W"], offsets, perm, ws, stream)
-            gg.replay()
-            ev[1].synchronize()
-            gu_ms.append(ev[0].elapsed_time(ev[1]))
+        # the dominant kernel: graphs A and B alternately (a sleep first, so that the timed
+        # region does not start before the host has queued the graph)
+        ab = {"a": [], "b": []}
+        for i in range(max(15, args.steps)):
+            for name, gr in (("a", g_a), ("b", g_b)):
+                torch.cuda._sleep(100000)
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                gr.replay()
+                e1.record(stream)
+                ab[name].append((e0, e1))
     torch.cuda.synchronize()
     clk = clocks.stop()
+    ta = statistics.median(e0.elapsed_time(e1) for e0, e1 in ab["a"])
+    tb = statistics.median(e0.elapsed_time(e1) for e0, e1 in ab["b"])
+    gu_ms = [(ta - tb) / n_layers]
     step_ms = [starts[i].elapsed_time(ends[i]) for i in range(args.steps)]
     total_s = max_over_ranks(sum(step_ms) / 1000.0, dist, dev)
     if dist is not None:
@@ -413,7 +424,7 @@ def run_gpu(args, w):
         }
         print(json.dumps(line), flush=True)
     if dist is not None:
-        del g_step, g_gu
+        del g_step, g_a, g_b
         dist.barrier()
         dist.destroy_process_group()
 
