@@ -62,15 +62,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
 }
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* m, int c0, int c1,
-                                            uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(bar)
-      : "memory");
-}
-// the same load with an L2 eviction-priority policy (from make_policy_*)
+// tiled TMA loads (2-D, 3-D) into shared memory, completing as transaction bytes on an
+// mbarrier, with an L2 eviction-priority policy (from make_policy_*)
 __device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap* m, int c0, int c1,
                                                  uint32_t bar, uint64_t policy) {
   asm volatile(
@@ -102,16 +95,6 @@ __device__ __forceinline__ uint64_t make_policy_evict_normal() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
   return p;
-}
-// 1-D bulk copy global -> shared (sizes and both addresses multiples of 16 bytes),
-// completing as transaction bytes on an mbarrier, with an L2 eviction-priority policy
-__device__ __forceinline__ void bulk_load_hint(uint32_t dst, const void* src, uint32_t bytes,
-                                               uint32_t bar, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1], %2, [%3], %4;" ::"r"(dst),
-      "l"(src), "r"(bytes), "r"(bar), "l"(policy)
-      : "memory");
 }
 __device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
@@ -225,11 +208,6 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2_f16x2(uint16_t v) {
   uint32_t r;
   asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
   return r;
-}
-__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
 }
 // warp-level D(16x8, fp32) = A(16x16, f16, row) x B(16x8, f16, col), from a zero accumulator
 __device__ __forceinline__ void mma_m16n8k16_f16_zero(float* d, uint32_t a0, uint32_t a1,
