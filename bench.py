@@ -371,7 +371,7 @@ def run_gpu(args, w):
     # single-token batches run the FP4 GEMV kernels (the library's default switch)
     gemv = T == 1 and d % 512 == 0 and f % 512 == 0
     kernel_file = os.path.join(ROOT, "bit_moe_routed_b200", "csrc", "gemv.cu" if gemv else "ffn.cu")
-    kernel_name = ("ffn gate/up (FP4 GEMV: bulk-copy stages, in-register e2m1 decode, "
+    kernel_name = ("ffn gate/up (FP4 GEMV: TMA-staged rows, in-register e2m1 decode, "
                    "mma.sync f16 -> fp32)") if gemv else "ffn gate/up (tcgen05 kind::mxf8f6f4)"
     traffic = kernel_traffic(kernel_file, "gate_up", w.name)
     if is_prefill:
