@@ -9,8 +9,8 @@
 // the tensor core itself: TMA unpacks the FP4 codes into byte containers in shared
 // memory and the MMA applies the ue8m0 block scales from TMEM.
 //
-// Tiles ("swap-AB"): a tile is (expert e, 128-row block of the weight matrix, token
-// tile of n <= NMAX rows).  The weight rows are the MMA's M = 128; the tokens are its N
+// Tiles ("swap-AB"): a tile is (expert e, block of 128 or 256 weight rows, token tile of
+// n <= NMAX rows).  The weight rows are the MMA's M (128 per MMA); the tokens are its N
 // (n rounded up to 16), so ragged expert groups waste at most 15 columns.  Phase 1
 // multiplies the gate AND up rows of the same 128 h-rows with one shared activation
 // tile, then computes h = silu(g) * u and re-quantises it per 128-block to e4m3;
@@ -33,14 +33,15 @@
 // L2: a layer's weights stream through once; the TMA loads mark them evict-first so the
 // activation rows, which every weight block of an expert reads again, stay in L2.
 //
-// Warp roles (384 threads, one CTA per SM, persistent):
+// Warp roles (32 * (10 + issuers) threads, one CTA per SM, persistent):
 //   warp 0   : TMA producer (weights, activations)
 //   warp 1   : TMEM allocator; lane 0 issues tcgen05.cp / tcgen05.mma / commits for the
-//              gate (phase 1) or down (phase 2) matrix
+//              first (matrix, 128-row block) of a tile
 //   warps 2-9: epilogue; warp w reads TMEM lanes 32*(w%4).., column half (w-2)/4
 //   warp 10  : scale loader: the weights' ue8m0 bytes (cp.async gather into the
 //              tcgen05.cp layout) and the tokens' fp32 activation scales of each chunk
-//   warp 11  : lane 0 issues the up matrix's tcgen05.cp / tcgen05.mma (phase 1)
+//   warps 11+: lane 0 issues for each further (matrix, 128-row block): the up matrix in
+//              phase 1, the second 128-row block of 256-row tiles
 // Every wait is bounded by a %globaltimer limit; on expiry the kernel records a
 // timeout in the status word, lets in-flight copies and MMAs land, frees TMEM and
 // returns.
