@@ -176,6 +176,29 @@ def oracle_sample(w, x, scores, seconds: float, layer_seed: int):
         f"FFN, combine), {elapsed:.1f} s of oracle time on {cores} threads"
 
 
+def oracle_extras(w, x, scores, layer_seed: int) -> dict:
+    """The oracle's routing + dispatch time for the whole batch, and one token's time on a
+    single thread (weights prepared beforehand, untimed)."""
+    import oracle
+    s_np = scores.numpy()
+    ta = time.perf_counter()
+    idx, gw = oracle.route_topk(s_np, w.k)
+    oracle.dispatch(idx, w.E)
+    route_s = time.perf_counter() - ta
+    need = set(idx[0].tolist()) | {w.E}
+    experts = {e: synth.host_expert(layer_seed, 0, e, w.d, w.f) for e in need}
+    cores = os.cpu_count() or 1
+    oracle.set_threads(1)
+    try:
+        ta = time.perf_counter()
+        oracle.moe_tokens(x, w.E, w.k, w.d, w.f, experts, idx, gw, [0])
+        one_s = time.perf_counter() - ta
+    finally:
+        oracle.set_threads(cores)
+    return {"route_dispatch_ms": 1000.0 * route_s,
+            "single_thread_tokens_per_s": 1.0 / one_s}
+
+
 def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -404,6 +427,8 @@ def run_gpu(args, w):
         oracle.build()
         rate, cores, desc = oracle_sample(w, x_cpu, s_cpu, args.cpu_seconds, w.seed(0))
         cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc}
+        if T <= 64:  # one token single-threaded is seconds at these sizes
+            cpu.update(oracle_extras(w, x_cpu, s_cpu, w.seed(0)))
 
     if rank == 0:
         layer_s = total_s / args.steps
