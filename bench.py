@@ -6,11 +6,17 @@
 One step = one pass of the whole layer over one batch of synthetic tokens, with the
 layer's weights resident in HBM.  Default workload: one decode layer, T=1 token,
 256 routed experts + 1 shared, top-6, d=4096, f=2048 (FP4 e2m1 weights, e4m3
-activations).  Each step is one layer; the steps rotate over several resident layers,
-each with its own weights and tokens, so that a step never finds its weights in L2 from
-before (inputs larger than L2).  Each layer's step is captured once in a CUDA graph and
-replayed.  Multi-GPU runs are replicas
-(each rank its own tokens and weights, no collective on the data path) -> weak scaling.
+activations).  The steps rotate over several resident layers, each with its own weights
+and tokens, so that a step never finds its weights in L2 from before (inputs larger than
+L2).  The K timed steps are captured back to back in one CUDA graph (as a model runs its
+layers) and timed with CUDA events; a second figure times each step as its own graph
+replay.  Multi-GPU runs are replicas (each rank its own tokens and weights, no collective
+on the data path) -> weak scaling.
+
+At one GPU the line also carries a `workloads` record: the batched-decode (T=64, Zipf 1.0),
+prefill (T=4096, uniform and Zipf 1.2) and 43-resident-layer (T=1 and T=32, Zipf 1.0)
+configurations, each with its step time, the dominant kernel's roofline, the layer-level
+fraction and an oracle sample; and `peaks`, the dense FP8 tensor rate measured on this GPU.
 
 Prints one JSON line (rank 0).  `--impl reference` times the oracle (the plain CPU
 implementation the tests check against) on the host cores instead.
@@ -38,6 +44,11 @@ import synth  # noqa: E402
 METRIC = "MoE-layer tokens/s; decode HBM GB/s and prefill TFLOPS as % of B200 peak"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
+SPEC_HBM_GBS = 8000.0          # B200 HBM3e, spec
+SPEC_FP8_TFLOPS = 4500.0       # B200 dense FP8, spec
+L2_BYTES = 126 * 2 ** 20
+EXTRA_WORKLOADS = ("decode_t64_zipf", "prefill_t4096_uniform", "prefill_t4096_zipf",
+                   "layers43_t1", "layers43_t32")
 
 
 def load_peaks():
@@ -152,6 +163,78 @@ def replica_seed(w, rank: int) -> int:
     return w.seed(0) + 100000 * rank
 
 
+def time_graph(g, stream, reps: int) -> list:
+    """Durations (ms) of `reps` replays of a CUDA graph, each after a short device sleep so
+    that the timed region does not start before the host has queued the replay."""
+    out = []
+    with torch.cuda.stream(stream):
+        for _ in range(reps):
+            torch.cuda._sleep(100000)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+            out.append((e0, e1))
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in out]
+
+
+# ------------------------------------------------------------------------ measured peaks
+def measure_fp8_peak(dev) -> dict:
+    """Dense FP8 (e4m3 x e4m3 -> bf16) GEMM rate of this GPU through torch._scaled_mm on
+    8192^3: with one scale per tensor, and block-scaled (one e8m0 scale per 32 elements
+    along K, the MX format) where the build supports it.  Timed alone (burst) with CUDA
+    events, median of 20 after 5 warm-ups."""
+    M = N = K = 8192
+    res = {"how": "torch._scaled_mm e4m3 x e4m3 -> bf16, 8192^3, CUDA events, median of 20"}
+    a = torch.randn(M, K, device=dev).to(torch.float8_e4m3fn)
+    b = torch.randn(N, K, device=dev).to(torch.float8_e4m3fn).t()
+    one = torch.tensor(1.0, device=dev)
+
+    def timed(fn):
+        for _ in range(5):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(20):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            ts.append((e0, e1))
+        torch.cuda.synchronize()
+        ms = statistics.median(x.elapsed_time(y) for x, y in ts)
+        return 2.0 * M * N * K / (ms * 1e-3) / 1e12
+
+    try:
+        res["fp8_tensorwise_tflops"] = timed(
+            lambda: torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16))
+    except Exception as e:  # noqa: BLE001 - recorded, not fatal
+        res["fp8_tensorwise_error"] = f"{type(e).__name__}: {str(e)[:160]}"
+    try:
+        e8 = torch.float8_e8m0fnu
+        sa = torch.full((M, K // 32), 127, dtype=torch.uint8, device=dev).view(e8)
+        sb = torch.full((N, K // 32), 127, dtype=torch.uint8, device=dev).view(e8)
+        res["mxfp8_tflops"] = timed(
+            lambda: torch._scaled_mm(a, b, scale_a=sa, scale_b=sb, out_dtype=torch.bfloat16))
+    except Exception as e:  # noqa: BLE001
+        res["mxfp8_error"] = f"{type(e).__name__}: {str(e)[:160]}"
+    del a, b
+    torch.cuda.empty_cache()
+    return res
+
+
+def fp8_peak_of(peaks: dict, bf16_peak: float):
+    if peaks.get("mxfp8_tflops"):
+        return peaks["mxfp8_tflops"], "measured dense MX block-scaled FP8 (torch._scaled_mm)"
+    if peaks.get("fp8_tensorwise_tflops"):
+        return peaks["fp8_tensorwise_tflops"], "measured dense FP8, one scale per tensor " \
+                                               "(torch._scaled_mm)"
+    return 2.0 * bf16_peak, "2 x bf16 burst (nominal fp8/bf16 ratio; FP8 not measurable)"
+
+
 # ------------------------------------------------------------------------ CPU oracle leg
 def oracle_sample(w, x, scores, seconds: float, layer_seed: int):
     """Time the oracle on whole tokens of this workload for about `seconds` seconds.
@@ -199,6 +282,16 @@ def oracle_extras(w, x, scores, layer_seed: int) -> dict:
             "single_thread_tokens_per_s": 1.0 / one_s}
 
 
+def cpu_baseline(w, x, scores, seconds, extras=False):
+    import oracle
+    oracle.build()
+    rate, cores, desc = oracle_sample(w, x, scores, seconds, w.seed(0))
+    cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc}
+    if extras:
+        cpu.update(oracle_extras(w, x, scores, w.seed(0)))
+    return cpu
+
+
 def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -234,6 +327,234 @@ def run_reference(args, w):
 
 
 # ------------------------------------------------------------------------ GPU leg
+class Layers:
+    """L resident layers of a workload on one device, each with its own weights and tokens."""
+
+    def __init__(self, bm, w, n_layers, rank, dev):
+        T, k, E, d, f = w.T, w.k, w.E, w.d, w.f
+        self.w = w
+        self.items = []
+        for l in range(n_layers):
+            seed = replica_seed(w, rank) + l if w.layers == 1 else w.seed(l)
+            if rank == 0 or w.layers > 1:
+                x_cpu, s_cpu = synth.gen_layer_inputs(w, l)
+            else:
+                x_cpu = synth.gen_x(T, d, seed)
+                s_cpu = synth.gen_scores_uniform(T, E, seed) if w.routing == "uniform" else \
+                    synth.gen_scores_zipf(T, E, w.zipf_s, seed)
+            W = bm.LayerWeights.from_dict(synth.device_layer_weights(w.seed(l), l, E, d, f))
+            self.items.append(dict(x_cpu=x_cpu, s_cpu=s_cpu, W=W, x=x_cpu.to(dev),
+                                   scores=s_cpu.to(dev)))
+        self.ws = bm.alloc_workspace(T, k, E, d, f, dev)
+        self.y = torch.empty((max(T * k, 1), d), dtype=torch.float32, device=dev)
+        self.ysh = torch.empty((T, d), dtype=torch.float32, device=dev)
+        self.out = torch.empty((T, d), dtype=torch.float32, device=dev)
+
+
+def resident_layers(w, max_layers):
+    """Layers to rotate through so that a step's weights have been evicted from L2 by the
+    other layers' since their last use (four times the L2 in between)."""
+    if w.layers > 1:
+        return w.layers
+    per_expert = synth.expert_bytes(w.d, w.f)
+    step_bytes = (min(w.E, w.T * w.k) + 1) * per_expert
+    return max(min(2, max_layers), min(max_layers, -(-4 * L2_BYTES // step_bytes) + 1))
+
+
+def measure(bm, w, args, dev, stream, rank, dist, steps, warmup, peaks, cpu_seconds,
+            headline=False):
+    """Time one workload; returns the record (and the layers, for the e2e leg)."""
+    T, k, E, d, f = w.T, w.k, w.E, w.d, w.f
+    n_layers = resident_layers(w, args.max_layers)
+    if w.layers > 1:
+        steps = w.layers * max(1, steps // w.layers)  # whole passes over the resident layers
+    Ls = Layers(bm, w, n_layers, rank, dev)
+
+    def step(L):
+        idx, gw = bm.route_topk(L["scores"], k, stream)
+        counts, offsets, perm, pos = bm.dispatch(idx, E, stream)
+        bm.expert_ffn(L["x"], k, L["W"], offsets, perm, Ls.ws, out=(Ls.y, Ls.ysh),
+                      stream=stream)
+        bm.combine(Ls.y, Ls.ysh, gw, pos, Ls.out, stream)
+        return counts
+
+    # one eager pass per layer (checks the status word and gives the routing counts)
+    works = []
+    for L in Ls.items:
+        with torch.cuda.stream(stream):
+            counts = step(L)
+        bm.sync_status(stream)
+        works.append(layer_work(w, counts.cpu().numpy()))
+    work = {key: sum(wk[key] for wk in works) / len(works) for key in works[0]}
+
+    # the K timed steps back to back in one graph (step i runs layer i % L), a graph of the
+    # warm-up steps, and one graph per layer for the isolated per-step figure
+    def chain(n):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(n):
+                step(Ls.items[i % n_layers])
+        return g
+
+    g_warm, g_timed = chain(warmup), chain(steps)
+    g_one = []
+    for L in Ls.items[:min(n_layers, 8)]:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step(L)
+        g_one.append(g)
+
+    # the dominant kernel's own duration: graph A runs route, dispatch, prepare and gate/up
+    # for every layer in turn, graph B the same without gate/up; gate/up per launch is
+    # (A - B) / layers.  Launch latencies cancel, and every gate/up meets its weights cold.
+    def pre(L):
+        idx, _ = bm.route_topk(L["scores"], k, stream)
+        _, offsets, perm, _ = bm.dispatch(idx, E, stream)
+        bm.ffn_prepare(L["x"], k, L["W"], offsets, perm, Ls.ws, stream)
+
+    g_a, g_b = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_a, stream=stream):
+        for L in Ls.items:
+            pre(L)
+            bm.ffn_gate_up(T, k, L["W"], Ls.ws, stream)
+    with torch.cuda.graph(g_b, stream=stream):
+        for L in Ls.items:
+            pre(L)
+    torch.cuda.synchronize()
+
+    with torch.cuda.stream(stream):
+        g_warm.replay()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+    clocks = None
+    if headline:
+        clocks = ClockSampler(int(str(dev).split(":")[-1]) if ":" in str(dev) else 0)
+        clocks.start()
+        time.sleep(0.3)
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(100000)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g_timed.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    timed_ms = e0.elapsed_time(e1)
+    one_ms = []
+    for i in range(max(len(g_one), 10)):
+        one_ms += time_graph(g_one[i % len(g_one)], stream, 1)
+    ab = {"a": [], "b": []}
+    for _ in range(max(7, min(15, steps))):
+        ab["a"] += time_graph(g_a, stream, 1)
+        ab["b"] += time_graph(g_b, stream, 1)
+    clk = clocks.stop() if clocks is not None else None
+    total_s = max_over_ranks(timed_ms / 1000.0, dist, dev)
+    world = dist.get_world_size() if dist is not None else 1
+    layer_s = total_s / steps
+    gu_s = (statistics.median(ab["a"]) - statistics.median(ab["b"])) / n_layers / 1000.0
+    is_prefill = T > 256
+    gemv = T == 1 and d % 512 == 0 and f % 512 == 0
+    kernel_file = os.path.join(ROOT, "bit_moe_routed_b200", "csrc", "gemv.cu" if gemv else "ffn.cu")
+    kernel_name = ("ffn gate/up (FP4 GEMV: TMA-staged rows, in-register e2m1 decode, "
+                   "mma.sync f16 -> fp32)") if gemv else "ffn gate/up (tcgen05 kind::mxf8f6f4)"
+    traffic = kernel_traffic(kernel_file, "gate_up", w.name)
+    hbm_peak, fp8_peak, fp8_src, peak_kind = peaks
+    if is_prefill:
+        achieved = work["flops_gu"] / gu_s / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
+                "frac": achieved / fp8_peak, "traffic": traffic, "kernel": kernel_name,
+                "peak_source": fp8_src}
+        layer_tf = (work["flops_gu"] + work["flops_dn"]) / layer_s / 1e12
+        layer = {"tflops": layer_tf, "frac_of_measured_fp8": layer_tf / fp8_peak,
+                 "frac_of_spec_fp8_4500": layer_tf / SPEC_FP8_TFLOPS,
+                 "weight_gb_per_s": work["weight_bytes"] / layer_s / 1e9}
+    else:
+        achieved = work["gu_bytes"] / gu_s / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved / hbm_peak, "traffic": traffic, "kernel": kernel_name,
+                "peak_source": f"{peak_kind} HBM copy"}
+        gbs = work["weight_bytes"] / layer_s / 1e9
+        layer = {"weight_gb_per_s": gbs, "weight_bytes": work["weight_bytes"],
+                 "frac_of_measured_hbm": gbs / hbm_peak, "frac_of_spec_hbm_8tbs": gbs / SPEC_HBM_GBS,
+                 "tflops": (work["flops_gu"] + work["flops_dn"]) / layer_s / 1e12}
+    roof["avg_launch_us"] = gu_s * 1e6
+    roof["algorithmic_per_launch"] = work["flops_gu"] if is_prefill else work["gu_bytes"]
+    rec = {
+        "value": world * T * steps / total_s, "unit": "tokens/s", "steps": steps,
+        "ms_per_step": 1000.0 * layer_s,
+        "ms_per_step_isolated": statistics.median(one_ms),
+        "config": {"workload": w.name, "T": T, "E": E, "k": k, "d": d, "f": f,
+                   "routing": w.routing, "zipf_s": w.zipf_s if w.routing == "zipf" else None,
+                   "active_experts": work["active"], "resident_layers": n_layers},
+        "layer": layer, "roofline": roof,
+    }
+    if clk is not None:
+        rec["clocks"] = clk
+    if rank == 0 and world == 1 and cpu_seconds > 0:
+        x_cpu, s_cpu = Ls.items[0]["x_cpu"], Ls.items[0]["s_cpu"]
+        rec["cpu_baseline"] = cpu_baseline(w, x_cpu, s_cpu, cpu_seconds, extras=T <= 64 and headline)
+    del g_warm, g_timed, g_one, g_a, g_b
+    return rec, Ls, step
+
+
+def e2e(bm, Ls, args, dev, stream, dist, world):
+    """The same metric through the public API with host buffers: each step copies x and the
+    scores from pinned host memory, runs the four calls and copies the output back, then
+    synchronises (a decode loop needs each output before its next input).  Measured as one
+    CUDA graph per layer, and eagerly (the four calls issued from Python each step)."""
+    w = Ls.w
+    T, k, d, E = w.T, w.k, w.d, w.E
+    for L in Ls.items:
+        L["x_h"] = L["x_cpu"].pin_memory()
+        L["s_h"] = L["s_cpu"].pin_memory()
+    out_h = torch.empty((T, d), dtype=torch.float32).pin_memory()
+
+    def body(L):
+        L["x"].copy_(L["x_h"], non_blocking=True)
+        L["scores"].copy_(L["s_h"], non_blocking=True)
+        r = bm.forward(L["x"], L["scores"], k, L["W"], Ls.ws, stream)
+        out_h.copy_(r["out"], non_blocking=True)
+
+    g_e2e = []
+    for L in Ls.items:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            body(L)
+        g_e2e.append(g)
+    torch.cuda.synchronize()
+    res = {}
+    for mode in ("graph", "eager"):
+        ms = []
+        for i in range(args.warmup + args.steps):
+            torch.cuda.synchronize()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                a.record(stream)
+                if mode == "graph":
+                    g_e2e[i % len(g_e2e)].replay()
+                else:
+                    body(Ls.items[i % len(Ls.items)])
+                b.record(stream)
+            b.synchronize()
+            if i >= args.warmup:
+                ms.append(a.elapsed_time(b))
+        s = max_over_ranks(sum(ms) / 1000.0, dist, dev)
+        res[mode] = world * T * args.steps / s
+    bm.sync_status(stream)
+    del g_e2e
+    return {"value": res["graph"], "unit": "tokens/s",
+            "h2d_bytes_per_step": T * d * 2 + T * E * 4, "d2h_bytes_per_step": T * d * 4,
+            "how": "per layer one CUDA graph of the pinned H2D copies of x and scores, the four "
+                   "calls and the D2H copy of out; synchronised every step",
+            "eager_value": res["eager"],
+            "eager_how": "the same copies and the four calls issued from Python (ctypes) every "
+                         "step, no graph: includes the host's launch costs"}
+
+
 def run_gpu(args, w):
     import bit_moe_routed_b200 as bm
     rank = int(os.environ.get("RANK", "0"))
@@ -246,220 +567,63 @@ def run_gpu(args, w):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     dev = torch.device("cuda", local)
-    hbm_peak, bf16_peak, bf16_sus, peak_kind = load_peaks()
-
-    # Working set: L layers resident in HBM, each with its own weights and tokens; step i
-    # runs layer i % L.  L is chosen so the other L-1 layers' weights exceed four times
-    # the L2, so a step's weights are never still in L2 from its previous use (read-only
-    # weights: no dirty lines to write back, unlike a write-flush).
-    T, k, E, d, f = w.T, w.k, w.E, w.d, w.f
-    per_expert = synth.expert_bytes(d, f)
-    est_active = min(E, T * k) + 1
-    step_bytes = est_active * per_expert
-    L2_BYTES = 126 * 2 ** 20
-    n_layers = max(min(2, args.max_layers), min(args.max_layers, -(-4 * L2_BYTES // step_bytes) + 1))
-    layers = []
-    for l in range(n_layers):
-        seed = replica_seed(w, rank) + l
-        if rank == 0:
-            x_cpu, s_cpu = synth.gen_layer_inputs(w, l)
-        else:
-            x_cpu = synth.gen_x(T, d, seed)
-            s_cpu = synth.gen_scores_uniform(T, E, seed) if w.routing == "uniform" else \
-                synth.gen_scores_zipf(T, E, w.zipf_s, seed)
-        W = bm.LayerWeights.from_dict(synth.device_layer_weights(w.seed(l), l, E, d, f))
-        layers.append(dict(x_cpu=x_cpu, s_cpu=s_cpu, W=W, x=x_cpu.to(dev), scores=s_cpu.to(dev)))
-    ws = bm.alloc_workspace(T, k, E, d, f, dev)
-    y = torch.empty((T * k, d), dtype=torch.float32, device=dev)
-    ysh = torch.empty((T, d), dtype=torch.float32, device=dev)
-    out = torch.empty((T, d), dtype=torch.float32, device=dev)
     stream = torch.cuda.Stream(dev)
+    hbm_peak, bf16_peak, bf16_sus, peak_kind = load_peaks()
+    fp8 = measure_fp8_peak(dev) if world == 1 and not args.no_workloads else {}
+    fp8_peak, fp8_src = fp8_peak_of(fp8, bf16_peak)
+    peaks = (hbm_peak, fp8_peak, fp8_src, peak_kind)
 
-    def step(L):
-        # route -> dispatch -> FFN (prepare | gate/up | down) -> combine
-        idx, gw = bm.route_topk(L["scores"], k, stream)
-        counts, offsets, perm, pos = bm.dispatch(idx, E, stream)
-        bm.expert_ffn(L["x"], k, L["W"], offsets, perm, ws, out=(y, ysh), stream=stream)
-        bm.combine(y, ysh, gw, pos, out, stream)
-        return counts
+    rec, Ls, _ = measure(bm, w, args, dev, stream, rank, dist, args.steps, args.warmup, peaks,
+                         0 if args.no_cpu_baseline else args.cpu_seconds, headline=True)
+    e2e_rec = e2e(bm, Ls, args, dev, stream, dist, world)
+    del Ls
+    torch.cuda.empty_cache()
 
-    # one eager pass per layer (checks the status word), then one graph per layer of the
-    # whole step, and one of the gate/up kernel alone (after its own prepare) per layer
-    works = []
-    for L in layers:
-        with torch.cuda.stream(stream):
-            counts = step(L)
-        bm.sync_status(stream)
-        works.append(layer_work(w, counts.cpu().numpy()))
-    work = works[0]
-    g_step = []
-    for L in layers:
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            step(L)
-        g_step.append(g)
-
-    # The dominant kernel's own duration: graph A runs route, dispatch, prepare and gate/up
-    # for every layer in turn, graph B the same without gate/up; gate/up per launch is
-    # (A - B) / layers.  Launch latencies cancel, and every gate/up meets its weights cold.
-    def pre(L):
-        idx, _ = bm.route_topk(L["scores"], k, stream)
-        _, offsets, perm, _ = bm.dispatch(idx, E, stream)
-        bm.ffn_prepare(L["x"], k, L["W"], offsets, perm, ws, stream)
-
-    g_a, g_b = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_a, stream=stream):
-        for L in layers:
-            pre(L)
-            bm.ffn_gate_up(T, k, L["W"], ws, stream)
-    with torch.cuda.graph(g_b, stream=stream):
-        for L in layers:
-            pre(L)
-    torch.cuda.synchronize()
-
-    for i in range(args.warmup):
-        with torch.cuda.stream(stream):
-            g_step[i % n_layers].replay()
-    torch.cuda.synchronize()
-    if dist is not None:
-        dist.barrier()
-    torch.cuda.synchronize()
-
-    clocks = ClockSampler(local)
-    clocks.start()
-    time.sleep(0.3)
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    with torch.cuda.stream(stream):
-        for i in range(args.steps):
-            starts[i].record(stream)
-            g_step[i % n_layers].replay()
-            ends[i].record(stream)
-        # the dominant kernel: graphs A and B alternately (a sleep first, so that the timed
-        # region does not start before the host has queued the graph)
-        ab = {"a": [], "b": []}
-        for i in range(max(15, args.steps)):
-            for name, gr in (("a", g_a), ("b", g_b)):
-                torch.cuda._sleep(100000)
-                e0 = torch.cuda.Event(enable_timing=True)
-                e1 = torch.cuda.Event(enable_timing=True)
-                e0.record(stream)
-                gr.replay()
-                e1.record(stream)
-                ab[name].append((e0, e1))
-    torch.cuda.synchronize()
-    clk = clocks.stop()
-    ta = statistics.median(e0.elapsed_time(e1) for e0, e1 in ab["a"])
-    tb = statistics.median(e0.elapsed_time(e1) for e0, e1 in ab["b"])
-    gu_ms = [(ta - tb) / n_layers]
-    step_ms = [starts[i].elapsed_time(ends[i]) for i in range(args.steps)]
-    total_s = max_over_ranks(sum(step_ms) / 1000.0, dist, dev)
-    if dist is not None:
-        dist.barrier()
-    value = world * T * args.steps / total_s
-
-    # e2e through the public API with host buffers: per layer one CUDA graph of the pinned
-    # H2D copies of x and scores, the four calls and the D2H copy of the layer output,
-    # replayed for step i (layer i % L) and synchronised before the next step, as a decode
-    # loop that needs each output before its next input would run it
-    for L in layers:
-        L["x_h"] = L["x_cpu"].pin_memory()
-        L["s_h"] = L["s_cpu"].pin_memory()
-    out_h = torch.empty((T, d), dtype=torch.float32).pin_memory()
-    g_e2e = []
-    for L in layers:
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            L["x"].copy_(L["x_h"], non_blocking=True)
-            L["scores"].copy_(L["s_h"], non_blocking=True)
-            r = bm.forward(L["x"], L["scores"], k, L["W"], ws, stream)
-            out_h.copy_(r["out"], non_blocking=True)
-        g_e2e.append(g)
-    torch.cuda.synchronize()
-    e2e_ms = []
-    for i in range(args.warmup + args.steps):
-        torch.cuda.synchronize()
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            a.record(stream)
-            g_e2e[i % n_layers].replay()
-            b.record(stream)
-        b.synchronize()
-        if i >= args.warmup:
-            e2e_ms.append(a.elapsed_time(b))
-    e2e_s = max_over_ranks(sum(e2e_ms) / 1000.0, dist, dev)
-    e2e_value = world * T * args.steps / e2e_s
-    bm.sync_status(stream)
-    x_cpu, s_cpu = layers[0]["x_cpu"], layers[0]["s_cpu"]
-
-    gu_avg_s = statistics.mean(gu_ms) / 1000.0
-    # per-launch algorithmic work averaged over the rotated layers
-    work = dict(work)
-    for key in ("gu_bytes", "dn_bytes", "flops_gu", "flops_dn", "weight_bytes", "active"):
-        work[key] = sum(wk[key] for wk in works) / len(works)
-    is_prefill = T > 256
-    # single-token batches run the FP4 GEMV kernels (the library's default switch)
-    gemv = T == 1 and d % 512 == 0 and f % 512 == 0
-    kernel_file = os.path.join(ROOT, "bit_moe_routed_b200", "csrc", "gemv.cu" if gemv else "ffn.cu")
-    kernel_name = ("ffn gate/up (FP4 GEMV: TMA-staged rows, in-register e2m1 decode, "
-                   "mma.sync f16 -> fp32)") if gemv else "ffn gate/up (tcgen05 kind::mxf8f6f4)"
-    traffic = kernel_traffic(kernel_file, "gate_up", w.name)
-    if is_prefill:
-        fp8_peak = bf16_peak * 2.0  # dense FP8 = 2x dense BF16 (nominal 4.5 / 2.25 PF)
-        achieved = work["flops_gu"] / gu_avg_s / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
-                "frac": achieved / fp8_peak, "traffic": traffic,
-                "kernel": "ffn gate/up (tcgen05 kind::mxf8f6f4)",
-                "peak_source": f"{peak_kind} bf16 burst x 2 (nominal fp8/bf16 ratio)"}
-    else:
-        achieved = work["gu_bytes"] / gu_avg_s / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                "frac": achieved / hbm_peak, "traffic": traffic,
-                "kernel": kernel_name,
-                "peak_source": f"{peak_kind} HBM copy"}
-    roof["avg_launch_us"] = gu_avg_s * 1e6
-    roof["algorithmic_per_launch"] = work["gu_bytes"] if not is_prefill else work["flops_gu"]
-
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        import oracle
-        oracle.build()
-        rate, cores, desc = oracle_sample(w, x_cpu, s_cpu, args.cpu_seconds, w.seed(0))
-        cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc}
-        if T <= 64:  # one token single-threaded is seconds at these sizes
-            cpu.update(oracle_extras(w, x_cpu, s_cpu, w.seed(0)))
+    workloads = {}
+    if world == 1 and not args.no_workloads:
+        names = EXTRA_WORKLOADS if args.workloads == "all" else \
+            [n for n in args.workloads.split(",") if n]
+        for name in names:
+            if name == w.name:
+                continue
+            wl = synth.WORKLOADS[name]
+            need = (wl.layers if wl.layers > 1 else 2) * synth.expert_bytes(wl.d, wl.f) * (wl.E + 1)
+            free, _ = torch.cuda.mem_get_info(dev)
+            if free < need + (6 << 30):
+                workloads[name] = {"skipped": f"needs {need / 1e9:.1f} GB, {free / 1e9:.1f} GB free"}
+                continue
+            r, Lw, _ = measure(bm, wl, args, dev, stream, rank, dist,
+                               args.extra_steps, 3, peaks, args.extra_cpu_seconds)
+            workloads[name] = r
+            del Lw
+            torch.cuda.empty_cache()
 
     if rank == 0:
-        layer_s = total_s / args.steps
         line = {
-            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * layer_s,
+            "metric": METRIC, "value": rec["value"], "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": rec["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "e2m1 x e4m3 -> f32", "data": "synthetic (seeded weights and tokens)",
-            "config": {"workload": w.name, "T": T, "E": E, "k": k, "d": d, "f": f,
-                       "routing": w.routing, "active_experts": work["active"],
-                       "l2": f"not flushed: step i runs layer i % {n_layers}, each with its own "
-                             f"weights ({n_layers * 257 * per_expert / 1e9:.1f} GB resident), so a "
-                             "step's weights were evicted by the other layers since their last use",
-                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "launch": "one CUDA graph of the 6 kernels per layer"},
-            "layer": {"weight_gb_per_s": work["weight_bytes"] / layer_s / 1e9,
-                      "weight_bytes": work["weight_bytes"],
-                      "tflops": (work["flops_gu"] + work["flops_dn"]) / layer_s / 1e12},
-            "roofline": roof,
-            "cpu_baseline": cpu,
-            "e2e": {"value": e2e_value, "unit": "tokens/s",
-                    "h2d_bytes_per_step": T * d * 2 + T * E * 4,
-                    "d2h_bytes_per_step": T * d * 4,
-                    "how": "per layer one CUDA graph of the pinned H2D copies of x and scores, "
-                           "the four calls and the D2H copy of out; synchronised every step"},
+            "config": dict(rec["config"], **{
+                "l2": f"not flushed: step i runs layer i % {rec['config']['resident_layers']}, "
+                      "each with its own weights, so a step's weights were evicted by the other "
+                      "layers since their last use (inputs larger than L2)",
+                "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                "launch": "the K timed steps captured back to back in one CUDA graph"}),
+            "ms_per_step_isolated": rec["ms_per_step_isolated"],
+            "layer": rec["layer"],
+            "roofline": rec["roofline"],
+            "cpu_baseline": rec.get("cpu_baseline"),
+            "e2e": e2e_rec,
             "gpu_launches": 6 * args.steps,
-            "clocks": clk,
+            "clocks": rec.get("clocks"),
+            "peaks": dict(fp8, hbm_gbs=hbm_peak, hbm_source=peak_kind,
+                          fp8_used_tflops=fp8_peak, fp8_used_source=fp8_src,
+                          bf16_burst_tflops=bf16_peak),
+            "workloads": workloads,
         }
         print(json.dumps(line), flush=True)
     if dist is not None:
-        del g_step, g_a, g_b, g_e2e
         dist.barrier()
         dist.destroy_process_group()
 
@@ -475,15 +639,17 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--max-layers", type=int, default=8,
                     help="most layers kept resident to rotate through (defeats L2 reuse)")
+    ap.add_argument("--workloads", default="all",
+                    help="extra workloads to record at one GPU: 'all' or a comma list")
+    ap.add_argument("--no-workloads", action="store_true", help="headline workload only")
+    ap.add_argument("--extra-steps", type=int, default=10)
+    ap.add_argument("--extra-cpu-seconds", type=float, default=4.0)
     ap.add_argument("--ref-seconds", type=float, default=None,
                     help="oracle seconds per step of the reference arm (default: fit ~1 min)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     w = synth.WORKLOADS[args.workload]
-    if w.layers > 1:
-        w = synth.Workload(w.name, w.T, w.E, w.k, w.d, w.f, w.routing, w.zipf_s, 1,
-                           w.config_id, w.draw)
     if args.impl == "reference":
         run_reference(args, w)
     else:

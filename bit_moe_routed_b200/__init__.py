@@ -27,12 +27,13 @@ MOE_ERR_WORKSPACE = -2
 MOE_ERR_CUDA = -3
 MOE_ERR_TIMEOUT = -4
 MOE_ERR_UNSUPPORTED = -5
+MOE_NOALLOC_SCRATCH_BYTES = 24 << 20  # the fixed scratch of moe_expert_ffn_noalloc
 
 EXPORTS = (
     "moe_route_topk", "moe_dispatch", "moe_act_quant", "moe_expert_ffn", "moe_ffn_prepare",
     "moe_ffn_gate_up", "moe_ffn_down", "moe_combine", "moe_workspace_size", "moe_last_error",
     "moe_set_wait_limit_ns", "moe_sync_status", "moe_expert_ffn_noalloc",
-    "moe_set_gemv_max_tokens",
+    "moe_set_gemv_max_tokens", "moe_workspace_offsets", "moe_set_test_stall",
 )
 
 
@@ -80,6 +81,8 @@ def lib():
             "moe_sync_status": [P],
             "moe_expert_ffn_noalloc": [P, I, I, W, P, P, P, P, P],
             "moe_set_gemv_max_tokens": [I],
+            "moe_workspace_offsets": [I, I, I, I, I, P],
+            "moe_set_test_stall": [I],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -150,6 +153,11 @@ def set_wait_limit_ns(n: int) -> None:
     _check(lib().moe_set_wait_limit_ns(int(n)))
 
 
+def set_test_stall(on: bool) -> None:
+    """Testing knob: make the single-token FFN kernels' bounded wait run out (see the header)."""
+    _check(lib().moe_set_test_stall(1 if on else 0))
+
+
 def set_gemv_max_tokens(t: int) -> None:
     """Batches up to t tokens (0 or 1) take the single-token FP4 GEMV path."""
     _check(lib().moe_set_gemv_max_tokens(int(t)))
@@ -161,6 +169,34 @@ def sync_status(stream=None) -> None:
 
 def workspace_size(T: int, k: int, E: int, d: int, f: int) -> int:
     return int(lib().moe_workspace_size(T, k, E, d, f))
+
+
+def workspace_offsets(T: int, k: int, E: int, d: int, f: int) -> dict:
+    """Byte offsets of qx, sx, qh, sh and h inside a workspace for (T, k, E, d, f); h is
+    None when the layout keeps no fp32 hidden state."""
+    off = (ctypes.c_size_t * 5)()
+    _check(lib().moe_workspace_offsets(T, k, E, d, f, off))
+    names = ("qx", "sx", "qh", "sh", "h")
+    return {n: (None if v == ctypes.c_size_t(-1).value else int(v)) for n, v in zip(names, off)}
+
+
+def workspace_views(ws: torch.Tensor, T: int, k: int, E: int, d: int, f: int) -> dict:
+    """Views of the intermediate results moe_expert_ffn leaves in `ws` (rows: routed pairs
+    in expert-sorted order, then the T shared-expert rows)."""
+    o = workspace_offsets(T, k, E, d, f)
+    R = T * k + T
+
+    def view(name, n, dtype):
+        nbytes = n * torch.empty((), dtype=dtype).element_size()
+        return ws[o[name]:o[name] + nbytes].view(dtype)
+
+    out = {"qx": view("qx", R * d, torch.uint8).view(R, d),
+           "sx": view("sx", R * (d // 128), torch.float32).view(R, d // 128),
+           "qh": view("qh", R * f, torch.uint8).view(R, f),
+           "sh": view("sh", R * (f // 128), torch.float32).view(R, f // 128)}
+    if o["h"] is not None:
+        out["h"] = view("h", R * f, torch.float32).view(R, f)
+    return out
 
 
 def alloc_workspace(T: int, k: int, E: int, d: int, f: int, device="cuda") -> torch.Tensor:

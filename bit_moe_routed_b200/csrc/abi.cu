@@ -22,6 +22,7 @@ namespace {
 thread_local std::string t_err;
 std::atomic<long long> g_wait_ns{2000000000LL};
 std::atomic<int> g_gemv_max_t{kGemvMaxT};  // batches up to this size take the GEMV path
+std::atomic<int> g_stall{0};                 // test knob: see moe_set_test_stall
 
 int fail(int code, const char* fmt, ...) {
   char buf[512];
@@ -156,6 +157,11 @@ int moe_set_wait_limit_ns(long long n) {
   return MOE_OK;
 }
 
+int moe_set_test_stall(int on) {
+  g_stall.store(on ? 1 : 0);
+  return MOE_OK;
+}
+
 int moe_set_gemv_max_tokens(int t) {
   if (t < 0) return fail(MOE_ERR_INVALID_ARG, "t=%d < 0", t);
   g_gemv_max_t.store(t);
@@ -165,6 +171,19 @@ int moe_set_gemv_max_tokens(int t) {
 size_t moe_workspace_size(int T, int k, int E, int d, int f) {
   if (T < 0 || k < 1 || E < 1 || d < 128 || f < 128 || d % 128 || f % 128) return 0;
   return workspace_layout(T, k, E, d, f).total;
+}
+
+int moe_workspace_offsets(int T, int k, int E, int d, int f, size_t off[5]) {
+  if (off == nullptr) return fail(MOE_ERR_INVALID_ARG, "off is NULL");
+  if (moe_workspace_size(T, k, E, d, f) == 0)
+    return fail(MOE_ERR_INVALID_ARG, "invalid sizes T=%d k=%d E=%d d=%d f=%d", T, k, E, d, f);
+  const WorkspaceLayout L = workspace_layout(T, k, E, d, f);
+  off[0] = L.qx;
+  off[1] = L.sx;
+  off[2] = L.qh;
+  off[3] = L.sh;
+  off[4] = T <= kGemvMaxT ? L.hbuf : (size_t)-1;
+  return MOE_OK;
 }
 
 int moe_sync_status(void* stream) {
@@ -309,12 +328,15 @@ GemvLaunch gemv_args(int T, int k, const moe_weights_t* w, const FfnCtx& c) {
   a.qx = c.ws + c.L.qx;
   a.sx = reinterpret_cast<const float*>(c.ws + c.L.sx);
   a.hbuf = reinterpret_cast<float*>(c.ws + c.L.hbuf);
+  a.qh = c.ws + c.L.qh;
+  a.sh = reinterpret_cast<float*>(c.ws + c.L.sh);
   a.E = w->E;
   a.d = w->d;
   a.f = w->f;
   a.P = T * k;
   a.wait_ns = g_wait_ns.load();
   a.status = c.di.status;
+  a.stall = g_stall.load();
   a.overlap = t_overlap;
   return a;
 }

@@ -63,9 +63,12 @@ struct GemvParams {
   float* hbuf;               // phase 1 out, phase 2 in: h [slot][f] fp32
   float* y_routed;           // phase 2 out: y rows [T*k][d] (expert-sorted order)
   float* y_shared;           // phase 2 out: the shared expert's row [d]
+  uint8_t* qh;               // phase 2 out: the re-quantised h [row][f] e4m3 and its
+  float* sh;                 //   scales [row][f/128] (row = output row, P for the shared)
   int E, K, rows_per_expert, f, d, P;
   long long wait_ns;
   int* status;
+  int stall;                 // test knob: warp 0 of CTA 0 waits on a barrier nothing completes
 };
 
 // Shared memory (from a 1024-byte aligned base): code rings [warp][stage] (each stage
@@ -90,9 +93,13 @@ struct GvSmem {
   __host__ __device__ static int off_misc(int phase, int K) {
     return off_plan(phase, K) + kGvPlanInts * 4;
   }
-  // misc: abort flag, then (expert, output row) of the range's slots
+  // misc: abort flag, then (expert, output row) of the range's slots, then (8-byte
+  // aligned) the barrier the test stall waits on
+  __host__ __device__ static int off_stall(int phase, int K) {
+    return (off_misc(phase, K) + 32 + 7) / 8 * 8;
+  }
   __host__ __device__ static size_t bytes(int phase, int K) {
-    return (size_t)off_misc(phase, K) + 32 + 1024;
+    return (size_t)off_misc(phase, K) + 48 + 1024;
   }
 };
 
@@ -152,7 +159,11 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_kernel(const __grid_consta
   }
   if (lane == 0)
     for (int s = 0; s < kGvStages; ++s) ptx::mbar_init(full(s), 1);
-  if (threadIdx.x == 0) *abort_flag = 0;
+  const uint32_t stall_bar = ptx::smem_u32(smem + GvSmem::off_stall(PHASE, K));
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    ptx::mbar_init(stall_bar, 1);  // never arrived on: only the test stall waits on it
+  }
   ptx::fence_mbar_init();
 
   // The plan comes from the prepare kernel, the activations of phase 1 too, and phase 2's
@@ -278,6 +289,14 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_kernel(const __grid_consta
       dst[0] = ptx::cvt_e4m3x2_f16x2(q01);
       dst[1] = ptx::cvt_e4m3x2_f16x2(q23);
       if (lane == 0) bs[sl * nb + j] = sc;
+      // the CTA whose range starts the expert's units also stores the codes and scales
+      if ((slot_lo + sl) * upe >= u_lo && slot_info[2 * sl + 1] >= -1) {
+        const int orow = slot_info[2 * sl + 1];
+        const size_t row = orow >= 0 ? (size_t)orow : (size_t)p.P;
+        *reinterpret_cast<uint32_t*>(p.qh + row * K + 128 * j + 4 * lane) =
+            (uint32_t)q01 | ((uint32_t)q23 << 16);
+        if (lane == 0) p.sh[row * nb + j] = sc;
+      }
     }
   }
   __syncthreads();
@@ -287,6 +306,12 @@ __global__ void __launch_bounds__(kGvThreads, 1) gemv_kernel(const __grid_consta
   int q = 0;
   for (; q < total; ++q) {
     const int st = q % kGvStages;
+    // test stall: a wait that no copy completes, so that its time limit runs out
+    if (p.stall && blockIdx.x == 0 && warp == 0 && q == 0 &&
+        !wait_warp(stall_bar, 0, p.wait_ns, abort_flag, p.status)) {
+      ok = false;
+      break;
+    }
     if (!wait_warp(full(st), (uint32_t)(q / kGvStages) & 1u, p.wait_ns, abort_flag, p.status)) {
       ok = false;
       break;
@@ -428,6 +453,8 @@ cudaError_t launch_gemv(int phase, const GemvLaunch& a, cudaStream_t s, int num_
   p.hbuf = a.hbuf;
   p.y_routed = a.y_routed;
   p.y_shared = a.y_shared;
+  p.qh = a.qh;
+  p.sh = a.sh;
   p.E = a.E;
   p.K = K;
   p.rows_per_expert = rpe;
@@ -436,6 +463,7 @@ cudaError_t launch_gemv(int phase, const GemvLaunch& a, cudaStream_t s, int num_
   p.P = a.P;
   p.wait_ns = a.wait_ns;
   p.status = a.status;
+  p.stall = a.stall;
   const size_t smem = GvSmem::bytes(phase, p.K);
   auto kern = phase == 1 ? gemv_kernel<1> : gemv_kernel<2>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -103,9 +103,12 @@ struct GemvLaunch {
   float* hbuf;               // h [active experts][f] fp32
   float* y_routed;
   float* y_shared;
+  uint8_t* qh;               // re-quantised h [row][f] and scales [row][f/128]
+  float* sh;
   int E, d, f, P;
   long long wait_ns;
   int* status;
+  int stall;                 // test knob (moe_set_test_stall)
   bool overlap;
 };
 cudaError_t launch_gemv(int phase, const GemvLaunch& a, cudaStream_t s, int num_sms);

@@ -155,6 +155,21 @@ int moe_combine(const float* y_routed, const float* y_shared, const float* topk_
 /* Bytes of workspace moe_expert_ffn needs (0 on invalid sizes). */
 size_t moe_workspace_size(int T, int k, int E, int d, int f);
 
+/* Where moe_expert_ffn leaves its intermediate results inside a workspace laid out for
+ * (T, k, E, d, f): byte offsets from the workspace start, for tests and tools that
+ * inspect them.  The pages have no counterpart.  Rows r < T*k are the routed pairs in
+ * expert-sorted order (row r = pair perm[r]); row T*k + t is token t's shared-expert row.
+ *   off[0] qx [rows][d]     e4m3 codes of the FFN's input rows (the single-token path
+ *                           writes row 0 only: the token)
+ *   off[1] sx [rows][d/128] fp32 scales of qx
+ *   off[2] qh [rows][f]     e4m3 codes of the re-quantised hidden state
+ *   off[3] sh [rows][f/128] fp32 scales of qh
+ *   off[4] h  [rows][f]     fp32 hidden state before re-quantisation; only the
+ *                           single-token path keeps it (SIZE_MAX otherwise)
+ * The contents are valid after moe_expert_ffn (or moe_forward) completes on the stream.
+ * Returns MOE_OK, or MOE_ERR_INVALID_ARG for sizes moe_workspace_size rejects. */
+int moe_workspace_offsets(int T, int k, int E, int d, int f, size_t off[5]);
+
 /* Thread-local message for the last error on this thread ("" if none). */
 const char* moe_last_error(void);
 
@@ -172,6 +187,15 @@ int moe_set_wait_limit_ns(long long n);
  * k + 1 <= the SM count; other shapes take the tile kernels.  Default 1.  Applies to
  * calls made after it. */
 int moe_set_gemv_max_tokens(int t);
+
+/* Testing knob; the pages have no counterpart.  While on, every launch of the
+ * single-token FFN kernels makes warp 0 of CTA 0 wait, before its first weight stage, on
+ * a shared-memory barrier that nothing completes, so that the wait's time limit
+ * (moe_set_wait_limit_ns) runs out: the kernel records MOE_ERR_TIMEOUT in the status word,
+ * lets the copies it issued land and returns, and the outputs of that call are
+ * incomplete.  This exercises the bounded-wait path without any fault.  0 (the default)
+ * turns it off.  Applies to launches made after the call. */
+int moe_set_test_stall(int on);
 
 /* Synchronise `stream`, then return MOE_ERR_CUDA for a pending CUDA error,
  * MOE_ERR_TIMEOUT if a device-side wait expired since the last call (clearing the

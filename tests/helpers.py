@@ -2,19 +2,42 @@
 and the comparison rules.
 
 Integers and codes (routing indices, dispatch permutation, activation codes and scales)
-must match bit-exactly.  Floating-point layer outputs must be within rel-L2 <= 1e-3 and
-max-abs <= 1e-2 * max|ref| of the oracle, with one allowance that the method itself
-makes necessary.
+must match bit-exactly.  Floating-point outputs are compared in two steps, because the
+method re-quantises the hidden state h = silu(g) * u to e4m3 (3 mantissa bits) from fp32
+and an element of h that lies next to an e4m3 rounding midpoint may round either way on
+a correct implementation:
 
-The hidden state h = silu(g) * u is re-quantised to e4m3 (3 mantissa bits) from fp32.
-The oracle sums g and u in double and the GPU in fp32, so their fp32 h can differ by a
-few 1e-7 relative.  An element whose h / s lies within TIE_REL of an e4m3 rounding
-midpoint may therefore round either way on a correct implementation: both codes are
-valid results.  For those elements only, the comparison allows the exact effect of the
-other rounding, |W_down[:, n]| * |code step| * s, propagated through the combine.
-Measured on a B200, GPU and oracle h codes differ in about 1 of 10^5 elements, always
-within 6e-7 of a midpoint; TIE_REL = 4e-6 leaves about 8x headroom and marks about
-0.1 element per (token, expert) pair.
+1. h codes.  The GPU's re-quantised h (codes qh and scales sh, read from the workspace)
+   must equal the oracle's, except for elements where the two differ by one code step
+   AND the oracle's value h/s lies within a derived error window of the midpoint between
+   the two codes.  The window comes from an a-priori bound on the GPU's fp32 error, not
+   from observed GPU behaviour (``h_error_bound``):
+     - g and u are fp32 dot products over K = d; every product of an e2m1 value, a power
+       of two and an e4m3 value is exact in fp32, so the error is that of the sums.  A
+       product passes through at most D = 128 + K/128 + 8 roundings on its way to the
+       result (<= 128 inside a 128-element chunk, whatever order the tensor core or the
+       MMA chain adds in; one fused multiply-add per chunk when the chunk is scaled by
+       the activation's fp32 block scale and added to the total; <= 8 to combine K-split
+       partials).  Each rounding errs by at most 2^-23 of its result (truncation
+       included), so |dg| <= D * 2^-23 * sum_k |W[n,k] x[k]| and likewise for u
+       (standard forward error bound of summation, gamma_D).
+     - h = g / (1 + exp(-g)) * u is then off by |u| |silu'(g)| dg + |silu(g)| du (plus the
+       second-order terms) and by the element-wise operations: expf (2 ulp), the add, the
+       fast divide (2 ulp) and the multiply; 9 ulp of |h| covers them and the oracle's own
+       rounding of h to fp32.
+     - s = amax / 448 differs by at most the bound of the block's largest elements plus one
+       rounding, and the quotient h / s (or h * (1/s)) adds 3 ulp.
+   A real mistake (a wrong code away from a tie, a dropped term) lands outside the window
+   or changes many codes: at most MAX_FLIPS_PER_VECTOR flips per vector and a fraction
+   MAX_FLIP_FRACTION of all compared codes are accepted.
+2. y and out.  y is compared with the oracle's down projection of the GPU's own codes
+   (``oracle.fp4_gemv`` on e4m3(qh) * sh), element by element within the same kind of
+   a-priori bound (D * 2^-23 * sum_n |W_down[m,n] h[n]|), and within the north-star
+   tolerance rel-L2 <= 1e-3, max-abs <= 1e-2 * max|ref|.  out is compared with the
+   oracle's combine of those references.
+
+Every check also reports the comparison against the oracle's own codes, with no tie rule
+(``pure``), and how many codes used the tie rule.
 """
 from __future__ import annotations
 
@@ -26,24 +49,35 @@ import synth
 
 REL_L2 = 1e-3
 MAX_ABS_FRAC = 1e-2
-TIE_REL = 4e-6
+U23 = 2.0 ** -23                  # largest relative error of one fp32 rounding (any mode)
+MAX_FLIPS_PER_VECTOR = 2
+MAX_FLIP_FRACTION = 1e-4
 
 _E4M3 = None
 
 
-def _e4m3_table():
+def e4m3_table():
     global _E4M3
     if _E4M3 is None:
         _E4M3 = np.array([oracle.e4m3_value(c) for c in range(256)])
     return _E4M3
 
 
-def close_report(got, ref, allow=None):
+def _sorted_values():
+    tab = e4m3_table()
+    return np.unique(tab[np.isfinite(tab)])  # -448 .. -0/+0 .. 448 (zeros merged)
+
+
+def acc_depth(K: int) -> int:
+    """Most fp32 roundings a product meets on its way into a dot product over K."""
+    return 128 + K // 128 + 8
+
+
+# --------------------------------------------------------------------------------- reports
+def close_report(got, ref):
     got = np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64)
     err = np.abs(got - ref)
-    if allow is not None:
-        err = np.maximum(0.0, err - np.asarray(allow, np.float64))
     nref = np.linalg.norm(ref)
     rel = np.linalg.norm(err) / (nref if nref > 0 else 1.0)
     mabs = float(err.max()) if err.size else 0.0
@@ -51,13 +85,29 @@ def close_report(got, ref, allow=None):
     return rel, mabs, bound
 
 
-def assert_close(got, ref, what="", allow=None):
+def assert_close(got, ref, what=""):
     assert np.isfinite(np.asarray(got, np.float64)).all(), f"{what}: non-finite output"
-    rel, mabs, bound = close_report(got, ref, allow)
+    rel, mabs, bound = close_report(got, ref)
     assert rel <= REL_L2 and mabs <= bound, \
         f"{what}: rel-L2 {rel:.3e} (<= {REL_L2}), max-abs {mabs:.3e} (<= {bound:.3e})"
+    return rel, mabs
 
 
+def assert_within(got, ref, bound, what=""):
+    """Element-wise |got - ref| <= bound; returns the largest |got - ref| / bound."""
+    got = np.asarray(got, np.float64)
+    err = np.abs(got - np.asarray(ref, np.float64))
+    bound = np.asarray(bound, np.float64)
+    ratio = err / np.maximum(bound, 1e-300)
+    worst = float(ratio.max()) if ratio.size else 0.0
+    if worst > 1.0:
+        i = np.unravel_index(int(np.argmax(ratio)), ratio.shape)
+        raise AssertionError(f"{what}: |got - ref| = {err[i]:.3e} exceeds its bound "
+                             f"{bound[i]:.3e} at {i} ({int((ratio > 1).sum())} elements)")
+    return worst
+
+
+# --------------------------------------------------------------------------------- inputs
 def device_weights(seed, layer, E, d, f):
     import bit_moe_routed_b200 as bm
     return bm.LayerWeights.from_dict(synth.device_layer_weights(seed, layer, E, d, f))
@@ -67,74 +117,150 @@ def host_experts(seed, layer, d, f, experts):
     return {int(e): synth.host_expert(seed, layer, int(e), d, f) for e in experts}
 
 
-def _down_column(ex, n: int) -> np.ndarray:
-    """Column n of the dequantised down matrix [d] (codes [d][f/2], scales [d][f/32])."""
-    byte = ex.down_codes[:, n // 2]
-    code = (byte >> 4) if (n & 1) else (byte & 0x0F)
-    e = (code >> 1) & 3
-    m = code & 1
-    mag = np.where(e == 0, 0.5 * m, np.ldexp(1.0 + m / 2.0, e - 1))
-    val = np.where(code & 8, -mag, mag)
-    return val * np.exp2(ex.down_scales[:, n // 32].astype(np.float64) - 127.0)
+def dequant_act(q: np.ndarray, s: np.ndarray) -> np.ndarray:
+    """x^ = e4m3(q) * s per 128-block, in double."""
+    return e4m3_table()[q] * np.repeat(np.asarray(s, np.float64), 128, axis=-1)
 
 
-def tie_allowance(ex, hq, hs, hf) -> np.ndarray:
-    """Bound on |y| change if any near-tie element of h rounds the other way [d]."""
-    tab = _e4m3_table()
-    mags = np.unique(np.abs(tab[np.isfinite(tab)]))
-    s = np.repeat(hs.astype(np.float64), 128)
-    a = np.abs(hf.astype(np.float64) / s)
-    i = np.clip(np.searchsorted(mags, a), 1, len(mags) - 1)
-    lo, hi = mags[i - 1], mags[i]
-    mid = (lo + hi) / 2
-    tie = (a < 448.0) & (np.abs(a - mid) <= TIE_REL * np.maximum(a, 1e-30))
-    allow = np.zeros(ex.down_codes.shape[0])
-    for n in np.nonzero(tie)[0]:
-        allow += np.abs(_down_column(ex, int(n))) * (hi[n] - lo[n]) * s[n]
-    return allow
+# --------------------------------------------------------------------------------- bounds
+def h_error_bound(ex, d: int, xhat: np.ndarray, rows):
+    """A-priori bound on |h_gpu - h_oracle| for the given rows of one expert and token,
+    and the exact g, u, h (double) of those rows."""
+    rows = np.asarray(rows, dtype=np.int64)
+    if rows.size == 0:
+        z = np.zeros(0)
+        return z, z, z, z
+    xabs = np.abs(xhat)
+    gc, gs = ex.gate_codes[rows], ex.gate_scales[rows]
+    uc, us = ex.up_codes[rows], ex.up_scales[rows]
+    g = oracle.fp4_gemv(gc, gs, xhat)
+    u = oracle.fp4_gemv(uc, us, xhat)
+    ag = oracle.fp4_gemv(gc & 0x77, gs, xabs)   # sum |W x| (sign bits cleared)
+    au = oracle.fp4_gemv(uc & 0x77, us, xabs)
+    D = acc_depth(d)
+    dg, du = D * U23 * ag, D * U23 * au
+    sig = 1.0 / (1.0 + np.exp(-g))
+    silu = g * sig
+    dsilu = sig * (1.0 + g * (1.0 - sig))
+    h = silu * u
+    B = 1.01 * (np.abs(u) * np.abs(dsilu) * dg + np.abs(silu) * du + 1.1 * dg * du
+                + 0.25 * dg * dg * np.abs(u)) + 9 * U23 * np.abs(h)
+    return B, g, u, h
 
 
-def oracle_pairs(x, scores, k, E, d, f, experts, tokens):
-    """Oracle per selected token: routing, y per routed pair, y_sh, out, and the tie
-    allowances of each, all from the oracle's own computation."""
-    idx, w = oracle.route_topk(scores.numpy(), k)
-    qx, sx = oracle.act_quant(x[torch.as_tensor(tokens)])
-    n = len(tokens)
-    y = np.zeros((n, k, d))
-    ysh = np.zeros((n, d))
-    ay = np.zeros((n, k, d))
-    ash = np.zeros((n, d))
-    out = np.zeros((n, d))
-    aout = np.zeros((n, d))
-    for i, t in enumerate(tokens):
-        for j in range(k + 1):
-            e = int(idx[t, j]) if j < k else E
-            yy, hq, hs, hf = oracle.expert_ffn_h(experts[e], d, f, qx[i:i + 1], sx[i:i + 1])
-            al = tie_allowance(experts[e], hq[0], hs[0], hf[0])
-            if j < k:
-                y[i, j], ay[i, j] = yy[0], al
-            else:
-                ysh[i], ash[i] = yy[0], al
-        out[i] = oracle.combine(ysh[i:i + 1], y[i:i + 1], w[t:t + 1])[0]
-        aout[i] = ash[i] + np.abs(w[t]) @ ay[i]
-    return idx, w, y, ysh, out, ay, ash, aout
+def y_error_bound(down_codes, down_scales, hhat: np.ndarray, K: int) -> np.ndarray:
+    """A-priori bound on |y_gpu - W_down h^| for an fp32 dot product over K = f."""
+    return 1.01 * acc_depth(K) * U23 * oracle.fp4_gemv(down_codes & 0x77, down_scales,
+                                                       np.abs(hhat))
 
 
-def gpu_layer(x, scores, k, weights, ws=None):
+class HStats:
+    """Counts of the tie rule's use over a test."""
+
+    def __init__(self):
+        self.codes = 0
+        self.flips = 0
+        self.max_flips_vector = 0
+        self.max_mid_rel = 0.0
+        self.max_window = 0.0
+        self.scales = 0
+        self.scales_diff = 0
+        self.max_scale_rel = 0.0
+
+    def line(self):
+        return (f"h codes: {self.flips} of {self.codes} rounded the other way at a tie "
+                f"(<= {self.max_flips_vector} per vector; largest |h/s - midpoint|/|h/s| "
+                f"{self.max_mid_rel:.2e}, window up to {self.max_window:.2e}); h scales: "
+                f"{self.scales_diff} of {self.scales} differ (largest rel {self.max_scale_rel:.2e})")
+
+
+def check_h_codes(qg, sg, qo, so, hf_o, ex, d, xhat, stats: HStats, what=""):
+    """Rule 1 for one vector (one token, one expert): GPU codes/scales (qg, sg) against the
+    oracle's (qo, so, and its fp32 h before quantisation hf_o)."""
+    tab = e4m3_table()
+    vals = _sorted_values()
+    qg = np.asarray(qg, np.uint8)
+    qo = np.asarray(qo, np.uint8)
+    sg = np.asarray(sg, np.float32)
+    so = np.asarray(so, np.float32)
+    nb = qo.size // 128
+    vg, vo = tab[qg], tab[qo]
+    flips = np.nonzero(vg != vo)[0]
+    diff_blocks = np.nonzero(sg != so)[0]
+    # rows whose bound is needed: every element that differs, and in blocks whose scale
+    # differs, the elements either side quantised to +-448 (the block's largest |h|)
+    need = set(int(n) for n in flips)
+    for b in diff_blocks:
+        blk = slice(128 * b, 128 * (b + 1))
+        top = np.nonzero((np.abs(vg[blk]) == 448.0) | (np.abs(vo[blk]) == 448.0))[0]
+        assert top.size > 0, f"{what}: block {b} has no element at +-448"
+        need |= set(int(128 * b + i) for i in top)
+    rows = np.array(sorted(need), dtype=np.int64)
+    B, _, _, _ = h_error_bound(ex, d, xhat, rows)
+    Bmap = dict(zip(rows.tolist(), B.tolist()))
+    srel = np.zeros(nb)
+    for b in diff_blocks:
+        blk = range(128 * b, 128 * (b + 1))
+        top = [n for n in blk if n in Bmap]
+        amax = float(np.abs(hf_o[128 * b:128 * (b + 1)]).max())
+        dmax = max(Bmap[n] for n in top)
+        allowed = dmax / amax + 2 * U23
+        rel = abs(float(sg[b]) - float(so[b])) / float(so[b])
+        assert rel <= allowed, f"{what}: h scale of block {b} differs by {rel:.3e} " \
+                               f"(derived bound {allowed:.3e})"
+        srel[b] = allowed
+        stats.max_scale_rel = max(stats.max_scale_rel, rel)
+    for n in flips:
+        b = n // 128
+        i_g = np.searchsorted(vals, vg[n])
+        i_o = np.searchsorted(vals, vo[n])
+        assert abs(int(i_g) - int(i_o)) == 1, \
+            f"{what}: h code {n} is {vg[n]} on the GPU, {vo[n]} in the oracle (not adjacent)"
+        v = float(hf_o[n]) / float(so[b])
+        mid = (vg[n] + vo[n]) / 2.0
+        window = Bmap[int(n)] / max(abs(float(hf_o[n])), 1e-300) + srel[b] + 3 * U23
+        mid_rel = abs(v - mid) / max(abs(v), 1e-300)
+        assert mid_rel <= window, \
+            f"{what}: h code {n} differs ({vg[n]} vs {vo[n]}) but h/s = {v!r} is " \
+            f"{mid_rel:.3e} from the midpoint (derived window {window:.3e})"
+        stats.max_mid_rel = max(stats.max_mid_rel, mid_rel)
+        stats.max_window = max(stats.max_window, window)
+    assert flips.size <= MAX_FLIPS_PER_VECTOR, \
+        f"{what}: {flips.size} h codes differ from the oracle's (at most " \
+        f"{MAX_FLIPS_PER_VECTOR} ties per vector)"
+    stats.codes += qo.size
+    stats.flips += int(flips.size)
+    stats.max_flips_vector = max(stats.max_flips_vector, int(flips.size))
+    stats.scales += nb
+    stats.scales_diff += int(diff_blocks.size)
+
+
+# --------------------------------------------------------------------------------- GPU runs
+def gpu_layer(x, scores, k, weights, ws=None, keep_device=False):
+    """One layer through the four calls; returns every result and the intermediates
+    moe_expert_ffn left in the workspace (on the host unless keep_device)."""
     import bit_moe_routed_b200 as bm
+    T, d = x.shape
+    E, f = weights.E, weights.f
+    if ws is None:
+        ws = bm.alloc_workspace(T, k, E, d, f)
     r = bm.forward(x.cuda(), scores.cuda(), k, weights, ws)
+    r.update({kk: v.clone() for kk, v in bm.workspace_views(ws, T, k, E, d, f).items()})
+    if keep_device:
+        return r
     bm.sync_status()
     return {kk: v.cpu() for kk, v in r.items()}
 
 
-def check_layer(g, x, scores, k, E, d, f, seed, layer, tokens, label="", experts=None):
-    """Compare GPU layer results against the oracle on the given tokens."""
-    idx_all, _ = oracle.route_topk(scores.numpy(), k)
-    if experts is None:
-        need = set(idx_all[tokens].ravel().tolist()) | {E}
-        experts = host_experts(seed, layer, d, f, need)
-    idx, w, y_pair, y_sh, out, ay, ash, aout = oracle_pairs(x, scores, k, E, d, f, experts,
-                                                            tokens)
+def check_layer(g, x, scores, k, E, d, f, seed, layer, tokens, label="", experts=None,
+                verbose=True):
+    """Compare GPU layer results against the oracle on the given tokens (see the module
+    docstring for the rules).  Returns a summary line."""
+    g = {kk: (v.cpu() if hasattr(v, "cpu") else v) for kk, v in g.items()}
+    T = x.shape[0]
+    P = T * k
+    tokens = [int(t) for t in tokens]
+    idx, w = oracle.route_topk(scores.numpy(), k)
     assert np.array_equal(g["idx"].numpy(), idx), f"{label}: routing indices differ"
     counts, offsets, perm, pos = oracle.dispatch(idx, E)
     assert np.array_equal(g["counts"].numpy(), counts), f"{label}: counts"
@@ -142,8 +268,141 @@ def check_layer(g, x, scores, k, E, d, f, seed, layer, tokens, label="", experts
     assert np.array_equal(g["perm"].numpy(), perm), f"{label}: perm"
     assert np.array_equal(g["pos"].numpy(), pos), f"{label}: pos"
     assert np.allclose(g["w"].numpy(), w, rtol=2e-6, atol=1e-7), f"{label}: gate weights"
+    if experts is None:
+        need = set(idx[tokens].ravel().tolist()) | {E}
+        experts = host_experts(seed, layer, d, f, need)
+    qx_o, sx_o = oracle.act_quant(x)
+    single = "h" in g  # the single-token path keeps its fp32 h and writes qx row 0 only
+    if single:
+        assert np.array_equal(g["qx"].numpy()[0], qx_o[0]), f"{label}: qx (token codes)"
+        assert np.array_equal(g["sx"].numpy()[0], sx_o[0]), f"{label}: sx (token scales)"
+    else:
+        src = np.concatenate([perm // k, np.arange(T)])
+        assert np.array_equal(g["qx"].numpy(), qx_o[src]), f"{label}: qx rows"
+        assert np.array_equal(g["sx"].numpy(), sx_o[src]), f"{label}: sx rows"
+    qh_g, sh_g = g["qh"].numpy(), g["sh"].numpy()
+    y_g, ysh_g, out_g = g["y"].numpy(), g["y_shared"].numpy(), g["out"].numpy()
+    tab = e4m3_table()
+    stats = HStats()
+    n = len(tokens)
+    y_ref = np.zeros((n, k, d))
+    y_pure = np.zeros((n, k, d))
+    y_bnd = np.zeros((n, k, d))
+    y_got = np.zeros((n, k, d))
+    ysh_ref = np.zeros((n, d))
+    ysh_pure = np.zeros((n, d))
+    ysh_bnd = np.zeros((n, d))
+    h_worst = 0.0
+    y_worst = 0.0
+    for i, t in enumerate(tokens):
+        xhat = dequant_act(qx_o[t], sx_o[t])
+        for j in range(k + 1):
+            e = int(idx[t, j]) if j < k else E
+            row = int(pos[t * k + j]) if j < k else P + t
+            ex = experts[e]
+            yo, hq_o, hs_o, hf_o = oracle.expert_ffn_h(ex, d, f, qx_o[t:t + 1], sx_o[t:t + 1])
+            what = f"{label}: token {t}, expert {e}"
+            check_h_codes(qh_g[row], sh_g[row], hq_o[0], hs_o[0], hf_o[0], ex, d, xhat, stats,
+                          what)
+            if single:  # the fp32 h itself, against the a-priori bound, every element
+                B, _, _, hx = h_error_bound(ex, d, xhat, np.arange(f))
+                h_worst = max(h_worst, assert_within(g["h"].numpy()[row], hx, B,
+                                                     f"{what}: fp32 h"))
+            hhat = tab[qh_g[row]] * np.repeat(sh_g[row].astype(np.float64), 128)
+            yr = oracle.fp4_gemv(ex.down_codes, ex.down_scales, hhat)
+            yb = y_error_bound(ex.down_codes, ex.down_scales, hhat, f)
+            got = y_g[row] if j < k else ysh_g[t]
+            y_worst = max(y_worst, assert_within(got, yr, yb, f"{what}: y"))
+            if j < k:
+                y_ref[i, j], y_pure[i, j], y_bnd[i, j], y_got[i, j] = yr, yo[0], yb, got
+            else:
+                ysh_ref[i], ysh_pure[i], ysh_bnd[i] = yr, yo[0], yb
+    assert stats.flips <= max(MAX_FLIPS_PER_VECTOR, MAX_FLIP_FRACTION * stats.codes), \
+        f"{label}: {stats.flips} of {stats.codes} h codes rounded the other way"
     tok = np.asarray(tokens)
-    y_gpu = g["y"].numpy()[pos.reshape(-1, k)[tok]]  # [n, k, d]
-    assert_close(y_gpu, y_pair, f"{label}: y_routed", ay)
-    assert_close(g["y_shared"].numpy()[tok], y_sh, f"{label}: y_shared", ash)
-    assert_close(g["out"].numpy()[tok], out, f"{label}: out", aout)
+    wt = w[tok]                                             # [n, k] double
+    out_ref = oracle.combine(ysh_ref, y_ref, wt)
+    out_pure = oracle.combine(ysh_pure, y_pure, wt)
+    out_bnd = ysh_bnd + np.einsum("nk,nkd->nd", np.abs(wt), y_bnd) + \
+        np.einsum("nk,nkd->nd", 2e-6 * np.abs(wt) + 1e-7, np.abs(y_ref)) + \
+        (k + 2) * U23 * (np.abs(ysh_ref) + np.einsum("nk,nkd->nd", np.abs(wt), np.abs(y_ref)))
+    out_worst = assert_within(out_g[tok], out_ref, out_bnd, f"{label}: out")
+    ry, my = assert_close(y_got, y_ref, f"{label}: y_routed")
+    rs, ms = assert_close(ysh_g[tok], ysh_ref, f"{label}: y_shared")
+    ro, mo = assert_close(out_g[tok], out_ref, f"{label}: out")
+    py = close_report(y_got, y_pure)
+    po = close_report(out_g[tok], out_pure)
+    line = (f"PARITY {label}: {n} tokens, {n * (k + 1)} (token, expert) vectors | {stats.line()}"
+            f" | y vs oracle on the GPU's h codes: rel-L2 {ry:.2e}, max-abs {my:.2e}, "
+            f"worst err/bound {y_worst:.2e}; y_shared rel-L2 {rs:.2e}; out rel-L2 {ro:.2e}, "
+            f"worst err/bound {out_worst:.2e}" +
+            (f"; fp32 h worst err/bound {h_worst:.2e}" if single else "") +
+            f" | vs the oracle's own codes (no tie rule): y rel-L2 {py[0]:.2e} max-abs "
+            f"{py[1]:.2e}, out rel-L2 {po[0]:.2e} max-abs {po[1]:.2e}")
+    if verbose:
+        print(line)
+    return line
+
+
+# --------------------------------------------------------------------------------- sampling
+def tile_plan(counts: np.ndarray, T: int, nmax: int):
+    """The FFN's token tiles of every expert (routed 0..E-1 by offsets, then the shared
+    expert's T rows): list of (expert, first row, rows) in plan order."""
+    E = counts.size
+    offs = np.concatenate([[0], np.cumsum(counts)])
+    P = int(offs[-1])
+    tiles = []
+    for e in range(E + 1):
+        n = int(counts[e]) if e < E else T
+        row = int(offs[e]) if e < E else P
+        if n == 0:
+            continue
+        nt = -(-n // nmax)
+        step = (-(-n // nt) + 15) // 16 * 16
+        for i in range(nt):
+            tiles.append((e, row + i * step, min(step, n - i * step)))
+    return tiles
+
+
+def tile_sample_tokens(idx: np.ndarray, E: int, n: int = 64, seed: int = 0):
+    """Tokens to check in a large batch, chosen to cover the tile kernels' edges: the
+    hottest expert's last tile, the last row of the last tile of the highest experts in
+    plan order (the tail the stream-K split cuts), the last row of the first tile of
+    experts with several tiles, the first and last tokens (the shared expert's first and
+    last tile), then seeded random tokens up to n."""
+    T, k = idx.shape
+    counts, offsets, perm, pos = oracle.dispatch(idx, E)
+    nmax = 32 if T <= 64 else 112
+    tiles = tile_plan(counts, T, nmax)
+    pick = []
+
+    def add_row(r):
+        t = int(perm[r]) // k if r < T * k else r - T * k
+        if t not in pick and len(pick) < n:
+            pick.append(t)
+
+    add_row(T * k)           # token 0 in the shared expert's first tile
+    add_row(T * k + T - 1)   # the last token: the shared expert's last tile, last row
+    hot = int(np.argmax(counts))
+    last = [tl for tl in tiles if tl[0] == hot][-1]
+    for r in range(last[1] + last[2] - 1, last[1] - 1, -1)[:16]:
+        add_row(r)
+    routed = [tl for tl in tiles if tl[0] < E]
+    ends = {}
+    for e, r0, m in routed:
+        ends[e] = r0 + m - 1
+    for e in sorted(ends)[::-1][:16]:
+        add_row(ends[e])
+    firsts = {}
+    for e, r0, m in routed:
+        if e not in firsts and int(counts[e]) > nmax:
+            firsts[e] = r0 + m - 1
+    for e in sorted(firsts)[:8]:
+        add_row(firsts[e])
+    rng = np.random.default_rng(seed)
+    for t in rng.permutation(T):
+        if len(pick) >= n:
+            break
+        if int(t) not in pick:
+            pick.append(int(t))
+    return sorted(pick)

@@ -26,3 +26,22 @@ def test_kernel_traffic_lookup(tmp_path):
     src.write_text("// not a recorded source\n")
     assert bench.kernel_traffic(str(src), "gate_up", "decode_t1") is None
     assert bench.kernel_traffic(str(src), "gate_up", "no_such_workload") is None
+
+
+def test_resident_layers_defeat_l2():
+    # decode: enough layers that the others' weights exceed four times the L2
+    w = synth.WORKLOADS["decode_t1"]
+    n = bench.resident_layers(w, 8)
+    per_step = 7 * synth.expert_bytes(w.d, w.f)
+    assert (n - 1) * per_step >= 4 * bench.L2_BYTES and n <= 8
+    # prefill reads the whole layer every step: two layers suffice; 43 layers stay 43
+    assert bench.resident_layers(synth.WORKLOADS["prefill_t4096_uniform"], 8) == 2
+    assert bench.resident_layers(synth.WORKLOADS["layers43_t32"], 8) == 43
+
+
+def test_fp8_peak_choice():
+    assert bench.fp8_peak_of({"mxfp8_tflops": 4000.0, "fp8_tensorwise_tflops": 4100.0},
+                             1600.0)[0] == 4000.0
+    assert bench.fp8_peak_of({"fp8_tensorwise_tflops": 4100.0}, 1600.0)[0] == 4100.0
+    peak, src = bench.fp8_peak_of({}, 1600.0)
+    assert peak == 3200.0 and "nominal" in src

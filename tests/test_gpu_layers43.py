@@ -1,13 +1,14 @@
 """43 independent MoE layers resident in HBM (147.7 GB of FP4 weights and scales), run back
 to back at T=1 and T=32 with Zipf(1.0) routing; every layer's output is checked against
-the oracle on sampled tokens (weights regenerated on the host for the experts used)."""
+the oracle on sampled tokens (weights regenerated on the host for the experts used): the
+one token at T=1, four tokens per layer at T=32 (chosen to cover the tiles' edges)."""
 import numpy as np
 import pytest
 import torch
 
 import oracle
 import synth
-from helpers import check_layer
+from helpers import check_layer, gpu_layer, tile_sample_tokens
 
 pytestmark = pytest.mark.gpu
 
@@ -32,8 +33,8 @@ def layers():
     torch.cuda.empty_cache()
 
 
-@pytest.mark.parametrize("name,tokens", [("layers43_t1", [0]), ("layers43_t32", [0, 31])])
-def test_43_layers_back_to_back(layers, name, tokens):
+@pytest.mark.parametrize("name,n_tokens", [("layers43_t1", 1), ("layers43_t32", 4)])
+def test_43_layers_back_to_back(layers, name, n_tokens):
     w_ = synth.WORKLOADS[name]
     base = synth.WORKLOADS["layers43_t1"]
     oracle.set_threads(8)
@@ -42,10 +43,11 @@ def test_43_layers_back_to_back(layers, name, tokens):
     results = []
     for l in range(w_.layers):  # all layers first, on the device, back to back
         x, s = inputs[l]
-        r = bm.forward(x.cuda(), s.cuda(), w_.k, layers[l], ws)
-        results.append({kk: v.cpu() for kk, v in r.items()})
+        results.append(gpu_layer(x, s, w_.k, layers[l], ws, keep_device=True))
     bm.sync_status()
     for l in range(w_.layers):
         x, s = inputs[l]
+        idx, _ = oracle.route_topk(s.numpy(), w_.k)
+        tokens = tile_sample_tokens(idx, w_.E, n_tokens, seed=l)
         check_layer(results[l], x, s, w_.k, w_.E, w_.d, w_.f, base.seed(l), l, tokens,
                     f"{name} layer {l}")

@@ -1,9 +1,13 @@
 """GPU parity: the CUDA library (through the C ABI) against the oracle.
 
 Routing indices, the dispatch permutation, offsets and the quantised activation codes
-and scales must match bit-exactly; FFN outputs (y_routed, y_shared, out) must be within
-rel-L2 <= 1e-3 and max-abs <= 1e-2 * max|ref|.  Small shapes are compared in full;
-the full-size workloads on sampled tokens the oracle computes one by one.
+and scales must match bit-exactly; the re-quantised hidden state must match the oracle's
+codes up to counted ties, and FFN outputs (y_routed, y_shared, out) must lie within
+derived element-wise bounds of the oracle evaluated on the GPU's codes and within rel-L2
+<= 1e-3, max-abs <= 1e-2 * max|ref| (helpers.py states the rules).  Small shapes are
+compared in full; decode_t64 on all its tokens; prefill on 64 tokens chosen to cover the
+tile kernels' edges (the hottest expert's last tile, the stream-K tail, the last rows of
+tiles), which the oracle computes one by one.
 """
 import numpy as np
 import pytest
@@ -11,7 +15,8 @@ import torch
 
 import oracle
 import synth
-from helpers import assert_close, check_layer, device_weights, gpu_layer, host_experts
+from helpers import (assert_close, check_layer, device_weights, gpu_layer, host_experts,
+                     tile_sample_tokens)
 
 pytestmark = pytest.mark.gpu
 
@@ -248,14 +253,17 @@ def test_device_generator_matches_host_generator():
 
 
 # ---------------------------------------------------------------- full-size workloads
-def _full_workload(name, tokens):
+def _full_workload(name, tokens=None, n_sample=64):
     w_ = synth.WORKLOADS[name]
     x, s = synth.gen_layer_inputs(w_, 0)
     W = device_weights(w_.seed(), 0, w_.E, w_.d, w_.f)
-    oracle.set_threads(8)
+    oracle.set_threads(max(8, (__import__("os").cpu_count() or 8)))
     g = gpu_layer(x, s, w_.k, W)
     del W
     torch.cuda.empty_cache()
+    if tokens is None:
+        idx, _ = oracle.route_topk(s.numpy(), w_.k)
+        tokens = tile_sample_tokens(idx, w_.E, n_sample, seed=w_.seed())
     check_layer(g, x, s, w_.k, w_.E, w_.d, w_.f, w_.seed(), 0, tokens, name)
     return g
 
@@ -269,14 +277,14 @@ def test_decode_t1_full(gemv):
         bm.set_gemv_max_tokens(1)
 
 
-def test_decode_t64_zipf_sampled():
-    g = _full_workload("decode_t64_zipf", [0, 9, 31, 63])
+def test_decode_t64_zipf_all_tokens():
+    g = _full_workload("decode_t64_zipf", list(range(64)))
     assert int(g["counts"].max()) > 16  # a hot expert serves many tokens
 
 
 @pytest.mark.parametrize("name", ["prefill_t4096_uniform", "prefill_t4096_zipf"])
 def test_prefill_t4096_sampled(name):
-    g = _full_workload(name, [0, 1, 1777, 4095])
+    g = _full_workload(name)
     w_ = synth.WORKLOADS[name]
     assert int(g["counts"].sum()) == w_.T * w_.k
     # every output row finite

@@ -1,12 +1,11 @@
 """Failure detection without a GPU fault: the FFN kernels bound every wait by a
 %globaltimer limit.  A 1 ns limit makes the first wait that is not already satisfied run
 out; the kernel must record MOE_ERR_TIMEOUT, release TMEM (tile kernels), drain its
-copies and return, leaving the context usable for the next (normal) call.  Both FFN
-implementations run with the tiny limit: the tile kernels (T = 8) and the single-token
-GEMV kernels (T = 1).  The GEMV kernels wait only on their own TMA stages, and one
-try_wait usually outlasts a stage's copy, so a tiny limit may or may not run out there:
-the GEMV test accepts either outcome, but a timeout must be reported and a clean run must
-be correct."""
+copies and return, leaving the context usable for the next (normal) call.  The tile
+kernels (T = 8) run with the tiny limit.  The single-token kernels wait only on their own
+TMA stages, and one try_wait usually outlasts a stage's copy, so there a tiny limit may or
+may not run out; their timeout path is exercised deterministically by the test stall
+(moe_set_test_stall), a wait on a barrier that nothing completes."""
 import numpy as np
 import pytest
 import torch
@@ -65,3 +64,29 @@ def test_gemv_tiny_wait_limit_reports_or_completes():
     bm.sync_status()
     g = gpu_layer(x, s, k, W)
     check_layer(g, x, s, k, E, d, f, 513, 0, [0], "after the tiny limit")
+
+
+def test_single_token_stall_times_out_and_recovers():
+    """The test stall makes one warp's bounded wait run out on every call: the status must
+    report MOE_ERR_TIMEOUT each time, and the next normal call must be correct."""
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    T, E, k, d, f = 1, 64, 6, 4096, 2048
+    x = synth.gen_x(T, d, seed=521)
+    s = synth.gen_scores_uniform(T, E, seed=522)
+    W = device_weights(523, 0, E, d, f)
+    bm.sync_status()
+    bm.set_wait_limit_ns(20_000_000)  # 20 ms
+    bm.set_test_stall(True)
+    try:
+        for _ in range(2):
+            bm.forward(x.cuda(), s.cuda(), k, W)
+            with pytest.raises(bm.MoeError) as ei:
+                bm.sync_status()
+            assert ei.value.code == bm.MOE_ERR_TIMEOUT
+    finally:
+        bm.set_test_stall(False)
+        bm.set_wait_limit_ns(0)
+    bm.sync_status()
+    g = gpu_layer(x, s, k, W)
+    check_layer(g, x, s, k, E, d, f, 523, 0, [0], "after the stall")
