@@ -346,9 +346,16 @@ class Layers:
             self.items.append(dict(x_cpu=x_cpu, s_cpu=s_cpu, W=W, x=x_cpu.to(dev),
                                    scores=s_cpu.to(dev)))
         self.ws = bm.alloc_workspace(T, k, E, d, f, dev)
-        self.y = torch.empty((max(T * k, 1), d), dtype=torch.float32, device=dev)
-        self.ysh = torch.empty((T, d), dtype=torch.float32, device=dev)
-        self.out = torch.empty((T, d), dtype=torch.float32, device=dev)
+        i32, f32 = torch.int32, torch.float32
+        self.outs = {"idx": torch.empty((T, k), dtype=i32, device=dev),
+                     "w": torch.empty((T, k), dtype=f32, device=dev),
+                     "counts": torch.empty((E,), dtype=i32, device=dev),
+                     "offsets": torch.empty((E + 1,), dtype=i32, device=dev),
+                     "perm": torch.empty((max(T * k, 1),), dtype=i32, device=dev),
+                     "pos": torch.empty((max(T * k, 1),), dtype=i32, device=dev),
+                     "y": torch.empty((max(T * k, 1), d), dtype=f32, device=dev),
+                     "y_shared": torch.empty((T, d), dtype=f32, device=dev),
+                     "out": torch.empty((T, d), dtype=f32, device=dev)}
 
 
 def resident_layers(w, max_layers):
@@ -370,13 +377,12 @@ def measure(bm, w, args, dev, stream, rank, dist, steps, warmup, peaks, cpu_seco
         steps = w.layers * max(1, steps // w.layers)  # whole passes over the resident layers
     Ls = Layers(bm, w, n_layers, rank, dev)
 
+    # one step = the whole layer in one call (moe_forward): one kernel for a single token,
+    # otherwise route, dispatch, prepare, gate/up, down and combine back to back
+    fused = T == 1 and d % 512 == 0 and f % 512 == 0
+
     def step(L):
-        idx, gw = bm.route_topk(L["scores"], k, stream)
-        counts, offsets, perm, pos = bm.dispatch(idx, E, stream)
-        bm.expert_ffn(L["x"], k, L["W"], offsets, perm, Ls.ws, out=(Ls.y, Ls.ysh),
-                      stream=stream)
-        bm.combine(Ls.y, Ls.ysh, gw, pos, Ls.out, stream)
-        return counts
+        return bm.forward(L["x"], L["scores"], k, L["W"], Ls.ws, stream, outs=Ls.outs)["counts"]
 
     # one eager pass per layer (checks the status word and gives the routing counts)
     works = []
@@ -413,13 +419,14 @@ def measure(bm, w, args, dev, stream, rank, dist, steps, warmup, peaks, cpu_seco
         bm.ffn_prepare(L["x"], k, L["W"], offsets, perm, Ls.ws, stream)
 
     g_a, g_b = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_a, stream=stream):
-        for L in Ls.items:
-            pre(L)
-            bm.ffn_gate_up(T, k, L["W"], Ls.ws, stream)
-    with torch.cuda.graph(g_b, stream=stream):
-        for L in Ls.items:
-            pre(L)
+    if not fused:
+        with torch.cuda.graph(g_a, stream=stream):
+            for L in Ls.items:
+                pre(L)
+                bm.ffn_gate_up(T, k, L["W"], Ls.ws, stream)
+        with torch.cuda.graph(g_b, stream=stream):
+            for L in Ls.items:
+                pre(L)
     torch.cuda.synchronize()
 
     with torch.cuda.stream(stream):
@@ -447,20 +454,30 @@ def measure(bm, w, args, dev, stream, rank, dist, steps, warmup, peaks, cpu_seco
     for i in range(max(len(g_one), 10)):
         one_ms += time_graph(g_one[i % len(g_one)], stream, 1)
     ab = {"a": [], "b": []}
-    for _ in range(max(7, min(15, steps))):
-        ab["a"] += time_graph(g_a, stream, 1)
-        ab["b"] += time_graph(g_b, stream, 1)
+    if not fused:
+        for _ in range(max(7, min(15, steps))):
+            ab["a"] += time_graph(g_a, stream, 1)
+            ab["b"] += time_graph(g_b, stream, 1)
     clk = clocks.stop() if clocks is not None else None
     total_s = max_over_ranks(timed_ms / 1000.0, dist, dev)
     world = dist.get_world_size() if dist is not None else 1
     layer_s = total_s / steps
-    gu_s = (statistics.median(ab["a"]) - statistics.median(ab["b"])) / n_layers / 1000.0
     is_prefill = T > 256
-    gemv = T == 1 and d % 512 == 0 and f % 512 == 0
-    kernel_file = os.path.join(ROOT, "bit_moe_routed_b200", "csrc", "gemv.cu" if gemv else "ffn.cu")
-    kernel_name = ("ffn gate/up (FP4 GEMV: TMA-staged rows, in-register e2m1 decode, "
-                   "mma.sync f16 -> fp32)") if gemv else "ffn gate/up (tcgen05 kind::mxf8f6f4)"
-    traffic = kernel_traffic(kernel_file, "gate_up", w.name)
+    if fused:
+        # the dominant kernel is the step itself: K launches back to back in one graph
+        gu_s = timed_ms / 1000.0 / steps
+        kernel_file = os.path.join(ROOT, "bit_moe_routed_b200", "csrc", "decode.cu")
+        kernel_name = ("decode_kernel: the whole layer in one cooperative kernel (routing, "
+                       "dispatch, quantisation, FP4 GEMVs with in-register e2m1 decode and "
+                       "mma.sync, combine)")
+        traffic = kernel_traffic(kernel_file, "layer", w.name)
+        io = 4 * E + 2 * d + 4 * d * (k + 2)  # scores, x; y_routed, y_shared and out
+        work["gu_bytes"] = work["weight_bytes"] + io
+    else:
+        gu_s = (statistics.median(ab["a"]) - statistics.median(ab["b"])) / n_layers / 1000.0
+        kernel_file = os.path.join(ROOT, "bit_moe_routed_b200", "csrc", "ffn.cu")
+        kernel_name = "ffn gate/up (tcgen05 kind::mxf8f6f4)"
+        traffic = kernel_traffic(kernel_file, "gate_up", w.name)
     hbm_peak, fp8_peak, fp8_src, peak_kind = peaks
     if is_prefill:
         achieved = work["flops_gu"] / gu_s / 1e12
@@ -483,6 +500,7 @@ def measure(bm, w, args, dev, stream, rank, dist, steps, warmup, peaks, cpu_seco
     roof["avg_launch_us"] = gu_s * 1e6
     roof["algorithmic_per_launch"] = work["flops_gu"] if is_prefill else work["gu_bytes"]
     rec = {
+        "fused": fused, "launches_per_step": 1 if fused else 6,
         "value": world * T * steps / total_s, "unit": "tokens/s", "steps": steps,
         "ms_per_step": 1000.0 * layer_s,
         "ms_per_step_isolated": statistics.median(one_ms),
@@ -615,7 +633,7 @@ def run_gpu(args, w):
             "roofline": rec["roofline"],
             "cpu_baseline": rec.get("cpu_baseline"),
             "e2e": e2e_rec,
-            "gpu_launches": 6 * args.steps,
+            "gpu_launches": rec["launches_per_step"] * args.steps,
             "clocks": rec.get("clocks"),
             "peaks": dict(fp8, hbm_gbs=hbm_peak, hbm_source=peak_kind,
                           fp8_used_tflops=fp8_peak, fp8_used_source=fp8_src,

@@ -7,8 +7,9 @@ if the library is missing or the device is not sm_100, calls raise.
 
     idx, w = route_topk(scores, k)              # step 1: top-k + sigmoid gate weights
     counts, offsets, perm, pos = dispatch(idx, E)  # step 2: stable grouping per expert
-    y, y_sh = expert_ffn(x, k, weights, offsets, perm)  # steps 3-7 (tcgen05 FFN)
+    y, y_sh = expert_ffn(x, k, weights, offsets, perm)  # steps 3-7 (FP4 x FP8 FFN)
     out = combine(y, y_sh, w, pos)              # step 8
+    r = forward(x, scores, k, weights)          # all of it in one call (one kernel at T=1)
 """
 from __future__ import annotations
 
@@ -33,7 +34,7 @@ EXPORTS = (
     "moe_route_topk", "moe_dispatch", "moe_act_quant", "moe_expert_ffn", "moe_ffn_prepare",
     "moe_ffn_gate_up", "moe_ffn_down", "moe_combine", "moe_workspace_size", "moe_last_error",
     "moe_set_wait_limit_ns", "moe_sync_status", "moe_expert_ffn_noalloc",
-    "moe_set_gemv_max_tokens", "moe_workspace_offsets", "moe_set_test_stall",
+    "moe_set_gemv_max_tokens", "moe_workspace_offsets", "moe_set_test_stall", "moe_forward",
 )
 
 
@@ -83,6 +84,7 @@ def lib():
             "moe_set_gemv_max_tokens": [I],
             "moe_workspace_offsets": [I, I, I, I, I, P],
             "moe_set_test_stall": [I],
+            "moe_forward": [P, P, I, I, W, P, P, P, P, P, P, P, P, P, P, Z, P],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -295,8 +297,37 @@ def combine(y_routed: torch.Tensor, y_shared: torch.Tensor, w: torch.Tensor, pos
 
 
 def forward(x: torch.Tensor, scores: torch.Tensor, k: int, w: LayerWeights,
-            ws: torch.Tensor | None = None, stream=None):
-    """The whole layer through the four calls; returns a dict of every intermediate."""
+            ws: torch.Tensor | None = None, stream=None, outs: dict | None = None):
+    """The whole layer in one call (moe_forward: one kernel for a single token, the four
+    calls back to back otherwise); returns a dict of every output.  `outs` may hold
+    preallocated outputs under the same names."""
+    T, d = x.shape
+    E = w.E
+    dev = x.device
+    if ws is None:
+        ws = alloc_workspace(T, k, E, w.d, w.f, dev)
+    o = dict(outs) if outs is not None else {}
+    shapes = {"idx": ((T, k), torch.int32), "w": ((T, k), torch.float32),
+              "counts": ((E,), torch.int32), "offsets": ((E + 1,), torch.int32),
+              "perm": ((max(T * k, 1),), torch.int32), "pos": ((max(T * k, 1),), torch.int32),
+              "y": ((max(T * k, 1), d), torch.float32), "y_shared": ((max(T, 1), d), torch.float32),
+              "out": ((max(T, 1), d), torch.float32)}
+    for name, (shape, dtype) in shapes.items():
+        if name not in o:
+            o[name] = torch.empty(shape, dtype=dtype, device=dev)
+    st = w.struct()
+    _check(lib().moe_forward(_p(scores), _p(x), T, k, ctypes.byref(st), _p(o["idx"]), _p(o["w"]),
+                             _p(o["counts"]), _p(o["offsets"]), _p(o["perm"]), _p(o["pos"]),
+                             _p(o["y"]), _p(o["y_shared"]), _p(o["out"]), _p(ws), ws.numel(),
+                             _stream(stream)))
+    return dict(idx=o["idx"], w=o["w"], counts=o["counts"], offsets=o["offsets"],
+                perm=o["perm"][:T * k], pos=o["pos"][:T * k], y=o["y"][:T * k],
+                y_shared=o["y_shared"][:T], out=o["out"][:T])
+
+
+def forward_calls(x: torch.Tensor, scores: torch.Tensor, k: int, w: LayerWeights,
+                  ws: torch.Tensor | None = None, stream=None):
+    """The whole layer through the four separate calls; returns a dict of every output."""
     idx, gw = route_topk(scores, k, stream)
     counts, offsets, perm, pos = dispatch(idx, w.E, stream)
     y, ysh = expert_ffn(x, k, w, offsets, perm, ws, stream=stream)

@@ -20,6 +20,14 @@ __device__ int g_status;  // device status word (kStatus* bits), one per device
 namespace {
 
 thread_local std::string t_err;
+// Set while a call issues kernels that follow another of this library's kernels on the
+// stream (see launch_pdl): they may start while it finishes.
+thread_local bool t_overlap = false;
+struct OverlapScope {
+  bool saved;
+  OverlapScope() : saved(t_overlap) { t_overlap = true; }
+  ~OverlapScope() { t_overlap = saved; }
+};
 std::atomic<long long> g_wait_ns{2000000000LL};
 std::atomic<int> g_gemv_max_t{kGemvMaxT};  // batches up to this size take the GEMV path
 std::atomic<int> g_stall{0};                 // test knob: see moe_set_test_stall
@@ -137,9 +145,12 @@ WorkspaceLayout workspace_layout(int T, int k, int E, int d, int f) {
   L.partials = o;
   const size_t tile_rows_max = nmax_for(T) == kNmaxSmall ? 256 : 128;
   o = align256(o + (size_t)kMaxCtas * 2 * (size_t)ncap_for(T) * 2 * tile_rows_max * 4);
-  // single-token path: h of every active expert, fp32
+  // single-token path: h of every active expert, fp32, and the combine counters of the
+  // single-token kernel (one per 16 output rows)
   L.hbuf = o;
   if (T <= kGemvMaxT) o = align256(o + R * f * 4);
+  L.done2 = o;
+  if (T <= kGemvMaxT) o = align256(o + 4 * (size_t)(d / 16));
   L.total = o;
   return L;
 }
@@ -200,8 +211,12 @@ int moe_sync_status(void* stream) {
     const int zero = 0;
     e = cudaMemcpy(di.status, &zero, sizeof(int), cudaMemcpyHostToDevice);
     if (e != cudaSuccess) return cuda_fail(e, "clear status");
-    if (host & kStatusTimeout)
+    if (host & kStatusTimeout) {
+      // a CTA that gave up may have left the single-token kernel's grid barrier mid-count
+      e = reset_grid_barrier();
+      if (e != cudaSuccess) return cuda_fail(e, "reset grid barrier");
       return fail(MOE_ERR_TIMEOUT, "a device-side wait exceeded its limit (status 0x%x)", host);
+    }
     return fail(MOE_ERR_INVALID_ARG, "an expert id or position was out of range (status 0x%x)",
                 host);
   }
@@ -240,7 +255,7 @@ int moe_dispatch(const int32_t* topk_idx, int T, int k, int E, int32_t* counts, 
   if (rc) return rc;
   // T == 0 still writes counts = 0 and offsets = 0 (the kernel handles P == 0)
   cudaError_t e = launch_dispatch(topk_idx, T, k, E, counts, offsets, perm, pos, di.status,
-                                  static_cast<cudaStream_t>(stream));
+                                  static_cast<cudaStream_t>(stream), t_overlap);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "dispatch launch");
 }
 
@@ -262,14 +277,12 @@ int moe_act_quant(const uint16_t* x_bf16, int T, int d, uint8_t* qx, float* sx, 
 
 namespace {
 
-// Set while moe_expert_ffn issues its second and third kernels (see launch_pdl).
-thread_local bool t_overlap = false;
-
 struct FfnCtx {
   DeviceInfo di;
   WorkspaceLayout L;
   int nmax;
-  bool gemv;  // single-token GEMV path (gemv.cu) instead of the tcgen05 tiles (ffn.cu)
+  bool gemv;   // single-token GEMV path (gemv.cu) instead of the tcgen05 tiles (ffn.cu)
+  bool fused;  // ... in one cooperative kernel (decode.cu), for the whole-call entry points
   uint8_t* ws;
 };
 
@@ -319,6 +332,9 @@ int ffn_check(int T, int k, const moe_weights_t* w, void* ws, size_t ws_bytes, F
     return fail(MOE_ERR_INVALID_ARG, "shape needs %zu bytes of shared memory (> %d)", need,
                 max_smem);
   c.gemv = use_gemv(T, k, w, c.di.sms, max_smem);
+  const int ctas = c.di.sms < kMaxCtas ? c.di.sms : kMaxCtas;
+  c.fused = c.gemv && decode_fits(k, w->d, w->f, ctas) &&
+            decode_smem_bytes(w->d, w->f) <= (size_t)max_smem;
   return MOE_OK;
 }
 
@@ -394,14 +410,14 @@ int moe_ffn_prepare(const uint16_t* x_bf16, int T, int k, const moe_weights_t* w
     cudaError_t e = launch_quant_rows(
         x_bf16, T, k, w->d, nullptr, 0, c.ws + c.L.qx, reinterpret_cast<float*>(c.ws + c.L.sx),
         offsets, w->E, c.nmax, reinterpret_cast<int32_t*>(c.ws + c.L.plan), nullptr, 0,
-        c.di.status, static_cast<cudaStream_t>(stream), 1);
+        c.di.status, static_cast<cudaStream_t>(stream), 1, t_overlap);
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "ffn prepare launch");
   }
   cudaError_t e = launch_quant_rows(
       x_bf16, T, k, w->d, perm, T * k, c.ws + c.L.qx, reinterpret_cast<float*>(c.ws + c.L.sx),
       offsets, w->E, c.nmax, reinterpret_cast<int32_t*>(c.ws + c.L.plan),
       reinterpret_cast<int*>(c.ws + c.L.counters), c.L.n_counters, c.di.status,
-      static_cast<cudaStream_t>(stream));
+      static_cast<cudaStream_t>(stream), 0, t_overlap);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "ffn prepare launch");
 }
 
@@ -450,20 +466,107 @@ int moe_ffn_down(int T, int k, const moe_weights_t* w, float* y_routed, float* y
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "ffn down launch");
 }
 
+namespace {
+
+DecodeLaunch decode_args(int k, const moe_weights_t* w, const FfnCtx& c) {
+  DecodeLaunch a{};
+  a.gate_codes = w->gate_codes;
+  a.gate_scales = w->gate_scales;
+  a.up_codes = w->up_codes;
+  a.up_scales = w->up_scales;
+  a.down_codes = w->down_codes;
+  a.down_scales = w->down_scales;
+  a.qx = c.ws + c.L.qx;
+  a.sx = reinterpret_cast<float*>(c.ws + c.L.sx);
+  a.qh = c.ws + c.L.qh;
+  a.sh = reinterpret_cast<float*>(c.ws + c.L.sh);
+  a.hbuf = reinterpret_cast<float*>(c.ws + c.L.hbuf);
+  a.done2 = reinterpret_cast<int*>(c.ws + c.L.done2);
+  a.E = w->E;
+  a.k = k;
+  a.d = w->d;
+  a.f = w->f;
+  a.wait_ns = g_wait_ns.load();
+  a.status = c.di.status;
+  a.stall = g_stall.load();
+  return a;
+}
+
+}  // namespace
+
 int moe_expert_ffn(const uint16_t* x_bf16, int T, int k, const moe_weights_t* w,
                    const int32_t* offsets, const int32_t* perm, float* y_routed, float* y_shared,
                    void* ws, size_t ws_bytes, void* stream) {
-  int rc = moe_ffn_prepare(x_bf16, T, k, w, offsets, perm, ws, ws_bytes, stream);
+  FfnCtx c;
+  int rc = ffn_check(T, k, w, ws, ws_bytes, c);
+  if (rc) return rc;
+  if (T > 0 && c.fused) {  // one token: the whole FFN in one kernel
+    if (!x_bf16 || !offsets || !perm || !y_routed || !y_shared)
+      return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned(x_bf16, 16) || !aligned(y_routed, 16) || !aligned(y_shared, 16))
+      return fail(MOE_ERR_INVALID_ARG, "x and the outputs must be 16-byte aligned");
+    DecodeLaunch a = decode_args(k, w, c);
+    a.forward = false;
+    a.x = x_bf16;
+    a.offsets_in = offsets;
+    a.y_routed = y_routed;
+    a.y_shared = y_shared;
+    cudaError_t e = launch_decode(a, static_cast<cudaStream_t>(stream), c.di.sms);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "single-token ffn launch");
+  }
+  rc = moe_ffn_prepare(x_bf16, T, k, w, offsets, perm, ws, ws_bytes, stream);
   if (rc) return rc;
   // gate/up and down follow a kernel of this call on the stream: they may start while it
   // finishes (their prologue overlaps its tail)
-  struct Overlap {
-    Overlap() { t_overlap = true; }
-    ~Overlap() { t_overlap = false; }
-  } guard;
+  OverlapScope guard;
   rc = moe_ffn_gate_up(T, k, w, ws, ws_bytes, stream);
   if (rc) return rc;
   return moe_ffn_down(T, k, w, y_routed, y_shared, ws, ws_bytes, stream);
+}
+
+int moe_forward(const float* scores, const uint16_t* x_bf16, int T, int k,
+                const moe_weights_t* w, int32_t* topk_idx, float* topk_w, int32_t* counts,
+                int32_t* offsets, int32_t* perm, int32_t* pos, float* y_routed, float* y_shared,
+                float* out, void* ws, size_t ws_bytes, void* stream) {
+  FfnCtx c;
+  int rc = ffn_check(T, k, w, ws, ws_bytes, c);
+  if (rc) return rc;
+  if (k > 32) return fail(MOE_ERR_INVALID_ARG, "k=%d outside [1, min(E, 32)]", k);
+  if (T > 0 && c.fused) {  // one token: the whole layer in one kernel
+    if (!scores || !x_bf16 || !topk_idx || !topk_w || !counts || !offsets || !perm || !pos ||
+        !y_routed || !y_shared || !out)
+      return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned(scores, 4) || !aligned(x_bf16, 16) || !aligned(y_routed, 16) ||
+        !aligned(y_shared, 16) || !aligned(out, 16) || !aligned(topk_idx, 4) ||
+        !aligned(topk_w, 4) || !aligned(counts, 4) || !aligned(offsets, 4) || !aligned(perm, 4) ||
+        !aligned(pos, 4))
+      return fail(MOE_ERR_INVALID_ARG, "misaligned pointer");
+    DecodeLaunch a = decode_args(k, w, c);
+    a.forward = true;
+    a.scores = scores;
+    a.x = x_bf16;
+    a.idx = topk_idx;
+    a.w_out = topk_w;
+    a.counts = counts;
+    a.offsets = offsets;
+    a.perm = perm;
+    a.pos = pos;
+    a.y_routed = y_routed;
+    a.y_shared = y_shared;
+    a.out = out;
+    cudaError_t e = launch_decode(a, static_cast<cudaStream_t>(stream), c.di.sms);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "single-token layer launch");
+  }
+  // otherwise the four calls; every kernel after the first may start under its
+  // predecessor's tail
+  rc = moe_route_topk(scores, T, w->E, k, topk_idx, topk_w, stream);
+  if (rc) return rc;
+  OverlapScope guard;
+  rc = moe_dispatch(topk_idx, T, k, w->E, counts, offsets, perm, pos, nullptr, 0, stream);
+  if (rc) return rc;
+  rc = moe_expert_ffn(x_bf16, T, k, w, offsets, perm, y_routed, y_shared, ws, ws_bytes, stream);
+  if (rc) return rc;
+  return moe_combine(y_routed, y_shared, topk_w, pos, T, k, w->d, out, stream);
 }
 
 int moe_combine(const float* y_routed, const float* y_shared, const float* topk_w,
@@ -480,7 +583,7 @@ int moe_combine(const float* y_routed, const float* y_shared, const float* topk_
   int rc = device_info(di);
   if (rc) return rc;
   cudaError_t e = launch_combine(y_routed, y_shared, topk_w, pos, T, k, d, out, di.status,
-                                 static_cast<cudaStream_t>(stream));
+                                 static_cast<cudaStream_t>(stream), t_overlap);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "combine launch");
 }
 

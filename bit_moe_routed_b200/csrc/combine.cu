@@ -55,11 +55,12 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
 // Grid: one row of CTAs per token, each CTA one float4 per thread of a slice of the row
 // (a short row needs one round of loads, whatever T is).
 cudaError_t launch_combine(const float* y, const float* ysh, const float* w, const int32_t* pos,
-                           int T, int k, int d, float* out, int* status, cudaStream_t s) {
+                           int T, int k, int d, float* out, int* status, cudaStream_t s,
+                           bool overlap) {
   int threads = d / 4 < 256 ? d / 4 : 256;
   threads = (threads + 31) / 32 * 32;
   const unsigned slices = (unsigned)((d / 4 + threads - 1) / threads);
-  return launch_pdl(combine_kernel, dim3((unsigned)T, slices), dim3(threads), 0, s, false, y, ysh, w, pos,
+  return launch_pdl(combine_kernel, dim3((unsigned)T, slices), dim3(threads), 0, s, overlap, y, ysh, w, pos,
                     T, k, d, out, status);
 }
 

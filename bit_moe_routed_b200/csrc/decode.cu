@@ -1,0 +1,836 @@
+// Single-token decode of the whole MoE layer in one kernel: routing, dispatch, activation
+// quantisation, gate/up FP4 GEMV, SwiGLU, re-quantisation, down FP4 GEMV and the
+// routing-weighted combine.
+//
+// At T = 1 the layer is bound by reading the k + 1 selected experts' FP4 codes and block
+// scales once (dpshk.com article, "核心实现三": an expert is read once for all its tokens;
+// "核心实现四": FP4 decoded inside the GEMV, gate and up on one quantised input).  As
+// separate kernels, the routing, dispatch, quantisation and combine steps and the
+// launch gaps between them cost as much as a third of the layer (ai-muninn.com post,
+// "一張 22G 老卡跑 284B": the fixed per-token cost of launches and round trips).  Here
+// they run inside one cooperative launch, and every SM starts streaming weights at once:
+//
+//   prologue  every CTA issues the copies of its share of the shared expert (always
+//             active, known before routing), then computes the top-k of the token's
+//             scores (warp 0) and quantises the token (warps 1-8) redundantly, so no
+//             grid-wide step precedes the weight stream; CTA 0 stores the routing,
+//             dispatch and quantisation outputs;
+//   phase 1   gate/up: units of 8 h-rows (8 gate + the same 8 up weight rows) x 512-wide
+//             K stages, as in the two-kernel GEMV path; h = silu(g) * u to the workspace;
+//   barrier   one bounded grid barrier (all h written); the down weights of each warp's
+//             first phase-2 stages stream into its ring during the phase-1 tail and the
+//             barrier;
+//   phase 2   each CTA quantises the h of its experts (amax / 448, IEEE divide, e4m3
+//             round to nearest even) and runs the down GEMV (units of 16 down rows);
+//   combine   per block of 16 output rows, the last of the k + 1 experts to write it
+//             sums out = y_shared + sum_j w_j y_j in fixed j order.
+//
+// Work split: the shared expert's units and the routed experts' units are each cut into
+// one contiguous range per CTA (so every CTA holds 1-2 shared units to stream before
+// routing is known), and a CTA's stages go round-robin to its 24 warps, each with a
+// private ring of 2 stages filled by TMA (3-D code boxes with the 128-byte swizzle, 2-D
+// scale boxes).  Per 32-element block the warp decodes e2m1 pairs to f16 in registers
+// and runs two mma.sync m16n8k16 (fp32 accumulate); block partials are scaled by the
+// row's ue8m0 scale (exact) and the activation's fp32 block scale, and each row's stage
+// partials are summed in K order after a CTA barrier: results do not depend on timing and
+// equal those of the two-kernel path bit for bit.
+//
+// Every wait is bounded (%globaltimer): an expired wait records MOE_ERR_TIMEOUT in the
+// status word, the CTA skips its remaining work, lets its issued copies land, still
+// takes part in the grid barrier and returns.
+#include "internal.cuh"
+#include "ptx.cuh"
+#include "waits.cuh"
+
+#include <cstring>
+
+namespace bitmoe {
+
+// Grid barrier of the single-token kernel, one per device (zero when the module loads):
+// high word = generation, low word = CTAs arrived in the current generation.  The last
+// CTA to arrive adds 2^32 - G, which clears the count and opens the next generation.  It
+// serves one launch at a time: a launch holds every SM (one CTA per SM, by its shared
+// memory) until all its CTAs have passed the barrier, so a later launch's CTAs cannot
+// arrive before the barrier has opened.
+__device__ unsigned long long g_grid_bar;
+
+namespace {
+
+constexpr int kDcWarps = 24;
+constexpr int kDcThreads = kDcWarps * 32;
+constexpr int kDcStages = 2;                       // ring depth per warp
+constexpr int kDcRows = 16;                        // weight rows per stage
+constexpr int kDcCodeBytes = kDcRows * 256;        // 512 FP4 elements per row
+constexpr int kDcScaleBytes = kDcRows * 16;        // 16 ue8m0 bytes per row
+constexpr int kDcStageBytes = kDcCodeBytes + kDcScaleBytes;
+constexpr int kDcMaxUnits = 16;                    // units per CTA and phase
+constexpr int kDcMaxSlots = 33;                    // active experts (k <= 32) + shared
+constexpr int kDcP2Slots = 3;                      // experts whose h a CTA holds in phase 2
+
+enum { kModeForward = 0, kModeFfn = 1 };
+
+struct DecodeParams {
+  CUtensorMap tm_gc, tm_gs, tm_uc, tm_us, tm_dc, tm_ds;  // codes (3-D) and scales (2-D)
+  const float* scores;        // forward: [E] router scores
+  const uint16_t* x;          // [d] bf16 token
+  const int32_t* offsets_in;  // ffn: [E+1] from moe_dispatch
+  int32_t* idx;               // forward outputs: [k], [k], [E], [E+1], [k], [k]
+  float* w;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* perm;
+  int32_t* pos;
+  float* y_routed;            // [k][d], row = pair's sorted position
+  float* y_shared;            // [d]
+  float* out;                 // forward: [d]
+  uint8_t* qx;                // workspace: the token's codes [d] and scales [d/128]
+  float* sx;
+  uint8_t* qh;                // workspace: re-quantised h [k+1][f], scales [k+1][f/128]
+  float* sh;
+  float* hbuf;                // workspace: h [active experts][f] fp32 (shared last)
+  int* done2;                 // workspace: [d/16] combine counters (forward)
+  int E, k, d, f;
+  long long wait_ns;
+  int* status;
+  int stall;
+};
+
+// Shared memory: rings (codes, then scales), the phase-dependent area (phase 1: token as
+// f16, its scales, stage partials; phase 2: up to three experts' h as f16, scales, stage
+// partials), barriers, routing facts.
+struct DcSmem {
+  int d, f;
+  static constexpr int kOffScales = kDcWarps * kDcStages * kDcCodeBytes;
+  static constexpr int kOffArea = kOffScales + kDcWarps * kDcStages * kDcScaleBytes;
+  __host__ __device__ int p1_bs() const { return kOffArea + 2 * d; }
+  __host__ __device__ int p1_part() const { return p1_bs() + d / 32; }
+  __host__ __device__ int p1_end() const { return p1_part() + kDcMaxUnits * (d / 512) * 64; }
+  __host__ __device__ int p2_bs() const { return kOffArea + kDcP2Slots * 2 * f; }
+  __host__ __device__ int p2_part() const { return p2_bs() + kDcP2Slots * (f / 32); }
+  __host__ __device__ int p2_end() const { return p2_part() + kDcMaxUnits * (f / 512) * 64; }
+  __host__ __device__ int bars() const {
+    const int e = p1_end() > p2_end() ? p1_end() : p2_end();
+    return (e + 7) / 8 * 8;
+  }
+  // ring barriers [warp][stage], the stall barrier
+  __host__ __device__ int info() const { return bars() + (kDcWarps * kDcStages + 1) * 8; }
+  // int words: abort, n_active, then per slot (expert, row0, rows), then per pair
+  // (weight, pos)
+  __host__ __device__ int bytes() const { return info() + 4 * (4 + 3 * kDcMaxSlots + 64) + 1024; }
+};
+
+__device__ __forceinline__ void ue8m0x4_f32(uint32_t w, float (&f)[4]) {
+  const uint32_t m = 0x7F800000u, e0 = 0x00400000u;
+  f[0] = __uint_as_float(max((w << 23) & m, e0));
+  f[1] = __uint_as_float(max((w << 15) & m, e0));
+  f[2] = __uint_as_float(max((w << 7) & m, e0));
+  f[3] = __uint_as_float(max((w >> 1) & m, e0));
+}
+
+// Byte offset in a stage of bytes 4t..4t+3 of 32-block b (0..15) of stage row r (phase 1:
+// rows 0-7 gate, 8-15 up, boxes [matrix][half][8 rows]; phase 2: boxes [half][16 rows]);
+// the 128-byte swizzle XORs the 16-byte chunk with the row index mod 8.
+template <int PH>
+__device__ __forceinline__ uint32_t code_offset(int r, int b, int t) {
+  const int half = b >> 3, chunk = b & 7;
+  uint32_t box, rb;
+  if (PH == 1) {
+    box = (uint32_t)((r >> 3) * 2 + half) * 1024u;
+    rb = (uint32_t)(r & 7);
+  } else {
+    box = (uint32_t)half * 2048u;
+    rb = (uint32_t)r;
+  }
+  return box + rb * 128u + ((uint32_t)(chunk ^ (r & 7)) << 4) + 4u * (uint32_t)t;
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ int atom_add_acq_rel(int* p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v)
+               : "memory");
+  return old;
+}
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// One CTA's share of a phase: M = (routed experts + 1) * upe units in all, CTA b taking
+// [b*M/G, (b+1)*M/G) of them; its first ns are the shared expert's units [s_lo, s_lo+ns)
+// (s_lo = b*upe/G, a share that does not depend on the routing), the rest the routed units
+// [r_lo, r_lo+nr) of the list that runs over the active routed experts in slot order.
+struct Range {
+  int s_lo, ns, r_lo, nr, upe;
+  __device__ Range(int upe_, int n_routed, int G, int b) {
+    upe = upe_;
+    s_lo = (int)((long long)b * upe / G);
+    ns = (int)((long long)(b + 1) * upe / G) - s_lo;
+    const long long M = (long long)(n_routed + 1) * upe;
+    const long long t_lo = b * M / G, t_hi = (b + 1) * M / G;
+    r_lo = (int)(t_lo - s_lo);
+    nr = (int)(t_hi - t_lo) - ns;
+  }
+  __device__ int units() const { return ns + nr; }
+};
+
+// The bounded grid barrier (see g_grid_bar); false if the wait ran out.  ok_s: a word of
+// shared memory that carries thread 0's result to the CTA.
+__device__ bool grid_barrier(long long limit, int* status, volatile int* ok_s) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    __threadfence();
+    const unsigned long long G = gridDim.x;
+    const unsigned long long old = atomicAdd(&g_grid_bar, 1ull);
+    const unsigned long long gen = old >> 32;
+    if ((old & 0xffffffffull) + 1 == G) {
+      atomicAdd(&g_grid_bar, (1ull << 32) - G);
+    } else {
+      const uint64_t t0 = ptx::globaltimer();
+      while ((ld_acquire_u64(&g_grid_bar) >> 32) == gen) {
+        if ((long long)(ptx::globaltimer() - t0) > limit) {
+          atomicOr(status, kStatusTimeout);
+          ok = 0;
+          break;
+        }
+      }
+    }
+    __threadfence();
+    *ok_s = ok;
+  }
+  __syncthreads();
+  return *ok_s != 0;
+}
+
+template <int MODE, int PL>
+__global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (ptx::smem_u32(smem_raw) & 1023)) & 1023);
+  const DcSmem L{p.d, p.f};
+  const int d = p.d, f = p.f, E = p.E, k = p.k;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int G = gridDim.x, b = blockIdx.x;
+
+  uint16_t* bx = reinterpret_cast<uint16_t*>(smem + DcSmem::kOffArea);  // f16 activations
+  float* bs1 = reinterpret_cast<float*>(smem + L.p1_bs());
+  float* part1 = reinterpret_cast<float*>(smem + L.p1_part());
+  float* bs2 = reinterpret_cast<float*>(smem + L.p2_bs());
+  float* part2 = reinterpret_cast<float*>(smem + L.p2_part());
+  const uint32_t bars = ptx::smem_u32(smem + L.bars());
+  const uint32_t stall_bar = bars + 8u * (kDcWarps * kDcStages);
+  int* info = reinterpret_cast<int*>(smem + L.info());
+  volatile int* abort_flag = info;
+  int* n_active = info + 1;
+  volatile int* barrier_ok = info + 2;
+  int* slot_e = info + 4;                      // [slot] expert
+  int* slot_row = slot_e + kDcMaxSlots;        // [slot] first output row
+  int* slot_n = slot_row + kDcMaxSlots;        // [slot] rows (pairs) of the expert
+  float* pair_w = reinterpret_cast<float*>(slot_n + kDcMaxSlots);  // [j] gate weight
+  int* pair_pos = slot_n + kDcMaxSlots + 32;   // [j] sorted position
+
+  auto full = [&](int s) { return bars + 8u * (uint32_t)(warp * kDcStages + s); };
+  auto codes_at = [&](int s) { return smem + (warp * kDcStages + s) * kDcCodeBytes; };
+  auto scales_at = [&](int s) {
+    return smem + DcSmem::kOffScales + (warp * kDcStages + s) * kDcScaleBytes;
+  };
+
+  if (threadIdx.x == 0) {
+    ptx::prefetch_tmap(&p.tm_gc);
+    ptx::prefetch_tmap(&p.tm_gs);
+    ptx::prefetch_tmap(&p.tm_uc);
+    ptx::prefetch_tmap(&p.tm_us);
+    ptx::prefetch_tmap(&p.tm_dc);
+    ptx::prefetch_tmap(&p.tm_ds);
+    *abort_flag = 0;
+    ptx::mbar_init(stall_bar, 1);  // never arrived on: only the test stall waits on it
+  }
+  if (lane == 0)
+    for (int s = 0; s < kDcStages; ++s) ptx::mbar_init(full(s), 1);
+  ptx::fence_mbar_init();
+  if (MODE == kModeForward && b == 0)  // combine counters start at zero (published by the
+    for (int i = threadIdx.x; i < d / 16; i += kDcThreads) p.done2[i] = 0;  // grid barrier)
+  __syncthreads();
+
+  const int S1 = d / 512, S2 = f / 512;
+  const int upe1 = f / 8, upe2 = d / 16;
+  const uint64_t pol = ptx::make_policy_evict_first();
+
+  // n_act routed experts (known after routing); ranges and task counts follow from it
+  int n_act = MODE == kModeForward ? k : 0;
+  Range r1(upe1, n_act, G, b), r2(upe2, n_act, G, b);
+  int q1 = 0, q2 = 0;
+
+  // copies of this warp's q-th stage (phase 1 while q < q1), issued by lane 0
+  auto issue = [&](int q) {
+    const int st = q % kDcStages;
+    const uint32_t dc = ptx::smem_u32(codes_at(st)), ds = ptx::smem_u32(scales_at(st));
+    ptx::mbar_arrive_expect_tx(full(st), kDcStageBytes);
+    if (q < q1) {
+      const int task = warp + q * kDcWarps;
+      const int ul = task / S1, c = task % S1;
+      int e, uin;
+      if (ul < r1.ns) {
+        e = E;
+        uin = r1.s_lo + ul;
+      } else {
+        const int ru = r1.r_lo + ul - r1.ns;
+        e = slot_e[ru / upe1];
+        uin = ru % upe1;
+      }
+      const int row = e * f + uin * 8;
+      ptx::tma_load_3d_hint(dc, &p.tm_gc, 0, row, 2 * c, full(st), pol);
+      ptx::tma_load_3d_hint(dc + 2048, &p.tm_uc, 0, row, 2 * c, full(st), pol);
+      ptx::tma_load_2d_hint(ds, &p.tm_gs, c * 16, row, full(st), pol);
+      ptx::tma_load_2d_hint(ds + 128, &p.tm_us, c * 16, row, full(st), pol);
+    } else {
+      const int task = warp + (q - q1) * kDcWarps;
+      const int ul = task / S2, c = task % S2;
+      int e, uin;
+      if (ul < r2.ns) {
+        e = E;
+        uin = r2.s_lo + ul;
+      } else {
+        const int ru = r2.r_lo + ul - r2.ns;
+        e = slot_e[ru / upe2];
+        uin = ru % upe2;
+      }
+      const int row = e * d + uin * 16;
+      ptx::tma_load_3d_hint(dc, &p.tm_dc, 0, row, 2 * c, full(st), pol);
+      ptx::tma_load_2d_hint(ds, &p.tm_ds, c * 16, row, full(st), pol);
+    }
+  };
+
+  // the shared expert's first stages go out before routing is known
+  int issued = 0;
+  {
+    q1 = r1.ns * S1 > warp ? (r1.ns * S1 - warp + kDcWarps - 1) / kDcWarps : 0;  // shared only
+    const int early = q1 < kDcStages ? q1 : kDcStages;
+    if (lane == 0)
+      for (int q = 0; q < early; ++q) issue(q);
+    issued = early;
+  }
+
+  // ---------------------------------------------------------------- routing / plan
+  if (warp == 0) {
+    if (MODE == kModeForward) {
+      // top-k of the E scores (each lane holds experts lane + 32 i): k rounds of a warp
+      // arg-max on (value desc, index asc); then w_j = sigmoid(s_j) / sum over the k
+      float v[PL];
+#pragma unroll
+      for (int i = 0; i < PL; ++i) {
+        const int e = lane + 32 * i;
+        v[i] = e < E ? __ldg(p.scores + e) : -INFINITY;
+      }
+      unsigned taken = 0;
+      float sel_v = 0.f;
+      int sel_i = 0;
+      for (int j = 0; j < k; ++j) {
+        float bv = -INFINITY;
+        int bi = 0x7FFFFFFF;
+#pragma unroll
+        for (int i = 0; i < PL; ++i) {
+          const int e = lane + 32 * i;
+          const bool ok = !((taken >> i) & 1u) && e < E;
+          if (ok && (v[i] > bv || (v[i] == bv && e < bi))) {
+            bv = v[i];
+            bi = e;
+          }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+          const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+          if (ov > bv || (ov == bv && oi < bi)) {
+            bv = ov;
+            bi = oi;
+          }
+        }
+        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+        if (lane == j) {
+          sel_v = bv;
+          sel_i = bi;
+        }
+      }
+      const float sig = lane < k ? 1.0f / (1.0f + expf(-sel_v)) : 0.0f;
+      float sum = sig;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+      // slot (= sorted position) of pair j: the number of selected experts below it
+      int rank = 0;
+      for (int j = 0; j < k; ++j) {
+        const int ej = __shfl_sync(0xffffffffu, sel_i, j);
+        rank += (lane < k && ej < sel_i) ? 1 : 0;
+      }
+      if (lane < k) {
+        slot_e[rank] = sel_i;
+        slot_row[rank] = rank;
+        slot_n[rank] = 1;
+        pair_w[lane] = sig / sum;
+        pair_pos[lane] = rank;
+        if (b == 0) {
+          p.idx[lane] = sel_i;
+          p.w[lane] = sig / sum;
+          p.perm[rank] = lane;
+          p.pos[lane] = rank;
+        }
+      }
+      if (lane == 0) *n_active = k;
+    } else {
+      // active experts from the dispatch offsets, ascending: (expert, first row, rows)
+      const int per = (E + 31) / 32;
+      const int e0 = lane * per, e1 = min(E, e0 + per);
+      int local = 0;
+      for (int e = e0; e < e1; ++e) local += p.offsets_in[e + 1] > p.offsets_in[e] ? 1 : 0;
+      int incl = local;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int tt = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += tt;
+      }
+      int i = incl - local;
+      for (int e = e0; e < e1; ++e) {
+        const int lo = p.offsets_in[e], hi = p.offsets_in[e + 1];
+        if (hi > lo) {
+          if (i < kDcMaxSlots - 1 && lo >= 0 && hi <= k) {
+            slot_e[i] = e;
+            slot_row[i] = lo;
+            slot_n[i] = hi - lo;
+          } else {
+            atomicOr(p.status, kStatusBadIndex);
+          }
+          ++i;
+        }
+      }
+      if (lane == 31) *n_active = incl < kDcMaxSlots - 1 ? incl : kDcMaxSlots - 1;
+    }
+  } else if (warp <= 8) {
+    // the token: s = amax / 448 per 128-block (IEEE divide; 1 if amax = 0), q = e4m3(x / s)
+    // rounded to nearest even; 8 threads per block, 16 values each; f16 copies in smem
+    const int tid = threadIdx.x - 32;
+    for (int c0 = tid * 16; c0 - (tid & 31) * 16 < d; c0 += 256 * 16) {
+      const bool act = c0 < d;
+      uint4 a = make_uint4(0, 0, 0, 0), bb = make_uint4(0, 0, 0, 0);
+      if (act) {
+        a = *reinterpret_cast<const uint4*>(p.x + c0);
+        bb = *reinterpret_cast<const uint4*>(p.x + c0 + 8);
+      }
+      const float v[16] = {bf16_lo(a.x), bf16_hi(a.x), bf16_lo(a.y), bf16_hi(a.y),
+                           bf16_lo(a.z), bf16_hi(a.z), bf16_lo(a.w), bf16_hi(a.w),
+                           bf16_lo(bb.x), bf16_hi(bb.x), bf16_lo(bb.y), bf16_hi(bb.y),
+                           bf16_lo(bb.z), bf16_hi(bb.z), bf16_lo(bb.w), bf16_hi(bb.w)};
+      float amax = 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+      const float sc = amax == 0.f ? 1.0f : __fdiv_rn(amax, 448.0f);
+      uint32_t packed[4], hx[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint16_t lo = ptx::cvt_e4m3x2(__fdiv_rn(v[4 * i], sc), __fdiv_rn(v[4 * i + 1], sc));
+        const uint16_t hi =
+            ptx::cvt_e4m3x2(__fdiv_rn(v[4 * i + 2], sc), __fdiv_rn(v[4 * i + 3], sc));
+        packed[i] = (uint32_t)lo | ((uint32_t)hi << 16);
+        hx[2 * i] = ptx::cvt_e4m3x2_f16x2(lo);
+        hx[2 * i + 1] = ptx::cvt_e4m3x2_f16x2(hi);
+      }
+      if (act) {
+        uint4* dst = reinterpret_cast<uint4*>(bx + c0);
+        dst[0] = make_uint4(hx[0], hx[1], hx[2], hx[3]);
+        dst[1] = make_uint4(hx[4], hx[5], hx[6], hx[7]);
+        if ((tid & 7) == 0) bs1[c0 / 128] = sc;
+        if (b == 0) {
+          *reinterpret_cast<uint4*>(p.qx + c0) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+          if ((tid & 7) == 0) p.sx[c0 / 128] = sc;
+        }
+      }
+    }
+  }
+  __syncthreads();
+
+  n_act = *n_active;
+  r1 = Range(upe1, n_act, G, b);
+  r2 = Range(upe2, n_act, G, b);
+  const int nt1 = r1.units() * S1, nt2 = r2.units() * S2;
+  q1 = nt1 > warp ? (nt1 - warp + kDcWarps - 1) / kDcWarps : 0;
+  q2 = nt2 > warp ? (nt2 - warp + kDcWarps - 1) / kDcWarps : 0;
+  // the host keeps every range within these limits; a plan that breaks them stops here
+  if (r1.units() > kDcMaxUnits || r2.units() > kDcMaxUnits || r2.nr > r2.upe + 1) {
+    if (threadIdx.x == 0) atomicOr(p.status, kStatusBadIndex);
+    *abort_flag = 1;
+  }
+  const int qt = q1 + q2;
+  if (!*abort_flag) {
+    if (lane == 0)
+      for (int q = issued; q < kDcStages && q < qt; ++q) issue(q);
+    issued = max(issued, min(kDcStages, qt));
+  }
+
+  // CTA 0 stores the dispatch of the token (forward)
+  if (MODE == kModeForward && b == 0) {
+    for (int e = threadIdx.x; e <= E; e += kDcThreads) {
+      int below = 0, hit = 0;
+      for (int s = 0; s < k; ++s) {
+        below += slot_e[s] < e ? 1 : 0;
+        hit += slot_e[s] == e ? 1 : 0;
+      }
+      p.offsets[e] = below;
+      if (e < E) p.counts[e] = hit;
+    }
+  }
+
+  // phase 2's experts held by this CTA: local slot 0 = shared, 1.. = routed slots
+  const int r2_slot0 = r2.r_lo / upe2;
+  auto p2_local = [&](int ul, int& e, int& uin, int& ls, int& slot) {
+    if (ul < r2.ns) {
+      e = E;
+      uin = r2.s_lo + ul;
+      ls = 0;
+      slot = n_act;
+    } else {
+      const int ru = r2.r_lo + ul - r2.ns;
+      slot = ru / upe2;
+      e = slot_e[slot];
+      uin = ru % upe2;
+      ls = 1 + slot - r2_slot0;
+    }
+  };
+
+  // ---------------------------------------------------------------- phases 1 and 2
+  const int r0 = g, rr1 = g + 8;
+  bool ok = !*abort_flag;
+  bool switched = false;
+  int q = 0;
+
+  // all warps arrive here once, after their phase-1 stages: h of this CTA's units to
+  // the workspace, the grid barrier, then the h of phase 2's experts staged as f16
+  auto phase_switch = [&]() {
+    switched = true;
+    __syncthreads();
+    if (!*abort_flag) {
+      for (int i = threadIdx.x; i < r1.units() * 8; i += kDcThreads) {
+        const int ul = i >> 3, r = i & 7;
+        float gg = 0.f, uu = 0.f;
+        for (int c = 0; c < S1; ++c) {
+          gg += part1[(ul * S1 + c) * kDcRows + r];
+          uu += part1[(ul * S1 + c) * kDcRows + 8 + r];
+        }
+        int slot, uin;
+        if (ul < r1.ns) {
+          slot = n_act;
+          uin = r1.s_lo + ul;
+        } else {
+          const int ru = r1.r_lo + ul - r1.ns;
+          slot = ru / upe1;
+          uin = ru % upe1;
+        }
+        const float h = __fdividef(gg, 1.0f + expf(-gg)) * uu;
+        p.hbuf[(size_t)slot * f + uin * 8 + r] = h;
+      }
+    }
+    if (!grid_barrier(p.wait_ns, p.status, barrier_ok)) *abort_flag = 1;
+    // stage h: one warp per (local slot, 128-block), 4 values per lane
+    const int nb = f / 128;
+    const int nls = 1 + (r2.nr > 0 ? (r2.r_lo + r2.nr - 1) / upe2 - r2_slot0 + 1 : 0);
+    if (!*abort_flag) {
+      for (int wi = warp; wi < nls * nb; wi += kDcWarps) {
+        const int ls = wi / nb, j = wi % nb;
+        if (ls == 0 && r2.ns == 0) continue;
+        const int slot = ls == 0 ? n_act : r2_slot0 + ls - 1;
+        const float4 h = __ldcg(reinterpret_cast<const float4*>(p.hbuf + (size_t)slot * f +
+                                                                128 * j + 4 * lane));
+        float amax = fmaxf(fmaxf(fabsf(h.x), fabsf(h.y)), fmaxf(fabsf(h.z), fabsf(h.w)));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        const float sc = amax == 0.f ? 1.0f : __fdiv_rn(amax, 448.0f);
+        const uint16_t q01 = ptx::cvt_e4m3x2(__fdiv_rn(h.x, sc), __fdiv_rn(h.y, sc));
+        const uint16_t q23 = ptx::cvt_e4m3x2(__fdiv_rn(h.z, sc), __fdiv_rn(h.w, sc));
+        uint32_t* dst = reinterpret_cast<uint32_t*>(bx + (size_t)ls * f + 128 * j + 4 * lane);
+        dst[0] = ptx::cvt_e4m3x2_f16x2(q01);
+        dst[1] = ptx::cvt_e4m3x2_f16x2(q23);
+        if (lane == 0) bs2[ls * nb + j] = sc;
+        // the CTA holding the expert's first unit also stores its codes and scales
+        const bool owner = ls == 0 ? r2.s_lo == 0 : slot * upe2 >= r2.r_lo;
+        if (owner) {
+          const uint32_t qw = (uint32_t)q01 | ((uint32_t)q23 << 16);
+          const int rows = ls == 0 ? 1 : slot_n[slot];
+          const int row0 = ls == 0 ? k : slot_row[slot];
+          for (int rr = 0; rr < rows; ++rr) {
+            *reinterpret_cast<uint32_t*>(p.qh + (size_t)(row0 + rr) * f + 128 * j + 4 * lane) = qw;
+            if (lane == 0) p.sh[(size_t)(row0 + rr) * nb + j] = sc;
+          }
+        }
+      }
+    }
+    __syncthreads();
+  };
+
+  for (; q < qt; ++q) {
+    if (q == q1) phase_switch();
+    if (__shfl_sync(0xffffffffu, *abort_flag, 0)) {  // another warp gave up: stop too
+      ok = false;
+      break;
+    }
+    const int st = q % kDcStages;
+    if (p.stall && b == 0 && warp == 0 && q == 0 &&
+        !wait_warp(stall_bar, 0, p.wait_ns, abort_flag, p.status)) {
+      ok = false;
+      break;
+    }
+    if (!wait_warp(full(st), (uint32_t)(q / kDcStages) & 1u, p.wait_ns, abort_flag, p.status)) {
+      ok = false;
+      break;
+    }
+    const uint8_t* cst = codes_at(st);
+    const uint8_t* sst = scales_at(st);
+    float acc0 = 0.f, acc1 = 0.f;  // rows g and g+8 of the stage, column 0 (the token)
+    if (q < q1) {
+      const int task = warp + q * kDcWarps;
+      const int ul = task / S1, c = task % S1;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int j = 4 * c + i;
+        float fa[4], fb[4];
+        ue8m0x4_f32(*reinterpret_cast<const uint32_t*>(sst + r0 * 16 + 4 * i), fa);
+        ue8m0x4_f32(*reinterpret_cast<const uint32_t*>(sst + rr1 * 16 + 4 * i), fb);
+        float pa = 0.f, pb = 0.f;
+#pragma unroll
+        for (int bb = 0; bb < 4; ++bb) {
+          const int blk = 4 * i + bb;
+          const uint32_t wa = *reinterpret_cast<const uint32_t*>(cst + code_offset<1>(r0, blk, t));
+          const uint32_t wb = *reinterpret_cast<const uint32_t*>(cst + code_offset<1>(rr1, blk, t));
+          uint32_t ha[4], hb[4];
+          ptx::cvt_e2m1x8_f16(wa, ha);
+          ptx::cvt_e2m1x8_f16(wb, hb);
+          const uint4 xv = *reinterpret_cast<const uint4*>(bx + 128 * j + 32 * bb + 8 * t);
+          float cb[4];
+          ptx::mma_m16n8k16_f16_zero(cb, ha[0], hb[0], ha[1], hb[1], xv.x, xv.y);
+          ptx::mma_m16n8k16_f16(cb, ha[2], hb[2], ha[3], hb[3], xv.z, xv.w);
+          pa = fmaf(fa[bb], cb[0], pa);
+          pb = fmaf(fb[bb], cb[2], pb);
+        }
+        const float sxj = bs1[j];
+        acc0 = fmaf(sxj, pa, acc0);
+        acc1 = fmaf(sxj, pb, acc1);
+      }
+      __syncwarp();
+      if (issued < qt) {
+        if (lane == 0) issue(issued);
+        ++issued;
+      }
+      if (t == 0) {
+        float* pp = part1 + (ul * S1 + c) * kDcRows;
+        pp[r0] = acc0;
+        pp[rr1] = acc1;
+      }
+    } else {
+      const int task = warp + (q - q1) * kDcWarps;
+      const int ul = task / S2, c = task % S2;
+      int e, uin, ls, slot;
+      p2_local(ul, e, uin, ls, slot);
+      const uint16_t* xb = bx + (size_t)ls * f;
+      const float* sxb = bs2 + ls * (f / 128);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int j = 4 * c + i;
+        float fa[4], fb[4];
+        ue8m0x4_f32(*reinterpret_cast<const uint32_t*>(sst + r0 * 16 + 4 * i), fa);
+        ue8m0x4_f32(*reinterpret_cast<const uint32_t*>(sst + rr1 * 16 + 4 * i), fb);
+        float pa = 0.f, pb = 0.f;
+#pragma unroll
+        for (int bb = 0; bb < 4; ++bb) {
+          const int blk = 4 * i + bb;
+          const uint32_t wa = *reinterpret_cast<const uint32_t*>(cst + code_offset<2>(r0, blk, t));
+          const uint32_t wb = *reinterpret_cast<const uint32_t*>(cst + code_offset<2>(rr1, blk, t));
+          uint32_t ha[4], hb[4];
+          ptx::cvt_e2m1x8_f16(wa, ha);
+          ptx::cvt_e2m1x8_f16(wb, hb);
+          const uint4 xv = *reinterpret_cast<const uint4*>(xb + 128 * j + 32 * bb + 8 * t);
+          float cb[4];
+          ptx::mma_m16n8k16_f16_zero(cb, ha[0], hb[0], ha[1], hb[1], xv.x, xv.y);
+          ptx::mma_m16n8k16_f16(cb, ha[2], hb[2], ha[3], hb[3], xv.z, xv.w);
+          pa = fmaf(fa[bb], cb[0], pa);
+          pb = fmaf(fb[bb], cb[2], pb);
+        }
+        const float sxj = sxb[j];
+        acc0 = fmaf(sxj, pa, acc0);
+        acc1 = fmaf(sxj, pb, acc1);
+      }
+      __syncwarp();
+      if (issued < qt) {
+        if (lane == 0) issue(issued);
+        ++issued;
+      }
+      if (t == 0) {
+        float* pp = part2 + (ul * S2 + c) * kDcRows;
+        pp[r0] = acc0;
+        pp[rr1] = acc1;
+      }
+    }
+  }
+  if (!ok) {  // let the copies this warp issued land before the CTA can exit
+    *abort_flag = 1;
+    if (lane == 0)
+      for (int r = q; r < issued; ++r) drain_wait(full(r % kDcStages), (uint32_t)(r / kDcStages) & 1u);
+    __syncwarp();
+  }
+  if (!switched) phase_switch();
+  __syncthreads();
+  if (*abort_flag) return;
+
+  // ---------------------------------------------------------------- phase-2 results
+  for (int i = threadIdx.x; i < r2.units() * kDcRows; i += kDcThreads) {
+    const int ul = i >> 4, r = i & 15;
+    float y = 0.f;
+    for (int c = 0; c < S2; ++c) y += part2[(ul * S2 + c) * kDcRows + r];
+    int e, uin, ls, slot;
+    p2_local(ul, e, uin, ls, slot);
+    const size_t m = (size_t)uin * 16 + r;
+    if (ls == 0) {
+      p.y_shared[m] = y;
+    } else {
+      for (int rr = 0; rr < slot_n[slot]; ++rr) p.y_routed[(size_t)(slot_row[slot] + rr) * d + m] = y;
+    }
+  }
+  if (MODE == kModeForward) {
+    // per 16-row output block, the last of the k + 1 experts to finish it sums out
+    __syncthreads();
+    for (int ul = warp; ul < r2.units(); ul += kDcWarps) {
+      int e, uin, ls, slot;
+      p2_local(ul, e, uin, ls, slot);
+      int last = 0;
+      if (lane == 0) {
+        __threadfence();
+        last = atom_add_acq_rel(p.done2 + uin, 1) == n_act ? 1 : 0;
+      }
+      last = __shfl_sync(0xffffffffu, last, 0);
+      if (last && lane < 16) {
+        const size_t m = (size_t)uin * 16 + lane;
+        float acc = __ldcg(p.y_shared + m);
+        for (int j = 0; j < k; ++j)
+          acc = fmaf(pair_w[j], __ldcg(p.y_routed + (size_t)pair_pos[j] * d + m), acc);
+        p.out[m] = acc;
+      }
+    }
+  }
+}
+
+// 2-D map over a byte matrix [rows][cols]; box = box_cols bytes x box_rows rows
+bool make_byte_map(CUtensorMap* m, const void* base, long long cols, long long rows, int box_cols,
+                   int box_rows) {
+  EncodeTiledFn fn = tensor_map_encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols};
+  const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+// 3-D map over FP4 code rows [rows][cols bytes] viewed as (128-byte piece, row, piece
+// index): a box of 2 pieces x box_rows rows lands as [piece][row][128 bytes], 128-byte
+// swizzle
+bool make_code_map(CUtensorMap* m, const void* base, long long cols, long long rows, int box_rows) {
+  EncodeTiledFn fn = tensor_map_encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {128u, (cuuint64_t)rows, (cuuint64_t)(cols / 128)};
+  const cuuint64_t strides[2] = {(cuuint64_t)cols, 128u};
+  const cuuint32_t box[3] = {128u, (cuuint32_t)box_rows, 2u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int MODE, int PL>
+cudaError_t launch_one(const DecodeParams& prm, cudaStream_t s, int grid) {
+  const DcSmem L{prm.d, prm.f};
+  const size_t smem = (size_t)L.bytes();
+  auto kern = decode_kernel<MODE, PL>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kDcThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;  // every CTA resident: the grid barrier
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, prm);
+}
+
+}  // namespace
+
+size_t decode_smem_bytes(int d, int f) { return (size_t)DcSmem{d, f}.bytes(); }
+
+bool decode_fits(int k, int d, int f, int ctas) {
+  if (k < 1 || k > 32 || d % 512 || f % 512 || ctas < 1) return false;
+  const long long upe1 = f / 8, upe2 = d / 16;
+  // the most units a CTA can get in either phase (fewer active experts give fewer)
+  auto most = [&](long long upe) { return ((long long)(k + 1) * upe + ctas - 1) / ctas; };
+  if (most(upe1) > kDcMaxUnits || most(upe2) > kDcMaxUnits) return false;
+  // a CTA's phase-2 routed range spans at most two experts
+  if (most(upe2) > upe2 + 1) return false;
+  return true;
+}
+
+cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t s, int num_sms) {
+  DecodeParams p;
+  memset(&p, 0, sizeof(p));
+  const long long rows1 = (long long)(a.E + 1) * a.f, rows2 = (long long)(a.E + 1) * a.d;
+  if (!make_code_map(&p.tm_gc, a.gate_codes, a.d / 2, rows1, 8) ||
+      !make_byte_map(&p.tm_gs, a.gate_scales, a.d / 32, rows1, 16, 8) ||
+      !make_code_map(&p.tm_uc, a.up_codes, a.d / 2, rows1, 8) ||
+      !make_byte_map(&p.tm_us, a.up_scales, a.d / 32, rows1, 16, 8) ||
+      !make_code_map(&p.tm_dc, a.down_codes, a.f / 2, rows2, 16) ||
+      !make_byte_map(&p.tm_ds, a.down_scales, a.f / 32, rows2, 16, 16))
+    return cudaErrorInvalidValue;
+  p.scores = a.scores;
+  p.x = a.x;
+  p.offsets_in = a.offsets_in;
+  p.idx = a.idx;
+  p.w = a.w_out;
+  p.counts = a.counts;
+  p.offsets = a.offsets;
+  p.perm = a.perm;
+  p.pos = a.pos;
+  p.y_routed = a.y_routed;
+  p.y_shared = a.y_shared;
+  p.out = a.out;
+  p.qx = a.qx;
+  p.sx = a.sx;
+  p.qh = a.qh;
+  p.sh = a.sh;
+  p.hbuf = a.hbuf;
+  p.done2 = a.done2;
+  p.E = a.E;
+  p.k = a.k;
+  p.d = a.d;
+  p.f = a.f;
+  p.wait_ns = a.wait_ns;
+  p.status = a.status;
+  p.stall = a.stall;
+  const int grid = num_sms < kMaxCtas ? num_sms : kMaxCtas;
+  if (a.forward) {
+    if (a.E <= 256) return launch_one<kModeForward, 8>(p, s, grid);
+    return launch_one<kModeForward, 32>(p, s, grid);
+  }
+  return launch_one<kModeFfn, 8>(p, s, grid);
+}
+
+cudaError_t reset_grid_barrier() {
+  const unsigned long long zero = 0;
+  return cudaMemcpyToSymbol(g_grid_bar, &zero, sizeof(zero));
+}
+
+}  // namespace bitmoe

@@ -120,12 +120,12 @@ __global__ void __launch_bounds__(1024, 1) dispatch_kernel(const int32_t* __rest
 
 cudaError_t launch_dispatch(const int32_t* idx, int T, int k, int E, int32_t* counts,
                             int32_t* offsets, int32_t* perm, int32_t* pos, int* status,
-                            cudaStream_t s) {
+                            cudaStream_t s, bool overlap) {
   const size_t smem = sizeof(int32_t) * ((size_t)kWarps * E + E + 1 + 32);
   cudaError_t err = cudaFuncSetAttribute(dispatch_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  return launch_pdl(dispatch_kernel, dim3(1), dim3(1024), smem, s, false, idx, T * k, E, counts, offsets,
+  return launch_pdl(dispatch_kernel, dim3(1), dim3(1024), smem, s, overlap, idx, T * k, E, counts, offsets,
                     perm, pos, status);
 }
 

@@ -39,7 +39,7 @@ inline size_t plan_ntmax(int R, int E) { return (size_t)R / 16 + (size_t)E + 2; 
 constexpr int kGemvMaxT = 1;
 
 struct WorkspaceLayout {
-  size_t plan, qx, sx, qh, sh, counters, partials, hbuf, total;
+  size_t plan, qx, sx, qh, sh, counters, partials, hbuf, done2, total;
   size_t n_counters;
 };
 WorkspaceLayout workspace_layout(int T, int k, int E, int d, int f);
@@ -49,7 +49,7 @@ cudaError_t launch_route_topk(const float* scores, int T, int E, int k, int32_t*
                               cudaStream_t s);
 cudaError_t launch_dispatch(const int32_t* idx, int T, int k, int E, int32_t* counts,
                             int32_t* offsets, int32_t* perm, int32_t* pos, int* status,
-                            cudaStream_t s);
+                            cudaStream_t s, bool overlap = false);
 // rows r < P = T*k take token perm[r]/k, rows P <= r < P+T take token r-P; perm may be
 // NULL with P = 0 for a plain quantisation of T rows.  If plan != NULL, one extra block
 // writes the token-tile plan (plan_mode 0) or the single-token path's list of active
@@ -57,9 +57,11 @@ cudaError_t launch_dispatch(const int32_t* idx, int T, int k, int E, int32_t* co
 cudaError_t launch_quant_rows(const uint16_t* x, int T, int k, int d, const int32_t* perm,
                               int nrows_routed, uint8_t* q, float* s, const int32_t* offsets,
                               int E, int nmax, int32_t* plan, int* counters, size_t n_counters,
-                              int* status, cudaStream_t st, int plan_mode = 0);
+                              int* status, cudaStream_t st, int plan_mode = 0,
+                              bool overlap = false);
 cudaError_t launch_combine(const float* y, const float* ysh, const float* w, const int32_t* pos,
-                           int T, int k, int d, float* out, int* status, cudaStream_t s);
+                           int T, int k, int d, float* out, int* status, cudaStream_t s,
+                           bool overlap = false);
 
 struct FfnArgs {
   const uint8_t* a0_codes;   // gate (phase 1) or down (phase 2) codes, all experts
@@ -116,6 +118,40 @@ size_t gemv_smem_bytes(int phase, int K);
 // a launch's units (8 h-rows in phase 1, 16 down rows in phase 2, of every active
 // expert) are cut into one range per CTA of at most this many units
 int gemv_max_units_per_cta();
+
+// Single-token layer in one cooperative kernel (decode.cu): forward = routing from the
+// scores, dispatch and combine included; otherwise the expert FFN from dispatch offsets.
+struct DecodeLaunch {
+  bool forward;
+  const uint8_t* gate_codes;
+  const uint8_t* gate_scales;
+  const uint8_t* up_codes;
+  const uint8_t* up_scales;
+  const uint8_t* down_codes;
+  const uint8_t* down_scales;
+  const float* scores;
+  const uint16_t* x;
+  const int32_t* offsets_in;
+  int32_t *idx, *counts, *offsets, *perm, *pos;
+  float* w_out;
+  float *y_routed, *y_shared, *out;
+  uint8_t* qx;
+  float* sx;
+  uint8_t* qh;
+  float* sh;
+  float* hbuf;
+  int* done2;
+  int E, k, d, f;
+  long long wait_ns;
+  int* status;
+  int stall;
+};
+cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t s, int num_sms);
+size_t decode_smem_bytes(int d, int f);
+// whether the single-token kernel's per-CTA limits hold for (k, d, f) on `ctas` CTAs
+bool decode_fits(int k, int d, int f, int ctas);
+// clears the single-token kernel's grid barrier (after a reported timeout)
+cudaError_t reset_grid_barrier();
 
 // Launch, with `overlap`, as a programmatic dependent launch: the kernel may start while
 // the previous kernel on the stream finishes (every kernel of this library calls

@@ -153,12 +153,12 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(
 cudaError_t launch_quant_rows(const uint16_t* x, int T, int k, int d, const int32_t* perm,
                               int nrows_routed, uint8_t* q, float* s, const int32_t* offsets,
                               int E, int nmax, int32_t* plan, int* counters, size_t n_counters,
-                              int* status, cudaStream_t st, int plan_mode) {
+                              int* status, cudaStream_t st, int plan_mode, bool overlap) {
   const int R = nrows_routed + T;
   const unsigned blocks = (unsigned)(R + (plan != nullptr ? 1 : 0));
   int threads = (d / 16 + 31) / 32 * 32;  // whole warps
   if (threads > 256) threads = 256;
-  return launch_pdl(quant_rows_kernel, dim3(blocks), dim3(threads), 0, st, false, x, T, k, d, perm,
+  return launch_pdl(quant_rows_kernel, dim3(blocks), dim3(threads), 0, st, overlap, x, T, k, d, perm,
                     nrows_routed, q, s, offsets, E, nmax, plan, counters, n_counters, status,
                     plan_mode);
 }

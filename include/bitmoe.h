@@ -38,6 +38,10 @@
  *   - T == 0 is a valid no-op.
  *   - Errors found on the device (a bounded wait that expired) are recorded in a
  *     device-side status word and returned by moe_sync_status().
+ *   - On first use on a device the library looks up and keeps the device addresses of its
+ *     own device variables (the status word, the single-token kernel's grid barrier, the
+ *     scratch of moe_expert_ffn_noalloc).  cudaDeviceReset unloads them: after a reset,
+ *     make no further call of this library on that device in the same process.
  */
 #ifndef BITMOE_H
 #define BITMOE_H
@@ -144,6 +148,25 @@ int moe_ffn_down(int T, int k, const moe_weights_t* w, float* y_routed, float* y
 int moe_expert_ffn_noalloc(const uint16_t* x_bf16, int T, int k, const moe_weights_t* w,
                            const int32_t* offsets, const int32_t* perm, float* y_routed,
                            float* y_shared, void* stream);
+
+/* Steps 1-8 in one call: route, dispatch, expert FFN and combine for T tokens, with the
+ * arguments, outputs and rules of the four calls above (the outputs are the same arrays:
+ * topk_idx [T][k], topk_w [T][k], counts [E], offsets [E+1], perm [T*k], pos [T*k],
+ * y_routed [T*k][d], y_shared [T][d], out [T][d]; ws as for moe_expert_ffn).  The pages
+ * describe the layer as this one sequence ([P2] "核心实现一" to "核心实现四").
+ * A single token (T = 1; d, f multiples of 512; scale arrays 16-byte aligned; k <= 32)
+ * runs as ONE cooperative kernel: routing, dispatch, quantisation, both FP4 GEMVs and
+ * the combine, streaming the selected experts' weights from its first instruction.  Its
+ * results equal those of the four calls bit for bit.  It needs every SM of the device for
+ * the duration of the kernel (one block per SM, all resident at once), which a launch
+ * under MPS limits or beside other resident work may not get: such a launch fails with
+ * MOE_ERR_CUDA (cooperative launch too large) instead of running.  Larger batches run the
+ * four calls back to back, each kernel after the first allowed to start under the tail
+ * of the one before it.  k <= 32. */
+int moe_forward(const float* scores, const uint16_t* x_bf16, int T, int k,
+                const moe_weights_t* w, int32_t* topk_idx, float* topk_w, int32_t* counts,
+                int32_t* offsets, int32_t* perm, int32_t* pos, float* y_routed, float* y_shared,
+                float* out, void* ws, size_t ws_bytes, void* stream);
 
 /* Step 8 — combine: out[t][m] = y_shared[t][m] + sum_{j<k} topk_w[t][j] *
  * y_routed[pos[t*k+j]][m], summed in fixed j order in fp32.

@@ -236,15 +236,17 @@ def check_h_codes(qg, sg, qo, so, hf_o, ex, d, xhat, stats: HStats, what=""):
 
 
 # --------------------------------------------------------------------------------- GPU runs
-def gpu_layer(x, scores, k, weights, ws=None, keep_device=False):
-    """One layer through the four calls; returns every result and the intermediates
-    moe_expert_ffn left in the workspace (on the host unless keep_device)."""
+def gpu_layer(x, scores, k, weights, ws=None, keep_device=False, calls=False):
+    """One layer through moe_forward (or, with calls=True, the four separate calls);
+    returns every result and the intermediates left in the workspace (on the host unless
+    keep_device)."""
     import bit_moe_routed_b200 as bm
     T, d = x.shape
     E, f = weights.E, weights.f
     if ws is None:
         ws = bm.alloc_workspace(T, k, E, d, f)
-    r = bm.forward(x.cuda(), scores.cuda(), k, weights, ws)
+    run = bm.forward_calls if calls else bm.forward
+    r = run(x.cuda(), scores.cuda(), k, weights, ws)
     r.update({kk: v.clone() for kk, v in bm.workspace_views(ws, T, k, E, d, f).items()})
     if keep_device:
         return r

@@ -1,0 +1,118 @@
+"""The single-token layer kernel (decode.cu) splits each phase's units over its CTAs: CTA b
+takes [b*M/G, (b+1)*M/G) of all M = (active routed experts + 1) * U units (U the units per
+expert: f/8 in phase 1, d/16 in phase 2), of which the first are its share of the shared
+expert's units [b*U/G, (b+1)*U/G) (streamed before routing is known) and the rest a
+contiguous range of the routed experts' units.  A CTA keeps at most 16 units' partial sums
+and, in phase 2, the hidden state of the shared expert and of at most two routed experts
+in shared memory.  This checks on the CPU, before any launch, that the host's condition
+(decode_fits in decode.cu) implies those limits for every shape it accepts and every
+number of active experts, that the ranges cover every unit exactly once, that every TMA
+box the kernel addresses lies inside its tensor, and that the shared-memory layout fits
+the 227 KB a B200 CTA may use at the decode workload's sizes."""
+import itertools
+
+import pytest
+
+MAX_UNITS = 16    # kDcMaxUnits
+P2_SLOTS = 3      # kDcP2Slots: shared + two routed
+WARPS = 24
+STAGE_BYTES = 16 * 256 + 16 * 16
+SMEM_LIMIT = 232448   # bytes of shared memory a CTA may opt into on sm_100
+
+
+def decode_fits(k, d, f, ctas):
+    """Mirror of decode_fits() in decode.cu."""
+    if k < 1 or k > 32 or d % 512 or f % 512 or ctas < 1:
+        return False
+
+    def most(upe):
+        return -(-((k + 1) * upe) // ctas)
+
+    upe1, upe2 = f // 8, d // 16
+    if most(upe1) > MAX_UNITS or most(upe2) > MAX_UNITS:
+        return False
+    return most(upe2) <= upe2 + 1
+
+
+def split(upe, n_routed, G, b):
+    """Mirror of the kernel's Range: (s_lo, ns, r_lo, nr)."""
+    s_lo = b * upe // G
+    ns = (b + 1) * upe // G - s_lo
+    M = (n_routed + 1) * upe
+    t_lo, t_hi = b * M // G, (b + 1) * M // G
+    return s_lo, ns, t_lo - s_lo, (t_hi - t_lo) - ns
+
+
+def smem_bytes(d, f):
+    """Mirror of DcSmem::bytes()."""
+    area = WARPS * 2 * STAGE_BYTES
+    p1_end = area + 2 * d + d // 32 + MAX_UNITS * (d // 512) * 64
+    p2_end = area + P2_SLOTS * 2 * f + P2_SLOTS * (f // 32) + MAX_UNITS * (f // 512) * 64
+    bars = (max(p1_end, p2_end) + 7) // 8 * 8
+    info = bars + (WARPS * 2 + 1) * 8
+    return info + 4 * (4 + 3 * 33 + 64) + 1024
+
+
+@pytest.mark.parametrize("ctas", [148, 132, 100])
+def test_accepted_shapes_fit_every_range(ctas):
+    checked = 0
+    for k, d, f in itertools.product(range(1, 33), (512, 1024, 2048, 4096, 7168, 8192),
+                                     (512, 1024, 1536, 2048, 4096)):
+        if not decode_fits(k, d, f, ctas):
+            continue
+        for n_act in range(1, k + 1):   # a caller's dispatch may repeat experts
+            for upe in (f // 8, d // 16):
+                shared, routed = [], []
+                for b in range(ctas):
+                    s_lo, ns, r_lo, nr = split(upe, n_act, ctas, b)
+                    assert nr >= 0 and ns + nr <= MAX_UNITS
+                    shared.extend(range(s_lo, s_lo + ns))
+                    routed.extend(range(r_lo, r_lo + nr))
+                    if upe == d // 16 and nr:
+                        slots = (r_lo + nr - 1) // upe - r_lo // upe + 1
+                        assert slots <= P2_SLOTS - 1
+                assert shared == list(range(upe))
+                assert routed == list(range(n_act * upe))
+                checked += 1
+    assert checked > 500
+
+
+def test_decode_workload_is_accepted_and_fits_shared_memory():
+    assert decode_fits(6, 4096, 2048, 148)
+    assert smem_bytes(4096, 2048) <= SMEM_LIMIT
+    # every CTA holds one or two shared units to stream before routing is known
+    for b in range(148):
+        s_lo, ns, r_lo, nr = split(2048 // 8, 6, 148, b)
+        assert 1 <= ns <= 2 and ns + nr in (12, 13)
+
+
+def test_tma_boxes_stay_inside_their_tensors():
+    """Phase 1 boxes: rows e*f + u*8 .. +8 of [(E+1)*f] rows, code pieces 2c, 2c+1 of d/256,
+    scale bytes 16c .. 16c+16 of d/32; phase 2 likewise with 16 rows, d and f swapped."""
+    for E, k, d, f in ((256, 6, 4096, 2048), (8, 2, 512, 512), (1024, 8, 1024, 512),
+                       (64, 32, 512, 512)):
+        assert decode_fits(k, d, f, 148)
+        for rows_box, upe, K, rows_per in ((8, f // 8, d, f), (16, d // 16, f, d)):
+            for e in (0, E):
+                last_row = e * rows_per + (upe - 1) * rows_box + rows_box
+                assert last_row <= (E + 1) * rows_per
+            for c in range(K // 512):
+                assert 2 * c + 1 < K // 256
+                assert 16 * c + 16 <= K // 32
+
+
+def test_every_warp_takes_its_tasks_once():
+    """Tasks go round-robin (task = warp + 24 q); the first two of each warp are issued
+    before routing only when they belong to the shared expert."""
+    S1 = 4096 // 512
+    for b in (0, 73, 147):
+        s_lo, ns, r_lo, nr = split(2048 // 8, 6, 148, b)
+        n_tasks = (ns + nr) * S1
+        seen = []
+        for w in range(WARPS):
+            q1 = -(-(n_tasks - w) // WARPS) if n_tasks > w else 0
+            seen.extend(w + WARPS * q for q in range(q1))
+            shared_q = -(-(ns * S1 - w) // WARPS) if ns * S1 > w else 0
+            for q in range(min(shared_q, 2)):
+                assert (w + WARPS * q) // S1 < ns
+        assert sorted(seen) == list(range(n_tasks))

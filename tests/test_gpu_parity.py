@@ -103,15 +103,16 @@ def test_act_quant_special_rows():
 
 
 # ---------------------------------------------------------------- whole layer, small shapes
-def _small_layer(T, E, k, d, f, routing="uniform", seed=5, zero_rows=()):
+def _small_layer(T, E, k, d, f, routing="uniform", seed=5, zero_rows=(), calls=False):
     x = synth.gen_x(T, d, seed=seed)
     for r in zero_rows:
         x[r] = 0
     s = synth.gen_scores_uniform(T, E, seed + 1) if routing == "uniform" else \
         synth.gen_scores_zipf(T, E, 1.2, seed + 1)
     W = device_weights(seed, 0, E, d, f)
-    g = gpu_layer(x, s, k, W)
-    check_layer(g, x, s, k, E, d, f, seed, 0, list(range(T)), f"T={T} E={E} k={k} d={d} f={f}")
+    g = gpu_layer(x, s, k, W, calls=calls)
+    check_layer(g, x, s, k, E, d, f, seed, 0, list(range(T)),
+                f"T={T} E={E} k={k} d={d} f={f}" + (" (four calls)" if calls else ""))
 
 
 def test_layer_tiny_workload():
@@ -182,14 +183,68 @@ def test_layer_extreme_weights():
 
 
 # ---------------------------------------------------------------- single-token GEMV path
+@pytest.mark.parametrize("calls", [False, True], ids=["forward", "calls"])
 @pytest.mark.parametrize("E,k,d,f", [
     (8, 2, 512, 512),       # one stage per row along d and along f
     (16, 4, 1024, 512),
     (32, 6, 512, 1536),     # three stages per down row
     (256, 6, 2048, 1024),   # CTA ranges that span two experts
+    (1024, 8, 1024, 512),   # many experts: top-k over 32 scores per lane
+    (64, 32, 512, 512),     # the most experts per token
 ])
-def test_gemv_single_token_shapes(E, k, d, f):
-    _small_layer(1, E, k, d, f, "uniform", seed=E + d + f)
+def test_gemv_single_token_shapes(E, k, d, f, calls):
+    _small_layer(1, E, k, d, f, "uniform", seed=E + d + f + k, calls=calls)
+
+
+def test_single_token_paths_agree_bit_for_bit():
+    """One token through moe_forward (one kernel), the four calls (the FFN as one kernel),
+    and the three exposed FFN stages (two GEMV kernels): identical results."""
+    E, k, d, f = 256, 6, 4096, 2048
+    x = synth.gen_x(1, d, seed=61)
+    s = synth.gen_scores_uniform(1, E, seed=62)
+    W = device_weights(63, 0, E, d, f)
+    a = gpu_layer(x, s, k, W)
+    b = gpu_layer(x, s, k, W, calls=True)
+    xd, sd = x.cuda(), s.cuda()
+    idx, gw = bm.route_topk(sd, k)
+    counts, offsets, perm, pos = bm.dispatch(idx, E)
+    ws = bm.alloc_workspace(1, k, E, d, f)
+    y = torch.empty((k, d), dtype=torch.float32, device="cuda")
+    ysh = torch.empty((1, d), dtype=torch.float32, device="cuda")
+    bm.ffn_prepare(xd, k, W, offsets, perm, ws)
+    bm.ffn_gate_up(1, k, W, ws)
+    bm.ffn_down(1, k, W, y, ysh, ws)
+    out = bm.combine(y, ysh, gw, pos)
+    c = dict(idx=idx, w=gw, counts=counts, offsets=offsets, perm=perm, pos=pos, y=y,
+             y_shared=ysh, out=out)
+    c.update(bm.workspace_views(ws, 1, k, E, d, f))
+    bm.sync_status()
+    for name in ("idx", "w", "counts", "offsets", "perm", "pos", "y", "y_shared", "out", "qh",
+                 "sh", "h"):
+        assert torch.equal(a[name].cpu(), b[name].cpu()), f"forward vs calls: {name}"
+        assert torch.equal(a[name].cpu(), c[name].cpu()), f"forward vs stages: {name}"
+    for name in ("qx", "sx"):  # the single-token path writes row 0, the token
+        assert torch.equal(a[name].cpu()[0], b[name].cpu()[0]), f"forward vs calls: {name}"
+        assert torch.equal(a[name].cpu()[0], c[name].cpu()[0]), f"forward vs stages: {name}"
+
+
+def test_single_token_repeated_expert_in_dispatch():
+    """moe_expert_ffn at one token with an expert listed twice in topk_idx (a caller's own
+    routing): both of its rows get the expert's output."""
+    E, k, d, f = 8, 3, 512, 512
+    x = synth.gen_x(1, d, seed=71)
+    W = device_weights(72, 0, E, d, f)
+    idx = torch.tensor([[5, 2, 5]], dtype=torch.int32, device="cuda")
+    counts, offsets, perm, pos = bm.dispatch(idx, E)
+    y, ysh = bm.expert_ffn(x.cuda(), k, W, offsets, perm)
+    bm.sync_status()
+    qx, sx = oracle.act_quant(x)
+    ex = host_experts(72, 0, d, f, [2, 5, E])
+    y_cpu = y.cpu().numpy()
+    for j, e in enumerate([5, 2, 5]):
+        yo = oracle.expert_ffn(ex[e], d, f, qx, sx)[0]
+        assert_close(y_cpu[int(pos[j])], yo, f"pair {j} (expert {e})")
+    assert_close(ysh.cpu().numpy()[0], oracle.expert_ffn(ex[E], d, f, qx, sx)[0], "shared")
 
 
 def _custom_layer_check(T, E, k, d, f, arrs, seed, label):
@@ -253,12 +308,12 @@ def test_device_generator_matches_host_generator():
 
 
 # ---------------------------------------------------------------- full-size workloads
-def _full_workload(name, tokens=None, n_sample=64):
+def _full_workload(name, tokens=None, n_sample=64, calls=False):
     w_ = synth.WORKLOADS[name]
     x, s = synth.gen_layer_inputs(w_, 0)
     W = device_weights(w_.seed(), 0, w_.E, w_.d, w_.f)
     oracle.set_threads(max(8, (__import__("os").cpu_count() or 8)))
-    g = gpu_layer(x, s, w_.k, W)
+    g = gpu_layer(x, s, w_.k, W, calls=calls)
     del W
     torch.cuda.empty_cache()
     if tokens is None:
@@ -268,11 +323,12 @@ def _full_workload(name, tokens=None, n_sample=64):
     return g
 
 
-@pytest.mark.parametrize("gemv", [1, 0], ids=["gemv", "tiles"])
-def test_decode_t1_full(gemv):
-    bm.set_gemv_max_tokens(gemv)
+@pytest.mark.parametrize("path", ["forward", "calls", "tiles"])
+def test_decode_t1_full(path):
+    """decode_t1 through moe_forward (one kernel), the four calls, and the tile kernels."""
+    bm.set_gemv_max_tokens(0 if path == "tiles" else 1)
     try:
-        _full_workload("decode_t1", [0])
+        _full_workload("decode_t1", [0], calls=path == "calls")
     finally:
         bm.set_gemv_max_tokens(1)
 

@@ -30,6 +30,7 @@ def test_ffn_stays_inside_workspace(T):
     counts, offsets, perm, pos = bm.dispatch(idx, E)
     y, ysh = bm.expert_ffn(x, k, W, offsets, perm, ws)
     bm.combine(y, ysh, gw, pos)
+    bm.forward(x, s, k, W, ws)  # the whole-layer call (one kernel at T = 1)
     bm.sync_status()
     tail = buf[n:]
     bad = int((tail != 0xA5).sum())
