@@ -29,6 +29,7 @@ MOE_ERR_CUDA = -3
 MOE_ERR_TIMEOUT = -4
 MOE_ERR_UNSUPPORTED = -5
 MOE_NOALLOC_SCRATCH_BYTES = 24 << 20  # the fixed scratch of moe_expert_ffn_noalloc
+GEMV_MAX_TOKENS = 64                  # default of moe_set_gemv_max_tokens
 
 EXPORTS = (
     "moe_route_topk", "moe_dispatch", "moe_act_quant", "moe_expert_ffn", "moe_ffn_prepare",
@@ -161,7 +162,8 @@ def set_test_stall(on: bool) -> None:
 
 
 def set_gemv_max_tokens(t: int) -> None:
-    """Batches up to t tokens (0 or 1) take the single-token FP4 GEMV path."""
+    """Batches up to t tokens (at most 64) take the FP4 GEMV paths; 0 sends every batch to
+    the tcgen05 tile kernels."""
     _check(lib().moe_set_gemv_max_tokens(int(t)))
 
 

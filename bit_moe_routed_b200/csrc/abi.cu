@@ -29,7 +29,7 @@ struct OverlapScope {
   ~OverlapScope() { t_overlap = saved; }
 };
 std::atomic<long long> g_wait_ns{2000000000LL};
-std::atomic<int> g_gemv_max_t{kGemvMaxT};  // batches up to this size take the GEMV path
+std::atomic<int> g_gemv_max_t{kBgMaxT};  // batches up to this size take a GEMV path
 std::atomic<int> g_stall{0};                 // test knob: see moe_set_test_stall
 
 int fail(int code, const char* fmt, ...) {
@@ -119,6 +119,49 @@ EncodeTiledFn tensor_map_encode_fn() {
   return fn;
 }
 
+// 2-D map over a byte matrix [rows][cols]; box = box_cols bytes x box_rows rows, no swizzle.
+bool make_byte_map(CUtensorMap* m, const void* base, long long cols, long long rows, int box_cols,
+                   int box_rows) {
+  EncodeTiledFn fn = tensor_map_encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols};
+  const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D map over byte rows [rows][cols] viewed as (128-byte piece, row, piece index): a box of
+// `pieces` pieces x box_rows rows lands as [piece][row][128 bytes] with the 128-byte swizzle
+// (16-byte chunk index XOR row mod 8).  Rows past the end read as zeros.
+bool make_code_map(CUtensorMap* m, const void* base, long long cols, long long rows, int box_rows,
+                   int pieces) {
+  EncodeTiledFn fn = tensor_map_encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {128u, (cuuint64_t)rows, (cuuint64_t)(cols / 128)};
+  const cuuint64_t strides[2] = {(cuuint64_t)cols, 128u};
+  const cuuint32_t box[3] = {128u, (cuuint32_t)box_rows, (cuuint32_t)pieces};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D map over an fp32 matrix [rows][cols]; box = cols x box_rows (cols*4 a multiple of 16).
+bool make_f32_map(CUtensorMap* m, const void* base, long long cols, long long rows, int box_rows) {
+  EncodeTiledFn fn = tensor_map_encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 4};
+  const cuuint32_t box[2] = {(cuuint32_t)cols, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Sets the message moe_last_error returns, for the library's other translation units.
 int record_error(int code, const char* msg) { return fail(code, "%s", msg); }
 
@@ -127,7 +170,10 @@ WorkspaceLayout workspace_layout(int T, int k, int E, int d, int f) {
   const size_t R = (size_t)T * k + T;
   size_t o = 0;
   L.plan = o;
-  o = align256(o + 4 * ((size_t)E + 2 + 2 * plan_ntmax((int)R, E)));
+  // the tile plan, or (batched GEMV) the slot count and (expert, row, rows) per slot
+  size_t plan_ints = (size_t)E + 2 + 2 * plan_ntmax((int)R, E);
+  if (T <= kBgMaxT && 1 + 3 * R > plan_ints) plan_ints = 1 + 3 * R;
+  o = align256(o + 4 * plan_ints);
   L.qx = o;
   o = align256(o + R * d);
   L.sx = o;
@@ -140,15 +186,17 @@ WorkspaceLayout workspace_layout(int T, int k, int E, int d, int f) {
   const size_t hb = (size_t)((d > f ? d : f) / 128);
   L.n_counters = plan_ntmax((int)R, E) * hb;
   o = align256(o + 4 * L.n_counters);
-  // stream-K partial slots: two per CTA, each [ncap columns][2 matrices][tile rows] fp32;
-  // small batches take tiles of up to 256 weight rows, large ones 128
+  // stream-K partial slots of the tile kernels: two per CTA, each [ncap columns][2 matrices]
+  // [tile rows] fp32 (small batches take tiles of up to 256 weight rows, large ones 128).
+  // The GEMV paths' fp32 hidden state (single token: per active expert; batched: per row)
+  // shares the area: a call runs either the tile kernels or a GEMV path, never both.
   L.partials = o;
-  const size_t tile_rows_max = nmax_for(T) == kNmaxSmall ? 256 : 128;
-  o = align256(o + (size_t)kMaxCtas * 2 * (size_t)ncap_for(T) * 2 * tile_rows_max * 4);
-  // single-token path: h of every active expert, fp32, and the combine counters of the
-  // single-token kernel (one per 16 output rows)
   L.hbuf = o;
-  if (T <= kGemvMaxT) o = align256(o + R * f * 4);
+  const size_t tile_rows_max = nmax_for(T) == kNmaxSmall ? 256 : 128;
+  size_t area = (size_t)kMaxCtas * 2 * (size_t)ncap_for(T) * 2 * tile_rows_max * 4;
+  if (T <= kBgMaxT && R * f * 4 > area) area = R * f * 4;
+  o = align256(o + area);
+  // the combine counters of the single-token kernel (one per 16 output rows)
   L.done2 = o;
   if (T <= kGemvMaxT) o = align256(o + 4 * (size_t)(d / 16));
   L.total = o;
@@ -193,7 +241,7 @@ int moe_workspace_offsets(int T, int k, int E, int d, int f, size_t off[5]) {
   off[1] = L.sx;
   off[2] = L.qh;
   off[3] = L.sh;
-  off[4] = T <= kGemvMaxT ? L.hbuf : (size_t)-1;
+  off[4] = T <= kBgMaxT ? L.hbuf : (size_t)-1;
   return MOE_OK;
 }
 
@@ -281,6 +329,7 @@ struct FfnCtx {
   DeviceInfo di;
   WorkspaceLayout L;
   int nmax;
+  bool bg;     // batched GEMV path (bgemv.cu) instead of the tcgen05 tiles (ffn.cu)
   bool gemv;   // single-token GEMV path (gemv.cu) instead of the tcgen05 tiles (ffn.cu)
   bool fused;  // ... in one cooperative kernel (decode.cu), for the whole-call entry points
   uint8_t* ws;
@@ -332,10 +381,29 @@ int ffn_check(int T, int k, const moe_weights_t* w, void* ws, size_t ws_bytes, F
     return fail(MOE_ERR_INVALID_ARG, "shape needs %zu bytes of shared memory (> %d)", need,
                 max_smem);
   c.gemv = use_gemv(T, k, w, c.di.sms, max_smem);
+  c.bg = T >= 2 && T <= g_gemv_max_t.load() && T <= kBgMaxT && w->d % 512 == 0 &&
+         w->f % 512 == 0 && aligned(w->gate_scales, 16) && aligned(w->up_scales, 16) &&
+         aligned(w->down_scales, 16) && bgemv_smem_bytes(w->d) <= (size_t)max_smem &&
+         bgemv_smem_bytes(w->f) <= (size_t)max_smem;
   const int ctas = c.di.sms < kMaxCtas ? c.di.sms : kMaxCtas;
   c.fused = c.gemv && decode_fits(k, w->d, w->f, ctas) &&
             decode_smem_bytes(w->d, w->f) <= (size_t)max_smem;
   return MOE_OK;
+}
+
+BgLaunch bg_args(int T, int k, const moe_weights_t* w, const FfnCtx& c) {
+  BgLaunch a{};
+  a.plan = reinterpret_cast<const int32_t*>(c.ws + c.L.plan);
+  a.hbuf = reinterpret_cast<float*>(c.ws + c.L.hbuf);
+  a.E = w->E;
+  a.d = w->d;
+  a.f = w->f;
+  a.P = T * k;
+  a.R = T * k + T;
+  a.wait_ns = g_wait_ns.load();
+  a.status = c.di.status;
+  a.overlap = t_overlap;
+  return a;
 }
 
 GemvLaunch gemv_args(int T, int k, const moe_weights_t* w, const FfnCtx& c) {
@@ -413,6 +481,13 @@ int moe_ffn_prepare(const uint16_t* x_bf16, int T, int k, const moe_weights_t* w
         c.di.status, static_cast<cudaStream_t>(stream), 1, t_overlap);
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "ffn prepare launch");
   }
+  if (c.bg) {  // the rows in expert-sorted order and the slot plan
+    cudaError_t e = launch_quant_rows(
+        x_bf16, T, k, w->d, perm, T * k, c.ws + c.L.qx, reinterpret_cast<float*>(c.ws + c.L.sx),
+        offsets, w->E, c.nmax, reinterpret_cast<int32_t*>(c.ws + c.L.plan), nullptr, 0,
+        c.di.status, static_cast<cudaStream_t>(stream), 2, t_overlap);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "ffn prepare launch");
+  }
   cudaError_t e = launch_quant_rows(
       x_bf16, T, k, w->d, perm, T * k, c.ws + c.L.qx, reinterpret_cast<float*>(c.ws + c.L.sx),
       offsets, w->E, c.nmax, reinterpret_cast<int32_t*>(c.ws + c.L.plan),
@@ -436,6 +511,17 @@ int moe_ffn_gate_up(int T, int k, const moe_weights_t* w, void* ws, size_t ws_by
     cudaError_t e = launch_gemv(1, a, static_cast<cudaStream_t>(stream), c.di.sms);
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "ffn gate/up launch");
   }
+  if (c.bg) {
+    BgLaunch a = bg_args(T, k, w, c);
+    a.a0_codes = w->gate_codes;
+    a.a0_scales = w->gate_scales;
+    a.a1_codes = w->up_codes;
+    a.a1_scales = w->up_scales;
+    a.act = c.ws + c.L.qx;
+    a.act_scales = reinterpret_cast<const float*>(c.ws + c.L.sx);
+    cudaError_t e = launch_bgemv(1, a, static_cast<cudaStream_t>(stream), c.di.sms);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "ffn gate/up launch");
+  }
   cudaError_t e = launch_ffn(1, c.nmax, ffn_args(1, T, k, w, c),
                              static_cast<cudaStream_t>(stream), c.di.sms);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "ffn gate/up launch");
@@ -457,6 +543,23 @@ int moe_ffn_down(int T, int k, const moe_weights_t* w, float* y_routed, float* y
     g.y_routed = y_routed;
     g.y_shared = y_shared;
     cudaError_t e = launch_gemv(2, g, static_cast<cudaStream_t>(stream), c.di.sms);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "ffn down launch");
+  }
+  if (c.bg) {  // re-quantise h, then the down GEMV
+    const int R = T * k + T;
+    cudaError_t e = launch_quant_h(reinterpret_cast<const float*>(c.ws + c.L.hbuf), R, w->f,
+                                   c.ws + c.L.qh, reinterpret_cast<float*>(c.ws + c.L.sh),
+                                   static_cast<cudaStream_t>(stream), t_overlap);
+    if (e != cudaSuccess) return cuda_fail(e, "ffn h quantisation launch");
+    BgLaunch b = bg_args(T, k, w, c);
+    b.a0_codes = w->down_codes;
+    b.a0_scales = w->down_scales;
+    b.act = c.ws + c.L.qh;
+    b.act_scales = reinterpret_cast<const float*>(c.ws + c.L.sh);
+    b.y_routed = y_routed;
+    b.y_shared = y_shared;
+    b.overlap = true;  // follows the quantisation kernel of this call
+    e = launch_bgemv(2, b, static_cast<cudaStream_t>(stream), c.di.sms);
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "ffn down launch");
   }
   FfnArgs a = ffn_args(2, T, k, w, c);

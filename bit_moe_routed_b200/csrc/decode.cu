@@ -721,33 +721,6 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
   }
 }
 
-// 2-D map over a byte matrix [rows][cols]; box = box_cols bytes x box_rows rows
-bool make_byte_map(CUtensorMap* m, const void* base, long long cols, long long rows, int box_cols,
-                   int box_rows) {
-  EncodeTiledFn fn = tensor_map_encode_fn();
-  if (fn == nullptr) return false;
-  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)cols};
-  const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
-  const cuuint32_t estr[2] = {1u, 1u};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-// 3-D map over FP4 code rows [rows][cols bytes] viewed as (128-byte piece, row, piece
-// index): a box of 2 pieces x box_rows rows lands as [piece][row][128 bytes], 128-byte
-// swizzle
-bool make_code_map(CUtensorMap* m, const void* base, long long cols, long long rows, int box_rows) {
-  EncodeTiledFn fn = tensor_map_encode_fn();
-  if (fn == nullptr) return false;
-  const cuuint64_t dims[3] = {128u, (cuuint64_t)rows, (cuuint64_t)(cols / 128)};
-  const cuuint64_t strides[2] = {(cuuint64_t)cols, 128u};
-  const cuuint32_t box[3] = {128u, (cuuint32_t)box_rows, 2u};
-  const cuuint32_t estr[3] = {1u, 1u, 1u};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 template <int MODE, int PL>
 cudaError_t launch_one(const DecodeParams& prm, cudaStream_t s, int grid) {

@@ -34,9 +34,12 @@ constexpr int kMaxCtas = 148;
 //   [E+2, E+2 + 2*ntmax)  tiles: (row0, n) per token tile
 inline size_t plan_ntmax(int R, int E) { return (size_t)R / 16 + (size_t)E + 2; }
 
-// Single-token batches (T = 1) run the expert FFN as two FP4 GEMV kernels (gemv.cu)
-// when the shapes allow it; larger batches use the tcgen05 tile kernels (ffn.cu).
+// Single-token batches (T = 1) run the expert FFN as FP4 GEMV kernels (decode.cu, gemv.cu)
+// when the shapes allow it; batches up to kBgMaxT run the batched FP4 GEMV (bgemv.cu);
+// larger ones use the tcgen05 tile kernels (ffn.cu).
 constexpr int kGemvMaxT = 1;
+constexpr int kBgMaxT = 64;
+constexpr int kBgSlotTokens = 8;  // tokens per slot of the batched GEMV (the MMA's N)
 
 struct WorkspaceLayout {
   size_t plan, qx, sx, qh, sh, counters, partials, hbuf, done2, total;
@@ -59,6 +62,9 @@ cudaError_t launch_quant_rows(const uint16_t* x, int T, int k, int d, const int3
                               int E, int nmax, int32_t* plan, int* counters, size_t n_counters,
                               int* status, cudaStream_t st, int plan_mode = 0,
                               bool overlap = false);
+// h [R][f] fp32 -> e4m3 codes [R][f] and scales [R][f/128] (batched GEMV path)
+cudaError_t launch_quant_h(const float* h, int R, int f, uint8_t* q, float* s, cudaStream_t st,
+                           bool overlap);
 cudaError_t launch_combine(const float* y, const float* ysh, const float* w, const int32_t* pos,
                            int T, int k, int d, float* out, int* status, cudaStream_t s,
                            bool overlap = false);
@@ -118,6 +124,28 @@ size_t gemv_smem_bytes(int phase, int K);
 // a launch's units (8 h-rows in phase 1, 16 down rows in phase 2, of every active
 // expert) are cut into one range per CTA of at most this many units
 int gemv_max_units_per_cta();
+
+// Batched FP4 GEMV path (bgemv.cu), 2 <= T <= kBgMaxT: phase 1 reads the activation rows
+// qx/sx and writes h [R][f] fp32; phase 2 reads qh/sh and writes y.  The plan holds the
+// slots (expert, first row, rows <= kBgSlotTokens) after their count.
+struct BgLaunch {
+  const uint8_t* a0_codes;   // gate (phase 1) or down (phase 2)
+  const uint8_t* a0_scales;
+  const uint8_t* a1_codes;   // up (phase 1)
+  const uint8_t* a1_scales;
+  const int32_t* plan;
+  const uint8_t* act;        // [R][K] e4m3 rows (qx or qh)
+  const float* act_scales;   // [R][K/128]
+  float* hbuf;
+  float* y_routed;
+  float* y_shared;
+  int E, d, f, P, R;
+  long long wait_ns;
+  int* status;
+  bool overlap;
+};
+cudaError_t launch_bgemv(int phase, const BgLaunch& a, cudaStream_t s, int num_sms);
+size_t bgemv_smem_bytes(int K);
 
 // Single-token layer in one cooperative kernel (decode.cu): forward = routing from the
 // scores, dispatch and combine included; otherwise the expert FFN from dispatch offsets.
@@ -180,6 +208,12 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn tensor_map_encode_fn();
+// Tensor maps the GEMV kernels use (defined in abi.cu; false if encoding fails).
+bool make_byte_map(CUtensorMap* m, const void* base, long long cols, long long rows, int box_cols,
+                   int box_rows);
+bool make_code_map(CUtensorMap* m, const void* base, long long cols, long long rows, int box_rows,
+                   int pieces = 2);
+bool make_f32_map(CUtensorMap* m, const void* base, long long cols, long long rows, int box_rows);
 
 // Defined in abi.cu: sets the thread-local message that moe_last_error returns.
 int record_error(int code, const char* msg);

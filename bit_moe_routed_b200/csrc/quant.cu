@@ -86,6 +86,38 @@ __device__ void write_gemv_plan(const int32_t* __restrict__ offsets, int E,
   }
 }
 
+// Slots of the batched FP4 GEMV: every expert's rows (routed experts with a group, in
+// ascending id, then the shared expert's T rows) cut into slots of at most kBgSlotTokens
+// rows.  plan[0] = slots, then (expert, first row, rows) per slot.
+__device__ void write_slot_plan(const int32_t* __restrict__ offsets, int E, int T, int P,
+                                int32_t* __restrict__ plan) {
+  const int lane = threadIdx.x & 31;
+  const int per = (E + 1 + 31) / 32;
+  const int e0 = lane * per, e1 = min(E + 1, e0 + per);
+  int local = 0;
+  for (int e = e0; e < e1; ++e) {
+    const int n = e < E ? offsets[e + 1] - offsets[e] : T;
+    local += (n + kBgSlotTokens - 1) / kBgSlotTokens;
+  }
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  int i = incl - local;
+  for (int e = e0; e < e1; ++e) {
+    const int n = e < E ? offsets[e + 1] - offsets[e] : T;
+    const int row = e < E ? offsets[e] : P;
+    for (int c = 0; c < n; c += kBgSlotTokens, ++i) {
+      plan[1 + 3 * i] = e;
+      plan[2 + 3 * i] = row + c;
+      plan[3 + 3 * i] = min(kBgSlotTokens, n - c);
+    }
+  }
+  if (lane == 31) plan[0] = incl;
+}
+
 __global__ void __launch_bounds__(256) quant_rows_kernel(
     const uint16_t* __restrict__ x, int T, int k, int d, const int32_t* __restrict__ perm, int P,
     uint8_t* __restrict__ q, float* __restrict__ s, const int32_t* __restrict__ offsets, int E,
@@ -102,6 +134,7 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(
   if (r == R) {  // the plan block
     if (threadIdx.x < 32) {
       if (plan_mode == 1) write_gemv_plan(offsets, E, plan);
+      else if (plan_mode == 2) write_slot_plan(offsets, E, T, P, plan);
       else write_plan(offsets, E, T, P, nmax, plan);
     }
     return;
@@ -148,7 +181,59 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(
   }
 }
 
+// The hidden state of the batched GEMV path, fp32 [R][f], re-quantised per row and
+// 128-block exactly as the activations: s = amax / 448 (IEEE divide; 1 if amax = 0),
+// q = e4m3(h / s) rounded to nearest even.  8 threads per block, 16 values each.
+__global__ void __launch_bounds__(256) quant_h_kernel(const float* __restrict__ h, int f,
+                                                      uint8_t* __restrict__ q,
+                                                      float* __restrict__ s) {
+  ptx::griddep_launch_dependents();
+  ptx::griddep_wait();  // h comes from the gate/up kernel
+  const float* hr = h + (size_t)blockIdx.x * f;
+  const int lane16 = (threadIdx.x & 31) * 16;
+  for (int c0 = threadIdx.x * 16; c0 - lane16 < f; c0 += blockDim.x * 16) {
+    const bool act = c0 < f;
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 a = act ? __ldcg(reinterpret_cast<const float4*>(hr + c0) + i)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+      v[4 * i] = a.x;
+      v[4 * i + 1] = a.y;
+      v[4 * i + 2] = a.z;
+      v[4 * i + 3] = a.w;
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+    const float sc = amax == 0.f ? 1.0f : __fdiv_rn(amax, 448.0f);
+    uint32_t packed[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint16_t lo = ptx::cvt_e4m3x2(__fdiv_rn(v[4 * i], sc), __fdiv_rn(v[4 * i + 1], sc));
+      const uint16_t hi =
+          ptx::cvt_e4m3x2(__fdiv_rn(v[4 * i + 2], sc), __fdiv_rn(v[4 * i + 3], sc));
+      packed[i] = (uint32_t)lo | ((uint32_t)hi << 16);
+    }
+    if (act) {
+      *reinterpret_cast<uint4*>(q + (size_t)blockIdx.x * f + c0) =
+          make_uint4(packed[0], packed[1], packed[2], packed[3]);
+      if ((threadIdx.x & 7) == 0) s[(size_t)blockIdx.x * (f / 128) + c0 / 128] = sc;
+    }
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_quant_h(const float* h, int R, int f, uint8_t* q, float* s, cudaStream_t st,
+                           bool overlap) {
+  int threads = (f / 16 + 31) / 32 * 32;
+  if (threads > 256) threads = 256;
+  return launch_pdl(quant_h_kernel, dim3((unsigned)R), dim3(threads), 0, st, overlap, h, f, q, s);
+}
 
 cudaError_t launch_quant_rows(const uint16_t* x, int T, int k, int d, const int32_t* perm,
                               int nrows_routed, uint8_t* q, float* s, const int32_t* offsets,

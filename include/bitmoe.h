@@ -202,13 +202,14 @@ const char* moe_last_error(void);
  * (2 s).  n <= 0 restores the default.  Applies to launches made after the call. */
 int moe_set_wait_limit_ns(long long n);
 
-/* Largest batch T that runs the expert FFN as two FP4 GEMV kernels (the single-token
- * decode path) instead of the tcgen05 tile kernels.  The pages have no counterpart: it
- * is a switch between two implementations of the same calls.  0 sends every batch to
- * the tile kernels; values above 1 act as 1 (the GEMV path takes T = 1 only).  The
- * GEMV path also needs d and f multiples of 512, 16-byte aligned scale arrays and
- * k + 1 <= the SM count; other shapes take the tile kernels.  Default 1.  Applies to
- * calls made after it. */
+/* Largest batch T that runs the expert FFN as FP4 GEMV kernels (CUDA-core e2m1 decode,
+ * mma.sync; the decode paths) instead of the tcgen05 tile kernels: T = 1 the single-token
+ * kernels, 2 <= T <= 64 the batched GEMV (groups of up to 8 tokens per expert).  The
+ * pages have no counterpart: it is a switch between implementations of the same calls.
+ * 0 sends every batch to the tile kernels; values above 64 act as 64.  The GEMV paths
+ * also need d and f multiples of 512 and 16-byte aligned scale arrays (the single-token
+ * kernel also k + 1 <= the SM count); other shapes take the tile kernels.  Default 64.
+ * Applies to calls made after it. */
 int moe_set_gemv_max_tokens(int t);
 
 /* Testing knob; the pages have no counterpart.  While on, every launch of the

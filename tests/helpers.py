@@ -274,7 +274,7 @@ def check_layer(g, x, scores, k, E, d, f, seed, layer, tokens, label="", experts
         need = set(idx[tokens].ravel().tolist()) | {E}
         experts = host_experts(seed, layer, d, f, need)
     qx_o, sx_o = oracle.act_quant(x)
-    single = "h" in g  # the single-token path keeps its fp32 h and writes qx row 0 only
+    single = T == 1 and "h" in g  # the single-token path writes qx row 0 only
     if single:
         assert np.array_equal(g["qx"].numpy()[0], qx_o[0]), f"{label}: qx (token codes)"
         assert np.array_equal(g["sx"].numpy()[0], sx_o[0]), f"{label}: sx (token scales)"

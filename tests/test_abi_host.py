@@ -93,13 +93,13 @@ def test_oracle_and_cuda_path_are_independent():
 def test_gemv_switch_host(L):
     """moe_set_gemv_max_tokens takes 0 (tile kernels only) or a positive bound, and
     rejects a negative one with a message; the workspace of a single token holds the
-    GEMV path's fp32 hidden state (k + 1 rows of f) on top of the tile path's needs."""
+    GEMV path's fp32 hidden state (k + 1 rows of f)."""
     assert L.moe_set_gemv_max_tokens(-1) == bm.MOE_ERR_INVALID_ARG
     assert b"t=-1" in L.moe_last_error()
     try:
         assert L.moe_set_gemv_max_tokens(0) == bm.MOE_OK
     finally:
-        assert L.moe_set_gemv_max_tokens(1) == bm.MOE_OK
+        assert L.moe_set_gemv_max_tokens(bm.GEMV_MAX_TOKENS) == bm.MOE_OK
     one = bm.workspace_size(1, 6, 256, 4096, 2048)
     two = bm.workspace_size(2, 6, 256, 4096, 2048)
     assert one >= 7 * 2048 * 4

@@ -134,6 +134,30 @@ def test_layer_ragged_shapes(T, E, k, d, f, routing):
     _small_layer(T, E, k, d, f, routing, seed=T + E)
 
 
+@pytest.mark.parametrize("T,E,k,d,f,routing", [
+    (2, 8, 2, 512, 512, "uniform"),
+    (7, 16, 3, 1024, 512, "zipf"),       # one slot per expert, fewer than 8 tokens
+    (16, 32, 4, 512, 1024, "zipf"),      # the shared expert in two slots
+    (33, 16, 6, 1024, 512, "zipf"),      # hot experts in several slots
+    (64, 256, 6, 2048, 1024, "zipf"),    # CTA ranges over many slots
+])
+def test_batched_gemv_shapes(T, E, k, d, f, routing):
+    """2 <= T <= 64 with d, f multiples of 512: the batched FP4 GEMV kernels."""
+    _small_layer(T, E, k, d, f, routing, seed=T + E + d)
+
+
+def test_batched_gemv_all_tokens_one_expert():
+    """40 tokens on one routed expert: five slots of 8 rows re-read its weights."""
+    T, E, k, d, f = 40, 8, 1, 512, 512
+    x = synth.gen_x(T, d, seed=95)
+    s = synth.gen_scores_uniform(T, E, seed=96)
+    s[:, 5] += 10.0
+    W = device_weights(97, 0, E, d, f)
+    g = gpu_layer(x, s, k, W)
+    assert g["counts"].tolist()[5] == T
+    check_layer(g, x, s, k, E, d, f, 97, 0, list(range(T)), "one expert, batched GEMV")
+
+
 def test_layer_zero_activations():
     _small_layer(6, 8, 2, 256, 128, seed=77, zero_rows=(0, 3))
 
@@ -278,7 +302,7 @@ def test_wide_scale_range_single_token(gemv):
     try:
         _custom_layer_check(1, E, k, d, f, arrs, 31, "wide scales")
     finally:
-        bm.set_gemv_max_tokens(1)
+        bm.set_gemv_max_tokens(bm.GEMV_MAX_TOKENS)
 
 
 def test_extreme_weights_single_token():
@@ -330,11 +354,17 @@ def test_decode_t1_full(path):
     try:
         _full_workload("decode_t1", [0], calls=path == "calls")
     finally:
-        bm.set_gemv_max_tokens(1)
+        bm.set_gemv_max_tokens(bm.GEMV_MAX_TOKENS)
 
 
-def test_decode_t64_zipf_all_tokens():
-    g = _full_workload("decode_t64_zipf", list(range(64)))
+@pytest.mark.parametrize("path", ["gemv", "tiles"])
+def test_decode_t64_zipf_all_tokens(path):
+    """decode_t64 through the batched GEMV kernels and through the tile kernels."""
+    bm.set_gemv_max_tokens(0 if path == "tiles" else bm.GEMV_MAX_TOKENS)
+    try:
+        g = _full_workload("decode_t64_zipf", list(range(64)))
+    finally:
+        bm.set_gemv_max_tokens(bm.GEMV_MAX_TOKENS)
     assert int(g["counts"].max()) > 16  # a hot expert serves many tokens
 
 
