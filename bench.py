@@ -380,6 +380,7 @@ def measure(bm, w, args, dev, stream, rank, dist, steps, warmup, peaks, cpu_seco
     # one step = the whole layer in one call (moe_forward): one kernel for a single token,
     # otherwise route, dispatch, prepare, gate/up, down and combine back to back
     fused = T == 1 and d % 512 == 0 and f % 512 == 0
+    batched = 2 <= T <= 64 and d % 512 == 0 and f % 512 == 0  # the batched GEMV path
 
     def step(L):
         return bm.forward(L["x"], L["scores"], k, L["W"], Ls.ws, stream, outs=Ls.outs)["counts"]
@@ -475,8 +476,13 @@ def measure(bm, w, args, dev, stream, rank, dist, steps, warmup, peaks, cpu_seco
         work["gu_bytes"] = work["weight_bytes"] + io
     else:
         gu_s = (statistics.median(ab["a"]) - statistics.median(ab["b"])) / n_layers / 1000.0
-        kernel_file = os.path.join(ROOT, "bit_moe_routed_b200", "csrc", "ffn.cu")
-        kernel_name = "ffn gate/up (tcgen05 kind::mxf8f6f4)"
+        if batched:
+            kernel_file = os.path.join(ROOT, "bit_moe_routed_b200", "csrc", "bgemv.cu")
+            kernel_name = ("bgemv gate/up + SwiGLU (batched FP4 GEMV: packed codes in shared "
+                           "memory, in-register e2m1 decode, tokens in mma.sync N columns)")
+        else:
+            kernel_file = os.path.join(ROOT, "bit_moe_routed_b200", "csrc", "ffn.cu")
+            kernel_name = "ffn gate/up (tcgen05 kind::mxf8f6f4)"
         traffic = kernel_traffic(kernel_file, "gate_up", w.name)
     hbm_peak, fp8_peak, fp8_src, peak_kind = peaks
     if is_prefill:
@@ -500,7 +506,7 @@ def measure(bm, w, args, dev, stream, rank, dist, steps, warmup, peaks, cpu_seco
     roof["avg_launch_us"] = gu_s * 1e6
     roof["algorithmic_per_launch"] = work["flops_gu"] if is_prefill else work["gu_bytes"]
     rec = {
-        "fused": fused, "launches_per_step": 1 if fused else 6,
+        "fused": fused, "launches_per_step": 1 if fused else (7 if batched else 6),
         "value": world * T * steps / total_s, "unit": "tokens/s", "steps": steps,
         "ms_per_step": 1000.0 * layer_s,
         "ms_per_step_isolated": statistics.median(one_ms),
