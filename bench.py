@@ -521,7 +521,7 @@ def measure(bm, w, args, dev, stream, rank, dist, steps, warmup, peaks, cpu_seco
         x_cpu, s_cpu = Ls.items[0]["x_cpu"], Ls.items[0]["s_cpu"]
         rec["cpu_baseline"] = cpu_baseline(w, x_cpu, s_cpu, cpu_seconds, extras=T <= 64 and headline)
     del g_warm, g_timed, g_one, g_a, g_b
-    return rec, Ls, step
+    return rec, Ls
 
 
 def e2e(bm, Ls, args, dev, stream, dist, world):
@@ -597,7 +597,7 @@ def run_gpu(args, w):
     fp8_peak, fp8_src = fp8_peak_of(fp8, bf16_peak)
     peaks = (hbm_peak, fp8_peak, fp8_src, peak_kind)
 
-    rec, Ls, _ = measure(bm, w, args, dev, stream, rank, dist, args.steps, args.warmup, peaks,
+    rec, Ls = measure(bm, w, args, dev, stream, rank, dist, args.steps, args.warmup, peaks,
                          0 if args.no_cpu_baseline else args.cpu_seconds, headline=True)
     e2e_rec = e2e(bm, Ls, args, dev, stream, dist, world)
     del Ls
@@ -616,10 +616,13 @@ def run_gpu(args, w):
             if free < need + (6 << 30):
                 workloads[name] = {"skipped": f"needs {need / 1e9:.1f} GB, {free / 1e9:.1f} GB free"}
                 continue
-            r, Lw, _ = measure(bm, wl, args, dev, stream, rank, dist,
-                               args.extra_steps, 3, peaks, args.extra_cpu_seconds)
+            r, Lw = measure(bm, wl, args, dev, stream, rank, dist,
+                            args.extra_steps, 3, peaks, args.extra_cpu_seconds)
             workloads[name] = r
             del Lw
+            import gc
+            gc.collect()
+            torch.cuda.synchronize()
             torch.cuda.empty_cache()
 
     if rank == 0:

@@ -28,6 +28,7 @@ MOE_ERR_WORKSPACE = -2
 MOE_ERR_CUDA = -3
 MOE_ERR_TIMEOUT = -4
 MOE_ERR_UNSUPPORTED = -5
+PATH_TILES, PATH_SINGLE, PATH_BATCHED = 0, 1, 2
 MOE_NOALLOC_SCRATCH_BYTES = 24 << 20  # the fixed scratch of moe_expert_ffn_noalloc
 GEMV_MAX_TOKENS = 64                  # default of moe_set_gemv_max_tokens
 
@@ -36,6 +37,7 @@ EXPORTS = (
     "moe_ffn_gate_up", "moe_ffn_down", "moe_combine", "moe_workspace_size", "moe_last_error",
     "moe_set_wait_limit_ns", "moe_sync_status", "moe_expert_ffn_noalloc",
     "moe_set_gemv_max_tokens", "moe_workspace_offsets", "moe_set_test_stall", "moe_forward",
+    "moe_ffn_path",
 )
 
 
@@ -86,6 +88,7 @@ def lib():
             "moe_workspace_offsets": [I, I, I, I, I, P],
             "moe_set_test_stall": [I],
             "moe_forward": [P, P, I, I, W, P, P, P, P, P, P, P, P, P, P, Z, P],
+            "moe_ffn_path": [I, I, W],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -173,6 +176,15 @@ def sync_status(stream=None) -> None:
 
 def workspace_size(T: int, k: int, E: int, d: int, f: int) -> int:
     return int(lib().moe_workspace_size(T, k, E, d, f))
+
+
+def ffn_path(T: int, k: int, w: "LayerWeights") -> int:
+    """PATH_TILES, PATH_SINGLE or PATH_BATCHED: the implementation moe_expert_ffn runs."""
+    st = w.struct()
+    rc = lib().moe_ffn_path(T, k, ctypes.byref(st))
+    if rc < 0:
+        _check(rc)
+    return rc
 
 
 def workspace_offsets(T: int, k: int, E: int, d: int, f: int) -> dict:

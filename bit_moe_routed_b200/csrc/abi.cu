@@ -362,7 +362,7 @@ int ffn_check(int T, int k, const moe_weights_t* w, void* ws, size_t ws_bytes, F
   rc = device_info(c.di);
   if (rc) return rc;
   c.L = workspace_layout(T, k, w->E, w->d, w->f);
-  if (T > 0) {
+  if (T > 0 && ws_bytes != (size_t)-1) {
     if (ws == nullptr || !aligned(ws, 256))
       return fail(MOE_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned");
     if (ws_bytes < c.L.total)
@@ -596,6 +596,15 @@ DecodeLaunch decode_args(int k, const moe_weights_t* w, const FfnCtx& c) {
 }
 
 }  // namespace
+
+int moe_ffn_path(int T, int k, const moe_weights_t* w) {
+  FfnCtx c;
+  const int rc = ffn_check(T, k, w, nullptr, (size_t)-1, c);  // no workspace: a query
+  if (rc) return rc;
+  if (T == 1 && c.fused) return MOE_PATH_SINGLE;
+  if (c.bg) return MOE_PATH_BATCHED;
+  return MOE_PATH_TILES;
+}
 
 int moe_expert_ffn(const uint16_t* x_bf16, int T, int k, const moe_weights_t* w,
                    const int32_t* offsets, const int32_t* perm, float* y_routed, float* y_shared,

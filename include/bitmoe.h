@@ -221,6 +221,16 @@ int moe_set_gemv_max_tokens(int t);
  * turns it off.  Applies to launches made after the call. */
 int moe_set_test_stall(int on);
 
+/* Which implementation moe_expert_ffn would run for T tokens with these weights on the
+ * current device, under the current moe_set_gemv_max_tokens: MOE_PATH_TILES (tcgen05
+ * tiles), MOE_PATH_SINGLE (the single-token kernels) or MOE_PATH_BATCHED (the batched
+ * GEMV); a negative MOE_ERR_* on invalid arguments.  The pages have no counterpart; tests
+ * and tools use it to know which intermediates a workspace holds. */
+#define MOE_PATH_TILES 0
+#define MOE_PATH_SINGLE 1
+#define MOE_PATH_BATCHED 2
+int moe_ffn_path(int T, int k, const moe_weights_t* w);
+
 /* Synchronise `stream`, then return MOE_ERR_CUDA for a pending CUDA error,
  * MOE_ERR_TIMEOUT if a device-side wait expired since the last call (clearing the
  * record), else MOE_OK. */

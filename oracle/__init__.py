@@ -61,6 +61,7 @@ def lib():
         L.oracle_quant_blocks.argtypes = [P, I, P, P]
         L.oracle_act_quant.argtypes = [P, I, I, P, P]
         L.oracle_route_topk.argtypes = [P, I, I, I, P, P]
+        L.oracle_router_scores.argtypes = [P, P, I, I, I, P]
         L.oracle_dispatch.argtypes = [P, I, I, I, P, P, P, P]
         L.oracle_fp4_gemv.argtypes = [P, P, I, I, P, P]
         L.oracle_expert_ffn.argtypes = [ctypes.POINTER(_Expert), I, I, P, P, I, P, P, P]
@@ -131,6 +132,17 @@ def act_quant(x):
     s = np.empty((T, d // 128), np.float32)
     lib().oracle_act_quant(xb.ctypes.data, T, d, q.ctypes.data, s.ctypes.data)
     return q, s
+
+
+def router_scores(x, w_router) -> np.ndarray:
+    """scores [T, E] (double) = x [T, d] . W_router [E, d]^T over bf16 inputs."""
+    xb = _bf16_bits(x)
+    wb = _bf16_bits(w_router)
+    T, d = xb.shape
+    E = wb.shape[0]
+    out = np.empty((T, E), np.float64)
+    lib().oracle_router_scores(xb.ctypes.data, wb.ctypes.data, T, d, E, out.ctypes.data)
+    return out
 
 
 def route_topk(scores: np.ndarray, k: int):

@@ -112,6 +112,21 @@ static int rank_before(float sa, int ia, float sb, int ib) {
     return ia < ib;
 }
 
+/* Router scores (dpshk.com article, "核心实现一": the router decides each token's experts
+ * from its hidden state): scores[t][e] = sum_i x[t][i] * W[e][i] over the bf16 inputs,
+ * summed in double (every product of two bf16 values is exact in double). */
+void oracle_router_scores(const uint16_t* x_bf16, const uint16_t* w_bf16, int T, int d, int E,
+                          double* scores) {
+    for (int t = 0; t < T; ++t)
+        for (int e = 0; e < E; ++e) {
+            double acc = 0.0;
+            for (int i = 0; i < d; ++i)
+                acc += (double)bf16_to_f32(x_bf16[(size_t)t * d + i]) *
+                       (double)bf16_to_f32(w_bf16[(size_t)e * d + i]);
+            scores[(size_t)t * E + e] = acc;
+        }
+}
+
 void oracle_route_topk(const float* scores, int T, int E, int k, int32_t* idx, double* w) {
     int* order = (int*)malloc(sizeof(int) * (size_t)E);
     for (int t = 0; t < T; ++t) {

@@ -63,6 +63,12 @@ void oracle_quant_blocks(const float* v, int n, uint8_t* q, float* s);
 /* bf16 activations [T][d] -> e4m3 codes [T][d], fp32 scales [T][d/128]. */
 void oracle_act_quant(const uint16_t* x_bf16, int T, int d, uint8_t* q, float* s);
 
+/* Router scores: scores[t][e] = sum_i x[t][i] * W_router[e][i] over bf16 x [T][d] and
+ * W_router [E][d], in double.  (dpshk.com article, "核心实现一": the router picks each
+ * token's experts.)  The selection is oracle_route_topk on these scores rounded to fp32. */
+void oracle_router_scores(const uint16_t* x_bf16, const uint16_t* w_bf16, int T, int d, int E,
+                          double* scores);
+
 /* Top-k routing: k largest scores per token, descending, ties to the lower expert
  * index; w_j = sigmoid(s_j) / sum_j' sigmoid(s_j') in double. */
 void oracle_route_topk(const float* scores, int T, int E, int k, int32_t* idx, double* w);

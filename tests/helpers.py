@@ -246,8 +246,12 @@ def gpu_layer(x, scores, k, weights, ws=None, keep_device=False, calls=False):
     if ws is None:
         ws = bm.alloc_workspace(T, k, E, d, f)
     run = bm.forward_calls if calls else bm.forward
+    path = bm.ffn_path(T, k, weights)
     r = run(x.cuda(), scores.cuda(), k, weights, ws)
-    r.update({kk: v.clone() for kk, v in bm.workspace_views(ws, T, k, E, d, f).items()})
+    views = bm.workspace_views(ws, T, k, E, d, f)
+    if path == bm.PATH_TILES:
+        views.pop("h", None)  # the tile kernels keep no fp32 h
+    r.update({kk: v.clone() for kk, v in views.items()})
     if keep_device:
         return r
     bm.sync_status()

@@ -70,3 +70,50 @@ def test_dispatch_empty_and_single_expert():
     assert perm.tolist() == [0, 1, 2, 3, 4]
     counts, offsets, perm, pos = oracle.dispatch(np.zeros((0, 3), np.int32), 4)
     assert counts.tolist() == [0, 0, 0, 0] and offsets.tolist() == [0] * 5 and perm.size == 0
+
+
+# ---------------------------------------------------------------- router scores (NEXT-1)
+def _bf16(a):
+    return torch.as_tensor(np.asarray(a, np.float32)).to(torch.bfloat16)
+
+
+def test_router_scores_match_float64_matmul():
+    """Against numpy's float64 matmul of the bf16-decoded inputs (a library routine)."""
+    rng = np.random.default_rng(5)
+    x = _bf16(rng.normal(size=(7, 384)))
+    w = _bf16(rng.normal(size=(40, 384)) * 0.05)
+    got = oracle.router_scores(x, w)
+    ref = x.float().numpy().astype(np.float64) @ w.float().numpy().astype(np.float64).T
+    assert np.allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_router_scores_closed_forms():
+    """One-hot tokens pick out columns of W; integer inputs give exact integer scores."""
+    d, E = 64, 9
+    rng = np.random.default_rng(6)
+    w = _bf16(rng.integers(-8, 9, size=(E, d)))
+    x = np.zeros((3, d), np.float32)
+    x[0, 5] = 1.0
+    x[1, 63] = -2.0
+    x[2] = rng.integers(-4, 5, size=d)
+    s = oracle.router_scores(_bf16(x), w)
+    wf = w.float().numpy().astype(np.float64)
+    assert np.array_equal(s[0], wf[:, 5])
+    assert np.array_equal(s[1], -2.0 * wf[:, 63])
+    assert np.array_equal(s[2], np.array([int(np.dot(x[2].astype(np.int64),
+                                                      wf[e].astype(np.int64))) for e in range(E)],
+                                         dtype=np.float64))
+
+
+def test_router_then_topk_selects_the_largest_dot_products():
+    """A planted winner: the experts whose rows align with the token are chosen in order."""
+    d, E, k = 128, 16, 3
+    rng = np.random.default_rng(7)
+    x = rng.normal(size=(1, d)).astype(np.float32)
+    w = rng.normal(size=(E, d)).astype(np.float32) * 0.01
+    w[11] = x[0]
+    w[2] = 0.5 * x[0]
+    w[7] = 0.25 * x[0]
+    s = oracle.router_scores(_bf16(x), _bf16(w)).astype(np.float32)
+    idx, _ = oracle.route_topk(s, k)
+    assert idx.tolist() == [[11, 2, 7]]
