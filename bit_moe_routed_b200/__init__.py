@@ -37,7 +37,7 @@ EXPORTS = (
     "moe_ffn_gate_up", "moe_ffn_down", "moe_combine", "moe_workspace_size", "moe_last_error",
     "moe_set_wait_limit_ns", "moe_sync_status", "moe_expert_ffn_noalloc",
     "moe_set_gemv_max_tokens", "moe_workspace_offsets", "moe_set_test_stall", "moe_forward",
-    "moe_ffn_path",
+    "moe_ffn_path", "moe_router_topk",
 )
 
 
@@ -89,6 +89,7 @@ def lib():
             "moe_set_test_stall": [I],
             "moe_forward": [P, P, I, I, W, P, P, P, P, P, P, P, P, P, P, Z, P],
             "moe_ffn_path": [I, I, W],
+            "moe_router_topk": [P, P, I, I, I, I, P, P, P, P],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -226,6 +227,18 @@ def route_topk(scores: torch.Tensor, k: int, stream=None):
     w = torch.empty((T, k), dtype=torch.float32, device=scores.device)
     _check(lib().moe_route_topk(_p(scores), T, E, k, _p(idx), _p(w), _stream(stream)))
     return idx, w
+
+
+def router_topk(x: torch.Tensor, w_router: torch.Tensor, k: int, stream=None):
+    """Router scores x . W_router^T (bf16 in, fp32 out) and their top-k: (scores, idx, w)."""
+    T, d = x.shape
+    E = w_router.shape[0]
+    scores = torch.empty((T, E), dtype=torch.float32, device=x.device)
+    idx = torch.empty((T, k), dtype=torch.int32, device=x.device)
+    w = torch.empty((T, k), dtype=torch.float32, device=x.device)
+    _check(lib().moe_router_topk(_p(x), _p(w_router), T, d, E, k, _p(scores), _p(idx), _p(w),
+                                 _stream(stream)))
+    return scores, idx, w
 
 
 def dispatch(idx: torch.Tensor, E: int, stream=None):

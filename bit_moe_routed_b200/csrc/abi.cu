@@ -288,6 +288,28 @@ int moe_route_topk(const float* scores, int T, int E, int k, int32_t* topk_idx, 
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "route_topk launch");
 }
 
+int moe_router_topk(const uint16_t* x_bf16, const uint16_t* w_router_bf16, int T, int d, int E,
+                    int k, float* scores, int32_t* topk_idx, float* topk_w, void* stream) {
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T=%d < 0", T);
+  if (E < 1 || E > 1024) return fail(MOE_ERR_INVALID_ARG, "E=%d outside [1, 1024]", E);
+  if (k < 1 || k > E || k > 32) return fail(MOE_ERR_INVALID_ARG, "k=%d outside [1, min(E, 32)]", k);
+  if (d < 128 || d % 128) return fail(MOE_ERR_INVALID_ARG, "d=%d must be a positive multiple of 128", d);
+  if (T == 0) return MOE_OK;
+  if (!x_bf16 || !w_router_bf16 || !scores || !topk_idx || !topk_w)
+    return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(x_bf16, 4) || !aligned(w_router_bf16, 4) || !aligned(scores, 4) ||
+      !aligned(topk_idx, 4) || !aligned(topk_w, 4))
+    return fail(MOE_ERR_INVALID_ARG, "pointers must be 4-byte aligned");
+  DeviceInfo di;
+  int rc = device_info(di);
+  if (rc) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_router(x_bf16, w_router_bf16, T, d, E, scores, s, t_overlap);
+  if (e != cudaSuccess) return cuda_fail(e, "router launch");
+  e = launch_route_topk(scores, T, E, k, topk_idx, topk_w, s, true);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "route_topk launch");
+}
+
 int moe_dispatch(const int32_t* topk_idx, int T, int k, int E, int32_t* counts, int32_t* offsets,
                  int32_t* perm, int32_t* pos, void* ws, size_t ws_bytes, void* stream) {
   (void)ws;

@@ -49,7 +49,10 @@ WorkspaceLayout workspace_layout(int T, int k, int E, int d, int f);
 
 // Host launchers (each returns a cudaError_t of the launch)
 cudaError_t launch_route_topk(const float* scores, int T, int E, int k, int32_t* idx, float* w,
-                              cudaStream_t s);
+                              cudaStream_t s, bool overlap = false);
+// scores [T][E] fp32 = x [T][d] bf16 . W_router [E][d] bf16 (router.cu)
+cudaError_t launch_router(const uint16_t* x, const uint16_t* w, int T, int d, int E, float* scores,
+                          cudaStream_t s, bool overlap = false);
 cudaError_t launch_dispatch(const int32_t* idx, int T, int k, int E, int32_t* counts,
                             int32_t* offsets, int32_t* perm, int32_t* pos, int* status,
                             cudaStream_t s, bool overlap = false);

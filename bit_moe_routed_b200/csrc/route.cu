@@ -71,14 +71,14 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ sco
 }  // namespace
 
 cudaError_t launch_route_topk(const float* scores, int T, int E, int k, int32_t* idx, float* w,
-                              cudaStream_t s) {
+                              cudaStream_t s, bool overlap) {
   const int warps_per_block = 8;
   const unsigned blocks = (unsigned)((T + warps_per_block - 1) / warps_per_block);
   if (E <= 256)
-    return launch_pdl(topk_kernel<8>, dim3(blocks), dim3(256), 0, s, false, scores, T, E, k, idx, w);
+    return launch_pdl(topk_kernel<8>, dim3(blocks), dim3(256), 0, s, overlap, scores, T, E, k, idx, w);
   if (E <= 512)
-    return launch_pdl(topk_kernel<16>, dim3(blocks), dim3(256), 0, s, false, scores, T, E, k, idx, w);
-  return launch_pdl(topk_kernel<32>, dim3(blocks), dim3(256), 0, s, false, scores, T, E, k, idx, w);
+    return launch_pdl(topk_kernel<16>, dim3(blocks), dim3(256), 0, s, overlap, scores, T, E, k, idx, w);
+  return launch_pdl(topk_kernel<32>, dim3(blocks), dim3(256), 0, s, overlap, scores, T, E, k, idx, w);
 }
 
 }  // namespace bitmoe

@@ -86,6 +86,18 @@ typedef struct {
 int moe_route_topk(const float* scores, int T, int E, int k, int32_t* topk_idx,
                    float* topk_w, void* stream);
 
+/* Router scoring + step 1 ([P2] "核心实现一": the router decides each token's experts
+ * from its hidden state): scores[t][e] = x[t] . W_router[e], summed in fp32 over bf16
+ * inputs, then the top-k of moe_route_topk on those scores.
+ *   x_bf16        [T][d] bf16 bit patterns; w_router_bf16 [E][d] bf16.
+ *   scores        [T][E] fp32 out (the router scores the selection used).
+ *   topk_idx, topk_w as for moe_route_topk.
+ * d % 128 == 0; 1 <= k <= min(E, 32); 1 <= E <= 1024; pointers 4-byte aligned.
+ * Two kernels: the scores (tiles of 16 tokens x 8 experts, bf16 mma.sync, fp32 sums in a
+ * fixed order), then top-k. */
+int moe_router_topk(const uint16_t* x_bf16, const uint16_t* w_router_bf16, int T, int d, int E,
+                    int k, float* scores, int32_t* topk_idx, float* topk_w, void* stream);
+
 /* Step 2 — dispatch ([P2] "核心实现三": group tokens by expert so each expert's
  * weights are read once for its whole group).  Stable counting sort of the T*k
  * (token, slot) pairs, flat id p = t*k + j, by expert.

@@ -249,6 +249,13 @@ def gen_scores(w: Workload, layer: int = 0) -> torch.Tensor:
     return gen_scores_uniform(w.T, w.E, w.seed(layer))
 
 
+def gen_router_weights(E: int, d: int, seed: int) -> torch.Tensor:
+    """W_router [E, d]: N(0, 1/d) drawn in fp32, rounded to bf16 (scores of unit-variance
+    tokens then have unit variance)."""
+    g = torch.Generator().manual_seed(int(seed) * 2 + 3)
+    return (torch.randn(E, d, generator=g, dtype=torch.float32) / math.sqrt(d)).to(torch.bfloat16)
+
+
 def gen_layer_inputs(w: Workload, layer: int = 0):
     """(x bf16 [T, d], scores fp32 [T, E]) for one layer of a workload, on the CPU."""
     return gen_x(w.T, w.d, w.seed(layer)), gen_scores(w, layer)
