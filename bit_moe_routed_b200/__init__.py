@@ -37,7 +37,7 @@ EXPORTS = (
     "moe_ffn_gate_up", "moe_ffn_down", "moe_combine", "moe_workspace_size", "moe_last_error",
     "moe_set_wait_limit_ns", "moe_sync_status", "moe_expert_ffn_noalloc",
     "moe_set_gemv_max_tokens", "moe_workspace_offsets", "moe_set_test_stall", "moe_forward",
-    "moe_ffn_path", "moe_router_topk",
+    "moe_ffn_path", "moe_router_topk", "moe_dispatch_workspace_size",
 )
 
 
@@ -90,12 +90,14 @@ def lib():
             "moe_forward": [P, P, I, I, W, P, P, P, P, P, P, P, P, P, P, Z, P],
             "moe_ffn_path": [I, I, W],
             "moe_router_topk": [P, P, I, I, I, I, P, P, P, P],
+            "moe_dispatch_workspace_size": [I, I, I],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
             fn.argtypes = args
             fn.restype = ctypes.c_int
         L.moe_workspace_size.restype = ctypes.c_size_t
+        L.moe_dispatch_workspace_size.restype = ctypes.c_size_t
         L.moe_last_error.restype = ctypes.c_char_p
         _lib = L
     return _lib
@@ -241,15 +243,18 @@ def router_topk(x: torch.Tensor, w_router: torch.Tensor, k: int, stream=None):
     return scores, idx, w
 
 
-def dispatch(idx: torch.Tensor, E: int, stream=None):
+def dispatch(idx: torch.Tensor, E: int, stream=None, multi: bool = True):
+    """Stable grouping per expert; large batches use the multi-CTA form unless multi=False."""
     T, k = idx.shape
     dev = idx.device
     counts = torch.empty(E, dtype=torch.int32, device=dev)
     offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
     perm = torch.empty(max(T * k, 1), dtype=torch.int32, device=dev)
     pos = torch.empty(max(T * k, 1), dtype=torch.int32, device=dev)
-    _check(lib().moe_dispatch(_p(idx), T, k, E, _p(counts), _p(offsets), _p(perm), _p(pos), None,
-                              0, _stream(stream)))
+    n = int(lib().moe_dispatch_workspace_size(T, k, E)) if multi else 0
+    ws = torch.empty(max(n, 4), dtype=torch.uint8, device=dev) if n else None
+    _check(lib().moe_dispatch(_p(idx), T, k, E, _p(counts), _p(offsets), _p(perm), _p(pos),
+                              _p(ws), n, _stream(stream)))
     return counts, offsets, perm[:T * k], pos[:T * k]
 
 

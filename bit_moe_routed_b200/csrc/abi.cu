@@ -199,6 +199,9 @@ WorkspaceLayout workspace_layout(int T, int k, int E, int d, int f) {
   // the combine counters of the single-token kernel (one per 16 output rows)
   L.done2 = o;
   if (T <= kGemvMaxT) o = align256(o + 4 * (size_t)(d / 16));
+  // the multi-CTA dispatch's counts (moe_forward on large batches)
+  L.dispatch = o;
+  o = align256(o + dispatch_ws_bytes(T, k, E));
   L.total = o;
   return L;
 }
@@ -225,6 +228,11 @@ int moe_set_gemv_max_tokens(int t) {
   if (t < 0) return fail(MOE_ERR_INVALID_ARG, "t=%d < 0", t);
   g_gemv_max_t.store(t);
   return MOE_OK;
+}
+
+size_t moe_dispatch_workspace_size(int T, int k, int E) {
+  if (T < 0 || k < 1 || E < 1) return 0;
+  return dispatch_ws_bytes(T, k, E);
 }
 
 size_t moe_workspace_size(int T, int k, int E, int d, int f) {
@@ -312,8 +320,6 @@ int moe_router_topk(const uint16_t* x_bf16, const uint16_t* w_router_bf16, int T
 
 int moe_dispatch(const int32_t* topk_idx, int T, int k, int E, int32_t* counts, int32_t* offsets,
                  int32_t* perm, int32_t* pos, void* ws, size_t ws_bytes, void* stream) {
-  (void)ws;
-  (void)ws_bytes;
   if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T=%d < 0", T);
   if (E < 1 || E > 1024) return fail(MOE_ERR_INVALID_ARG, "E=%d outside [1, 1024]", E);
   if (k < 1 || k > E) return fail(MOE_ERR_INVALID_ARG, "k=%d outside [1, E]", k);
@@ -323,6 +329,13 @@ int moe_dispatch(const int32_t* topk_idx, int T, int k, int E, int32_t* counts, 
   DeviceInfo di;
   int rc = device_info(di);
   if (rc) return rc;
+  const size_t need = dispatch_ws_bytes(T, k, E);
+  if (need > 0 && ws != nullptr && ws_bytes >= need && aligned(ws, 4)) {
+    cudaError_t e = launch_dispatch_multi(topk_idx, T, k, E, counts, offsets, perm, pos,
+                                          static_cast<int32_t*>(ws), di.status,
+                                          static_cast<cudaStream_t>(stream), t_overlap);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "dispatch launch");
+  }
   // T == 0 still writes counts = 0 and offsets = 0 (the kernel handles P == 0)
   cudaError_t e = launch_dispatch(topk_idx, T, k, E, counts, offsets, perm, pos, di.status,
                                   static_cast<cudaStream_t>(stream), t_overlap);
@@ -696,7 +709,8 @@ int moe_forward(const float* scores, const uint16_t* x_bf16, int T, int k,
   rc = moe_route_topk(scores, T, w->E, k, topk_idx, topk_w, stream);
   if (rc) return rc;
   OverlapScope guard;
-  rc = moe_dispatch(topk_idx, T, k, w->E, counts, offsets, perm, pos, nullptr, 0, stream);
+  rc = moe_dispatch(topk_idx, T, k, w->E, counts, offsets, perm, pos, c.ws + c.L.dispatch,
+                    dispatch_ws_bytes(T, k, w->E), stream);
   if (rc) return rc;
   rc = moe_expert_ffn(x_bf16, T, k, w, offsets, perm, y_routed, y_shared, ws, ws_bytes, stream);
   if (rc) return rc;

@@ -42,7 +42,7 @@ constexpr int kBgMaxT = 64;
 constexpr int kBgSlotTokens = 8;  // tokens per slot of the batched GEMV (the MMA's N)
 
 struct WorkspaceLayout {
-  size_t plan, qx, sx, qh, sh, counters, partials, hbuf, done2, total;
+  size_t plan, qx, sx, qh, sh, counters, partials, hbuf, done2, dispatch, total;
   size_t n_counters;
 };
 WorkspaceLayout workspace_layout(int T, int k, int E, int d, int f);
@@ -56,6 +56,13 @@ cudaError_t launch_router(const uint16_t* x, const uint16_t* w, int T, int d, in
 cudaError_t launch_dispatch(const int32_t* idx, int T, int k, int E, int32_t* counts,
                             int32_t* offsets, int32_t* perm, int32_t* pos, int* status,
                             cudaStream_t s, bool overlap = false);
+// Multi-CTA dispatch for large batches (T*k >= kDispatchMultiMin pairs): its workspace
+// holds one count per (segment of pairs, expert); 0 below the threshold.
+constexpr long long kDispatchMultiMin = 8192;
+size_t dispatch_ws_bytes(int T, int k, int E);
+cudaError_t launch_dispatch_multi(const int32_t* idx, int T, int k, int E, int32_t* counts,
+                                  int32_t* offsets, int32_t* perm, int32_t* pos, int32_t* cnt,
+                                  int* status, cudaStream_t s, bool overlap);
 // rows r < P = T*k take token perm[r]/k, rows P <= r < P+T take token r-P; perm may be
 // NULL with P = 0 for a plain quantisation of T rows.  If plan != NULL, one extra block
 // writes the token-tile plan (plan_mode 0) or the single-token path's list of active

@@ -106,7 +106,11 @@ int moe_router_topk(const uint16_t* x_bf16, const uint16_t* w_router_bf16, int T
  *   perm    [T*k] int32 out: perm[r] = flat id at sorted position r; pairs of one
  *           expert keep ascending flat-id order.
  *   pos     [T*k] int32 out: inverse of perm.
- * topk_idx values must lie in [0, E).  ws/ws_bytes are unused (may be NULL/0). */
+ * topk_idx values must lie in [0, E).
+ * ws/ws_bytes: optional scratch (may be NULL/0).  With at least
+ * moe_dispatch_workspace_size(T, k, E) bytes (nonzero from 8192 pairs up), a large batch
+ * runs a multi-CTA form (per-segment counts, then a scatter) instead of one CTA; the
+ * result is the same permutation.  The scratch needs no initial contents. */
 int moe_dispatch(const int32_t* topk_idx, int T, int k, int E, int32_t* counts,
                  int32_t* offsets, int32_t* perm, int32_t* pos, void* ws, size_t ws_bytes,
                  void* stream);
@@ -186,6 +190,10 @@ int moe_forward(const float* scores, const uint16_t* x_bf16, int T, int k,
  * d % 4 == 0; y_routed, y_shared and out 16-byte aligned. */
 int moe_combine(const float* y_routed, const float* y_shared, const float* topk_w,
                 const int32_t* pos, int T, int k, int d, float* out, void* stream);
+
+/* Bytes of scratch the multi-CTA dispatch uses for T*k pairs over E experts (0 when a
+ * batch that small runs the one-CTA form, or on invalid sizes). */
+size_t moe_dispatch_workspace_size(int T, int k, int E);
 
 /* Bytes of workspace moe_expert_ffn needs (0 on invalid sizes). */
 size_t moe_workspace_size(int T, int k, int E, int d, int f);

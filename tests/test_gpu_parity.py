@@ -63,6 +63,24 @@ def test_route_and_dispatch_odd_shapes(T, E, k):
     assert np.array_equal(perm.cpu().numpy(), perm_o)
 
 
+@pytest.mark.parametrize("T,E,k", [(1366, 256, 6), (4096, 256, 6), (2000, 1024, 8),
+                                   (9000, 7, 1), (4096, 256, 6)])
+def test_multi_cta_dispatch_matches_oracle_and_one_cta(T, E, k):
+    """Large batches: the multi-CTA dispatch (per-segment counts, then a scatter) gives the
+    oracle's stable permutation, bit for bit, and the same as the one-CTA kernel."""
+    assert bm.lib().moe_dispatch_workspace_size(T, k, E) > 0
+    s = synth.gen_scores_zipf(T, E, 1.2, seed=T + E) if E > 8 else \
+        synth.gen_scores_uniform(T, E, seed=T)
+    idx_o, _ = oracle.route_topk(s.numpy(), k)
+    idx = torch.from_numpy(idx_o).cuda()
+    multi = bm.dispatch(idx, E)
+    one = bm.dispatch(idx, E, multi=False)
+    ref = oracle.dispatch(idx_o, E)
+    for a, b_, r, name in zip(multi, one, ref, ("counts", "offsets", "perm", "pos")):
+        assert np.array_equal(a.cpu().numpy(), r), f"multi-CTA {name}"
+        assert torch.equal(a, b_), f"multi vs one CTA: {name}"
+
+
 def test_route_ties_go_to_lower_index():
     s = torch.tensor([[0.5, 0.9, 0.9, 0.1, 0.9] + [0.0] * 27], dtype=torch.float32)
     idx, _ = bm.route_topk(s.cuda(), 4)
