@@ -43,6 +43,7 @@
 #include "waits.cuh"
 
 #include <cstring>
+#include <type_traits>
 
 namespace bitmoe {
 
@@ -504,14 +505,12 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
 
   // ---------------------------------------------------------------- phases 1 and 2
   const int r0 = g, rr1 = g + 8;
-  bool ok = !*abort_flag;
-  bool switched = false;
+  const bool ok = !*abort_flag;
   int q = 0;
 
   // all warps arrive here once, after their phase-1 stages: h of this CTA's units to
   // the workspace, the grid barrier, then the h of phase 2's experts staged as f16
   auto phase_switch = [&]() {
-    switched = true;
     __syncthreads();
     if (!*abort_flag) {
       for (int i = threadIdx.x; i < r1.units() * 8; i += kDcThreads) {
@@ -571,28 +570,32 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
     __syncthreads();
   };
 
-  for (; q < qt; ++q) {
-    if (q == q1) phase_switch();
-    if (__shfl_sync(0xffffffffu, *abort_flag, 0)) {  // another warp gave up: stop too
-      ok = false;
-      break;
-    }
-    const int st = q % kDcStages;
-    if (p.stall && b == 0 && warp == 0 && q == 0 &&
-        !wait_warp(stall_bar, 0, p.wait_ns, abort_flag, p.status)) {
-      ok = false;
-      break;
-    }
-    if (!wait_warp(full(st), (uint32_t)(q / kDcStages) & 1u, p.wait_ns, abort_flag, p.status)) {
-      ok = false;
-      break;
-    }
-    const uint8_t* cst = codes_at(st);
-    const uint8_t* sst = scales_at(st);
-    float acc0 = 0.f, acc1 = 0.f;  // rows g and g+8 of the stage, column 0 (the token)
-    if (q < q1) {
-      const int task = warp + q * kDcWarps;
-      const int ul = task / S1, c = task % S1;
+  // one phase's stages of this warp (PH: 1 = gate/up, 2 = down), from q up to q_end;
+  // returns false if a wait ran out or another warp gave up
+  auto run = [&](auto phc, int q_end) -> bool {
+    constexpr int PH = decltype(phc)::value;
+    for (; q < q_end; ++q) {
+      if (__shfl_sync(0xffffffffu, *abort_flag, 0)) return false;  // another warp gave up
+      const int st = q % kDcStages;
+      if (p.stall && b == 0 && warp == 0 && q == 0 &&
+          !wait_warp(stall_bar, 0, p.wait_ns, abort_flag, p.status))
+        return false;
+      if (!wait_warp(full(st), (uint32_t)(q / kDcStages) & 1u, p.wait_ns, abort_flag, p.status))
+        return false;
+      const uint8_t* cst = codes_at(st);
+      const uint8_t* sst = scales_at(st);
+      const int task = warp + (PH == 1 ? q : q - q1) * kDcWarps;
+      const int S = PH == 1 ? S1 : S2;
+      const int ul = task / S, c = task % S;
+      const uint16_t* xb = bx;
+      const float* sxb = bs1;
+      if (PH == 2) {
+        int e, uin, ls, slot;
+        p2_local(ul, e, uin, ls, slot);
+        xb = bx + (size_t)ls * f;
+        sxb = bs2 + ls * (f / 128);
+      }
+      float acc0 = 0.f, acc1 = 0.f;  // rows g and g+8 of the stage, column 0 (the token)
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int j = 4 * c + i;
@@ -603,51 +606,8 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
 #pragma unroll
         for (int bb = 0; bb < 4; ++bb) {
           const int blk = 4 * i + bb;
-          const uint32_t wa = *reinterpret_cast<const uint32_t*>(cst + code_offset<1>(r0, blk, t));
-          const uint32_t wb = *reinterpret_cast<const uint32_t*>(cst + code_offset<1>(rr1, blk, t));
-          uint32_t ha[4], hb[4];
-          ptx::cvt_e2m1x8_f16(wa, ha);
-          ptx::cvt_e2m1x8_f16(wb, hb);
-          const uint4 xv = *reinterpret_cast<const uint4*>(bx + 128 * j + 32 * bb + 8 * t);
-          float cb[4];
-          ptx::mma_m16n8k16_f16_zero(cb, ha[0], hb[0], ha[1], hb[1], xv.x, xv.y);
-          ptx::mma_m16n8k16_f16(cb, ha[2], hb[2], ha[3], hb[3], xv.z, xv.w);
-          pa = fmaf(fa[bb], cb[0], pa);
-          pb = fmaf(fb[bb], cb[2], pb);
-        }
-        const float sxj = bs1[j];
-        acc0 = fmaf(sxj, pa, acc0);
-        acc1 = fmaf(sxj, pb, acc1);
-      }
-      __syncwarp();
-      if (issued < qt) {
-        if (lane == 0) issue(issued);
-        ++issued;
-      }
-      if (t == 0) {
-        float* pp = part1 + (ul * S1 + c) * kDcRows;
-        pp[r0] = acc0;
-        pp[rr1] = acc1;
-      }
-    } else {
-      const int task = warp + (q - q1) * kDcWarps;
-      const int ul = task / S2, c = task % S2;
-      int e, uin, ls, slot;
-      p2_local(ul, e, uin, ls, slot);
-      const uint16_t* xb = bx + (size_t)ls * f;
-      const float* sxb = bs2 + ls * (f / 128);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int j = 4 * c + i;
-        float fa[4], fb[4];
-        ue8m0x4_f32(*reinterpret_cast<const uint32_t*>(sst + r0 * 16 + 4 * i), fa);
-        ue8m0x4_f32(*reinterpret_cast<const uint32_t*>(sst + rr1 * 16 + 4 * i), fb);
-        float pa = 0.f, pb = 0.f;
-#pragma unroll
-        for (int bb = 0; bb < 4; ++bb) {
-          const int blk = 4 * i + bb;
-          const uint32_t wa = *reinterpret_cast<const uint32_t*>(cst + code_offset<2>(r0, blk, t));
-          const uint32_t wb = *reinterpret_cast<const uint32_t*>(cst + code_offset<2>(rr1, blk, t));
+          const uint32_t wa = *reinterpret_cast<const uint32_t*>(cst + code_offset<PH>(r0, blk, t));
+          const uint32_t wb = *reinterpret_cast<const uint32_t*>(cst + code_offset<PH>(rr1, blk, t));
           uint32_t ha[4], hb[4];
           ptx::cvt_e2m1x8_f16(wa, ha);
           ptx::cvt_e2m1x8_f16(wb, hb);
@@ -662,25 +622,31 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
         acc0 = fmaf(sxj, pa, acc0);
         acc1 = fmaf(sxj, pb, acc1);
       }
-      __syncwarp();
+      __syncwarp();  // every lane is done with the stage: it may be refilled
       if (issued < qt) {
         if (lane == 0) issue(issued);
         ++issued;
       }
       if (t == 0) {
-        float* pp = part2 + (ul * S2 + c) * kDcRows;
+        float* pp = (PH == 1 ? part1 + (ul * S1 + c) * kDcRows : part2 + (ul * S2 + c) * kDcRows);
         pp[r0] = acc0;
         pp[rr1] = acc1;
       }
     }
-  }
-  if (!ok) {  // let the copies this warp issued land before the CTA can exit
+    return true;
+  };
+  // let the copies this warp issued land before the CTA can go on or exit
+  auto give_up = [&]() {
     *abort_flag = 1;
     if (lane == 0)
       for (int r = q; r < issued; ++r) drain_wait(full(r % kDcStages), (uint32_t)(r / kDcStages) & 1u);
     __syncwarp();
-  }
-  if (!switched) phase_switch();
+    q = issued;
+  };
+
+  if (!(ok && run(std::integral_constant<int, 1>(), q1))) give_up();
+  phase_switch();
+  if (!run(std::integral_constant<int, 2>(), qt)) give_up();
   __syncthreads();
   if (*abort_flag) return;
 
