@@ -57,9 +57,12 @@ __device__ unsigned long long g_grid_bar;
 
 namespace {
 
-constexpr int kDcWarps = 24;
+// 16 warps x 3 ring stages: the same 204 KB in flight per SM as 24 x 2, and room for 128
+// registers per thread, so the inner loop does not spill (measured: 34.9 vs 37.0 us per
+// decode layer at d = 4096, f = 2048, k = 6)
+constexpr int kDcWarps = 16;
 constexpr int kDcThreads = kDcWarps * 32;
-constexpr int kDcStages = 2;                       // ring depth per warp
+constexpr int kDcStages = 3;                       // ring depth per warp
 constexpr int kDcRows = 16;                        // weight rows per stage
 constexpr int kDcCodeBytes = kDcRows * 256;        // 512 FP4 elements per row
 constexpr int kDcScaleBytes = kDcRows * 16;        // 16 ue8m0 bytes per row
@@ -505,6 +508,12 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
 
   // ---------------------------------------------------------------- phases 1 and 2
   const int r0 = g, rr1 = g + 8;
+  // the lane's 8 swizzled code offsets within a 128-byte row group: 16-byte chunk c of rows
+  // g and g + 8 (both g mod 8) lies at ((c ^ g) << 4), plus 4t for the lane's 4 bytes; the
+  // box and half offsets are compile-time constants (see code_offset)
+  uint32_t off8[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) off8[c] = (uint32_t)g * 128u + ((uint32_t)(c ^ g) << 4) + 4u * t;
   const bool ok = !*abort_flag;
   int q = 0;
 
@@ -606,8 +615,13 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
 #pragma unroll
         for (int bb = 0; bb < 4; ++bb) {
           const int blk = 4 * i + bb;
-          const uint32_t wa = *reinterpret_cast<const uint32_t*>(cst + code_offset<PH>(r0, blk, t));
-          const uint32_t wb = *reinterpret_cast<const uint32_t*>(cst + code_offset<PH>(rr1, blk, t));
+          // rows g and g + 8: boxes [matrix][half][8 rows] (phase 1) or [half][16 rows]
+          const uint32_t half = (uint32_t)(blk >> 3);
+          const uint32_t ba = PH == 1 ? half * 1024u : half * 2048u;
+          const uint32_t bbx = PH == 1 ? 2048u + half * 1024u : half * 2048u + 1024u;
+          const uint8_t* cp = cst + off8[blk & 7];
+          const uint32_t wa = *reinterpret_cast<const uint32_t*>(cp + ba);
+          const uint32_t wb = *reinterpret_cast<const uint32_t*>(cp + bbx);
           uint32_t ha[4], hb[4];
           ptx::cvt_e2m1x8_f16(wa, ha);
           ptx::cvt_e2m1x8_f16(wb, hb);

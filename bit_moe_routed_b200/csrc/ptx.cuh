@@ -96,6 +96,13 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* m, 
       "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
       : "memory");
 }
+// bring [src, src + bytes) into L2 (no shared-memory destination); 16-byte aligned, bytes a
+// multiple of 16
+__device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)),
+               "r"(bytes)
+               : "memory");
+}
 // L2 cache policies covering every access they are given to
 __device__ __forceinline__ uint64_t make_policy_evict_first() {
   uint64_t p;

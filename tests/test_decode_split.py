@@ -15,8 +15,9 @@ import pytest
 
 MAX_UNITS = 16    # kDcMaxUnits
 P2_SLOTS = 3      # kDcP2Slots: shared + two routed
-WARPS = 24
+WARPS = 16
 STAGE_BYTES = 16 * 256 + 16 * 16
+STAGES = 3
 SMEM_LIMIT = 232448   # bytes of shared memory a CTA may opt into on sm_100
 
 
@@ -45,11 +46,11 @@ def split(upe, n_routed, G, b):
 
 def smem_bytes(d, f):
     """Mirror of DcSmem::bytes()."""
-    area = WARPS * 2 * STAGE_BYTES
+    area = WARPS * STAGES * STAGE_BYTES
     p1_end = area + 2 * d + d // 32 + MAX_UNITS * (d // 512) * 64
     p2_end = area + P2_SLOTS * 2 * f + P2_SLOTS * (f // 32) + MAX_UNITS * (f // 512) * 64
     bars = (max(p1_end, p2_end) + 7) // 8 * 8
-    info = bars + (WARPS * 2 + 1) * 8
+    info = bars + (WARPS * STAGES + 1) * 8
     return info + 4 * (4 + 3 * 33 + 64) + 1024
 
 
@@ -102,8 +103,8 @@ def test_tma_boxes_stay_inside_their_tensors():
 
 
 def test_every_warp_takes_its_tasks_once():
-    """Tasks go round-robin (task = warp + 24 q); the first two of each warp are issued
-    before routing only when they belong to the shared expert."""
+    """Tasks go round-robin (task = warp + 16 q); the first ones of each warp (as many as its
+    ring holds) are issued before routing only when they belong to the shared expert."""
     S1 = 4096 // 512
     for b in (0, 73, 147):
         s_lo, ns, r_lo, nr = split(2048 // 8, 6, 148, b)
@@ -113,6 +114,6 @@ def test_every_warp_takes_its_tasks_once():
             q1 = -(-(n_tasks - w) // WARPS) if n_tasks > w else 0
             seen.extend(w + WARPS * q for q in range(q1))
             shared_q = -(-(ns * S1 - w) // WARPS) if ns * S1 > w else 0
-            for q in range(min(shared_q, 2)):
+            for q in range(min(shared_q, STAGES)):
                 assert (w + WARPS * q) // S1 < ns
         assert sorted(seen) == list(range(n_tasks))
