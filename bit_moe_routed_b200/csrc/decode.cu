@@ -27,8 +27,8 @@
 //
 // Work split: the shared expert's units and the routed experts' units are each cut into
 // one contiguous range per CTA (so every CTA holds 1-2 shared units to stream before
-// routing is known), and a CTA's stages go round-robin to its 24 warps, each with a
-// private ring of 2 stages filled by TMA (3-D code boxes with the 128-byte swizzle, 2-D
+// routing is known), and a CTA's stages go round-robin to its 16 warps, each with a
+// private ring of 3 stages filled by TMA (3-D code boxes with the 128-byte swizzle, 2-D
 // scale boxes).  Per 32-element block the warp decodes e2m1 pairs to f16 in registers
 // and runs two mma.sync m16n8k16 (fp32 accumulate); block partials are scaled by the
 // row's ue8m0 scale (exact) and the activation's fp32 block scale, and each row's stage
@@ -157,6 +157,13 @@ __device__ __forceinline__ int atom_add_acq_rel(int* p, int v) {
                : "memory");
   return old;
 }
+__device__ __forceinline__ unsigned long long atom_add_acq_rel_u64(unsigned long long* p,
+                                                                   unsigned long long v) {
+  unsigned long long old;
+  asm volatile("atom.acq_rel.gpu.global.add.u64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(v)
+               : "memory");
+  return old;
+}
 __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
   unsigned long long v;
   asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
@@ -182,17 +189,20 @@ struct Range {
 };
 
 // The bounded grid barrier (see g_grid_bar); false if the wait ran out.  ok_s: a word of
-// shared memory that carries thread 0's result to the CTA.
+// shared memory that carries thread 0's result to the CTA.  The CTA barrier orders the
+// CTA's writes before thread 0's arrival, an acq_rel atomic that releases them at GPU
+// scope; the last arrival (acq_rel: it has acquired every other arrival) opens the next
+// generation, and the waiters' acquire loads of it order their later reads after all
+// arrivals.
 __device__ bool grid_barrier(long long limit, int* status, volatile int* ok_s) {
   __syncthreads();
   if (threadIdx.x == 0) {
     int ok = 1;
-    __threadfence();
     const unsigned long long G = gridDim.x;
-    const unsigned long long old = atomicAdd(&g_grid_bar, 1ull);
+    const unsigned long long old = atom_add_acq_rel_u64(&g_grid_bar, 1ull);
     const unsigned long long gen = old >> 32;
     if ((old & 0xffffffffull) + 1 == G) {
-      atomicAdd(&g_grid_bar, (1ull << 32) - G);
+      atom_add_acq_rel_u64(&g_grid_bar, (1ull << 32) - G);
     } else {
       const uint64_t t0 = ptx::globaltimer();
       while ((ld_acquire_u64(&g_grid_bar) >> 32) == gen) {
@@ -203,7 +213,6 @@ __device__ bool grid_barrier(long long limit, int* status, volatile int* ok_s) {
         }
       }
     }
-    __threadfence();
     *ok_s = ok;
   }
   __syncthreads();
@@ -323,41 +332,41 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
   if (warp == 0) {
     if (MODE == kModeForward) {
       // top-k of the E scores (each lane holds experts lane + 32 i): k rounds of a warp
-      // arg-max on (value desc, index asc); then w_j = sigmoid(s_j) / sum over the k
+      // arg-max on (value desc, index asc), as a max of order-preserving integer keys and
+      // then a min of the indices holding it (two warp reductions a round); then
+      // w_j = sigmoid(s_j) / sum over the k
       float v[PL];
 #pragma unroll
       for (int i = 0; i < PL; ++i) {
         const int e = lane + 32 * i;
         v[i] = e < E ? __ldg(p.scores + e) : -INFINITY;
       }
+      // keys: a larger score has a larger key (sign-magnitude to offset order); NaN and
+      // padding get 0, below every number, so they are taken only after all numbers
+      uint32_t key[PL];
+#pragma unroll
+      for (int i = 0; i < PL; ++i) {
+        const uint32_t u = __float_as_uint(v[i] == 0.f ? 0.f : v[i]);  // -0 ties +0
+        key[i] = (v[i] != v[i] || lane + 32 * i >= E) ? 0u : ((u & 0x80000000u) ? ~u : (u | 0x80000000u));
+      }
       unsigned taken = 0;
       float sel_v = 0.f;
       int sel_i = 0;
       for (int j = 0; j < k; ++j) {
-        float bv = -INFINITY;
-        int bi = 0x7FFFFFFF;
+        uint32_t bk = 0u, bidx = 0xFFFFFFFFu;
 #pragma unroll
         for (int i = 0; i < PL; ++i) {
-          const int e = lane + 32 * i;
-          const bool ok = !((taken >> i) & 1u) && e < E;
-          if (ok && (v[i] > bv || (v[i] == bv && e < bi))) {
-            bv = v[i];
-            bi = e;
+          if (!((taken >> i) & 1u) && (key[i] > bk || bidx == 0xFFFFFFFFu)) {
+            bk = key[i];
+            bidx = (uint32_t)(lane + 32 * i);
           }
         }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-          const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-          const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-          if (ov > bv || (ov == bv && oi < bi)) {
-            bv = ov;
-            bi = oi;
-          }
-        }
-        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+        const uint32_t kmax = __reduce_max_sync(0xffffffffu, bk);
+        const uint32_t imin = __reduce_min_sync(0xffffffffu, bk == kmax ? bidx : 0xFFFFFFFFu);
+        if ((int)(imin & 31u) == lane) taken |= 1u << (imin >> 5);
         if (lane == j) {
-          sel_v = bv;
-          sel_i = bi;
+          sel_v = __uint_as_float((kmax & 0x80000000u) ? (kmax ^ 0x80000000u) : ~kmax);
+          sel_i = (int)imin;
         }
       }
       const float sig = lane < k ? 1.0f / (1.0f + expf(-sel_v)) : 0.0f;
@@ -543,35 +552,51 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
       }
     }
     if (!grid_barrier(p.wait_ns, p.status, barrier_ok)) *abort_flag = 1;
-    // stage h: one warp per (local slot, 128-block), 4 values per lane
+    // stage h: one warp per (local slot, 128-block), 4 values per lane; a warp loads the
+    // h of up to four of its tasks before quantising any, so their L2 latencies overlap
     const int nb = f / 128;
     const int nls = 1 + (r2.nr > 0 ? (r2.r_lo + r2.nr - 1) / upe2 - r2_slot0 + 1 : 0);
     if (!*abort_flag) {
-      for (int wi = warp; wi < nls * nb; wi += kDcWarps) {
-        const int ls = wi / nb, j = wi % nb;
-        if (ls == 0 && r2.ns == 0) continue;
-        const int slot = ls == 0 ? n_act : r2_slot0 + ls - 1;
-        const float4 h = __ldcg(reinterpret_cast<const float4*>(p.hbuf + (size_t)slot * f +
-                                                                128 * j + 4 * lane));
-        float amax = fmaxf(fmaxf(fabsf(h.x), fabsf(h.y)), fmaxf(fabsf(h.z), fabsf(h.w)));
+      for (int w0 = warp; w0 < nls * nb; w0 += 4 * kDcWarps) {
+        float4 hv[4];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        const float sc = amax == 0.f ? 1.0f : __fdiv_rn(amax, 448.0f);
-        const uint16_t q01 = ptx::cvt_e4m3x2(__fdiv_rn(h.x, sc), __fdiv_rn(h.y, sc));
-        const uint16_t q23 = ptx::cvt_e4m3x2(__fdiv_rn(h.z, sc), __fdiv_rn(h.w, sc));
-        uint32_t* dst = reinterpret_cast<uint32_t*>(bx + (size_t)ls * f + 128 * j + 4 * lane);
-        dst[0] = ptx::cvt_e4m3x2_f16x2(q01);
-        dst[1] = ptx::cvt_e4m3x2_f16x2(q23);
-        if (lane == 0) bs2[ls * nb + j] = sc;
-        // the CTA holding the expert's first unit also stores its codes and scales
-        const bool owner = ls == 0 ? r2.s_lo == 0 : slot * upe2 >= r2.r_lo;
-        if (owner) {
-          const uint32_t qw = (uint32_t)q01 | ((uint32_t)q23 << 16);
-          const int rows = ls == 0 ? 1 : slot_n[slot];
-          const int row0 = ls == 0 ? k : slot_row[slot];
-          for (int rr = 0; rr < rows; ++rr) {
-            *reinterpret_cast<uint32_t*>(p.qh + (size_t)(row0 + rr) * f + 128 * j + 4 * lane) = qw;
-            if (lane == 0) p.sh[(size_t)(row0 + rr) * nb + j] = sc;
+        for (int u = 0; u < 4; ++u) {
+          const int wi = w0 + u * kDcWarps;
+          const int ls = wi / nb, j = wi % nb;
+          hv[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (wi < nls * nb && !(ls == 0 && r2.ns == 0)) {
+            const int slot = ls == 0 ? n_act : r2_slot0 + ls - 1;
+            hv[u] = __ldcg(reinterpret_cast<const float4*>(p.hbuf + (size_t)slot * f + 128 * j +
+                                                           4 * lane));
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int wi = w0 + u * kDcWarps;
+          const int ls = wi / nb, j = wi % nb;
+          if (wi >= nls * nb || (ls == 0 && r2.ns == 0)) continue;
+          const int slot = ls == 0 ? n_act : r2_slot0 + ls - 1;
+          const float4 h = hv[u];
+          float amax = fmaxf(fmaxf(fabsf(h.x), fabsf(h.y)), fmaxf(fabsf(h.z), fabsf(h.w)));
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+          const float sc = amax == 0.f ? 1.0f : __fdiv_rn(amax, 448.0f);
+          const uint16_t q01 = ptx::cvt_e4m3x2(__fdiv_rn(h.x, sc), __fdiv_rn(h.y, sc));
+          const uint16_t q23 = ptx::cvt_e4m3x2(__fdiv_rn(h.z, sc), __fdiv_rn(h.w, sc));
+          uint32_t* dst = reinterpret_cast<uint32_t*>(bx + (size_t)ls * f + 128 * j + 4 * lane);
+          dst[0] = ptx::cvt_e4m3x2_f16x2(q01);
+          dst[1] = ptx::cvt_e4m3x2_f16x2(q23);
+          if (lane == 0) bs2[ls * nb + j] = sc;
+          // the CTA holding the expert's first unit also stores its codes and scales
+          const bool owner = ls == 0 ? r2.s_lo == 0 : slot * upe2 >= r2.r_lo;
+          if (owner) {
+            const uint32_t qw = (uint32_t)q01 | ((uint32_t)q23 << 16);
+            const int rows = ls == 0 ? 1 : slot_n[slot];
+            const int row0 = ls == 0 ? k : slot_row[slot];
+            for (int rr = 0; rr < rows; ++rr) {
+              *reinterpret_cast<uint32_t*>(p.qh + (size_t)(row0 + rr) * f + 128 * j + 4 * lane) = qw;
+              if (lane == 0) p.sh[(size_t)(row0 + rr) * nb + j] = sc;
+            }
           }
         }
       }
