@@ -35,9 +35,13 @@ def build(force: bool = False) -> str:
     return SO
 
 
+FP4, Q2 = 0, 1  # weight codecs (oracle.h: ORACLE_FP4, ORACLE_Q2)
+
+
 class _Expert(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
-        "gate_codes", "gate_scales", "up_codes", "up_scales", "down_codes", "down_scales")]
+        "gate_codes", "gate_scales", "up_codes", "up_scales", "down_codes", "down_scales")] + [
+        ("codec", ctypes.c_int)]
 
 
 _lib = None
@@ -56,6 +60,8 @@ def lib():
         L.oracle_e4m3_value.restype = ctypes.c_double
         L.oracle_ue8m0_value.argtypes = [I]
         L.oracle_ue8m0_value.restype = ctypes.c_double
+        L.oracle_q2_value.argtypes = [I]
+        L.oracle_q2_value.restype = ctypes.c_double
         L.oracle_e4m3_encode.argtypes = [ctypes.c_float]
         L.oracle_e4m3_encode.restype = ctypes.c_uint8
         L.oracle_quant_blocks.argtypes = [P, I, P, P]
@@ -64,6 +70,7 @@ def lib():
         L.oracle_router_scores.argtypes = [P, P, I, I, I, P]
         L.oracle_dispatch.argtypes = [P, I, I, I, P, P, P, P]
         L.oracle_fp4_gemv.argtypes = [P, P, I, I, P, P]
+        L.oracle_q2_gemv.argtypes = [P, P, I, I, P, P]
         L.oracle_expert_ffn.argtypes = [ctypes.POINTER(_Expert), I, I, P, P, I, P, P, P]
         L.oracle_expert_ffn_h.argtypes = [ctypes.POINTER(_Expert), I, I, P, P, I, P, P, P, P]
         L.oracle_combine_token.argtypes = [P, P, P, I, I, P]
@@ -100,6 +107,10 @@ def e4m3_value(code: int) -> float:
 
 def ue8m0_value(code: int) -> float:
     return lib().oracle_ue8m0_value(int(code))
+
+
+def q2_value(code: int) -> float:
+    return lib().oracle_q2_value(int(code))
 
 
 def e4m3_encode(v) -> np.ndarray:
@@ -177,11 +188,23 @@ def fp4_gemv(codes: np.ndarray, scales: np.ndarray, xhat: np.ndarray) -> np.ndar
     return out
 
 
+def q2_gemv(codes: np.ndarray, scales: np.ndarray, xhat: np.ndarray) -> np.ndarray:
+    """2-bit matrix (codes [rows, K/4], scales [rows, K/128]) times xhat, in double."""
+    codes, pc = _c(codes, np.uint8)
+    scales, psc = _c(scales, np.uint8)
+    xhat, px = _c(xhat, np.float64)
+    rows, K = codes.shape[0], codes.shape[1] * 4
+    out = np.empty(rows, np.float64)
+    lib().oracle_q2_gemv(pc, psc, rows, K, px, out.ctypes.data)
+    return out
+
+
 class ExpertSet:
     """Holds numpy weight arrays alive and exposes a ctypes array of experts.
 
     ``experts`` maps expert index -> object with gate_codes, gate_scales, up_codes,
-    up_scales, down_codes, down_scales (uint8 numpy arrays); missing experts are NULL.
+    up_scales, down_codes, down_scales (uint8 numpy arrays) and optionally ``codec``
+    (FP4 when absent); missing experts are NULL.
     """
 
     def __init__(self, n: int, experts: dict):
@@ -194,7 +217,7 @@ class ExpertSet:
                 a = np.ascontiguousarray(getattr(ex, name), dtype=np.uint8)
                 self._keep.append(a)
                 vals.append(a.ctypes.data)
-            self.arr[e] = _Expert(*vals)
+            self.arr[e] = _Expert(*vals, int(getattr(ex, "codec", FP4)))
 
 
 def expert_ffn(ex, d: int, f: int, qx: np.ndarray, sx: np.ndarray, want_h: bool = False):

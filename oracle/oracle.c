@@ -187,6 +187,18 @@ static inline double fp4_weight(const uint8_t* codes, const uint8_t* scales, int
     return oracle_e2m1_value(code) * oracle_ue8m0_value(scales[(size_t)r * (K / 32) + c / 32]);
 }
 
+/* 2-bit routed-expert codec (ai-muninn.com post "一張 22G 老卡跑 284B": IQ2_XXS routed
+ * experts at 2.0625 bits per weight; the code book is this library's reading, see
+ * oracle.h): value = code - 1.5, one ue8m0 scale per 128 elements. */
+double oracle_q2_value(int code) { return (double)(code & 3) - 1.5; }
+
+static inline double q2_weight(const uint8_t* codes, const uint8_t* scales, int K, int r,
+                               int c) {
+    uint8_t byte = codes[(size_t)r * (K / 4) + c / 4];
+    int code = (byte >> (2 * (c & 3))) & 3;
+    return oracle_q2_value(code) * oracle_ue8m0_value(scales[(size_t)r * (K / 128) + c / 128]);
+}
+
 static int g_threads = 1;
 void oracle_set_threads(int n) { g_threads = n < 1 ? 1 : n; }
 int oracle_get_threads(void) { return g_threads; }
@@ -201,10 +213,22 @@ void oracle_fp4_gemv(const uint8_t* codes, const uint8_t* scales, int rows, int 
     }
 }
 
-/* Decode one FP4 row into doubles. */
-static void decode_row(const uint8_t* codes, const uint8_t* scales, int K, int r,
+void oracle_q2_gemv(const uint8_t* codes, const uint8_t* scales, int rows, int K,
+                    const double* xhat, double* out) {
+#pragma omp parallel for num_threads(g_threads) schedule(static)
+    for (int r = 0; r < rows; ++r) {
+        double acc = 0.0;
+        for (int c = 0; c < K; ++c) acc += q2_weight(codes, scales, K, r, c) * xhat[c];
+        out[r] = acc;
+    }
+}
+
+/* Decode one weight row (FP4 or 2-bit codec) into doubles. */
+static void decode_row(int codec, const uint8_t* codes, const uint8_t* scales, int K, int r,
                        double* dst) {
-    for (int c = 0; c < K; ++c) dst[c] = fp4_weight(codes, scales, K, r, c);
+    for (int c = 0; c < K; ++c)
+        dst[c] = codec == ORACLE_Q2 ? q2_weight(codes, scales, K, r, c)
+                                    : fp4_weight(codes, scales, K, r, c);
 }
 
 /* One expert over a group of tokens: g = Wg xhat, u = Wu xhat, h = silu(g) * u
@@ -237,8 +261,8 @@ void oracle_expert_ffn_h(const oracle_expert_t* w, int d, int f, const uint8_t* 
         double* ru = (double*)malloc(sizeof(double) * (size_t)d);
 #pragma omp for schedule(static)
         for (int n = 0; n < f; ++n) {
-            decode_row(w->gate_codes, w->gate_scales, d, n, rg);
-            decode_row(w->up_codes, w->up_scales, d, n, ru);
+            decode_row(w->codec, w->gate_codes, w->gate_scales, d, n, rg);
+            decode_row(w->codec, w->up_codes, w->up_scales, d, n, ru);
             for (int t = 0; t < ntok; ++t) {
                 const double* xt = xhat + (size_t)t * d;
                 double ag = 0.0, au = 0.0;
@@ -275,7 +299,7 @@ void oracle_expert_ffn_h(const oracle_expert_t* w, int d, int f, const uint8_t* 
         double* rd = (double*)malloc(sizeof(double) * (size_t)f);
 #pragma omp for schedule(static)
         for (int m = 0; m < d; ++m) {
-            decode_row(w->down_codes, w->down_scales, f, m, rd);
+            decode_row(w->codec, w->down_codes, w->down_scales, f, m, rd);
             for (int t = 0; t < ntok; ++t) {
                 const double* ht = hhat + (size_t)t * f;
                 double acc = 0.0;

@@ -23,6 +23,14 @@
  *    fp32, combine weight = sigmoid of the selected scores renormalised to 1,
  *    shared expert added with weight 1.
  *  Formats: OCP Microscaling Formats (MX) Specification v1.0 (e2m1, e4m3, e8m0).
+ *  - "一張 22G 老卡跑 284B" post (ai-muninn.com): the routed experts of the deployed model
+ *    are 2-bit (IQ2_XXS, 2.0625 bits per weight) while the always-resident weights
+ *    (shared expert included) stay at higher precision; the "2-bit routed experts only"
+ *    of the ds4 engine (smzdm.com post) is the same split.  The pages name the bit rate,
+ *    not the code book, so the 2-bit codec here is read as: four 2-bit codes per byte
+ *    (element i of a byte in bits 2i..2i+1), value = code - 1.5 (the uniform
+ *    four-level grid -1.5, -0.5, 0.5, 1.5), times one ue8m0 scale per 128 consecutive
+ *    elements along the reduction axis: 2 + 8/128 = 2.0625 bits per weight.
  *
  * Floating point: all sums are in double.  Activation quantisation is done in
  * fp32 arithmetic (divide, then round to nearest e4m3, ties to even mantissa,
@@ -37,8 +45,11 @@
 extern "C" {
 #endif
 
-/* Per-expert weight pointers: codes [rows][K/2] bytes, scales [rows][K/32] bytes.
- * gate/up: rows = f, K = d.  down: rows = d, K = f. */
+/* Per-expert weight pointers.  gate/up: rows = f, K = d.  down: rows = d, K = f.
+ * codec ORACLE_FP4: codes [rows][K/2] bytes, scales [rows][K/32] bytes.
+ * codec ORACLE_Q2:  codes [rows][K/4] bytes, scales [rows][K/128] bytes. */
+#define ORACLE_FP4 0
+#define ORACLE_Q2 1
 typedef struct {
     const uint8_t* gate_codes;
     const uint8_t* gate_scales;
@@ -46,12 +57,14 @@ typedef struct {
     const uint8_t* up_scales;
     const uint8_t* down_codes;
     const uint8_t* down_scales;
+    int codec;
 } oracle_expert_t;
 
 /* Format decoding from bit fields (OCP MX v1.0). */
 double oracle_e2m1_value(int code);   /* code in [0,16) */
 double oracle_e4m3_value(int code);   /* code in [0,256); NaN for 0x7F/0xFF */
 double oracle_ue8m0_value(int code);  /* code in [0,256); NaN for 0xFF */
+double oracle_q2_value(int code);     /* code in [0,4): code - 1.5 */
 
 /* fp32 -> e4m3fn code: round to nearest, ties to even mantissa, saturate to +-448. */
 uint8_t oracle_e4m3_encode(float v);
@@ -81,6 +94,11 @@ void oracle_dispatch(const int32_t* idx, int T, int k, int E, int32_t* counts,
  * W[r,k] = e2m1(code) * ue8m0(scale[r, k/32]), in double. */
 void oracle_fp4_gemv(const uint8_t* codes, const uint8_t* scales, int rows, int K,
                      const double* xhat, double* out);
+
+/* The same for a 2-bit matrix: W[r,k] = q2(code) * ue8m0(scale[r, k/128]), code of
+ * element k in bits 2(k%4)..2(k%4)+1 of byte codes[r, k/4]; in double. */
+void oracle_q2_gemv(const uint8_t* codes, const uint8_t* scales, int rows, int K,
+                    const double* xhat, double* out);
 
 /* One expert FFN over a group of ntok tokens that share its weights (layer-major:
  * each weight row is decoded once and dotted with every token of the group).

@@ -197,6 +197,60 @@ def device_layer_weights(seed: int, layer: int, E: int, d: int, f: int, device="
 
 
 # --------------------------------------------------------------------------------------
+# 2-bit routed-expert weights: codes [rows, K/4] (four 2-bit codes per byte) and scales
+# [rows, K/128], drawn by the same generator as the FP4 bytes from seeds seed ^ Q2_SEED
+# (other streams than the FP4 weights of the same layer).  Any byte is four valid codes;
+# scale bytes are 121 + (byte AND 3), as for FP4.
+# --------------------------------------------------------------------------------------
+Q2_SEED = 0x5132
+
+
+def q2_cols(which: int, kind: int, d: int, f: int) -> int:
+    r, K = matrix_shape(which, d, f)
+    return K // 4 if kind == CODES else K // 128
+
+
+def expert_matrix_host_q2(seed: int, layer: int, expert: int, which: int, kind: int, d: int,
+                          f: int) -> np.ndarray:
+    r, _ = matrix_shape(which, d, f)
+    out = np.empty((r, q2_cols(which, kind, d, f)), dtype=np.uint8)
+    _host_lib().synth_fill(seed ^ Q2_SEED, layer, expert, which, kind, out.ctypes.data, 0,
+                           out.size)
+    return out
+
+
+def host_expert_q2(seed: int, layer: int, expert: int, d: int, f: int) -> HostExpert:
+    g = lambda m, k: expert_matrix_host_q2(seed, layer, expert, m, k, d, f)  # noqa: E731
+    return HostExpert(g(GATE, CODES), g(GATE, SCALES), g(UP, CODES), g(UP, SCALES),
+                      g(DOWN, CODES), g(DOWN, SCALES))
+
+
+def device_layer_weights_q2(seed: int, layer: int, E: int, d: int, f: int, device="cuda",
+                            stream=None):
+    """The E routed experts of a layer in the 2-bit codec, in device memory (torch uint8
+    tensors [E, rows, cols]); the same bytes as host_expert_q2."""
+    lib = _dev_lib()
+    out = {}
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    for name, which in (("gate", GATE), ("up", UP), ("down", DOWN)):
+        r, _ = matrix_shape(which, d, f)
+        for kind, suffix in ((CODES, "codes"), (SCALES, "scales")):
+            cols = q2_cols(which, kind, d, f)
+            t = torch.empty((E, r, cols), dtype=torch.uint8, device=device)
+            rc = lib.synth_fill_dev(seed ^ Q2_SEED, layer, E, which, kind, r * cols, t.data_ptr(),
+                                    ctypes.c_void_p(s.cuda_stream))
+            if rc != 0:
+                raise RuntimeError(f"synth_fill_dev failed: {rc}")
+            out[f"{name}_{suffix}"] = t
+    return out
+
+
+def q2_expert_bytes(d: int, f: int) -> int:
+    return sum(matrix_shape(m, d, f)[0] * (q2_cols(m, CODES, d, f) + q2_cols(m, SCALES, d, f))
+               for m in (GATE, UP, DOWN))
+
+
+# --------------------------------------------------------------------------------------
 # Activations and router scores (torch CPU generators, fp32 then rounded where stated)
 # --------------------------------------------------------------------------------------
 def gen_x(T: int, d: int, seed: int) -> torch.Tensor:
