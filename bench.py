@@ -48,7 +48,7 @@ SPEC_HBM_GBS = 8000.0          # B200 HBM3e, spec
 SPEC_FP8_TFLOPS = 4500.0       # B200 dense FP8, spec
 L2_BYTES = 126 * 2 ** 20
 EXTRA_WORKLOADS = ("decode_t64_zipf", "prefill_t4096_uniform", "prefill_t4096_zipf",
-                   "layers43_t1", "layers43_t32")
+                   "layers43_t1", "layers43_t32", "decode_t1_q2")
 
 
 def load_peaks():
@@ -124,12 +124,16 @@ def layer_work(w, counts: np.ndarray):
     R = T * k + T
     gu_w = 2 * (f * d // 2 + f * d // 32)            # gate + up codes and scales per expert
     dn_w = d * f // 2 + d * f // 32
+    weight_bytes = active * (gu_w + dn_w)
+    if w.routed_codec == "q2":  # routed experts 2-bit (codes K/4, scales K/128 per row)
+        q2_w = 3 * (f * d // 4 + f * d // 128)
+        weight_bytes = (active - 1) * q2_w + gu_w + dn_w
     gu_bytes = active * gu_w + R * d + R * (d // 128) * 4 + R * f + R * (f // 128) * 4
     dn_bytes = active * dn_w + R * f + R * (f // 128) * 4 + R * d * 4
     flops_gu = 2 * 2 * R * d * f
     flops_dn = 2 * R * d * f
     return dict(active=active, gu_bytes=gu_bytes, dn_bytes=dn_bytes, flops_gu=flops_gu,
-                flops_dn=flops_dn, weight_bytes=active * (gu_w + dn_w))
+                flops_dn=flops_dn, weight_bytes=weight_bytes)
 
 
 def kernel_traffic(kernel_file: str, name: str, workload: str):
@@ -236,6 +240,19 @@ def fp8_peak_of(peaks: dict, bf16_peak: float):
 
 
 # ------------------------------------------------------------------------ CPU oracle leg
+def host_expert_for(w, layer_seed: int, e: int):
+    """Host copy of expert e as the oracle takes it (2-bit routed experts tagged with
+    their codec; the shared expert, index E, is FP4)."""
+    import oracle
+    if w.routed_codec == "q2" and e < w.E:
+        he = synth.host_expert_q2(layer_seed, 0, e, w.d, w.f)
+        ex = type("Q2Expert", (), {})()
+        ex.__dict__.update(he.__dict__)
+        ex.codec = oracle.Q2
+        return ex
+    return synth.host_expert(layer_seed, 0, e, w.d, w.f)
+
+
 def oracle_sample(w, x, scores, seconds: float, layer_seed: int):
     """Time the oracle on whole tokens of this workload for about `seconds` seconds.
     Returns (tokens/s, cores, description)."""
@@ -249,7 +266,7 @@ def oracle_sample(w, x, scores, seconds: float, layer_seed: int):
         need = set(idx[t].tolist()) | {w.E}
         for e in need:  # weight generation is input preparation, not timed
             if e not in cache:
-                cache[e] = synth.host_expert(layer_seed, 0, e, w.d, w.f)
+                cache[e] = host_expert_for(w, layer_seed, e)
         ta = time.perf_counter()
         oracle.moe_tokens(x, w.E, w.k, w.d, w.f, {e: cache[e] for e in need}, idx, gw, [t])
         elapsed += time.perf_counter() - ta
@@ -269,7 +286,7 @@ def oracle_extras(w, x, scores, layer_seed: int) -> dict:
     oracle.dispatch(idx, w.E)
     route_s = time.perf_counter() - ta
     need = set(idx[0].tolist()) | {w.E}
-    experts = {e: synth.host_expert(layer_seed, 0, e, w.d, w.f) for e in need}
+    experts = {e: host_expert_for(w, layer_seed, e) for e in need}
     cores = os.cpu_count() or 1
     oracle.set_threads(1)
     try:
@@ -343,7 +360,9 @@ class Layers:
                 s_cpu = synth.gen_scores_uniform(T, E, seed) if w.routing == "uniform" else \
                     synth.gen_scores_zipf(T, E, w.zipf_s, seed)
             W = bm.LayerWeights.from_dict(synth.device_layer_weights(w.seed(l), l, E, d, f))
-            self.items.append(dict(x_cpu=x_cpu, s_cpu=s_cpu, W=W, x=x_cpu.to(dev),
+            Q = bm.Q2Experts.from_dict(synth.device_layer_weights_q2(w.seed(l), l, E, d, f)) \
+                if w.routed_codec == "q2" else None
+            self.items.append(dict(x_cpu=x_cpu, s_cpu=s_cpu, W=W, Q=Q, x=x_cpu.to(dev),
                                    scores=s_cpu.to(dev)))
         self.ws = bm.alloc_workspace(T, k, E, d, f, dev)
         i32, f32 = torch.int32, torch.float32
@@ -364,7 +383,8 @@ def resident_layers(w, max_layers):
     if w.layers > 1:
         return w.layers
     per_expert = synth.expert_bytes(w.d, w.f)
-    step_bytes = (min(w.E, w.T * w.k) + 1) * per_expert
+    routed = synth.q2_expert_bytes(w.d, w.f) if w.routed_codec == "q2" else per_expert
+    step_bytes = min(w.E, w.T * w.k) * routed + per_expert
     return max(min(2, max_layers), min(max_layers, -(-4 * L2_BYTES // step_bytes) + 1))
 
 
@@ -381,8 +401,12 @@ def measure(bm, w, args, dev, stream, rank, dist, steps, warmup, peaks, cpu_seco
     # otherwise route, dispatch, prepare, gate/up, down and combine back to back
     fused = T == 1 and d % 512 == 0 and f % 512 == 0
     batched = 2 <= T <= 64 and d % 512 == 0 and f % 512 == 0  # the batched GEMV path
+    q2 = w.routed_codec == "q2"
 
     def step(L):
+        if q2:
+            return bm.forward_q2(L["x"], L["scores"], k, L["W"], L["Q"], Ls.ws, stream,
+                                 outs=Ls.outs)["counts"]
         return bm.forward(L["x"], L["scores"], k, L["W"], Ls.ws, stream, outs=Ls.outs)["counts"]
 
     # one eager pass per layer (checks the status word and gives the routing counts)
@@ -471,6 +495,10 @@ def measure(bm, w, args, dev, stream, rank, dist, steps, warmup, peaks, cpu_seco
         kernel_name = ("decode_kernel: the whole layer in one cooperative kernel (routing, "
                        "dispatch, quantisation, FP4 GEMVs with in-register e2m1 decode and "
                        "mma.sync, combine)")
+        if q2:
+            kernel_name = ("decode_kernel, Q2 form: the whole layer in one cooperative kernel, "
+                           "2-bit routed experts (byte-permute decode to e4m3, mma.sync e4m3) "
+                           "and the FP4 shared expert")
         traffic = kernel_traffic(kernel_file, "layer", w.name)
         io = 4 * E + 2 * d + 4 * d * (k + 2)  # scores, x; y_routed, y_shared and out
         work["gu_bytes"] = work["weight_bytes"] + io

@@ -37,7 +37,7 @@ EXPORTS = (
     "moe_ffn_gate_up", "moe_ffn_down", "moe_combine", "moe_workspace_size", "moe_last_error",
     "moe_set_wait_limit_ns", "moe_sync_status", "moe_expert_ffn_noalloc",
     "moe_set_gemv_max_tokens", "moe_workspace_offsets", "moe_set_test_stall", "moe_forward",
-    "moe_ffn_path", "moe_router_topk", "moe_dispatch_workspace_size",
+    "moe_ffn_path", "moe_router_topk", "moe_dispatch_workspace_size", "moe_forward_q2",
 )
 
 
@@ -45,6 +45,11 @@ class MoeError(RuntimeError):
     def __init__(self, code: int, msg: str):
         super().__init__(f"bitmoe error {code}: {msg}")
         self.code = code
+
+
+class _Q2Experts(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "gate_codes", "gate_scales", "up_codes", "up_scales", "down_codes", "down_scales")]
 
 
 class _Weights(ctypes.Structure):
@@ -91,6 +96,8 @@ def lib():
             "moe_ffn_path": [I, I, W],
             "moe_router_topk": [P, P, I, I, I, I, P, P, P, P],
             "moe_dispatch_workspace_size": [I, I, I],
+            "moe_forward_q2": [P, P, I, W, ctypes.POINTER(_Q2Experts), P, P, P, P, P, P, P, P,
+                               P, P, Z, P],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -155,6 +162,29 @@ class LayerWeights:
     @staticmethod
     def from_dict(d: dict) -> "LayerWeights":
         return LayerWeights(**{k: d[k] for k in (
+            "gate_codes", "gate_scales", "up_codes", "up_scales", "down_codes", "down_scales")})
+
+
+@dataclass
+class Q2Experts:
+    """The E routed experts of a layer in the 2-bit codec on the device: gate_codes /
+    up_codes [E, f, d/4], gate_scales / up_scales [E, f, d/128], down_codes [E, d, f/4],
+    down_scales [E, d, f/128] (uint8)."""
+    gate_codes: torch.Tensor
+    gate_scales: torch.Tensor
+    up_codes: torch.Tensor
+    up_scales: torch.Tensor
+    down_codes: torch.Tensor
+    down_scales: torch.Tensor
+
+    def struct(self) -> _Q2Experts:
+        return _Q2Experts(*(t.data_ptr() for t in (
+            self.gate_codes, self.gate_scales, self.up_codes, self.up_scales, self.down_codes,
+            self.down_scales)))
+
+    @staticmethod
+    def from_dict(d: dict) -> "Q2Experts":
+        return Q2Experts(**{k: d[k] for k in (
             "gate_codes", "gate_scales", "up_codes", "up_scales", "down_codes", "down_scales")})
 
 
@@ -355,6 +385,36 @@ def forward(x: torch.Tensor, scores: torch.Tensor, k: int, w: LayerWeights,
     return dict(idx=o["idx"], w=o["w"], counts=o["counts"], offsets=o["offsets"],
                 perm=o["perm"][:T * k], pos=o["pos"][:T * k], y=o["y"][:T * k],
                 y_shared=o["y_shared"][:T], out=o["out"][:T])
+
+
+def forward_q2(x: torch.Tensor, scores: torch.Tensor, k: int, w: LayerWeights, q2: Q2Experts,
+               ws: torch.Tensor | None = None, stream=None, outs: dict | None = None):
+    """One token through the layer with 2-bit routed experts (moe_forward_q2): the routed
+    experts from `q2`, the shared expert from `w` (FP4, index E).  Returns the dict of
+    `forward`."""
+    T, d = x.shape
+    if T != 1:
+        raise ValueError("moe_forward_q2 takes one token")
+    E = w.E
+    dev = x.device
+    if ws is None:
+        ws = alloc_workspace(1, k, E, w.d, w.f, dev)
+    o = dict(outs) if outs is not None else {}
+    shapes = {"idx": ((1, k), torch.int32), "w": ((1, k), torch.float32),
+              "counts": ((E,), torch.int32), "offsets": ((E + 1,), torch.int32),
+              "perm": ((k,), torch.int32), "pos": ((k,), torch.int32),
+              "y": ((k, d), torch.float32), "y_shared": ((1, d), torch.float32),
+              "out": ((1, d), torch.float32)}
+    for name, (shape, dtype) in shapes.items():
+        if name not in o:
+            o[name] = torch.empty(shape, dtype=dtype, device=dev)
+    st, qs = w.struct(), q2.struct()
+    _check(lib().moe_forward_q2(_p(scores), _p(x), k, ctypes.byref(st), ctypes.byref(qs),
+                                _p(o["idx"]), _p(o["w"]), _p(o["counts"]), _p(o["offsets"]),
+                                _p(o["perm"]), _p(o["pos"]), _p(o["y"]), _p(o["y_shared"]),
+                                _p(o["out"]), _p(ws), ws.numel(), _stream(stream)))
+    return dict(idx=o["idx"], w=o["w"], counts=o["counts"], offsets=o["offsets"],
+                perm=o["perm"], pos=o["pos"], y=o["y"], y_shared=o["y_shared"], out=o["out"])
 
 
 def forward_calls(x: torch.Tensor, scores: torch.Tensor, k: int, w: LayerWeights,

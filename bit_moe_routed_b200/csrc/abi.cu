@@ -717,6 +717,64 @@ int moe_forward(const float* scores, const uint16_t* x_bf16, int T, int k,
   return moe_combine(y_routed, y_shared, topk_w, pos, T, k, w->d, out, stream);
 }
 
+int moe_forward_q2(const float* scores, const uint16_t* x_bf16, int k, const moe_weights_t* w,
+                   const moe_q2_experts_t* q2, int32_t* topk_idx, float* topk_w,
+                   int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* pos,
+                   float* y_routed, float* y_shared, float* out, void* ws, size_t ws_bytes,
+                   void* stream) {
+  if (!q2) return fail(MOE_ERR_INVALID_ARG, "NULL 2-bit expert descriptor");
+  FfnCtx c;
+  int rc = ffn_check(1, k, w, ws, ws_bytes, c);
+  if (rc) return rc;
+  if (k > 32) return fail(MOE_ERR_INVALID_ARG, "k=%d outside [1, min(E, 32)]", k);
+  if (w->d % 2048 || w->f % 2048)
+    return fail(MOE_ERR_INVALID_ARG, "d=%d, f=%d must be multiples of 2048", w->d, w->f);
+  if (!q2->gate_codes || !q2->gate_scales || !q2->up_codes || !q2->up_scales ||
+      !q2->down_codes || !q2->down_scales)
+    return fail(MOE_ERR_INVALID_ARG, "NULL 2-bit weight pointer");
+  if (!aligned(q2->gate_codes, 16) || !aligned(q2->up_codes, 16) || !aligned(q2->down_codes, 16) ||
+      !aligned(q2->gate_scales, 16) || !aligned(q2->up_scales, 16) || !aligned(q2->down_scales, 16) ||
+      !aligned(w->gate_scales, 16) || !aligned(w->up_scales, 16) || !aligned(w->down_scales, 16))
+    return fail(MOE_ERR_INVALID_ARG, "weight arrays must be 16-byte aligned");
+  if (!scores || !x_bf16 || !topk_idx || !topk_w || !counts || !offsets || !perm || !pos ||
+      !y_routed || !y_shared || !out)
+    return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(scores, 4) || !aligned(x_bf16, 16) || !aligned(y_routed, 16) ||
+      !aligned(y_shared, 16) || !aligned(out, 16) || !aligned(topk_idx, 4) ||
+      !aligned(topk_w, 4) || !aligned(counts, 4) || !aligned(offsets, 4) || !aligned(perm, 4) ||
+      !aligned(pos, 4))
+    return fail(MOE_ERR_INVALID_ARG, "misaligned pointer");
+  int max_smem = 0, dev = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  const int ctas = c.di.sms < kMaxCtas ? c.di.sms : kMaxCtas;
+  if (!decode_fits(k, w->d, w->f, ctas, true) ||
+      decode_smem_bytes(w->d, w->f, true) > (size_t)max_smem)
+    return fail(MOE_ERR_INVALID_ARG, "shape (k=%d, d=%d, f=%d) does not fit the single-token kernel",
+                k, w->d, w->f);
+  DecodeLaunch a = decode_args(k, w, c);
+  a.forward = true;
+  a.scores = scores;
+  a.x = x_bf16;
+  a.idx = topk_idx;
+  a.w_out = topk_w;
+  a.counts = counts;
+  a.offsets = offsets;
+  a.perm = perm;
+  a.pos = pos;
+  a.y_routed = y_routed;
+  a.y_shared = y_shared;
+  a.out = out;
+  a.q2_gate_codes = q2->gate_codes;
+  a.q2_gate_scales = q2->gate_scales;
+  a.q2_up_codes = q2->up_codes;
+  a.q2_up_scales = q2->up_scales;
+  a.q2_down_codes = q2->down_codes;
+  a.q2_down_scales = q2->down_scales;
+  cudaError_t e = launch_decode(a, static_cast<cudaStream_t>(stream), c.di.sms);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "single-token 2-bit layer launch");
+}
+
 int moe_combine(const float* y_routed, const float* y_shared, const float* topk_w,
                 const int32_t* pos, int T, int k, int d, float* out, void* stream) {
   if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T=%d < 0", T);

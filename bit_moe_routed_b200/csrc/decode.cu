@@ -35,6 +35,18 @@
 // partials are summed in K order after a CTA barrier: results do not depend on timing and
 // equal those of the two-kernel path bit for bit.
 //
+// 2-bit routed experts (the Q2 form, moe_forward_q2): the deployed model of the
+// ai-muninn.com post ("一張 22G 老卡跑 284B") keeps its routed experts at 2 bits per weight
+// (IQ2_XXS, 2.0625 bpw) and the shared expert at higher precision.  In this form the
+// routed experts' units stream a 2-bit codec (four codes per byte, value code - 1.5, one
+// ue8m0 scale per 128 elements) while the shared expert stays FP4.  A 2-bit stage holds
+// the same 4 KB of codes per 16 rows as an FP4 stage but 1024 elements per row; per
+// 128-element chunk a lane turns its 2 x 16 codes of rows g and g + 8 into e4m3 bytes with
+// byte permutes (a 4-entry table indexed by the codes) and runs four mma.sync m16n8k32
+// e4m3 against the token's e4m3 codes, accumulating the chunk's 128 products in the
+// tensor core, then applies the chunk's ue8m0 weight scale (exact) and the token's fp32
+// block scale.  A shared unit counts twice in the work split (twice the stages).
+//
 // Every wait is bounded (%globaltimer): an expired wait records MOE_ERR_TIMEOUT in the
 // status word, the CTA skips its remaining work, lets its issued copies land, still
 // takes part in the grid barrier and returns.
@@ -75,6 +87,7 @@ enum { kModeForward = 0, kModeFfn = 1 };
 
 struct DecodeParams {
   CUtensorMap tm_gc, tm_gs, tm_uc, tm_us, tm_dc, tm_ds;  // codes (3-D) and scales (2-D)
+  CUtensorMap tm_gq, tm_gqs, tm_uq, tm_uqs, tm_dq, tm_dqs;  // 2-bit routed experts (Q2 form)
   const float* scores;        // forward: [E] router scores
   const uint16_t* x;          // [d] bf16 token
   const int32_t* offsets_in;  // ffn: [E+1] from moe_dispatch
@@ -100,16 +113,25 @@ struct DecodeParams {
 };
 
 // Shared memory: rings (codes, then scales), the phase-dependent area (phase 1: token as
-// f16, its scales, stage partials; phase 2: up to three experts' h as f16, scales, stage
-// partials), barriers, routing facts.
+// f16 [and, Q2 form, as e4m3 codes in 8-group order], its scales, stage partials;
+// phase 2: up to three experts' h as f16 [Q2 form: the shared expert's as f16, two
+// routed experts' as e4m3 codes in 8-group order], scales, stage partials), barriers,
+// routing facts.  8-group order: each 8 consecutive codes as the 4 even then the 4 odd
+// elements, the order of the 2-bit decode's e4m3 words.
 struct DcSmem {
   int d, f;
+  bool q2;
   static constexpr int kOffScales = kDcWarps * kDcStages * kDcCodeBytes;
   static constexpr int kOffArea = kOffScales + kDcWarps * kDcStages * kDcScaleBytes;
-  __host__ __device__ int p1_bs() const { return kOffArea + 2 * d; }
+  __host__ __device__ int p1_q8() const { return kOffArea + 2 * d; }  // Q2 form
+  __host__ __device__ int p1_bs() const { return kOffArea + (q2 ? 3 : 2) * d; }
   __host__ __device__ int p1_part() const { return p1_bs() + d / 32; }
   __host__ __device__ int p1_end() const { return p1_part() + kDcMaxUnits * (d / 512) * 64; }
-  __host__ __device__ int p2_bs() const { return kOffArea + kDcP2Slots * 2 * f; }
+  // phase 2: byte offset of local slot ls's activations
+  __host__ __device__ int p2_act(int ls) const {
+    return kOffArea + (q2 && ls > 0 ? 2 * f + (ls - 1) * f : ls * 2 * f);
+  }
+  __host__ __device__ int p2_bs() const { return kOffArea + (q2 ? 4 : 2 * kDcP2Slots) * f; }
   __host__ __device__ int p2_part() const { return p2_bs() + kDcP2Slots * (f / 32); }
   __host__ __device__ int p2_end() const { return p2_part() + kDcMaxUnits * (f / 512) * 64; }
   __host__ __device__ int bars() const {
@@ -170,22 +192,24 @@ __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long
   return v;
 }
 
-// One CTA's share of a phase: M = (routed experts + 1) * upe units in all, CTA b taking
-// [b*M/G, (b+1)*M/G) of them; its first ns are the shared expert's units [s_lo, s_lo+ns)
-// (s_lo = b*upe/G, a share that does not depend on the routing), the rest the routed units
-// [r_lo, r_lo+nr) of the list that runs over the active routed experts in slot order.
+// One CTA's share of a phase.  A shared unit weighs wsh (1; 2 in the Q2 form, where it
+// has twice the stages of a routed unit), a routed unit 1: M = (n_routed + wsh) * upe in
+// all, CTA b taking the weight range [b*M/G, (b+1)*M/G).  Its first ns units are the
+// shared expert's [s_lo, s_lo+ns) (s_lo = b*upe/G, a share that does not depend on the
+// routing), the rest the routed units [r_lo, r_lo+nr) of the list that runs over the
+// active routed experts in slot order (r_lo = b*M/G - wsh*s_lo).
 struct Range {
   int s_lo, ns, r_lo, nr, upe;
-  __device__ Range(int upe_, int n_routed, int G, int b) {
+  __host__ __device__ Range(int upe_, int n_routed, int G, int b, int wsh) {
     upe = upe_;
     s_lo = (int)((long long)b * upe / G);
     ns = (int)((long long)(b + 1) * upe / G) - s_lo;
-    const long long M = (long long)(n_routed + 1) * upe;
+    const long long M = (long long)(n_routed + wsh) * upe;
     const long long t_lo = b * M / G, t_hi = (b + 1) * M / G;
-    r_lo = (int)(t_lo - s_lo);
-    nr = (int)(t_hi - t_lo) - ns;
+    r_lo = (int)(t_lo - (long long)wsh * s_lo);
+    nr = (int)(t_hi - t_lo) - wsh * ns;
   }
-  __device__ int units() const { return ns + nr; }
+  __host__ __device__ int units() const { return ns + nr; }
 };
 
 // The bounded grid barrier (see g_grid_bar); false if the wait ran out.  ok_s: a word of
@@ -219,17 +243,60 @@ __device__ bool grid_barrier(long long limit, int* status, volatile int* ok_s) {
   return *ok_s != 0;
 }
 
-template <int MODE, int PL>
+// Unit ul / chunk c of task `task` in a CTA range whose first ns units have S stages each
+// (the shared expert's) and the rest Sq (the routed experts'); true for a routed unit.
+__device__ __forceinline__ bool locate(int task, int ns, int S, int Sq, int& ul, int& c) {
+  if (task < ns * S) {
+    ul = task / S;
+    c = task % S;
+    return false;
+  }
+  const int r = task - ns * S;
+  ul = ns + r / Sq;
+  c = r % Sq;
+  return true;
+}
+
+// e4m3 bytes of the 2-bit values -1.5, -0.5, 0.5, 1.5 (byte i = code i), the table of the
+// byte-permute decode
+constexpr uint32_t kQ2Lut = 0x3C30B0BCu;
+
+// One 128-element chunk of weight rows g and g + 8 (2-bit codes) against the token: lane
+// (g, t) holds code bytes 8t..8t+7 of the chunk of both rows (wa, wb: codes 32t..32t+31,
+// code i of a word in bits 2i..2i+1) and the token's e4m3 codes of elements 32t..32t+31 in
+// 8-group order (x01: elements 32t..32t+15, x23: 32t+16..32t+31).  Masking a word with
+// 0x33333333 leaves its even codes in the low 2 bits of its nibbles, the word shifted right
+// by 2 its odd codes; a byte permute indexed by 4 such nibbles looks up 4 e4m3 bytes.  MMA
+// m takes elements 32t + 8m .. 32t + 8m + 7 of every lane t, the even ones in k-slots
+// 4t..4t+3 and the odd ones in 16+4t..16+4t+3 of both operands, so the four MMAs sum each
+// of the 128 products once (fp32 accumulation in the tensor core).
+__device__ __forceinline__ void q2_chunk_dot(uint2 wa, uint2 wb, uint4 x01, uint4 x23,
+                                             float (&c)[4]) {
+  const uint32_t ea0 = wa.x & 0x33333333u, oa0 = (wa.x >> 2) & 0x33333333u;
+  const uint32_t ea1 = wa.y & 0x33333333u, oa1 = (wa.y >> 2) & 0x33333333u;
+  const uint32_t eb0 = wb.x & 0x33333333u, ob0 = (wb.x >> 2) & 0x33333333u;
+  const uint32_t eb1 = wb.y & 0x33333333u, ob1 = (wb.y >> 2) & 0x33333333u;
+  auto lut = [](uint32_t sel) { return ptx::prmt(kQ2Lut, 0u, sel); };
+  ptx::mma_m16n8k32_e4m3_zero(c, lut(ea0), lut(eb0), lut(oa0), lut(ob0), x01.x, x01.y);
+  ptx::mma_m16n8k32_e4m3(c, lut(ea0 >> 16), lut(eb0 >> 16), lut(oa0 >> 16), lut(ob0 >> 16),
+                         x01.z, x01.w);
+  ptx::mma_m16n8k32_e4m3(c, lut(ea1), lut(eb1), lut(oa1), lut(ob1), x23.x, x23.y);
+  ptx::mma_m16n8k32_e4m3(c, lut(ea1 >> 16), lut(eb1 >> 16), lut(oa1 >> 16), lut(ob1 >> 16),
+                         x23.z, x23.w);
+}
+
+template <int MODE, int PL, bool RQ>
 __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (ptx::smem_u32(smem_raw) & 1023)) & 1023);
-  const DcSmem L{p.d, p.f};
+  const DcSmem L{p.d, p.f, RQ};
   const int d = p.d, f = p.f, E = p.E, k = p.k;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int G = gridDim.x, b = blockIdx.x;
 
   uint16_t* bx = reinterpret_cast<uint16_t*>(smem + DcSmem::kOffArea);  // f16 activations
+  uint8_t* bxq = smem + L.p1_q8();  // Q2 form: the token's e4m3 codes in 8-group order
   float* bs1 = reinterpret_cast<float*>(smem + L.p1_bs());
   float* part1 = reinterpret_cast<float*>(smem + L.p1_part());
   float* bs2 = reinterpret_cast<float*>(smem + L.p2_bs());
@@ -259,6 +326,14 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
     ptx::prefetch_tmap(&p.tm_us);
     ptx::prefetch_tmap(&p.tm_dc);
     ptx::prefetch_tmap(&p.tm_ds);
+    if (RQ) {
+      ptx::prefetch_tmap(&p.tm_gq);
+      ptx::prefetch_tmap(&p.tm_gqs);
+      ptx::prefetch_tmap(&p.tm_uq);
+      ptx::prefetch_tmap(&p.tm_uqs);
+      ptx::prefetch_tmap(&p.tm_dq);
+      ptx::prefetch_tmap(&p.tm_dqs);
+    }
     *abort_flag = 0;
     ptx::mbar_init(stall_bar, 1);  // never arrived on: only the test stall waits on it
   }
@@ -269,13 +344,17 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
     for (int i = threadIdx.x; i < d / 16; i += kDcThreads) p.done2[i] = 0;  // grid barrier)
   __syncthreads();
 
+  // stages per unit: shared (FP4, 512-element stages) and routed (FP4, or 2-bit with
+  // 1024-element stages in the Q2 form)
   const int S1 = d / 512, S2 = f / 512;
+  const int S1q = RQ ? d / 1024 : S1, S2q = RQ ? f / 1024 : S2;
+  const int wsh = RQ ? 2 : 1;
   const int upe1 = f / 8, upe2 = d / 16;
   const uint64_t pol = ptx::make_policy_evict_first();
 
   // n_act routed experts (known after routing); ranges and task counts follow from it
   int n_act = MODE == kModeForward ? k : 0;
-  Range r1(upe1, n_act, G, b), r2(upe2, n_act, G, b);
+  Range r1(upe1, n_act, G, b, wsh), r2(upe2, n_act, G, b, wsh);
   int q1 = 0, q2 = 0;
 
   // copies of this warp's q-th stage (phase 1 while q < q1), issued by lane 0
@@ -284,10 +363,10 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
     const uint32_t dc = ptx::smem_u32(codes_at(st)), ds = ptx::smem_u32(scales_at(st));
     ptx::mbar_arrive_expect_tx(full(st), kDcStageBytes);
     if (q < q1) {
-      const int task = warp + q * kDcWarps;
-      const int ul = task / S1, c = task % S1;
+      int ul, c;
+      const bool routed = locate(warp + q * kDcWarps, r1.ns, S1, S1q, ul, c);
       int e, uin;
-      if (ul < r1.ns) {
+      if (!routed) {
         e = E;
         uin = r1.s_lo + ul;
       } else {
@@ -295,16 +374,26 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
         e = slot_e[ru / upe1];
         uin = ru % upe1;
       }
-      const int row = e * f + uin * 8;
-      ptx::tma_load_3d_hint(dc, &p.tm_gc, 0, row, 2 * c, full(st), pol);
-      ptx::tma_load_3d_hint(dc + 2048, &p.tm_uc, 0, row, 2 * c, full(st), pol);
-      ptx::tma_load_2d_hint(ds, &p.tm_gs, c * 16, row, full(st), pol);
-      ptx::tma_load_2d_hint(ds + 128, &p.tm_us, c * 16, row, full(st), pol);
+      if (RQ && routed) {
+        // 2-bit stage: 2 x 128 code bytes (1024 elements) per row; the 16-byte scale box
+        // covers 2048 elements, of which this stage uses bytes 8(c % 2)..+8
+        const int row = e * f + uin * 8;
+        ptx::tma_load_3d_hint(dc, &p.tm_gq, 0, row, 2 * c, full(st), pol);
+        ptx::tma_load_3d_hint(dc + 2048, &p.tm_uq, 0, row, 2 * c, full(st), pol);
+        ptx::tma_load_2d_hint(ds, &p.tm_gqs, (c >> 1) * 16, row, full(st), pol);
+        ptx::tma_load_2d_hint(ds + 128, &p.tm_uqs, (c >> 1) * 16, row, full(st), pol);
+      } else {
+        const int row = e * f + uin * 8;
+        ptx::tma_load_3d_hint(dc, &p.tm_gc, 0, row, 2 * c, full(st), pol);
+        ptx::tma_load_3d_hint(dc + 2048, &p.tm_uc, 0, row, 2 * c, full(st), pol);
+        ptx::tma_load_2d_hint(ds, &p.tm_gs, c * 16, row, full(st), pol);
+        ptx::tma_load_2d_hint(ds + 128, &p.tm_us, c * 16, row, full(st), pol);
+      }
     } else {
-      const int task = warp + (q - q1) * kDcWarps;
-      const int ul = task / S2, c = task % S2;
+      int ul, c;
+      const bool routed = locate(warp + (q - q1) * kDcWarps, r2.ns, S2, S2q, ul, c);
       int e, uin;
-      if (ul < r2.ns) {
+      if (!routed) {
         e = E;
         uin = r2.s_lo + ul;
       } else {
@@ -313,8 +402,13 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
         uin = ru % upe2;
       }
       const int row = e * d + uin * 16;
-      ptx::tma_load_3d_hint(dc, &p.tm_dc, 0, row, 2 * c, full(st), pol);
-      ptx::tma_load_2d_hint(ds, &p.tm_ds, c * 16, row, full(st), pol);
+      if (RQ && routed) {
+        ptx::tma_load_3d_hint(dc, &p.tm_dq, 0, row, 2 * c, full(st), pol);
+        ptx::tma_load_2d_hint(ds, &p.tm_dqs, (c >> 1) * 16, row, full(st), pol);
+      } else {
+        ptx::tma_load_3d_hint(dc, &p.tm_dc, 0, row, 2 * c, full(st), pol);
+        ptx::tma_load_2d_hint(ds, &p.tm_ds, c * 16, row, full(st), pol);
+      }
     }
   };
 
@@ -458,6 +552,10 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
         dst[0] = make_uint4(hx[0], hx[1], hx[2], hx[3]);
         dst[1] = make_uint4(hx[4], hx[5], hx[6], hx[7]);
         if ((tid & 7) == 0) bs1[c0 / 128] = sc;
+        if (RQ)  // the 16 codes in 8-group order: even then odd elements of each 8
+          *reinterpret_cast<uint4*>(bxq + c0) =
+              make_uint4(ptx::prmt(packed[0], packed[1], 0x6420u), ptx::prmt(packed[0], packed[1], 0x7531u),
+                         ptx::prmt(packed[2], packed[3], 0x6420u), ptx::prmt(packed[2], packed[3], 0x7531u));
         if (b == 0) {
           *reinterpret_cast<uint4*>(p.qx + c0) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
           if ((tid & 7) == 0) p.sx[c0 / 128] = sc;
@@ -468,13 +566,14 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
   __syncthreads();
 
   n_act = *n_active;
-  r1 = Range(upe1, n_act, G, b);
-  r2 = Range(upe2, n_act, G, b);
-  const int nt1 = r1.units() * S1, nt2 = r2.units() * S2;
+  r1 = Range(upe1, n_act, G, b, wsh);
+  r2 = Range(upe2, n_act, G, b, wsh);
+  const int nt1 = r1.ns * S1 + r1.nr * S1q, nt2 = r2.ns * S2 + r2.nr * S2q;
   q1 = nt1 > warp ? (nt1 - warp + kDcWarps - 1) / kDcWarps : 0;
   q2 = nt2 > warp ? (nt2 - warp + kDcWarps - 1) / kDcWarps : 0;
   // the host keeps every range within these limits; a plan that breaks them stops here
-  if (r1.units() > kDcMaxUnits || r2.units() > kDcMaxUnits || r2.nr > r2.upe + 1) {
+  if (r1.nr < 0 || r2.nr < 0 || r1.units() > kDcMaxUnits || r2.units() > kDcMaxUnits ||
+      r2.nr > r2.upe + 1) {
     if (threadIdx.x == 0) atomicOr(p.status, kStatusBadIndex);
     *abort_flag = 1;
   }
@@ -534,7 +633,8 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
       for (int i = threadIdx.x; i < r1.units() * 8; i += kDcThreads) {
         const int ul = i >> 3, r = i & 7;
         float gg = 0.f, uu = 0.f;
-        for (int c = 0; c < S1; ++c) {
+        const int Su = ul < r1.ns ? S1 : S1q;
+        for (int c = 0; c < Su; ++c) {
           gg += part1[(ul * S1 + c) * kDcRows + r];
           uu += part1[(ul * S1 + c) * kDcRows + 8 + r];
         }
@@ -583,14 +683,22 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
           const float sc = amax == 0.f ? 1.0f : __fdiv_rn(amax, 448.0f);
           const uint16_t q01 = ptx::cvt_e4m3x2(__fdiv_rn(h.x, sc), __fdiv_rn(h.y, sc));
           const uint16_t q23 = ptx::cvt_e4m3x2(__fdiv_rn(h.z, sc), __fdiv_rn(h.w, sc));
-          uint32_t* dst = reinterpret_cast<uint32_t*>(bx + (size_t)ls * f + 128 * j + 4 * lane);
-          dst[0] = ptx::cvt_e4m3x2_f16x2(q01);
-          dst[1] = ptx::cvt_e4m3x2_f16x2(q23);
+          const uint32_t qw = (uint32_t)q01 | ((uint32_t)q23 << 16);
+          if (RQ && ls > 0) {
+            // a 2-bit expert's h: codes in 8-group order; lanes 2m and 2m + 1 hold elements
+            // 8m..8m+7, the even lane stores the even ones, the odd lane the odd ones
+            const uint32_t qo = __shfl_xor_sync(0xffffffffu, qw, 1);
+            *reinterpret_cast<uint32_t*>(smem + L.p2_act(ls) + 128 * j + 4 * lane) =
+                (lane & 1) ? ptx::prmt(qo, qw, 0x7531u) : ptx::prmt(qw, qo, 0x6420u);
+          } else {
+            uint32_t* dst = reinterpret_cast<uint32_t*>(smem + L.p2_act(ls) + 2 * (128 * j + 4 * lane));
+            dst[0] = ptx::cvt_e4m3x2_f16x2(q01);
+            dst[1] = ptx::cvt_e4m3x2_f16x2(q23);
+          }
           if (lane == 0) bs2[ls * nb + j] = sc;
           // the CTA holding the expert's first unit also stores its codes and scales
           const bool owner = ls == 0 ? r2.s_lo == 0 : slot * upe2 >= r2.r_lo;
           if (owner) {
-            const uint32_t qw = (uint32_t)q01 | ((uint32_t)q23 << 16);
             const int rows = ls == 0 ? 1 : slot_n[slot];
             const int row0 = ls == 0 ? k : slot_row[slot];
             for (int rr = 0; rr < rows; ++rr) {
@@ -619,17 +727,50 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
       const uint8_t* cst = codes_at(st);
       const uint8_t* sst = scales_at(st);
       const int task = warp + (PH == 1 ? q : q - q1) * kDcWarps;
-      const int S = PH == 1 ? S1 : S2;
-      const int ul = task / S, c = task % S;
+      int ul, c;
+      const bool routed = PH == 1 ? locate(task, r1.ns, S1, S1q, ul, c)
+                                  : locate(task, r2.ns, S2, S2q, ul, c);
       const uint16_t* xb = bx;
+      const uint8_t* xq = bxq;
       const float* sxb = bs1;
       if (PH == 2) {
         int e, uin, ls, slot;
         p2_local(ul, e, uin, ls, slot);
-        xb = bx + (size_t)ls * f;
+        xb = reinterpret_cast<const uint16_t*>(smem + L.p2_act(ls));
+        xq = smem + L.p2_act(ls);
         sxb = bs2 + ls * (f / 128);
       }
       float acc0 = 0.f, acc1 = 0.f;  // rows g and g+8 of the stage, column 0 (the token)
+      if (RQ && routed) {
+        // 2-bit stage: 16 rows x 1024 elements, 8 chunks of 128; this stage's 8 scale bytes
+        // of each row are bytes 8(c % 2)..8(c % 2)+7 of its 16-byte scale box row
+        const uint2 sa = *reinterpret_cast<const uint2*>(sst + r0 * 16 + 8 * (c & 1));
+        const uint2 sb = *reinterpret_cast<const uint2*>(sst + rr1 * 16 + 8 * (c & 1));
+#pragma unroll 2
+        for (int jj = 0; jj < 8; ++jj) {
+          const int j = 8 * c + jj;  // the token's 128-block
+          // the lane's 8 code bytes of chunk jj (16-byte chunks 2 (jj % 4), 2 (jj % 4) + 1
+          // of the rows' 128-byte piece jj / 4): bytes 8t..8t+7, in 16-byte chunk
+          // 2 (jj % 4) + t / 2 (swizzled with the row index mod 8) at byte 8 (t % 2)
+          const uint32_t piece = (uint32_t)(jj >> 2);
+          const uint32_t ba = PH == 1 ? piece * 1024u : piece * 2048u;
+          const uint32_t bbx = PH == 1 ? 2048u + piece * 1024u : piece * 2048u + 1024u;
+          const uint8_t* cp = cst + g * 128 + ((((2 * (jj & 3)) + (t >> 1)) ^ g) << 4) + 8 * (t & 1);
+          const uint2 wa = *reinterpret_cast<const uint2*>(cp + ba);
+          const uint2 wb = *reinterpret_cast<const uint2*>(cp + bbx);
+          const uint4 x01 = *reinterpret_cast<const uint4*>(xq + 128 * j + 32 * t);
+          const uint4 x23 = *reinterpret_cast<const uint4*>(xq + 128 * j + 32 * t + 16);
+          float cq[4];
+          q2_chunk_dot(wa, wb, x01, x23, cq);
+          const uint32_t ea = ((jj < 4 ? sa.x : sa.y) >> (8 * (jj & 3))) & 0xFFu;
+          const uint32_t eb = ((jj < 4 ? sb.x : sb.y) >> (8 * (jj & 3))) & 0xFFu;
+          const float fa = __uint_as_float(max(ea << 23, 0x00400000u));  // 2^(e-127), exact
+          const float fb = __uint_as_float(max(eb << 23, 0x00400000u));
+          const float sxj = sxb[j];
+          acc0 = fmaf(sxj, fa * cq[0], acc0);
+          acc1 = fmaf(sxj, fb * cq[2], acc1);
+        }
+      } else {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int j = 4 * c + i;
@@ -660,6 +801,7 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
         const float sxj = sxb[j];
         acc0 = fmaf(sxj, pa, acc0);
         acc1 = fmaf(sxj, pb, acc1);
+      }
       }
       __syncwarp();  // every lane is done with the stage: it may be refilled
       if (issued < qt) {
@@ -693,7 +835,8 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
   for (int i = threadIdx.x; i < r2.units() * kDcRows; i += kDcThreads) {
     const int ul = i >> 4, r = i & 15;
     float y = 0.f;
-    for (int c = 0; c < S2; ++c) y += part2[(ul * S2 + c) * kDcRows + r];
+    const int Su = ul < r2.ns ? S2 : S2q;
+    for (int c = 0; c < Su; ++c) y += part2[(ul * S2 + c) * kDcRows + r];
     int e, uin, ls, slot;
     p2_local(ul, e, uin, ls, slot);
     const size_t m = (size_t)uin * 16 + r;
@@ -727,11 +870,11 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
 }
 
 
-template <int MODE, int PL>
+template <int MODE, int PL, bool RQ>
 cudaError_t launch_one(const DecodeParams& prm, cudaStream_t s, int grid) {
-  const DcSmem L{prm.d, prm.f};
+  const DcSmem L{prm.d, prm.f, RQ};
   const size_t smem = (size_t)L.bytes();
-  auto kern = decode_kernel<MODE, PL>;
+  auto kern = decode_kernel<MODE, PL, RQ>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -749,16 +892,23 @@ cudaError_t launch_one(const DecodeParams& prm, cudaStream_t s, int grid) {
 
 }  // namespace
 
-size_t decode_smem_bytes(int d, int f) { return (size_t)DcSmem{d, f}.bytes(); }
+size_t decode_smem_bytes(int d, int f, bool q2) { return (size_t)DcSmem{d, f, q2}.bytes(); }
 
-bool decode_fits(int k, int d, int f, int ctas) {
+bool decode_fits(int k, int d, int f, int ctas, bool q2) {
   if (k < 1 || k > 32 || d % 512 || f % 512 || ctas < 1) return false;
-  const long long upe1 = f / 8, upe2 = d / 16;
-  // the most units a CTA can get in either phase (fewer active experts give fewer)
-  auto most = [&](long long upe) { return ((long long)(k + 1) * upe + ctas - 1) / ctas; };
-  if (most(upe1) > kDcMaxUnits || most(upe2) > kDcMaxUnits) return false;
-  // a CTA's phase-2 routed range spans at most two experts
-  if (most(upe2) > upe2 + 1) return false;
+  // 2-bit stages hold 1024 elements and read 16-byte scale boxes (2048 elements)
+  if (q2 && (d % 2048 || f % 2048)) return false;
+  const int upe1 = f / 8, upe2 = d / 16, wsh = q2 ? 2 : 1;
+  // every CTA's ranges, for every count of active experts the kernel can meet: at most
+  // kDcMaxUnits units per phase, a routed share that is not negative, and a phase-2 routed
+  // range over at most two experts
+  for (int n = 1; n <= k; ++n)
+    for (int b = 0; b < ctas; ++b) {
+      const Range r1(upe1, n, ctas, b, wsh), r2(upe2, n, ctas, b, wsh);
+      if (r1.nr < 0 || r2.nr < 0 || r1.units() > kDcMaxUnits || r2.units() > kDcMaxUnits)
+        return false;
+      if (r2.nr > upe2 + 1) return false;
+    }
   return true;
 }
 
@@ -773,6 +923,17 @@ cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t s, int num_sms) {
       !make_code_map(&p.tm_dc, a.down_codes, a.f / 2, rows2, 16) ||
       !make_byte_map(&p.tm_ds, a.down_scales, a.f / 32, rows2, 16, 16))
     return cudaErrorInvalidValue;
+  const bool q2 = a.q2_gate_codes != nullptr;
+  if (q2) {  // the E routed experts in the 2-bit codec: codes [rows][K/4], scales [rows][K/128]
+    const long long q1 = (long long)a.E * a.f, q2r = (long long)a.E * a.d;
+    if (!make_code_map(&p.tm_gq, a.q2_gate_codes, a.d / 4, q1, 8) ||
+        !make_byte_map(&p.tm_gqs, a.q2_gate_scales, a.d / 128, q1, 16, 8) ||
+        !make_code_map(&p.tm_uq, a.q2_up_codes, a.d / 4, q1, 8) ||
+        !make_byte_map(&p.tm_uqs, a.q2_up_scales, a.d / 128, q1, 16, 8) ||
+        !make_code_map(&p.tm_dq, a.q2_down_codes, a.f / 4, q2r, 16) ||
+        !make_byte_map(&p.tm_dqs, a.q2_down_scales, a.f / 128, q2r, 16, 16))
+      return cudaErrorInvalidValue;
+  }
   p.scores = a.scores;
   p.x = a.x;
   p.offsets_in = a.offsets_in;
@@ -799,11 +960,16 @@ cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t s, int num_sms) {
   p.status = a.status;
   p.stall = a.stall;
   const int grid = num_sms < kMaxCtas ? num_sms : kMaxCtas;
-  if (a.forward) {
-    if (a.E <= 256) return launch_one<kModeForward, 8>(p, s, grid);
-    return launch_one<kModeForward, 32>(p, s, grid);
+  if (q2) {  // forward only
+    if (!a.forward) return cudaErrorInvalidValue;
+    if (a.E <= 256) return launch_one<kModeForward, 8, true>(p, s, grid);
+    return launch_one<kModeForward, 32, true>(p, s, grid);
   }
-  return launch_one<kModeFfn, 8>(p, s, grid);
+  if (a.forward) {
+    if (a.E <= 256) return launch_one<kModeForward, 8, false>(p, s, grid);
+    return launch_one<kModeForward, 32, false>(p, s, grid);
+  }
+  return launch_one<kModeFfn, 8, false>(p, s, grid);
 }
 
 cudaError_t reset_grid_barrier() {

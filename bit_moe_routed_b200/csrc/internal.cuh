@@ -183,11 +183,20 @@ struct DecodeLaunch {
   long long wait_ns;
   int* status;
   int stall;
+  // Q2 form (forward only): the E routed experts in the 2-bit codec; NULL otherwise, and
+  // then the FP4 arrays hold all E + 1 experts (in the Q2 form only the shared one, E)
+  const uint8_t* q2_gate_codes = nullptr;
+  const uint8_t* q2_gate_scales = nullptr;
+  const uint8_t* q2_up_codes = nullptr;
+  const uint8_t* q2_up_scales = nullptr;
+  const uint8_t* q2_down_codes = nullptr;
+  const uint8_t* q2_down_scales = nullptr;
 };
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t s, int num_sms);
-size_t decode_smem_bytes(int d, int f);
+size_t decode_smem_bytes(int d, int f, bool q2 = false);
 // whether the single-token kernel's per-CTA limits hold for (k, d, f) on `ctas` CTAs
-bool decode_fits(int k, int d, int f, int ctas);
+// (q2: with 2-bit routed experts)
+bool decode_fits(int k, int d, int f, int ctas, bool q2 = false);
 // clears the single-token kernel's grid barrier (after a reported timeout)
 cudaError_t reset_grid_barrier();
 

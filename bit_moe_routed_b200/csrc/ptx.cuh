@@ -252,6 +252,35 @@ __device__ __forceinline__ void mma_m16n8k16_f16(float* c, uint32_t a0, uint32_t
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
+// warp-level D(16x8, fp32) = A(16x32, e4m3, row) x B(32x8, e4m3, col), from a zero
+// accumulator; lane (g, t): a0 / a1 rows g / g+8 at k 4t..4t+3, a2 / a3 at k 16+4t..;
+// b0 k 4t..4t+3, b1 k 16+4t.., column g
+__device__ __forceinline__ void mma_m16n8k32_e4m3_zero(float* d, uint32_t a0, uint32_t a1,
+                                                       uint32_t a2, uint32_t a3, uint32_t b0,
+                                                       uint32_t b1) {
+  const float z = 0.0f;
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0, %1, %2, %3},"
+      " {%4, %5, %6, %7}, {%8, %9}, {%10, %10, %10, %10};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(z));
+}
+// warp-level D(16x8, fp32) += A(16x32, e4m3, row) x B(32x8, e4m3, col)
+__device__ __forceinline__ void mma_m16n8k32_e4m3(float* c, uint32_t a0, uint32_t a1, uint32_t a2,
+                                                  uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0, %1, %2, %3},"
+      " {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// byte permute: result byte i = byte sel[4i+3:4i] of {b, a} (a = bytes 0-3); only the low
+// 16 bits of sel are read
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
 
 }  // namespace ptx
 }  // namespace bitmoe

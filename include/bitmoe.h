@@ -184,6 +184,40 @@ int moe_forward(const float* scores, const uint16_t* x_bf16, int T, int k,
                 int32_t* offsets, int32_t* perm, int32_t* pos, float* y_routed, float* y_shared,
                 float* out, void* ws, size_t ws_bytes, void* stream);
 
+/* 2-bit routed experts (NEXT-2): the ai-muninn.com post "一張 22G 老卡跑 284B" runs the
+ * model with its routed experts at 2 bits per weight (IQ2_XXS, 2.0625 bpw) and the
+ * always-resident weights, the shared expert among them, at higher precision (the
+ * smzdm.com post's "2-bit routed experts only" of the ds4 engine is the same split).  The
+ * pages fix the bit rate, not the code book; this library's 2-bit codec is: four 2-bit
+ * codes per byte (element i of a byte in bits 2i..2i+1), value code - 1.5 (-1.5, -0.5,
+ * 0.5, 1.5), times one ue8m0 scale byte per 128 consecutive elements along the reduction
+ * axis (2 + 8/128 = 2.0625 bits per weight).  The E routed experts, contiguous per matrix:
+ *   gate_codes, up_codes  [E][f][d/4]   gate_scales, up_scales  [E][f][d/128]
+ *   down_codes            [E][d][f/4]   down_scales             [E][d][f/128]
+ * All six arrays 16-byte aligned. */
+typedef struct {
+  const uint8_t* gate_codes;
+  const uint8_t* gate_scales;
+  const uint8_t* up_codes;
+  const uint8_t* up_scales;
+  const uint8_t* down_codes;
+  const uint8_t* down_scales;
+} moe_q2_experts_t;
+
+/* moe_forward for one token (T = 1) with 2-bit routed experts: the routed experts come
+ * from `q2` (the same E, d, f as `w`), the shared expert from `w` (FP4, index E; w's
+ * routed experts are not read).  Outputs, workspace and rules as for moe_forward at T = 1,
+ * in ONE cooperative kernel: the routed experts' units stream the 2-bit codes (decoded to
+ * e4m3 in registers, mma.sync e4m3 x e4m3 with fp32 sums per 128-element chunk, then the
+ * chunk's weight scale and the token's activation scale), the shared expert's the FP4
+ * codes.  d and f multiples of 2048; k <= 32; the shape must fit the single-token kernel
+ * (MOE_ERR_INVALID_ARG otherwise). */
+int moe_forward_q2(const float* scores, const uint16_t* x_bf16, int k, const moe_weights_t* w,
+                   const moe_q2_experts_t* q2, int32_t* topk_idx, float* topk_w,
+                   int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* pos,
+                   float* y_routed, float* y_shared, float* out, void* ws, size_t ws_bytes,
+                   void* stream);
+
 /* Step 8 — combine: out[t][m] = y_shared[t][m] + sum_{j<k} topk_w[t][j] *
  * y_routed[pos[t*k+j]][m], summed in fixed j order in fp32.
  *   y_routed [T*k][d], y_shared [T][d], topk_w [T][k], pos [T*k], out [T][d] fp32.

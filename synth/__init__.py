@@ -49,6 +49,7 @@ class Workload:
     layers: int = 1
     config_id: int = 0
     draw: int = 0
+    routed_codec: str = "fp4"  # "fp4", or "q2": routed experts in the 2-bit codec
 
     def seed(self, layer: int = 0) -> int:
         return 1000 * self.config_id + 10 * self.draw + layer
@@ -63,6 +64,10 @@ WORKLOADS = {
                                       f=2048, config_id=3, draw=0),
     "prefill_t4096_zipf": Workload("prefill_t4096_zipf", T=4096, E=256, k=6, d=4096, f=2048,
                                    routing="zipf", zipf_s=1.2, config_id=3, draw=1),
+    # decode_t1's token, scores and shared expert with the routed experts in the 2-bit
+    # codec (the deployed model of the ai-muninn.com post: IQ2_XXS routed experts)
+    "decode_t1_q2": Workload("decode_t1_q2", T=1, E=256, k=6, d=4096, f=2048, config_id=1,
+                             routed_codec="q2"),
     "layers43_t1": Workload("layers43_t1", T=1, E=256, k=6, d=4096, f=2048, routing="zipf",
                             zipf_s=1.0, layers=43, config_id=4, draw=0),
     "layers43_t32": Workload("layers43_t32", T=32, E=256, k=6, d=4096, f=2048,

@@ -117,6 +117,36 @@ def host_experts(seed, layer, d, f, experts):
     return {int(e): synth.host_expert(seed, layer, int(e), d, f) for e in experts}
 
 
+def host_experts_q2(seed, layer, d, f, experts):
+    """Routed experts in the 2-bit codec (host copies of synth's bytes), tagged for the
+    oracle."""
+    out = {}
+    for e in experts:
+        he = synth.host_expert_q2(seed, layer, int(e), d, f)
+        ns = type("Q2Expert", (), {})()
+        ns.__dict__.update(he.__dict__)
+        ns.codec = oracle.Q2
+        out[int(e)] = ns
+    return out
+
+
+def _gemv(codes, scales, x, codec):
+    return oracle.q2_gemv(codes, scales, x) if codec == oracle.Q2 else \
+        oracle.fp4_gemv(codes, scales, x)
+
+
+def _abs_codes(codes, codec):
+    """Codes of |W|: FP4 clears the sign bits; 2-bit codes c < 2 (the negative values)
+    become 3 - c."""
+    if codec != oracle.Q2:
+        return codes & 0x77
+    out = codes.copy()
+    for i in range(4):
+        neg = ((codes >> (2 * i + 1)) & 1) == 0
+        out = np.where(neg, out ^ np.uint8(3 << (2 * i)), out).astype(np.uint8)
+    return out
+
+
 def dequant_act(q: np.ndarray, s: np.ndarray) -> np.ndarray:
     """x^ = e4m3(q) * s per 128-block, in double."""
     return e4m3_table()[q] * np.repeat(np.asarray(s, np.float64), 128, axis=-1)
@@ -131,12 +161,13 @@ def h_error_bound(ex, d: int, xhat: np.ndarray, rows):
         z = np.zeros(0)
         return z, z, z, z
     xabs = np.abs(xhat)
+    codec = getattr(ex, "codec", oracle.FP4)
     gc, gs = ex.gate_codes[rows], ex.gate_scales[rows]
     uc, us = ex.up_codes[rows], ex.up_scales[rows]
-    g = oracle.fp4_gemv(gc, gs, xhat)
-    u = oracle.fp4_gemv(uc, us, xhat)
-    ag = oracle.fp4_gemv(gc & 0x77, gs, xabs)   # sum |W x| (sign bits cleared)
-    au = oracle.fp4_gemv(uc & 0x77, us, xabs)
+    g = _gemv(gc, gs, xhat, codec)
+    u = _gemv(uc, us, xhat, codec)
+    ag = _gemv(_abs_codes(gc, codec), gs, xabs, codec)   # sum |W x|
+    au = _gemv(_abs_codes(uc, codec), us, xabs, codec)
     D = acc_depth(d)
     dg, du = D * U23 * ag, D * U23 * au
     sig = 1.0 / (1.0 + np.exp(-g))
@@ -148,10 +179,11 @@ def h_error_bound(ex, d: int, xhat: np.ndarray, rows):
     return B, g, u, h
 
 
-def y_error_bound(down_codes, down_scales, hhat: np.ndarray, K: int) -> np.ndarray:
+def y_error_bound(down_codes, down_scales, hhat: np.ndarray, K: int,
+                  codec=oracle.FP4) -> np.ndarray:
     """A-priori bound on |y_gpu - W_down h^| for an fp32 dot product over K = f."""
-    return 1.01 * acc_depth(K) * U23 * oracle.fp4_gemv(down_codes & 0x77, down_scales,
-                                                       np.abs(hhat))
+    return 1.01 * acc_depth(K) * U23 * _gemv(_abs_codes(down_codes, codec), down_scales,
+                                             np.abs(hhat), codec)
 
 
 class HStats:
@@ -258,6 +290,21 @@ def gpu_layer(x, scores, k, weights, ws=None, keep_device=False, calls=False):
     return {kk: v.cpu() for kk, v in r.items()}
 
 
+def gpu_layer_q2(x, scores, k, weights, q2, ws=None):
+    """One token through moe_forward_q2 (2-bit routed experts `q2`, FP4 shared expert in
+    `weights`); results and workspace intermediates on the host."""
+    import bit_moe_routed_b200 as bm
+    T, d = x.shape
+    E, f = weights.E, weights.f
+    if ws is None:
+        ws = bm.alloc_workspace(T, k, E, d, f)
+    r = bm.forward_q2(x.cuda(), scores.cuda(), k, weights, q2, ws)
+    views = bm.workspace_views(ws, T, k, E, d, f)
+    r.update({kk: v.clone() for kk, v in views.items()})
+    bm.sync_status()
+    return {kk: v.cpu() for kk, v in r.items()}
+
+
 def check_layer(g, x, scores, k, E, d, f, seed, layer, tokens, label="", experts=None,
                 verbose=True):
     """Compare GPU layer results against the oracle on the given tokens (see the module
@@ -315,8 +362,9 @@ def check_layer(g, x, scores, k, E, d, f, seed, layer, tokens, label="", experts
                 h_worst = max(h_worst, assert_within(g["h"].numpy()[row], hx, B,
                                                      f"{what}: fp32 h"))
             hhat = tab[qh_g[row]] * np.repeat(sh_g[row].astype(np.float64), 128)
-            yr = oracle.fp4_gemv(ex.down_codes, ex.down_scales, hhat)
-            yb = y_error_bound(ex.down_codes, ex.down_scales, hhat, f)
+            codec = getattr(ex, "codec", oracle.FP4)
+            yr = _gemv(ex.down_codes, ex.down_scales, hhat, codec)
+            yb = y_error_bound(ex.down_codes, ex.down_scales, hhat, f, codec)
             got = y_g[row] if j < k else ysh_g[t]
             y_worst = max(y_worst, assert_within(got, yr, yb, f"{what}: y"))
             if j < k:

@@ -21,34 +21,41 @@ STAGES = 3
 SMEM_LIMIT = 232448   # bytes of shared memory a CTA may opt into on sm_100
 
 
-def decode_fits(k, d, f, ctas):
-    """Mirror of decode_fits() in decode.cu."""
-    if k < 1 or k > 32 or d % 512 or f % 512 or ctas < 1:
-        return False
-
-    def most(upe):
-        return -(-((k + 1) * upe) // ctas)
-
-    upe1, upe2 = f // 8, d // 16
-    if most(upe1) > MAX_UNITS or most(upe2) > MAX_UNITS:
-        return False
-    return most(upe2) <= upe2 + 1
-
-
-def split(upe, n_routed, G, b):
-    """Mirror of the kernel's Range: (s_lo, ns, r_lo, nr)."""
+def split(upe, n_routed, G, b, wsh=1):
+    """Mirror of the kernel's Range: (s_lo, ns, r_lo, nr); a shared unit weighs wsh."""
     s_lo = b * upe // G
     ns = (b + 1) * upe // G - s_lo
-    M = (n_routed + 1) * upe
+    M = (n_routed + wsh) * upe
     t_lo, t_hi = b * M // G, (b + 1) * M // G
-    return s_lo, ns, t_lo - s_lo, (t_hi - t_lo) - ns
+    return s_lo, ns, t_lo - wsh * s_lo, (t_hi - t_lo) - wsh * ns
 
 
-def smem_bytes(d, f):
+def decode_fits(k, d, f, ctas, q2=False):
+    """Mirror of decode_fits() in decode.cu: every CTA's ranges, for every count of active
+    experts, within the per-CTA limits."""
+    if k < 1 or k > 32 or d % 512 or f % 512 or ctas < 1:
+        return False
+    if q2 and (d % 2048 or f % 2048):
+        return False
+    wsh = 2 if q2 else 1
+    upe1, upe2 = f // 8, d // 16
+    for n in range(1, k + 1):
+        for b in range(ctas):
+            for upe in (upe1, upe2):
+                _, ns, _, nr = split(upe, n, ctas, b, wsh)
+                if nr < 0 or ns + nr > MAX_UNITS:
+                    return False
+            if split(upe2, n, ctas, b, wsh)[3] > upe2 + 1:
+                return False
+    return True
+
+
+def smem_bytes(d, f, q2=False):
     """Mirror of DcSmem::bytes()."""
     area = WARPS * STAGES * STAGE_BYTES
-    p1_end = area + 2 * d + d // 32 + MAX_UNITS * (d // 512) * 64
-    p2_end = area + P2_SLOTS * 2 * f + P2_SLOTS * (f // 32) + MAX_UNITS * (f // 512) * 64
+    p1_end = area + (3 if q2 else 2) * d + d // 32 + MAX_UNITS * (d // 512) * 64
+    p2_end = area + (4 if q2 else 2 * P2_SLOTS) * f + P2_SLOTS * (f // 32) + \
+        MAX_UNITS * (f // 512) * 64
     bars = (max(p1_end, p2_end) + 7) // 8 * 8
     info = bars + (WARPS * STAGES + 1) * 8
     return info + 4 * (4 + 3 * 33 + 64) + 1024
@@ -117,3 +124,30 @@ def test_every_warp_takes_its_tasks_once():
             for q in range(min(shared_q, STAGES)):
                 assert (w + WARPS * q) // S1 < ns
         assert sorted(seen) == list(range(n_tasks))
+
+
+@pytest.mark.parametrize("ctas", [148, 132])
+def test_q2_form_ranges_cover_every_unit_once(ctas):
+    """The Q2 form (2-bit routed experts, a shared unit weighing 2): for every accepted
+    shape and count of active experts, the ranges cover the shared and the routed units
+    once each, with at most 16 units per CTA and a phase-2 routed range over at most two
+    experts; the decode workload is accepted and fits shared memory."""
+    checked = 0
+    for k, d, f in itertools.product(range(1, 12), (2048, 4096, 8192), (2048, 4096)):
+        if not decode_fits(k, d, f, ctas, q2=True):
+            continue
+        for n_act in range(1, k + 1):
+            for upe in (f // 8, d // 16):
+                shared, routed = [], []
+                for b in range(ctas):
+                    s_lo, ns, r_lo, nr = split(upe, n_act, ctas, b, 2)
+                    assert nr >= 0 and ns + nr <= MAX_UNITS
+                    shared.extend(range(s_lo, s_lo + ns))
+                    routed.extend(range(r_lo, r_lo + nr))
+                assert shared == list(range(upe))
+                assert routed == list(range(n_act * upe))
+                checked += 1
+    assert checked > 50
+    assert decode_fits(6, 4096, 2048, 148, q2=True)
+    assert smem_bytes(4096, 2048, q2=True) <= SMEM_LIMIT
+    assert not decode_fits(6, 1024, 2048, 148, q2=True)
