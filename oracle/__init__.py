@@ -35,7 +35,7 @@ def build(force: bool = False) -> str:
     return SO
 
 
-FP4, Q2 = 0, 1  # weight codecs (oracle.h: ORACLE_FP4, ORACLE_Q2)
+FP4, Q2, FP8 = 0, 1, 2  # weight codecs (oracle.h: ORACLE_FP4, ORACLE_Q2, ORACLE_FP8)
 
 
 class _Expert(ctypes.Structure):
@@ -71,6 +71,7 @@ def lib():
         L.oracle_dispatch.argtypes = [P, I, I, I, P, P, P, P]
         L.oracle_fp4_gemv.argtypes = [P, P, I, I, P, P]
         L.oracle_q2_gemv.argtypes = [P, P, I, I, P, P]
+        L.oracle_fp8_gemm.argtypes = [P, P, I, P, P, I, I, P]
         L.oracle_expert_ffn.argtypes = [ctypes.POINTER(_Expert), I, I, P, P, I, P, P, P]
         L.oracle_expert_ffn_h.argtypes = [ctypes.POINTER(_Expert), I, I, P, P, I, P, P, P, P]
         L.oracle_combine_token.argtypes = [P, P, P, I, I, P]
@@ -199,6 +200,20 @@ def q2_gemv(codes: np.ndarray, scales: np.ndarray, xhat: np.ndarray) -> np.ndarr
     return out
 
 
+def fp8_gemm(A: np.ndarray, sa: np.ndarray, B: np.ndarray, sb: np.ndarray) -> np.ndarray:
+    """C [M, N] (double) = (e4m3(A) * sa per 128-block) . (e4m3(B) * sb per 128x128 block)^T;
+    A [M, K], B [N, K] e4m3 codes, sa [M, K/128], sb [N/128, K/128] fp32."""
+    A, pa = _c(A, np.uint8)
+    B, pb = _c(B, np.uint8)
+    sa, psa = _c(sa, np.float32)
+    sb, psb = _c(sb, np.float32)
+    M, K = A.shape
+    N = B.shape[0]
+    C = np.empty((M, N), np.float64)
+    lib().oracle_fp8_gemm(pa, psa, M, pb, psb, N, K, C.ctypes.data)
+    return C
+
+
 class ExpertSet:
     """Holds numpy weight arrays alive and exposes a ctypes array of experts.
 
@@ -212,9 +227,11 @@ class ExpertSet:
         self.arr = (_Expert * n)()
         for e, ex in experts.items():
             vals = []
+            codec = int(getattr(ex, "codec", FP4))
             for name in ("gate_codes", "gate_scales", "up_codes", "up_scales", "down_codes",
                          "down_scales"):
-                a = np.ascontiguousarray(getattr(ex, name), dtype=np.uint8)
+                dt = np.float32 if (codec == FP8 and name.endswith("scales")) else np.uint8
+                a = np.ascontiguousarray(getattr(ex, name), dtype=dt)
                 self._keep.append(a)
                 vals.append(a.ctypes.data)
             self.arr[e] = _Expert(*vals, int(getattr(ex, "codec", FP4)))

@@ -213,6 +213,29 @@ void oracle_fp4_gemv(const uint8_t* codes, const uint8_t* scales, int rows, int 
     }
 }
 
+/* FP8 weights (tcti.cn post, "补齐软件栈缺失": fp8_gemm): e4m3 codes, one fp32 scale per
+ * 128 x 128 block. */
+static inline double fp8_weight(const uint8_t* codes, const uint8_t* scales, int K, int r,
+                                int c) {
+    const float* s = (const float*)scales;
+    return oracle_e4m3_value(codes[(size_t)r * K + c]) *
+           (double)s[(size_t)(r / 128) * (K / 128) + c / 128];
+}
+
+void oracle_fp8_gemm(const uint8_t* A, const float* sa, int M, const uint8_t* B,
+                     const float* sb, int N, int K, double* C) {
+#pragma omp parallel for num_threads(g_threads) schedule(static)
+    for (int n = 0; n < N; ++n) {
+        for (int m = 0; m < M; ++m) {
+            double acc = 0.0;
+            for (int k = 0; k < K; ++k)
+                acc += oracle_e4m3_value(A[(size_t)m * K + k]) * (double)sa[(size_t)m * (K / 128) + k / 128] *
+                       fp8_weight(B, (const uint8_t*)sb, K, n, k);
+            C[(size_t)m * N + n] = acc;
+        }
+    }
+}
+
 void oracle_q2_gemv(const uint8_t* codes, const uint8_t* scales, int rows, int K,
                     const double* xhat, double* out) {
 #pragma omp parallel for num_threads(g_threads) schedule(static)
@@ -228,7 +251,8 @@ static void decode_row(int codec, const uint8_t* codes, const uint8_t* scales, i
                        double* dst) {
     for (int c = 0; c < K; ++c)
         dst[c] = codec == ORACLE_Q2 ? q2_weight(codes, scales, K, r, c)
-                                    : fp4_weight(codes, scales, K, r, c);
+                 : codec == ORACLE_FP8 ? fp8_weight(codes, scales, K, r, c)
+                                       : fp4_weight(codes, scales, K, r, c);
 }
 
 /* One expert over a group of tokens: g = Wg xhat, u = Wu xhat, h = silu(g) * u

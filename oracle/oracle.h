@@ -31,6 +31,11 @@
  *    (element i of a byte in bits 2i..2i+1), value = code - 1.5 (the uniform
  *    four-level grid -1.5, -0.5, 0.5, 1.5), times one ue8m0 scale per 128 consecutive
  *    elements along the reduction axis: 2 + 8/128 = 2.0625 bits per weight.
+ *  - tcti.cn post, section "补齐软件栈缺失": fp8_gemm (FP8 activation x FP8 weight) for the
+ *    model's FP8 linears; the SURVEY's NEXT-3 reads the shared expert as one of them.  The
+ *    page gives no scale layout; read here as e4m3 weights with one fp32 scale per
+ *    128 x 128 block (rows x reduction) and activations quantised per token and 128-block
+ *    exactly as for the FP4 path.
  *
  * Floating point: all sums are in double.  Activation quantisation is done in
  * fp32 arithmetic (divide, then round to nearest e4m3, ties to even mantissa,
@@ -47,9 +52,12 @@ extern "C" {
 
 /* Per-expert weight pointers.  gate/up: rows = f, K = d.  down: rows = d, K = f.
  * codec ORACLE_FP4: codes [rows][K/2] bytes, scales [rows][K/32] bytes.
- * codec ORACLE_Q2:  codes [rows][K/4] bytes, scales [rows][K/128] bytes. */
+ * codec ORACLE_Q2:  codes [rows][K/4] bytes, scales [rows][K/128] bytes.
+ * codec ORACLE_FP8: codes [rows][K] e4m3 bytes; the scales pointer points to fp32 values
+ *                   [rows/128][K/128] (one per 128 x 128 block). */
 #define ORACLE_FP4 0
 #define ORACLE_Q2 1
+#define ORACLE_FP8 2
 typedef struct {
     const uint8_t* gate_codes;
     const uint8_t* gate_scales;
@@ -99,6 +107,12 @@ void oracle_fp4_gemv(const uint8_t* codes, const uint8_t* scales, int rows, int 
  * element k in bits 2(k%4)..2(k%4)+1 of byte codes[r, k/4]; in double. */
 void oracle_q2_gemv(const uint8_t* codes, const uint8_t* scales, int rows, int K,
                     const double* xhat, double* out);
+
+/* fp8_gemm: C[m][n] = sum_k (e4m3(A[m,k]) * sa[m, k/128]) * (e4m3(B[n,k]) * sb[n/128, k/128])
+ * in double; A [M][K] and B [N][K] e4m3 codes, sa [M][K/128], sb [N/128][K/128] fp32,
+ * C [M][N].  K and N multiples of 128. */
+void oracle_fp8_gemm(const uint8_t* A, const float* sa, int M, const uint8_t* B,
+                     const float* sb, int N, int K, double* C);
 
 /* One expert FFN over a group of ntok tokens that share its weights (layer-major:
  * each weight row is decoded once and dotted with every token of the group).
