@@ -38,6 +38,8 @@ EXPORTS = (
     "moe_set_wait_limit_ns", "moe_sync_status", "moe_expert_ffn_noalloc",
     "moe_set_gemv_max_tokens", "moe_workspace_offsets", "moe_set_test_stall", "moe_forward",
     "moe_ffn_path", "moe_router_topk", "moe_dispatch_workspace_size", "moe_forward_q2",
+    "moe_fp8_gemm", "moe_fp8_gemm_workspace_size", "moe_shared_expert_fp8",
+    "moe_shared_expert_fp8_workspace_size", "moe_shared_expert_fp8_offsets",
 )
 
 
@@ -50,6 +52,12 @@ class MoeError(RuntimeError):
 class _Q2Experts(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "gate_codes", "gate_scales", "up_codes", "up_scales", "down_codes", "down_scales")]
+
+
+class _Fp8Expert(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "gate", "gate_scales", "up", "up_scales", "down", "down_scales")] + [
+        ("d", ctypes.c_int), ("f", ctypes.c_int)]
 
 
 class _Weights(ctypes.Structure):
@@ -98,6 +106,11 @@ def lib():
             "moe_dispatch_workspace_size": [I, I, I],
             "moe_forward_q2": [P, P, I, W, ctypes.POINTER(_Q2Experts), P, P, P, P, P, P, P, P,
                                P, P, Z, P],
+            "moe_fp8_gemm": [P, P, I, I, P, P, I, P, P, Z, P],
+            "moe_fp8_gemm_workspace_size": [I, I, I],
+            "moe_shared_expert_fp8": [P, I, ctypes.POINTER(_Fp8Expert), P, P, Z, P],
+            "moe_shared_expert_fp8_workspace_size": [I, I, I],
+            "moe_shared_expert_fp8_offsets": [I, I, I, P],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -105,6 +118,8 @@ def lib():
             fn.restype = ctypes.c_int
         L.moe_workspace_size.restype = ctypes.c_size_t
         L.moe_dispatch_workspace_size.restype = ctypes.c_size_t
+        L.moe_fp8_gemm_workspace_size.restype = ctypes.c_size_t
+        L.moe_shared_expert_fp8_workspace_size.restype = ctypes.c_size_t
         L.moe_last_error.restype = ctypes.c_char_p
         _lib = L
     return _lib
@@ -186,6 +201,77 @@ class Q2Experts:
     def from_dict(d: dict) -> "Q2Experts":
         return Q2Experts(**{k: d[k] for k in (
             "gate_codes", "gate_scales", "up_codes", "up_scales", "down_codes", "down_scales")})
+
+
+@dataclass
+class Fp8Expert:
+    """An FP8-weight expert on the device: gate / up [f, d] and down [d, f] e4m3 codes
+    (uint8), gate_scales / up_scales [f/128, d/128] and down_scales [d/128, f/128] fp32."""
+    gate: torch.Tensor
+    gate_scales: torch.Tensor
+    up: torch.Tensor
+    up_scales: torch.Tensor
+    down: torch.Tensor
+    down_scales: torch.Tensor
+
+    @property
+    def d(self) -> int:
+        return self.gate.shape[1]
+
+    @property
+    def f(self) -> int:
+        return self.gate.shape[0]
+
+    def struct(self) -> _Fp8Expert:
+        return _Fp8Expert(*(t.data_ptr() for t in (
+            self.gate, self.gate_scales, self.up, self.up_scales, self.down, self.down_scales)),
+            self.d, self.f)
+
+    @staticmethod
+    def from_dict(d: dict) -> "Fp8Expert":
+        return Fp8Expert(**{k: d[k] for k in (
+            "gate", "gate_scales", "up", "up_scales", "down", "down_scales")})
+
+
+def fp8_gemm(A: torch.Tensor, sa: torch.Tensor, B: torch.Tensor, sb: torch.Tensor,
+             ws: torch.Tensor | None = None, stream=None, out: torch.Tensor | None = None):
+    """C [M, N] fp32 = FP8 A [M, K] (scales sa [M, K/128]) times FP8 B [N, K] (scales
+    sb [N/128, K/128]) transposed (moe_fp8_gemm)."""
+    M, K = A.shape
+    N = B.shape[0]
+    if ws is None:
+        n = int(lib().moe_fp8_gemm_workspace_size(M, N, K))
+        ws = torch.empty(max(n, 256), dtype=torch.uint8, device=A.device)
+    C = out if out is not None else torch.empty((M, N), dtype=torch.float32, device=A.device)
+    _check(lib().moe_fp8_gemm(_p(A), _p(sa), M, K, _p(B), _p(sb), N, _p(C), _p(ws), ws.numel(),
+                              _stream(stream)))
+    return C
+
+
+def shared_expert_fp8(x: torch.Tensor, w: Fp8Expert, ws: torch.Tensor | None = None,
+                      stream=None, out: torch.Tensor | None = None):
+    """y_shared [T, d] fp32 of the FP8-weight expert for bf16 tokens x [T, d]
+    (moe_shared_expert_fp8)."""
+    T, d = x.shape
+    if ws is None:
+        n = int(lib().moe_shared_expert_fp8_workspace_size(T, w.d, w.f))
+        ws = torch.empty(max(n, 256), dtype=torch.uint8, device=x.device)
+    y = out if out is not None else torch.empty((T, d), dtype=torch.float32, device=x.device)
+    st = w.struct()
+    _check(lib().moe_shared_expert_fp8(_p(x), T, ctypes.byref(st), _p(y), _p(ws), ws.numel(),
+                                       _stream(stream)))
+    return y
+
+
+def shared_expert_fp8_views(ws: torch.Tensor, T: int, d: int, f: int) -> dict:
+    """Views of moe_shared_expert_fp8's intermediates in its workspace: qx, sx, h, qh, sh."""
+    off = (ctypes.c_size_t * 5)()
+    _check(lib().moe_shared_expert_fp8_offsets(T, d, f, off))
+    u8 = lambda o, n: ws[o:o + n]  # noqa: E731
+    f32 = lambda o, n: ws[o:o + 4 * n].view(torch.float32)  # noqa: E731
+    return {"qx": u8(off[0], T * d).view(T, d), "sx": f32(off[1], T * (d // 128)).view(T, -1),
+            "h": f32(off[2], T * f).view(T, f), "qh": u8(off[3], T * f).view(T, f),
+            "sh": f32(off[4], T * (f // 128)).view(T, -1)}
 
 
 def set_wait_limit_ns(n: int) -> None:

@@ -775,6 +775,141 @@ int moe_forward_q2(const float* scores, const uint16_t* x_bf16, int k, const moe
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "single-token 2-bit layer launch");
 }
 
+size_t moe_fp8_gemm_workspace_size(int M, int N, int K) {
+  if (M < 1 || M > 64 || N < 128 || N % 128 || K < 512 || K % 512) return 0;
+  return fp8_gemm_ws_bytes(M, N, K, false);
+}
+
+int moe_fp8_gemm(const uint8_t* A, const float* sa, int M, int K, const uint8_t* B,
+                 const float* sb, int N, float* C, void* ws, size_t ws_bytes, void* stream) {
+  if (M < 0 || M > 64) return fail(MOE_ERR_INVALID_ARG, "M=%d outside [0, 64]", M);
+  if (N < 128 || N % 128 || K < 512 || K % 512)
+    return fail(MOE_ERR_INVALID_ARG, "N=%d must be a multiple of 128, K=%d of 512", N, K);
+  if (M == 0) return MOE_OK;
+  if (!A || !sa || !B || !sb || !C || !ws) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(A, 16) || !aligned(B, 16) || !aligned(C, 8) || !aligned(sa, 4) ||
+      !aligned(sb, 4) || !aligned(ws, 256))
+    return fail(MOE_ERR_INVALID_ARG, "A, B 16-byte, C 8-byte, ws 256-byte aligned");
+  const size_t need = fp8_gemm_ws_bytes(M, N, K, false);
+  if (ws_bytes < need)
+    return fail(MOE_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, need);
+  DeviceInfo di;
+  int rc = device_info(di);
+  if (rc) return rc;
+  Fp8Launch a{};
+  a.A = A;
+  a.sa = sa;
+  a.B0 = B;
+  a.sb0 = sb;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.C = C;
+  a.ws = static_cast<uint8_t*>(ws);
+  a.zero_counters = true;
+  cudaError_t e = launch_fp8_gemm(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "fp8_gemm launch");
+}
+
+namespace {
+// workspace of moe_shared_expert_fp8: qx, sx, h, qh, sh, then each GEMM's partials and
+// counters (separate regions: a counter must not sit in the other GEMM's partials)
+struct SharedFp8Layout {
+  size_t qx, sx, h, qh, sh, g1, g2, total;
+};
+SharedFp8Layout shared_fp8_layout(int T, int d, int f) {
+  SharedFp8Layout L{};
+  auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+  size_t o = 0;
+  L.qx = o; o = up(o + (size_t)T * d);
+  L.sx = o; o = up(o + (size_t)T * (d / 128) * 4);
+  L.h = o;  o = up(o + (size_t)T * f * 4);
+  L.qh = o; o = up(o + (size_t)T * f);
+  L.sh = o; o = up(o + (size_t)T * (f / 128) * 4);
+  L.g1 = o; o = up(o + fp8_gemm_ws_bytes(T, f, d, true));
+  L.g2 = o; o = up(o + fp8_gemm_ws_bytes(T, d, f, false));
+  L.total = o;
+  return L;
+}
+}  // namespace
+
+int moe_shared_expert_fp8_offsets(int T, int d, int f, size_t off[5]) {
+  if (!off) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  if (T < 1 || T > 64 || d < 512 || d % 512 || f < 512 || f % 512)
+    return fail(MOE_ERR_INVALID_ARG, "T=%d, d=%d, f=%d outside the accepted shapes", T, d, f);
+  const SharedFp8Layout L = shared_fp8_layout(T, d, f);
+  off[0] = L.qx;
+  off[1] = L.sx;
+  off[2] = L.h;
+  off[3] = L.qh;
+  off[4] = L.sh;
+  return MOE_OK;
+}
+
+size_t moe_shared_expert_fp8_workspace_size(int T, int d, int f) {
+  if (T < 1 || T > 64 || d < 512 || d % 512 || f < 512 || f % 512) return 0;
+  return shared_fp8_layout(T, d, f).total;
+}
+
+int moe_shared_expert_fp8(const uint16_t* x_bf16, int T, const moe_fp8_expert_t* w,
+                          float* y_shared, void* ws, size_t ws_bytes, void* stream) {
+  if (!w) return fail(MOE_ERR_INVALID_ARG, "NULL weights");
+  const int d = w->d, f = w->f;
+  if (T < 0 || T > 64) return fail(MOE_ERR_INVALID_ARG, "T=%d outside [0, 64]", T);
+  if (d < 512 || d % 512 || f < 512 || f % 512)
+    return fail(MOE_ERR_INVALID_ARG, "d=%d, f=%d must be multiples of 512", d, f);
+  if (T == 0) return MOE_OK;
+  if (!x_bf16 || !y_shared || !ws || !w->gate || !w->up || !w->down || !w->gate_scales ||
+      !w->up_scales || !w->down_scales)
+    return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(x_bf16, 16) || !aligned(y_shared, 8) || !aligned(ws, 256) ||
+      !aligned(w->gate, 16) || !aligned(w->up, 16) || !aligned(w->down, 16))
+    return fail(MOE_ERR_INVALID_ARG, "misaligned pointer");
+  const SharedFp8Layout L = shared_fp8_layout(T, d, f);
+  if (ws_bytes < L.total)
+    return fail(MOE_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, L.total);
+  DeviceInfo di;
+  int rc = device_info(di);
+  if (rc) return rc;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* qx = base + L.qx;
+  float* sx = reinterpret_cast<float*>(base + L.sx);
+  float* h = reinterpret_cast<float*>(base + L.h);
+  uint8_t* qh = base + L.qh;
+  float* sh = reinterpret_cast<float*>(base + L.sh);
+  cudaError_t e = launch_quant_rows(x_bf16, T, 1, d, nullptr, 0, qx, sx, nullptr, 0, 0, nullptr,
+                                    nullptr, 0, di.status, s);
+  Fp8Launch a{};
+  a.A = qx;
+  a.sa = sx;
+  a.B0 = w->gate;
+  a.sb0 = w->gate_scales;
+  a.B1 = w->up;
+  a.sb1 = w->up_scales;
+  a.M = T;
+  a.N = f;
+  a.K = d;
+  a.C = h;
+  a.ws = base + L.g1;
+  a.zero_counters = true;
+  if (e == cudaSuccess) e = launch_fp8_gemm(a, s);
+  if (e == cudaSuccess) e = launch_quant_h(h, T, f, qh, sh, s, true);
+  Fp8Launch b{};
+  b.A = qh;
+  b.sa = sh;
+  b.B0 = w->down;
+  b.sb0 = w->down_scales;
+  b.M = T;
+  b.N = d;
+  b.K = f;
+  b.C = y_shared;
+  b.ws = base + L.g2;
+  b.zero_counters = true;
+  if (e == cudaSuccess) e = launch_fp8_gemm(b, s);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "shared expert fp8 launch");
+}
+
 int moe_combine(const float* y_routed, const float* y_shared, const float* topk_w,
                 const int32_t* pos, int T, int k, int d, float* out, void* stream) {
   if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T=%d < 0", T);

@@ -197,6 +197,27 @@ size_t decode_smem_bytes(int d, int f, bool q2 = false);
 // whether the single-token kernel's per-CTA limits hold for (k, d, f) on `ctas` CTAs
 // (q2: with 2-bit routed experts)
 bool decode_fits(int k, int d, int f, int ctas, bool q2 = false);
+// FP8 x FP8 GEMM for M <= 64 rows of A (fp8.cu): C[m][n] = sum_kb sa[m][kb] sb[n/128][kb]
+// sum_k A[m][k] B[n][k], A [M][K] and B [N][K] e4m3, sa [M][K/128], sb [N/128][K/128] fp32.
+// With B1 (the up projection beside B0 = gate) C = silu(A B0^T) * (A B1^T).  K % 512 == 0,
+// N % 128 == 0; the workspace holds the partial sums and the row blocks' counters, which
+// must be zero on entry (zero_counters: the launch clears them first; every launch leaves
+// them zero).
+struct Fp8Launch {
+  const uint8_t* A;
+  const float* sa;
+  const uint8_t* B0;
+  const float* sb0;
+  const uint8_t* B1;
+  const float* sb1;
+  int M, N, K;
+  float* C;
+  uint8_t* ws;
+  bool zero_counters;
+  bool overlap;
+};
+size_t fp8_gemm_ws_bytes(int M, int N, int K, bool fused);
+cudaError_t launch_fp8_gemm(const Fp8Launch& a, cudaStream_t s);
 // clears the single-token kernel's grid barrier (after a reported timeout)
 cudaError_t reset_grid_barrier();
 

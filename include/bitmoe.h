@@ -218,6 +218,54 @@ int moe_forward_q2(const float* scores, const uint16_t* x_bf16, int k, const moe
                    float* y_routed, float* y_shared, float* out, void* ws, size_t ws_bytes,
                    void* stream);
 
+/* FP8 x FP8 GEMM (NEXT-3): the pages' fp8_gemm beside fp4_gemm ([P1] "补齐软件栈缺失":
+ * FP8 activations times FP8 weights, the format of the model's non-FP4 linears).  The
+ * page gives no scale layout; read here as e4m3 weights with one fp32 scale per 128 x 128
+ * block (rows x reduction) and e4m3 activations with one fp32 scale per row and 128-block
+ * (moe_act_quant's codes):
+ *   C[m][n] = sum_kb sa[m][kb] * sb[n/128][kb] * sum_{k in block kb} A[m][k] * B[n][k].
+ *   A [M][K] e4m3 codes (16-byte aligned), sa [M][K/128] fp32; B [N][K] e4m3 codes
+ *   (16-byte aligned), sb [N/128][K/128] fp32; C [M][N] fp32 out (8-byte aligned).
+ *   ws: at least moe_fp8_gemm_workspace_size(M, N, K) bytes, 256-byte aligned, contents
+ *   need not be initialised (the call clears what it needs).
+ * 0 <= M <= 64 (a decode-sized batch: one weight read serves every row of A); N % 128 == 0;
+ * K % 512 == 0.  Reads B once (mma.sync e4m3 on the codes, 128-element sums in the tensor
+ * core, scales applied in fp32, per-row-block partials added in reduction order). */
+size_t moe_fp8_gemm_workspace_size(int M, int N, int K);
+int moe_fp8_gemm(const uint8_t* A, const float* sa, int M, int K, const uint8_t* B,
+                 const float* sb, int N, float* C, void* ws, size_t ws_bytes, void* stream);
+
+/* An FP8-weight expert (NEXT-3: the real model's shared expert is FP8, not FP4):
+ *   gate, up [f][d] e4m3, gate_scales, up_scales [f/128][d/128] fp32;
+ *   down [d][f] e4m3, down_scales [d/128][f/128] fp32.  Code arrays 16-byte aligned. */
+typedef struct {
+  const uint8_t* gate;
+  const float* gate_scales;
+  const uint8_t* up;
+  const float* up_scales;
+  const uint8_t* down;
+  const float* down_scales;
+  int d;
+  int f;
+} moe_fp8_expert_t;
+
+/* The shared expert with FP8 weights for T tokens: x quantised as in moe_act_quant, then
+ * h = silu(g) * u with g, u from one fused FP8 GEMM over the gate and up rows, h
+ * re-quantised per 128-block (amax / 448, IEEE divide, round to nearest even), and
+ * y_shared = W_down h^ by a second FP8 GEMM.
+ *   x_bf16 [T][d] bf16 (16-byte aligned); y_shared [T][d] fp32 out (8-byte aligned).
+ *   ws: at least moe_shared_expert_fp8_workspace_size(T, d, f) bytes, 256-byte aligned.
+ * 0 <= T <= 64; d, f multiples of 512.  Four kernels on the stream. */
+size_t moe_shared_expert_fp8_workspace_size(int T, int d, int f);
+/* Where moe_shared_expert_fp8 leaves its intermediates in a workspace laid out for
+ * (T, d, f), for tests and tools (the pages have no counterpart): byte offsets of
+ * off[0] qx [T][d] e4m3, off[1] sx [T][d/128] fp32, off[2] h [T][f] fp32 (silu(g) * u
+ * before re-quantisation), off[3] qh [T][f] e4m3, off[4] sh [T][f/128] fp32.
+ * MOE_ERR_INVALID_ARG for shapes the call rejects. */
+int moe_shared_expert_fp8_offsets(int T, int d, int f, size_t off[5]);
+int moe_shared_expert_fp8(const uint16_t* x_bf16, int T, const moe_fp8_expert_t* w,
+                          float* y_shared, void* ws, size_t ws_bytes, void* stream);
+
 /* Step 8 — combine: out[t][m] = y_shared[t][m] + sum_{j<k} topk_w[t][j] *
  * y_routed[pos[t*k+j]][m], summed in fixed j order in fp32.
  *   y_routed [T*k][d], y_shared [T][d], topk_w [T][k], pos [T*k], out [T][d] fp32.

@@ -250,6 +250,62 @@ def device_layer_weights_q2(seed: int, layer: int, E: int, d: int, f: int, devic
     return out
 
 
+# --------------------------------------------------------------------------------------
+# FP8 shared expert: e4m3 codes [rows, K] and fp32 scales [rows/128, K/128], from the same
+# generator with seeds seed ^ FP8_SEED.  A code byte b becomes (b AND 0x87) OR
+# ((4 + ((b >> 3) AND 7)) << 3): sign and mantissa from b, exponent field 4..11 (values
+# 2^-3 .. 15, no NaN); a scale is 2^(e - 127) with e the generator's scale byte (121..124).
+# --------------------------------------------------------------------------------------
+FP8_SEED = 0xF8F8
+
+
+def _fp8_codes(raw):
+    return (raw & 0x87) | ((4 + ((raw >> 3) & 7)) << 3)
+
+
+def host_expert_fp8(seed: int, layer: int, d: int, f: int) -> dict:
+    """The FP8 shared expert as numpy arrays: gate/up/down codes (uint8) and scales
+    (float32); drawn from the streams of expert 0 under the FP8 seed."""
+    out = {}
+    for name, which in (("gate", GATE), ("up", UP), ("down", DOWN)):
+        r, K = matrix_shape(which, d, f)
+        raw = np.empty((r, K), np.uint8)
+        _host_lib().synth_fill(seed ^ FP8_SEED, layer, 0, which, CODES, raw.ctypes.data, 0,
+                               raw.size)
+        sb = np.empty((r // 128, K // 128), np.uint8)
+        _host_lib().synth_fill(seed ^ FP8_SEED, layer, 0, which, SCALES, sb.ctypes.data, 0,
+                               sb.size)
+        out[name] = _fp8_codes(raw).astype(np.uint8)
+        out[f"{name}_scales"] = np.ldexp(1.0, sb.astype(np.int32) - 127).astype(np.float32)
+    return out
+
+
+def device_expert_fp8(seed: int, layer: int, d: int, f: int, device="cuda",
+                      stream=None) -> dict:
+    """The same expert generated in device memory (torch tensors)."""
+    lib = _dev_lib()
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    out = {}
+    for name, which in (("gate", GATE), ("up", UP), ("down", DOWN)):
+        r, K = matrix_shape(which, d, f)
+        raw = torch.empty((r, K), dtype=torch.uint8, device=device)
+        sb = torch.empty((r // 128, K // 128), dtype=torch.uint8, device=device)
+        for t, kind in ((raw, CODES), (sb, SCALES)):
+            rc = lib.synth_fill_dev(seed ^ FP8_SEED, layer, 1, which, kind, t.numel(),
+                                    t.data_ptr(), ctypes.c_void_p(s.cuda_stream))
+            if rc != 0:
+                raise RuntimeError(f"synth_fill_dev failed: {rc}")
+        with torch.cuda.stream(s):
+            out[name] = _fp8_codes(raw.to(torch.int32)).to(torch.uint8)
+            out[f"{name}_scales"] = torch.ldexp(torch.ones_like(sb, dtype=torch.float32),
+                                                sb.to(torch.int32) - 127)
+    return out
+
+
+def fp8_expert_bytes(d: int, f: int) -> int:
+    return 3 * d * f + 3 * (d // 128) * (f // 128) * 4
+
+
 def q2_expert_bytes(d: int, f: int) -> int:
     return sum(matrix_shape(m, d, f)[0] * (q2_cols(m, CODES, d, f) + q2_cols(m, SCALES, d, f))
                for m in (GATE, UP, DOWN))

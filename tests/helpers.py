@@ -206,9 +206,22 @@ class HStats:
                 f"{self.scales_diff} of {self.scales} differ (largest rel {self.max_scale_rel:.2e})")
 
 
-def check_h_codes(qg, sg, qo, so, hf_o, ex, d, xhat, stats: HStats, what=""):
+def h_bound_from(g, u, ag, au, D):
+    """The a-priori bound on |h_gpu - h| from exact g, u, sum |W x| (ag, au) and the
+    depth D of the dot products (see the module docstring)."""
+    dg, du = D * U23 * ag, D * U23 * au
+    sig = 1.0 / (1.0 + np.exp(-g))
+    silu = g * sig
+    dsilu = sig * (1.0 + g * (1.0 - sig))
+    h = silu * u
+    return 1.01 * (np.abs(u) * np.abs(dsilu) * dg + np.abs(silu) * du + 1.1 * dg * du
+                   + 0.25 * dg * dg * np.abs(u)) + 9 * U23 * np.abs(h)
+
+
+def check_h_codes(qg, sg, qo, so, hf_o, ex, d, xhat, stats: HStats, what="", bound_fn=None):
     """Rule 1 for one vector (one token, one expert): GPU codes/scales (qg, sg) against the
-    oracle's (qo, so, and its fp32 h before quantisation hf_o)."""
+    oracle's (qo, so, and its fp32 h before quantisation hf_o).  bound_fn(rows), if given,
+    returns the h bound of those rows instead of h_error_bound(ex, d, xhat, rows)."""
     tab = e4m3_table()
     vals = _sorted_values()
     qg = np.asarray(qg, np.uint8)
@@ -228,7 +241,7 @@ def check_h_codes(qg, sg, qo, so, hf_o, ex, d, xhat, stats: HStats, what=""):
         assert top.size > 0, f"{what}: block {b} has no element at +-448"
         need |= set(int(128 * b + i) for i in top)
     rows = np.array(sorted(need), dtype=np.int64)
-    B, _, _, _ = h_error_bound(ex, d, xhat, rows)
+    B = bound_fn(rows) if bound_fn is not None else h_error_bound(ex, d, xhat, rows)[0]
     Bmap = dict(zip(rows.tolist(), B.tolist()))
     srel = np.zeros(nb)
     for b in diff_blocks:
