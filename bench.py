@@ -552,6 +552,40 @@ def measure(bm, w, args, dev, stream, rank, dist, steps, warmup, peaks, cpu_seco
     return rec, Ls
 
 
+def measure_shared_fp8(bm, dev, stream, T: int, hbm_peak: float, peak_kind: str,
+                       steps: int = 20) -> dict:
+    """The FP8-weight shared expert (moe_shared_expert_fp8) at d = 4096, f = 2048 for T
+    tokens: `steps` calls back to back in one CUDA graph, each on its own copy of the
+    weights (enough copies that a copy's 25 MB were evicted from L2 since its last use)."""
+    d, f = 4096, 2048
+    wbytes = synth.fp8_expert_bytes(d, f)
+    n = max(2, -(-4 * L2_BYTES // wbytes) + 1)
+    experts = [bm.Fp8Expert.from_dict(synth.device_expert_fp8(2000 + i, 0, d, f)) for i in range(n)]
+    x = synth.gen_x(T, d, seed=77).to(dev)
+    ws = torch.empty(int(bm.lib().moe_shared_expert_fp8_workspace_size(T, d, f)), dtype=torch.uint8,
+                     device=dev)
+    y = torch.empty((T, d), dtype=torch.float32, device=dev)
+    with torch.cuda.stream(stream):
+        for i in range(n):  # eager pass over every copy (checks the status word)
+            bm.shared_expert_fp8(x, experts[i], ws=ws, stream=stream, out=y)
+    bm.sync_status(stream)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(steps):
+            bm.shared_expert_fp8(x, experts[i % n], ws=ws, stream=stream, out=y)
+    time_graph(g, stream, 3)
+    ms = statistics.median(time_graph(g, stream, 5)) / steps
+    s = ms / 1000.0
+    gbs = wbytes / s / 1e9
+    del g
+    return {"T": T, "d": d, "f": f, "ms_per_step": ms, "steps": steps, "resident_copies": n,
+            "value": T / s, "unit": "tokens/s", "launches_per_step": 4,
+            "weight_bytes": wbytes, "weight_gb_per_s": gbs, "frac_of_measured_hbm": gbs / hbm_peak,
+            "peak_source": f"{peak_kind} HBM copy",
+            "kernels": "quant_rows (x -> e4m3), fp8_gemm gate+up -> h, quant_h, fp8_gemm down "
+                       "(mma.sync e4m3 on the codes, cp.async weight tiles)"}
+
+
 def e2e(bm, Ls, args, dev, stream, dist, world):
     """The same metric through the public API with host buffers: each step copies x and the
     scores from pinned host memory, runs the four calls and copies the output back, then
@@ -651,6 +685,11 @@ def run_gpu(args, w):
             import gc
             gc.collect()
             torch.cuda.synchronize()
+            torch.cuda.empty_cache()
+        if args.workloads == "all" or "shared_fp8" in args.workloads:
+            for Tf in (1, 64):  # NEXT-3: the FP8-weight shared expert on fp8_gemm
+                workloads[f"shared_fp8_t{Tf}"] = measure_shared_fp8(bm, dev, stream, Tf, hbm_peak,
+                                                                     peak_kind)
             torch.cuda.empty_cache()
 
     if rank == 0:
