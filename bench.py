@@ -670,7 +670,7 @@ def run_gpu(args, w):
         names = EXTRA_WORKLOADS if args.workloads == "all" else \
             [n for n in args.workloads.split(",") if n]
         for name in names:
-            if name == w.name:
+            if name == w.name or name not in synth.WORKLOADS:
                 continue
             wl = synth.WORKLOADS[name]
             need = (wl.layers if wl.layers > 1 else 2) * synth.expert_bytes(wl.d, wl.f) * (wl.E + 1)
