@@ -815,7 +815,7 @@ namespace {
 // workspace of moe_shared_expert_fp8: qx, sx, h, qh, sh, then each GEMM's partials and
 // counters (separate regions: a counter must not sit in the other GEMM's partials)
 struct SharedFp8Layout {
-  size_t qx, sx, h, qh, sh, g1, g2, total;
+  size_t qx, sx, h, qh, sh, g1, g2, cnt, total;
 };
 SharedFp8Layout shared_fp8_layout(int T, int d, int f) {
   SharedFp8Layout L{};
@@ -828,6 +828,7 @@ SharedFp8Layout shared_fp8_layout(int T, int d, int f) {
   L.sh = o; o = up(o + (size_t)T * (f / 128) * 4);
   L.g1 = o; o = up(o + fp8_gemm_ws_bytes(T, f, d, true));
   L.g2 = o; o = up(o + fp8_gemm_ws_bytes(T, d, f, false));
+  L.cnt = o; o = up(o + (fp8_gemm_counters(f, true) + fp8_gemm_counters(d, false)) * sizeof(int));
   L.total = o;
   return L;
 }
@@ -878,8 +879,13 @@ int moe_shared_expert_fp8(const uint16_t* x_bf16, int T, const moe_fp8_expert_t*
   float* h = reinterpret_cast<float*>(base + L.h);
   uint8_t* qh = base + L.qh;
   float* sh = reinterpret_cast<float*>(base + L.sh);
-  cudaError_t e = launch_quant_rows(x_bf16, T, 1, d, nullptr, 0, qx, sx, nullptr, 0, 0, nullptr,
-                                    nullptr, 0, di.status, s);
+  // both GEMMs' counters in one clear; every launch leaves its counters zero again
+  int* cnt = reinterpret_cast<int*>(base + L.cnt);
+  const size_t n1 = fp8_gemm_counters(f, true), n2 = fp8_gemm_counters(d, false);
+  cudaError_t e = cudaMemsetAsync(cnt, 0, (n1 + n2) * sizeof(int), s);
+  if (e == cudaSuccess)
+    e = launch_quant_rows(x_bf16, T, 1, d, nullptr, 0, qx, sx, nullptr, 0, 0, nullptr, nullptr, 0,
+                          di.status, s);
   Fp8Launch a{};
   a.A = qx;
   a.sa = sx;
@@ -892,7 +898,8 @@ int moe_shared_expert_fp8(const uint16_t* x_bf16, int T, const moe_fp8_expert_t*
   a.K = d;
   a.C = h;
   a.ws = base + L.g1;
-  a.zero_counters = true;
+  a.cnt = cnt;
+  a.overlap = true;
   if (e == cudaSuccess) e = launch_fp8_gemm(a, s);
   if (e == cudaSuccess) e = launch_quant_h(h, T, f, qh, sh, s, true);
   Fp8Launch b{};
@@ -905,7 +912,8 @@ int moe_shared_expert_fp8(const uint16_t* x_bf16, int T, const moe_fp8_expert_t*
   b.K = f;
   b.C = y_shared;
   b.ws = base + L.g2;
-  b.zero_counters = true;
+  b.cnt = cnt + n1;
+  b.overlap = true;
   if (e == cudaSuccess) e = launch_fp8_gemm(b, s);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "shared expert fp8 launch");
 }

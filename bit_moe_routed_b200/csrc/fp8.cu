@@ -8,10 +8,12 @@
 // scale amax / 448, as for the FP4 path:
 //   C[m][n] = sum_kb sa[m][kb] sb[n/128][kb] sum_{k in kb} A[m][k] B[n][k].
 //
-// For M <= 64 tokens the product is bound by reading B once.  One warp takes one task,
-// 16 weight rows x 512 reduction elements: it copies the 8 KB of e4m3 rows into its own
-// shared-memory tile with 16-byte cp.async (rows padded to 544 bytes so that the eight
-// rows one load touches fall on different banks), then per 32-element block runs one
+// For M <= 64 tokens the product is bound by reading B once.  Work is cut into tasks of
+// 16 weight rows x 512 reduction elements; a CTA of four warps takes four tasks of the
+// same 512-element chunk, one per warp.  The CTA copies the chunk of every token's row
+// (M x 512 bytes) and each warp its task's 16 weight rows (8 KB) into shared memory with
+// 16-byte cp.async, rows padded to 544 bytes so that the eight rows one 8-byte read
+// touches fall on different banks.  Per 32-element block the warp then runs one
 // mma.sync m16n8k32 e4m3 per group of 8 tokens straight on the codes (no decode): lane
 // (g, t) holds bytes 8t..8t+7 of the block in rows g and g+8 (k-slots 4t..4t+3 and
 // 16+4t..16+4t+3) and the same 8 bytes of token g's row.  Four blocks (128 elements) sum
@@ -52,33 +54,46 @@ __device__ __forceinline__ int atom_add_acq_rel(int* p, int v) {
   return old;
 }
 
+// shared memory of a CTA: four weight tiles, then the tokens' rows of the chunk
+__host__ __device__ constexpr int fp8_smem_bytes(int M) {
+  return kF8Warps * kF8Rows * kF8Pitch + ((M + 7) / 8 * 8) * kF8Pitch;
+}
+
 template <int NS, bool FUSED>
 __global__ void __launch_bounds__(kF8Warps * 32) fp8_gemm_kernel(const Fp8Params p) {
-  __shared__ __align__(16) uint8_t tile[kF8Warps][kF8Rows * kF8Pitch];
+  extern __shared__ __align__(16) uint8_t f8_smem[];
   ptx::griddep_launch_dependents();
-  ptx::griddep_wait();  // A comes from earlier work on the stream
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int K = p.K, M = p.M, kc = K / kF8K, nkb = K / 128;
   const int M8 = NS * 8;
-  const int units = FUSED ? p.N / 8 : p.N / 16;
-  const int task = blockIdx.x * kF8Warps + warp;
-  if (task >= units * kc) return;  // whole warps only; no CTA barrier follows
-  const int unit = task / kc, chunk = task % kc;
+  const int units = FUSED ? p.N / 8 : p.N / 16;  // a multiple of kF8Warps (N % 128 == 0)
+  const int per_chunk = units / kF8Warps;
+  const int chunk = blockIdx.x / per_chunk;
+  const int unit = (blockIdx.x % per_chunk) * kF8Warps + warp;
   const int row0 = FUSED ? 8 * unit : 16 * unit;  // first weight row (of each matrix)
-  uint8_t* sm = tile[warp];
+  uint8_t* wt = f8_smem + warp * kF8Rows * kF8Pitch;
+  uint8_t* at = f8_smem + kF8Warps * kF8Rows * kF8Pitch;
 
-  // the task's 16 rows x 512 bytes: 16-byte copies, 16 per lane
+  // this warp's 16 weight rows (they do not depend on earlier work: copied while the
+  // previous kernel on the stream may still run), then the CTA's tokens (M rows x 512
+  // bytes of the chunk)
   for (int i = lane; i < kF8Rows * (kF8K / 16); i += 32) {
     const int r = i / (kF8K / 16), c16 = i % (kF8K / 16);
     const uint8_t* src = FUSED ? (r < 8 ? p.B0 + (size_t)(row0 + r) * K
                                         : p.B1 + (size_t)(row0 + r - 8) * K)
                                : p.B0 + (size_t)(row0 + r) * K;
-    ptx::cp_async_16(ptx::smem_u32(sm + r * kF8Pitch + 16 * c16), src + chunk * kF8K + 16 * c16);
+    ptx::cp_async_16(ptx::smem_u32(wt + r * kF8Pitch + 16 * c16), src + chunk * kF8K + 16 * c16);
+  }
+  ptx::griddep_wait();  // A, its scales and the counters come from earlier work
+  for (int i = threadIdx.x; i < M * (kF8K / 16); i += kF8Warps * 32) {
+    const int r = i / (kF8K / 16), c16 = i % (kF8K / 16);
+    ptx::cp_async_16(ptx::smem_u32(at + r * kF8Pitch + 16 * c16),
+                     p.A + (size_t)r * K + chunk * kF8K + 16 * c16);
   }
   ptx::cp_async_commit();
   ptx::cp_async_wait_all();
-  __syncwarp();
+  __syncthreads();  // every thread's copies of the tokens have landed
 
   // rows g and g+8 of the task; tokens 8s + 2t, 8s + 2t + 1 of group s
   float acc[NS][4];
@@ -87,21 +102,20 @@ __global__ void __launch_bounds__(kF8Warps * 32) fp8_gemm_kernel(const Fp8Params
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc[s][i] = 0.f;
   const int rowblk = row0 / 128;
-#pragma unroll 1
+#pragma unroll
   for (int sc = 0; sc < kF8K / 128; ++sc) {
     const int kb = chunk * (kF8K / 128) + sc;  // the 128-block of the reduction
     float cq[NS][4];
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
       const int kk = sc * 128 + b * 32 + 8 * t;  // lane's 8 bytes of the 32-block
-      const uint2 wa = *reinterpret_cast<const uint2*>(sm + g * kF8Pitch + kk);
-      const uint2 wb = *reinterpret_cast<const uint2*>(sm + (g + 8) * kF8Pitch + kk);
+      const uint2 wa = *reinterpret_cast<const uint2*>(wt + g * kF8Pitch + kk);
+      const uint2 wb = *reinterpret_cast<const uint2*>(wt + (g + 8) * kF8Pitch + kk);
 #pragma unroll
       for (int s = 0; s < NS; ++s) {
         const int tok = 8 * s + g;
         uint2 xv = make_uint2(0u, 0u);
-        if (tok < M)
-          xv = __ldg(reinterpret_cast<const uint2*>(p.A + (size_t)tok * K + chunk * kF8K + kk));
+        if (tok < M) xv = *reinterpret_cast<const uint2*>(at + tok * kF8Pitch + kk);
         if (b == 0)
           ptx::mma_m16n8k32_e4m3_zero(cq[s], wa.x, wb.x, wa.y, wb.y, xv.x, xv.y);
         else
@@ -159,16 +173,24 @@ __global__ void __launch_bounds__(kF8Warps * 32) fp8_gemm_kernel(const Fp8Params
   if (lane == 0) p.cnt[unit] = 0;  // ready for the next launch on the stream
 }
 
+template <int NS, bool FUSED>
+cudaError_t launch_kern(const Fp8Params& prm, cudaStream_t s, bool overlap) {
+  const int units = FUSED ? prm.N / 8 : prm.N / 16;
+  const int ctas = units / kF8Warps * (prm.K / kF8K);
+  const size_t smem = (size_t)fp8_smem_bytes(prm.M);
+  auto kern = fp8_gemm_kernel<NS, FUSED>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(kern, dim3((unsigned)ctas), dim3(kF8Warps * 32), smem, s, overlap, prm);
+}
+
 template <bool FUSED>
 cudaError_t launch_ns(const Fp8Params& prm, int ns, cudaStream_t s, bool overlap) {
-  const int units = FUSED ? prm.N / 8 : prm.N / 16;
-  const int tasks = units * (prm.K / kF8K);
-  const dim3 grid((unsigned)((tasks + kF8Warps - 1) / kF8Warps)), block(kF8Warps * 32);
   switch (ns) {
-    case 1: return launch_pdl(fp8_gemm_kernel<1, FUSED>, grid, block, 0, s, overlap, prm);
-    case 2: return launch_pdl(fp8_gemm_kernel<2, FUSED>, grid, block, 0, s, overlap, prm);
-    case 4: return launch_pdl(fp8_gemm_kernel<4, FUSED>, grid, block, 0, s, overlap, prm);
-    default: return launch_pdl(fp8_gemm_kernel<8, FUSED>, grid, block, 0, s, overlap, prm);
+    case 1: return launch_kern<1, FUSED>(prm, s, overlap);
+    case 2: return launch_kern<2, FUSED>(prm, s, overlap);
+    case 4: return launch_kern<4, FUSED>(prm, s, overlap);
+    default: return launch_kern<8, FUSED>(prm, s, overlap);
   }
 }
 
@@ -177,13 +199,19 @@ int groups_for(int M) {
   return n <= 1 ? 1 : n <= 2 ? 2 : n <= 4 ? 4 : 8;
 }
 
+size_t part_bytes(int M, int N, int K, bool fused) {
+  const int units = fused ? N / 8 : N / 16;
+  return (size_t)units * (K / kF8K) * kF8Rows * (groups_for(M) * 8) * sizeof(float);
+}
+
 }  // namespace
 
 size_t fp8_gemm_ws_bytes(int M, int N, int K, bool fused) {
   const int units = fused ? N / 8 : N / 16;
-  const size_t part = (size_t)units * (K / kF8K) * kF8Rows * (groups_for(M) * 8) * sizeof(float);
-  return (part + 255) / 256 * 256 + (size_t)units * sizeof(int);
+  return (part_bytes(M, N, K, fused) + 255) / 256 * 256 + (size_t)units * sizeof(int);
 }
+
+size_t fp8_gemm_counters(int N, bool fused) { return (size_t)(fused ? N / 8 : N / 16); }
 
 cudaError_t launch_fp8_gemm(const Fp8Launch& a, cudaStream_t s) {
   Fp8Params p;
@@ -197,13 +225,12 @@ cudaError_t launch_fp8_gemm(const Fp8Launch& a, cudaStream_t s) {
   p.N = a.N;
   p.K = a.K;
   const bool fused = a.B1 != nullptr;
-  const int units = fused ? a.N / 8 : a.N / 16;
-  const size_t part = (size_t)units * (a.K / kF8K) * kF8Rows * (groups_for(a.M) * 8) * sizeof(float);
   p.part = reinterpret_cast<float*>(a.ws);
-  p.cnt = reinterpret_cast<int*>(a.ws + (part + 255) / 256 * 256);
+  p.cnt = a.cnt ? a.cnt
+                : reinterpret_cast<int*>(a.ws + (part_bytes(a.M, a.N, a.K, fused) + 255) / 256 * 256);
   p.C = a.C;
   if (a.zero_counters) {
-    cudaError_t e = cudaMemsetAsync(p.cnt, 0, (size_t)units * sizeof(int), s);
+    cudaError_t e = cudaMemsetAsync(p.cnt, 0, fp8_gemm_counters(a.N, fused) * sizeof(int), s);
     if (e != cudaSuccess) return e;
   }
   const int ns = groups_for(a.M);

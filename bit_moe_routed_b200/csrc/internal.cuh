@@ -213,10 +213,12 @@ struct Fp8Launch {
   int M, N, K;
   float* C;
   uint8_t* ws;
+  int* cnt;            // the row blocks' counters (NULL: at the end of ws)
   bool zero_counters;
   bool overlap;
 };
 size_t fp8_gemm_ws_bytes(int M, int N, int K, bool fused);
+size_t fp8_gemm_counters(int N, bool fused);  // counters (ints) a launch uses
 cudaError_t launch_fp8_gemm(const Fp8Launch& a, cudaStream_t s);
 // clears the single-token kernel's grid barrier (after a reported timeout)
 cudaError_t reset_grid_barrier();
