@@ -311,3 +311,47 @@ def moe_layer(x, E: int, k: int, d: int, f: int, experts: dict, idx: np.ndarray,
     lib().oracle_moe_layer(xb.ctypes.data, T, d, f, E, k, es.arr, pi, pw, y_pair.ctypes.data,
                            y_sh.ctypes.data, out.ctypes.data)
     return y_pair, y_sh, out
+
+
+# ---- expert cache (NEXT-4: routed experts streamed from host memory) -----------------
+def lru_cache_steps(selections, E: int, S: int):
+    """The expert cache's decisions over a sequence of steps, plainly: a cache of S slots,
+    each holding one routed expert or nothing; at step n (n = 1, 2, ...) the selected
+    experts, taken in ascending id, are first marked used (hits), then each expert not
+    resident gets the least recently used slot (smallest last-use step, ties to the lower
+    slot; empty slots count as never used) among the slots not holding an expert of this
+    step, whose expert is evicted.  (dpshk.com article, "核心实现一": experts are read as
+    they are needed and kept under an LRU share.)  Returns, per step, (hits, misses, fills)
+    with fills = [(expert, slot)], and the final (slot_of [E], expert_of [S], last_use [S]).
+    """
+    slot_of = [-1] * E
+    expert_of = [-1] * S
+    last_use = [0] * S
+    out = []
+    for n, sel in enumerate(selections, start=1):
+        sel = sorted(set(int(e) for e in sel))
+        hits, misses, fills = [], [], []
+        for e in sel:
+            if slot_of[e] >= 0:
+                last_use[slot_of[e]] = n
+                hits.append(e)
+        for e in sel:
+            if slot_of[e] >= 0:
+                continue
+            best = None
+            for s in range(S):
+                if expert_of[s] in sel:
+                    continue
+                if best is None or last_use[s] < last_use[best]:
+                    best = s
+            if best is None:
+                raise ValueError("fewer slots than selected experts")
+            if expert_of[best] >= 0:
+                slot_of[expert_of[best]] = -1
+            expert_of[best] = e
+            slot_of[e] = best
+            last_use[best] = n
+            misses.append(e)
+            fills.append((e, best))
+        out.append((hits, misses, fills))
+    return out, (slot_of, expert_of, last_use)
