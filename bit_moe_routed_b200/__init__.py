@@ -40,6 +40,7 @@ EXPORTS = (
     "moe_ffn_path", "moe_router_topk", "moe_dispatch_workspace_size", "moe_forward_q2",
     "moe_fp8_gemm", "moe_fp8_gemm_workspace_size", "moe_shared_expert_fp8",
     "moe_shared_expert_fp8_workspace_size", "moe_shared_expert_fp8_offsets",
+    "moe_expert_cache_reset", "moe_forward_streamed",
 )
 
 
@@ -111,6 +112,10 @@ def lib():
             "moe_shared_expert_fp8": [P, I, ctypes.POINTER(_Fp8Expert), P, P, Z, P],
             "moe_shared_expert_fp8_workspace_size": [I, I, I],
             "moe_shared_expert_fp8_offsets": [I, I, I, P],
+            "moe_expert_cache_reset": [ctypes.POINTER(_ExpertCache), P],
+            "moe_forward_streamed": [P, P, I, ctypes.POINTER(_HostExperts),
+                                     ctypes.POINTER(_ExpertCache), P, P, P, P, P, P, P, P, P,
+                                     P, Z, P],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -144,6 +149,16 @@ def _p(t: torch.Tensor | None):
 
 
 @dataclass
+class _HostExperts(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "gate_codes", "gate_scales", "up_codes", "up_scales", "down_codes", "down_scales")]
+
+
+class _ExpertCache(ctypes.Structure):
+    _fields_ = [("slots", _Weights)] + [(n, ctypes.c_void_p) for n in (
+        "slot_of", "expert_of", "last_use", "clock", "fetch", "stats")] + [("E", ctypes.c_int)]
+
+
 class LayerWeights:
     """One layer's FP4 weights on the device, E+1 experts (index E = shared).
 
@@ -272,6 +287,101 @@ def shared_expert_fp8_views(ws: torch.Tensor, T: int, d: int, f: int) -> dict:
     return {"qx": u8(off[0], T * d).view(T, d), "sx": f32(off[1], T * (d // 128)).view(T, -1),
             "h": f32(off[2], T * f).view(T, f), "qh": u8(off[3], T * f).view(T, f),
             "sh": f32(off[4], T * (f // 128)).view(T, -1)}
+
+
+_NAMES6 = ("gate_codes", "gate_scales", "up_codes", "up_scales", "down_codes", "down_scales")
+
+
+@dataclass
+class HostExperts:
+    """The E routed experts of a layer in pinned host memory (uint8 tensors with the
+    LayerWeights layout, [E, ...] per matrix), which the device reads through unified
+    addressing."""
+    gate_codes: torch.Tensor
+    gate_scales: torch.Tensor
+    up_codes: torch.Tensor
+    up_scales: torch.Tensor
+    down_codes: torch.Tensor
+    down_scales: torch.Tensor
+
+    def struct(self) -> _HostExperts:
+        return _HostExperts(*(getattr(self, n).data_ptr() for n in _NAMES6))
+
+    @staticmethod
+    def from_layer(w: "LayerWeights") -> "HostExperts":
+        """Pinned host copies of a device layer's routed experts (expert E excluded)."""
+        out = {}
+        for n in _NAMES6:
+            t = getattr(w, n)[:w.E]
+            h = torch.empty(t.shape, dtype=torch.uint8, pin_memory=True)
+            h.copy_(t)
+            out[n] = h
+        return HostExperts(**out)
+
+
+class ExpertCache:
+    """The HBM expert cache (moe_expert_cache_t): S + 1 slots (slot S holds the shared
+    expert), the expert/slot tables, the LRU clock and the hit/miss counters."""
+
+    def __init__(self, E: int, S: int, d: int, f: int, shared: "LayerWeights", device="cuda",
+                 stream=None):
+        self.E, self.S = E, S
+        shp = {"gate_codes": (f, d // 2), "gate_scales": (f, d // 32), "up_codes": (f, d // 2),
+               "up_scales": (f, d // 32), "down_codes": (d, f // 2), "down_scales": (d, f // 32)}
+        sl = {}
+        for n, (r, c) in shp.items():
+            t = torch.empty((S + 1, r, c), dtype=torch.uint8, device=device)
+            t[S].copy_(getattr(shared, n)[shared.E])  # the shared expert, resident
+            sl[n] = t
+        self.slots = LayerWeights(**sl)
+        i32, i64 = torch.int32, torch.int64
+        self.slot_of = torch.empty(E, dtype=i32, device=device)
+        self.expert_of = torch.empty(S, dtype=i32, device=device)
+        self.last_use = torch.empty(S, dtype=i64, device=device)
+        self.clock = torch.empty(1, dtype=i64, device=device)
+        self.fetch = torch.empty(1 + 2 * 32, dtype=i32, device=device)
+        self.stats = torch.empty(2, dtype=i64, device=device)
+        self.reset(stream)
+
+    def struct(self) -> _ExpertCache:
+        return _ExpertCache(self.slots.struct(), *(t.data_ptr() for t in (
+            self.slot_of, self.expert_of, self.last_use, self.clock, self.fetch, self.stats)),
+            self.E)
+
+    def reset(self, stream=None) -> None:
+        st = self.struct()
+        _check(lib().moe_expert_cache_reset(ctypes.byref(st), _stream(stream)))
+
+
+def forward_streamed(x: torch.Tensor, scores: torch.Tensor, k: int, host: HostExperts,
+                     cache: ExpertCache, ws: torch.Tensor | None = None, stream=None,
+                     outs: dict | None = None):
+    """One token through the layer with the routed experts streamed from host memory
+    through the cache (moe_forward_streamed); returns the dict of `forward`."""
+    T, d = x.shape
+    if T != 1:
+        raise ValueError("moe_forward_streamed takes one token")
+    E, f = cache.E, cache.slots.f
+    dev = x.device
+    if ws is None:
+        ws = alloc_workspace(1, k, E, d, f, dev)
+    o = dict(outs) if outs is not None else {}
+    shapes = {"idx": ((1, k), torch.int32), "w": ((1, k), torch.float32),
+              "counts": ((E,), torch.int32), "offsets": ((E + 1,), torch.int32),
+              "perm": ((k,), torch.int32), "pos": ((k,), torch.int32),
+              "y": ((k, d), torch.float32), "y_shared": ((1, d), torch.float32),
+              "out": ((1, d), torch.float32)}
+    for name, (shape, dtype) in shapes.items():
+        if name not in o:
+            o[name] = torch.empty(shape, dtype=dtype, device=dev)
+    hs, cs = host.struct(), cache.struct()
+    _check(lib().moe_forward_streamed(_p(scores), _p(x), k, ctypes.byref(hs), ctypes.byref(cs),
+                                      _p(o["idx"]), _p(o["w"]), _p(o["counts"]),
+                                      _p(o["offsets"]), _p(o["perm"]), _p(o["pos"]), _p(o["y"]),
+                                      _p(o["y_shared"]), _p(o["out"]), _p(ws), ws.numel(),
+                                      _stream(stream)))
+    return dict(idx=o["idx"], w=o["w"], counts=o["counts"], offsets=o["offsets"],
+                perm=o["perm"], pos=o["pos"], y=o["y"], y_shared=o["y_shared"], out=o["out"])
 
 
 def set_wait_limit_ns(n: int) -> None:

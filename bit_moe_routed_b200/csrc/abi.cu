@@ -918,6 +918,94 @@ int moe_shared_expert_fp8(const uint16_t* x_bf16, int T, const moe_fp8_expert_t*
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "shared expert fp8 launch");
 }
 
+int moe_expert_cache_reset(const moe_expert_cache_t* c, void* stream) {
+  if (!c || !c->slot_of || !c->expert_of || !c->last_use || !c->clock || !c->stats || !c->fetch)
+    return fail(MOE_ERR_INVALID_ARG, "NULL cache pointer");
+  if (c->E < 1 || c->slots.E < 1) return fail(MOE_ERR_INVALID_ARG, "E=%d, S=%d", c->E, c->slots.E);
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(c->slot_of, 0xFF, (size_t)c->E * sizeof(int32_t), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(c->expert_of, 0xFF, (size_t)c->slots.E * sizeof(int32_t), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(c->last_use, 0, (size_t)c->slots.E * sizeof(int64_t), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(c->clock, 0, sizeof(int64_t), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(c->stats, 0, 2 * sizeof(int64_t), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(c->fetch, 0, sizeof(int32_t), s);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "cache reset");
+}
+
+int moe_forward_streamed(const float* scores, const uint16_t* x_bf16, int k,
+                         const moe_host_experts_t* host, const moe_expert_cache_t* cache,
+                         int32_t* topk_idx, float* topk_w, int32_t* counts, int32_t* offsets,
+                         int32_t* perm, int32_t* pos, float* y_routed, float* y_shared,
+                         float* out, void* ws, size_t ws_bytes, void* stream) {
+  if (!host || !cache) return fail(MOE_ERR_INVALID_ARG, "NULL descriptor");
+  const moe_weights_t& sl = cache->slots;
+  const int E = cache->E, S = sl.E;
+  if (k < 1 || k > 32 || k > S || k > E)
+    return fail(MOE_ERR_INVALID_ARG, "k=%d outside [1, min(32, S=%d, E=%d)]", k, S, E);
+  // the routed view: E experts scored and routed, workspace laid out for them
+  moe_weights_t wr = sl;
+  wr.E = E;
+  FfnCtx c;
+  int rc = ffn_check(1, k, &wr, ws, ws_bytes, c);
+  if (rc) return rc;
+  if (!c.fused)
+    return fail(MOE_ERR_INVALID_ARG, "shape (k=%d, d=%d, f=%d) does not fit the single-token kernel",
+                k, sl.d, sl.f);
+  if (!host->gate_codes || !host->gate_scales || !host->up_codes || !host->up_scales ||
+      !host->down_codes || !host->down_scales || !cache->slot_of || !cache->expert_of ||
+      !cache->last_use || !cache->clock || !cache->fetch || !cache->stats)
+    return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  const uint8_t* src[6] = {host->gate_codes, host->gate_scales, host->up_codes, host->up_scales,
+                           host->down_codes, host->down_scales};
+  uint8_t* dst[6] = {const_cast<uint8_t*>(sl.gate_codes), const_cast<uint8_t*>(sl.gate_scales),
+                     const_cast<uint8_t*>(sl.up_codes), const_cast<uint8_t*>(sl.up_scales),
+                     const_cast<uint8_t*>(sl.down_codes), const_cast<uint8_t*>(sl.down_scales)};
+  const long long d = sl.d, f = sl.f;
+  const long long bytes[6] = {f * d / 2, f * d / 32, f * d / 2, f * d / 32, d * f / 2, d * f / 32};
+  for (int a = 0; a < 6; ++a) {
+    if (!aligned(src[a], 16) || !aligned(dst[a], 16))
+      return fail(MOE_ERR_INVALID_ARG, "expert arrays must be 16-byte aligned");
+    // the copy kernel reads the host arrays directly: they must be pinned host memory that
+    // the device addresses at the same pointer (unified addressing), not pageable memory
+    cudaPointerAttributes at{};
+    if (cudaPointerGetAttributes(&at, src[a]) != cudaSuccess || at.type != cudaMemoryTypeHost ||
+        at.devicePointer != src[a]) {
+      cudaGetLastError();
+      return fail(MOE_ERR_INVALID_ARG, "host expert array %d is not pinned, device-mapped memory", a);
+    }
+  }
+  if (!x_bf16 || !counts || !offsets || !perm || !pos || !y_routed || !y_shared || !out)
+    return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(x_bf16, 16) || !aligned(y_routed, 16) || !aligned(y_shared, 16) || !aligned(out, 16))
+    return fail(MOE_ERR_INVALID_ARG, "misaligned pointer");
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  rc = moe_route_topk(scores, 1, E, k, topk_idx, topk_w, stream);
+  if (rc) return rc;
+  cudaError_t e = launch_cache(topk_idx, k, S, cache->slot_of, cache->expert_of,
+                               reinterpret_cast<long long*>(cache->last_use),
+                               reinterpret_cast<long long*>(cache->clock), cache->fetch,
+                               reinterpret_cast<long long*>(cache->stats), c.di.status, s);
+  if (e == cudaSuccess) e = launch_fetch(src, dst, bytes, cache->fetch, c.di.sms, s);
+  if (e != cudaSuccess) return cuda_fail(e, "expert cache launch");
+  DecodeLaunch a = decode_args(k, &wr, c);
+  a.forward = true;
+  a.scores = scores;
+  a.x = x_bf16;
+  a.idx = topk_idx;
+  a.w_out = topk_w;
+  a.counts = counts;
+  a.offsets = offsets;
+  a.perm = perm;
+  a.pos = pos;
+  a.y_routed = y_routed;
+  a.y_shared = y_shared;
+  a.out = out;
+  a.slot_of = cache->slot_of;
+  a.maps_E = S;
+  e = launch_decode(a, s, c.di.sms);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "single-token streamed layer launch");
+}
+
 int moe_combine(const float* y_routed, const float* y_shared, const float* topk_w,
                 const int32_t* pos, int T, int k, int d, float* out, void* stream) {
   if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T=%d < 0", T);

@@ -110,6 +110,10 @@ struct DecodeParams {
   long long wait_ns;
   int* status;
   int stall;
+  // weight rows: expert e's are at slot_of[e] (the expert cache) or e; the shared expert's
+  // at sh_e (E, or the cache's slot count)
+  const int32_t* slot_of;
+  int sh_e;
 };
 
 // Shared memory: rings (codes, then scales), the phase-dependent area (phase 1: token as
@@ -367,11 +371,12 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
       const bool routed = locate(warp + q * kDcWarps, r1.ns, S1, S1q, ul, c);
       int e, uin;
       if (!routed) {
-        e = E;
+        e = p.sh_e;
         uin = r1.s_lo + ul;
       } else {
         const int ru = r1.r_lo + ul - r1.ns;
         e = slot_e[ru / upe1];
+        if (p.slot_of) e = p.slot_of[e];
         uin = ru % upe1;
       }
       if (RQ && routed) {
@@ -394,11 +399,12 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
       const bool routed = locate(warp + (q - q1) * kDcWarps, r2.ns, S2, S2q, ul, c);
       int e, uin;
       if (!routed) {
-        e = E;
+        e = p.sh_e;
         uin = r2.s_lo + ul;
       } else {
         const int ru = r2.r_lo + ul - r2.ns;
         e = slot_e[ru / upe2];
+        if (p.slot_of) e = p.slot_of[e];
         uin = ru % upe2;
       }
       const int row = e * d + uin * 16;
@@ -915,7 +921,8 @@ bool decode_fits(int k, int d, int f, int ctas, bool q2) {
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t s, int num_sms) {
   DecodeParams p;
   memset(&p, 0, sizeof(p));
-  const long long rows1 = (long long)(a.E + 1) * a.f, rows2 = (long long)(a.E + 1) * a.d;
+  const int maps_e = a.maps_E >= 0 ? a.maps_E : a.E;  // experts of the FP4 maps, shared last
+  const long long rows1 = (long long)(maps_e + 1) * a.f, rows2 = (long long)(maps_e + 1) * a.d;
   if (!make_code_map(&p.tm_gc, a.gate_codes, a.d / 2, rows1, 8) ||
       !make_byte_map(&p.tm_gs, a.gate_scales, a.d / 32, rows1, 16, 8) ||
       !make_code_map(&p.tm_uc, a.up_codes, a.d / 2, rows1, 8) ||
@@ -959,6 +966,8 @@ cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t s, int num_sms) {
   p.wait_ns = a.wait_ns;
   p.status = a.status;
   p.stall = a.stall;
+  p.slot_of = a.slot_of;
+  p.sh_e = maps_e;
   const int grid = num_sms < kMaxCtas ? num_sms : kMaxCtas;
   if (q2) {  // forward only
     if (!a.forward) return cudaErrorInvalidValue;

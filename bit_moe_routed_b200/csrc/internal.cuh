@@ -191,6 +191,10 @@ struct DecodeLaunch {
   const uint8_t* q2_up_scales = nullptr;
   const uint8_t* q2_down_codes = nullptr;
   const uint8_t* q2_down_scales = nullptr;
+  // expert cache: the FP4 arrays hold maps_E + 1 slots (the shared expert in the last);
+  // routed expert e's weights are in slot slot_of[e].  maps_E < 0: the plain layout.
+  const int32_t* slot_of = nullptr;
+  int maps_E = -1;
 };
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t s, int num_sms);
 size_t decode_smem_bytes(int d, int f, bool q2 = false);
@@ -220,6 +224,15 @@ struct Fp8Launch {
 size_t fp8_gemm_ws_bytes(int M, int N, int K, bool fused);
 size_t fp8_gemm_counters(int N, bool fused);  // counters (ints) a launch uses
 cudaError_t launch_fp8_gemm(const Fp8Launch& a, cudaStream_t s);
+// Expert cache (stream.cu): the LRU decisions of one token's step (one thread) and the
+// copy of the listed experts from host memory into their slots.  fetch = [count, then
+// (expert, slot) pairs]; stats = [hits, misses] accumulated.
+cudaError_t launch_cache(const int32_t* idx, int k, int S, int32_t* slot_of, int32_t* expert_of,
+                         long long* last_use, long long* clock, int32_t* fetch, long long* stats,
+                         int* status, cudaStream_t s);
+cudaError_t launch_fetch(const uint8_t* const src[6], uint8_t* const dst[6],
+                         const long long bytes[6], const int32_t* fetch, int num_sms,
+                         cudaStream_t s);
 // clears the single-token kernel's grid barrier (after a reported timeout)
 cudaError_t reset_grid_barrier();
 

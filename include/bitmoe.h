@@ -266,6 +266,61 @@ int moe_shared_expert_fp8_offsets(int T, int d, int f, size_t off[5]);
 int moe_shared_expert_fp8(const uint16_t* x_bf16, int T, const moe_fp8_expert_t* w,
                           float* y_shared, void* ws, size_t ws_bytes, void* stream);
 
+/* Expert streaming (NEXT-4, one GPU): routed experts that live in host memory
+ * ([P1] "DeepSeek-V4-Flash的可能性": routed experts in host RAM, the shared expert and
+ * attention resident; [P2] "核心实现一": experts streamed in as they are needed, kept
+ * under an LRU share).  The routed experts are in pinned host memory that the device can
+ * read (cudaHostAlloc, or cudaHostRegister with cudaHostRegisterMapped; pass the device
+ * pointers): the moe_weights_t layout for E experts, [E][...] per matrix, each array
+ * 16-byte aligned. */
+typedef struct {
+  const uint8_t* gate_codes;
+  const uint8_t* gate_scales;
+  const uint8_t* up_codes;
+  const uint8_t* up_scales;
+  const uint8_t* down_codes;
+  const uint8_t* down_scales;
+} moe_host_experts_t;
+
+/* The HBM expert cache, device memory owned by the caller:
+ *   slots      moe_weights_t of S + 1 expert slots (slots.E = S): slots 0..S-1 hold
+ *              routed experts, slot S the shared expert (the caller fills it once);
+ *   slot_of    [E] int32: slot of each routed expert, -1 when not resident;
+ *   expert_of  [S] int32: expert in each slot, -1 when empty;
+ *   last_use   [S] int64: step of each slot's last use;
+ *   clock      [1] int64: steps so far;
+ *   fetch      [1 + 2*32] int32 scratch: this step's fills (count, then expert, slot);
+ *   stats      [2] int64: hits and misses accumulated.
+ * E routed experts; k <= S. */
+typedef struct {
+  moe_weights_t slots;
+  int32_t* slot_of;
+  int32_t* expert_of;
+  int64_t* last_use;
+  int64_t* clock;
+  int32_t* fetch;
+  int64_t* stats;
+  int E;
+} moe_expert_cache_t;
+
+/* Empty cache: slot_of and expert_of to -1, last_use, clock and stats to 0 (enqueued). */
+int moe_expert_cache_reset(const moe_expert_cache_t* c, void* stream);
+
+/* moe_forward for one token with the routed experts streamed from `host` through the
+ * cache: the top-k of the scores (into topk_idx, topk_w), the cache's LRU step (the
+ * selected experts, ascending id, are marked used; each missing one takes the least
+ * recently used slot not holding an expert of this token, empty slots first, ties to the
+ * lower slot; its expert is evicted), the copy of the missing experts from host memory
+ * into their slots (a kernel reading the host arrays over PCIe), then the single-token
+ * layer kernel on the slots.  Outputs, workspace (moe_workspace_size(1, k, c->E, d, f))
+ * and rules as moe_forward at T = 1; results equal moe_forward's on resident weights bit
+ * for bit.  Everything is enqueued on `stream`; the host never waits. */
+int moe_forward_streamed(const float* scores, const uint16_t* x_bf16, int k,
+                         const moe_host_experts_t* host, const moe_expert_cache_t* c,
+                         int32_t* topk_idx, float* topk_w, int32_t* counts, int32_t* offsets,
+                         int32_t* perm, int32_t* pos, float* y_routed, float* y_shared,
+                         float* out, void* ws, size_t ws_bytes, void* stream);
+
 /* Step 8 — combine: out[t][m] = y_shared[t][m] + sum_{j<k} topk_w[t][j] *
  * y_routed[pos[t*k+j]][m], summed in fixed j order in fp32.
  *   y_routed [T*k][d], y_shared [T][d], topk_w [T][k], pos [T*k], out [T][d] fp32.
