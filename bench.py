@@ -586,6 +586,61 @@ def measure_shared_fp8(bm, dev, stream, T: int, hbm_peak: float, peak_kind: str,
                        "(mma.sync e4m3 on the codes, cp.async weight tiles)"}
 
 
+def measure_streamed(bm, dev, stream, S: int = 64, steps: int = 64, zipf_s: float = 1.0) -> dict:
+    """Decode T = 1 with the 256 routed experts in pinned host memory and an HBM cache of S
+    slots (moe_forward_streamed): `steps` tokens with Zipf(zipf_s) routing, one CUDA graph,
+    after as many untimed tokens to fill the cache.  Also the H2D copy rate of pinned host
+    memory (the bound of the fetches)."""
+    w = synth.WORKLOADS["decode_t1"]
+    E, k, d, f = w.E, w.k, w.d, w.f
+    W = bm.LayerWeights.from_dict(synth.device_layer_weights(w.seed(0), 0, E, d, f))
+    host = bm.HostExperts.from_layer(W)
+    cache = bm.ExpertCache(E, S, d, f, W)
+    del W
+    torch.cuda.empty_cache()
+    ws = bm.alloc_workspace(1, k, E, d, f, dev)
+    xs = [synth.gen_x(1, d, seed=9000 + i).to(dev) for i in range(2 * steps)]
+    ss = [synth.gen_scores_zipf(1, E, zipf_s, seed=9000 + i).to(dev) for i in range(2 * steps)]
+    outs = None
+    with torch.cuda.stream(stream):
+        for i in range(steps):  # untimed: fill the cache
+            outs = bm.forward_streamed(xs[i], ss[i], k, host, cache, ws, stream, outs=outs)
+    bm.sync_status(stream)
+    st0 = cache.stats.cpu().tolist()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(steps, 2 * steps):
+            bm.forward_streamed(xs[i], ss[i], k, host, cache, ws, stream, outs=outs)
+    ms = time_graph(g, stream, 1)[0]
+    bm.sync_status(stream)
+    st1 = cache.stats.cpu().tolist()
+    hits, misses = st1[0] - st0[0], st1[1] - st0[1]
+    per_expert = synth.expert_bytes(d, f)
+    # pinned host -> device copy rate, 1 GiB (the PCIe bound of the fetches)
+    hb = torch.empty(1 << 30, dtype=torch.uint8, pin_memory=True)
+    db = torch.empty(1 << 30, dtype=torch.uint8, device=dev)
+    with torch.cuda.stream(stream):
+        db.copy_(hb, non_blocking=True)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        db.copy_(hb, non_blocking=True)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    h2d = (1 << 30) / (e0.elapsed_time(e1) / 1000.0) / 1e9
+    s_step = ms / 1000.0 / steps
+    fetched = misses * per_expert / steps
+    del g, hb, db, host, cache
+    torch.cuda.empty_cache()
+    return {"T": 1, "E": E, "k": k, "d": d, "f": f, "slots": S, "zipf_s": zipf_s,
+            "steps": steps, "ms_per_step": ms / steps, "value": 1.0 / s_step,
+            "unit": "tokens/s", "hit_rate": hits / max(hits + misses, 1),
+            "fetched_bytes_per_step": fetched, "fetch_gb_per_s": fetched / s_step / 1e9,
+            "h2d_copy_gb_per_s": h2d, "frac_of_h2d_copy": fetched / s_step / 1e9 / h2d,
+            "launches_per_step": 4,
+            "how": "route, cache (LRU), fetch (host-mapped reads) and the single-token layer "
+                   "kernel per token, in one CUDA graph; the H2D rate is a 1 GiB pinned copy"}
+
+
 def e2e(bm, Ls, args, dev, stream, dist, world):
     """The same metric through the public API with host buffers: each step copies x and the
     scores from pinned host memory, runs the four calls and copies the output back, then
@@ -685,6 +740,9 @@ def run_gpu(args, w):
             import gc
             gc.collect()
             torch.cuda.synchronize()
+            torch.cuda.empty_cache()
+        if args.workloads == "all" or "streamed" in args.workloads:
+            workloads["streamed_t1"] = measure_streamed(bm, dev, stream)
             torch.cuda.empty_cache()
         if args.workloads == "all" or "shared_fp8" in args.workloads:
             for Tf in (1, 64):  # NEXT-3: the FP8-weight shared expert on fp8_gemm

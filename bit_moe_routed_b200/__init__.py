@@ -148,7 +148,6 @@ def _p(t: torch.Tensor | None):
     return ctypes.c_void_p(t.data_ptr())
 
 
-@dataclass
 class _HostExperts(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "gate_codes", "gate_scales", "up_codes", "up_scales", "down_codes", "down_scales")]
@@ -159,6 +158,7 @@ class _ExpertCache(ctypes.Structure):
         "slot_of", "expert_of", "last_use", "clock", "fetch", "stats")] + [("E", ctypes.c_int)]
 
 
+@dataclass
 class LayerWeights:
     """One layer's FP4 weights on the device, E+1 experts (index E = shared).
 

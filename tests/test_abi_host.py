@@ -104,3 +104,20 @@ def test_gemv_switch_host(L):
     two = bm.workspace_size(2, 6, 256, 4096, 2048)
     assert one >= 7 * 2048 * 4
     assert two > 0
+
+
+def test_binding_descriptors_marshal_on_the_host():
+    """The binding's weight descriptors build their C structs from tensors (no GPU)."""
+    import torch
+    import bit_moe_routed_b200 as bm
+    E, d, f = 3, 512, 256
+    mk = lambda *s: torch.zeros(s, dtype=torch.uint8)  # noqa: E731
+    w = bm.LayerWeights(mk(E + 1, f, d // 2), mk(E + 1, f, d // 32), mk(E + 1, f, d // 2),
+                        mk(E + 1, f, d // 32), mk(E + 1, d, f // 2), mk(E + 1, d, f // 32))
+    st = w.struct()
+    assert (w.E, w.d, w.f) == (E, d, f) and (st.E, st.d, st.f) == (E, d, f)
+    q = bm.Q2Experts(mk(E, f, d // 4), mk(E, f, d // 128), mk(E, f, d // 4), mk(E, f, d // 128),
+                     mk(E, d, f // 4), mk(E, d, f // 128))
+    assert q.struct().gate_codes == q.gate_codes.data_ptr()
+    h = bm.HostExperts(*(getattr(w, n)[:E] for n in bm._NAMES6))
+    assert h.struct().down_scales == w.down_scales.data_ptr()
