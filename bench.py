@@ -495,6 +495,12 @@ def measure(bm, w, args, dev, stream, rank, dist, steps, warmup, peaks, cpu_seco
         kernel_name = ("decode_kernel: the whole layer in one cooperative kernel (routing, "
                        "dispatch, quantisation, FP4 GEMVs with in-register e2m1 decode and "
                        "mma.sync, combine)")
+        if not q2 and bm.forward_path(1, k, Ls.items[0]["W"]) == bm.PATH_SINGLE_TC:
+            kernel_file = os.path.join(ROOT, "bit_moe_routed_b200", "csrc", "decode_tc.cu")
+            kernel_name = ("decode_tc_kernel: the whole layer in one cooperative kernel "
+                           "(routing, dispatch, quantisation, tcgen05 block-scaled FP4 x e4m3 "
+                           "MMAs on TMA-unpacked codes against block-diagonal token tiles, "
+                           "combine)")
         if q2:
             kernel_name = ("decode_kernel, Q2 form: the whole layer in one cooperative kernel, "
                            "2-bit routed experts (byte-permute decode to e4m3, mma.sync e4m3) "

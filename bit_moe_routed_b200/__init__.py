@@ -28,7 +28,7 @@ MOE_ERR_WORKSPACE = -2
 MOE_ERR_CUDA = -3
 MOE_ERR_TIMEOUT = -4
 MOE_ERR_UNSUPPORTED = -5
-PATH_TILES, PATH_SINGLE, PATH_BATCHED = 0, 1, 2
+PATH_TILES, PATH_SINGLE, PATH_BATCHED, PATH_SINGLE_TC = 0, 1, 2, 3
 MOE_NOALLOC_SCRATCH_BYTES = 24 << 20  # the fixed scratch of moe_expert_ffn_noalloc
 GEMV_MAX_TOKENS = 64                  # default of moe_set_gemv_max_tokens
 
@@ -37,6 +37,7 @@ EXPORTS = (
     "moe_ffn_gate_up", "moe_ffn_down", "moe_combine", "moe_workspace_size", "moe_last_error",
     "moe_set_wait_limit_ns", "moe_sync_status", "moe_expert_ffn_noalloc",
     "moe_set_gemv_max_tokens", "moe_workspace_offsets", "moe_set_test_stall", "moe_forward",
+    "moe_set_decode_engine", "moe_forward_path",
     "moe_ffn_path", "moe_router_topk", "moe_dispatch_workspace_size", "moe_forward_q2",
     "moe_fp8_gemm", "moe_fp8_gemm_workspace_size", "moe_shared_expert_fp8",
     "moe_shared_expert_fp8_workspace_size", "moe_shared_expert_fp8_offsets",
@@ -99,6 +100,8 @@ def lib():
             "moe_sync_status": [P],
             "moe_expert_ffn_noalloc": [P, I, I, W, P, P, P, P, P],
             "moe_set_gemv_max_tokens": [I],
+            "moe_set_decode_engine": [I],
+            "moe_forward_path": [I, I, W],
             "moe_workspace_offsets": [I, I, I, I, I, P],
             "moe_set_test_stall": [I],
             "moe_forward": [P, P, I, I, W, P, P, P, P, P, P, P, P, P, P, Z, P],
@@ -399,12 +402,28 @@ def set_gemv_max_tokens(t: int) -> None:
     _check(lib().moe_set_gemv_max_tokens(int(t)))
 
 
+def set_decode_engine(engine: int) -> None:
+    """The single-token layer kernel of moe_forward: 0 (the default) on the CUDA cores, 1 on
+    the tensor cores where the shapes allow it."""
+    _check(lib().moe_set_decode_engine(int(engine)))
+
+
 def sync_status(stream=None) -> None:
     _check(lib().moe_sync_status(_stream(stream)))
 
 
 def workspace_size(T: int, k: int, E: int, d: int, f: int) -> int:
     return int(lib().moe_workspace_size(T, k, E, d, f))
+
+
+def forward_path(T: int, k: int, w: "LayerWeights") -> int:
+    """ffn_path for moe_forward: PATH_SINGLE_TC where the single-token layer kernel runs on
+    the tensor cores."""
+    st = w.struct()
+    rc = lib().moe_forward_path(T, k, ctypes.byref(st))
+    if rc < 0:
+        _check(rc)
+    return rc
 
 
 def ffn_path(T: int, k: int, w: "LayerWeights") -> int:

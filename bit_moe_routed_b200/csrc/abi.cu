@@ -31,6 +31,7 @@ struct OverlapScope {
 std::atomic<long long> g_wait_ns{2000000000LL};
 std::atomic<int> g_gemv_max_t{kBgMaxT};  // batches up to this size take a GEMV path
 std::atomic<int> g_stall{0};                 // test knob: see moe_set_test_stall
+std::atomic<int> g_decode_engine{0};         // see moe_set_decode_engine
 
 int fail(int code, const char* fmt, ...) {
   char buf[512];
@@ -199,6 +200,9 @@ WorkspaceLayout workspace_layout(int T, int k, int E, int d, int f) {
   // the combine counters of the single-token kernel (one per 16 output rows)
   L.done2 = o;
   if (T <= kGemvMaxT) o = align256(o + 4 * (size_t)(d / 16));
+  // the pieces and counters of the tensor-core single-token kernel
+  L.dtc = o;
+  if (T <= kGemvMaxT) o = align256(o + decode_tc_ws_bytes(k, d, f));
   // the multi-CTA dispatch's counts (moe_forward on large batches)
   L.dispatch = o;
   o = align256(o + dispatch_ws_bytes(T, k, E));
@@ -221,6 +225,12 @@ int moe_set_wait_limit_ns(long long n) {
 
 int moe_set_test_stall(int on) {
   g_stall.store(on ? 1 : 0);
+  return MOE_OK;
+}
+
+int moe_set_decode_engine(int engine) {
+  if (engine != 0 && engine != 1) return fail(MOE_ERR_INVALID_ARG, "engine=%d is not 0 or 1", engine);
+  g_decode_engine.store(engine);
   return MOE_OK;
 }
 
@@ -270,6 +280,7 @@ int moe_sync_status(void* stream) {
     if (host & kStatusTimeout) {
       // a CTA that gave up may have left the single-token kernel's grid barrier mid-count
       e = reset_grid_barrier();
+      if (e == cudaSuccess) e = reset_tc_barrier();
       if (e != cudaSuccess) return cuda_fail(e, "reset grid barrier");
       return fail(MOE_ERR_TIMEOUT, "a device-side wait exceeded its limit (status 0x%x)", host);
     }
@@ -367,6 +378,7 @@ struct FfnCtx {
   bool bg;     // batched GEMV path (bgemv.cu) instead of the tcgen05 tiles (ffn.cu)
   bool gemv;   // single-token GEMV path (gemv.cu) instead of the tcgen05 tiles (ffn.cu)
   bool fused;  // ... in one cooperative kernel (decode.cu), for the whole-call entry points
+  bool tc;     // ... whose forward form runs on the tensor cores (decode_tc.cu)
   uint8_t* ws;
 };
 
@@ -423,6 +435,8 @@ int ffn_check(int T, int k, const moe_weights_t* w, void* ws, size_t ws_bytes, F
   const int ctas = c.di.sms < kMaxCtas ? c.di.sms : kMaxCtas;
   c.fused = c.gemv && decode_fits(k, w->d, w->f, ctas) &&
             decode_smem_bytes(w->d, w->f) <= (size_t)max_smem;
+  c.tc = c.fused && g_decode_engine.load() == 1 && decode_tc_fits(k, w->d, w->f, ctas) &&
+         decode_tc_smem_bytes(w->d, w->f) <= (size_t)max_smem;
   return MOE_OK;
 }
 
@@ -620,6 +634,7 @@ DecodeLaunch decode_args(int k, const moe_weights_t* w, const FfnCtx& c) {
   a.sh = reinterpret_cast<float*>(c.ws + c.L.sh);
   a.hbuf = reinterpret_cast<float*>(c.ws + c.L.hbuf);
   a.done2 = reinterpret_cast<int*>(c.ws + c.L.done2);
+  a.tc_ws = c.tc ? c.ws + c.L.dtc : nullptr;
   a.E = w->E;
   a.k = k;
   a.d = w->d;
@@ -639,6 +654,14 @@ int moe_ffn_path(int T, int k, const moe_weights_t* w) {
   if (T == 1 && c.fused) return MOE_PATH_SINGLE;
   if (c.bg) return MOE_PATH_BATCHED;
   return MOE_PATH_TILES;
+}
+
+int moe_forward_path(int T, int k, const moe_weights_t* w) {
+  FfnCtx c;
+  const int rc = ffn_check(T, k, w, nullptr, (size_t)-1, c);
+  if (rc) return rc;
+  if (T == 1 && c.fused && c.tc && k <= 32) return MOE_PATH_SINGLE_TC;
+  return moe_ffn_path(T, k, w);
 }
 
 int moe_expert_ffn(const uint16_t* x_bf16, int T, int k, const moe_weights_t* w,

@@ -52,6 +52,7 @@
 // takes part in the grid barrier and returns.
 #include "internal.cuh"
 #include "ptx.cuh"
+#include "single_token.cuh"
 #include "waits.cuh"
 
 #include <cstring>
@@ -195,26 +196,6 @@ __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long
   asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
   return v;
 }
-
-// One CTA's share of a phase.  A shared unit weighs wsh (1; 2 in the Q2 form, where it
-// has twice the stages of a routed unit), a routed unit 1: M = (n_routed + wsh) * upe in
-// all, CTA b taking the weight range [b*M/G, (b+1)*M/G).  Its first ns units are the
-// shared expert's [s_lo, s_lo+ns) (s_lo = b*upe/G, a share that does not depend on the
-// routing), the rest the routed units [r_lo, r_lo+nr) of the list that runs over the
-// active routed experts in slot order (r_lo = b*M/G - wsh*s_lo).
-struct Range {
-  int s_lo, ns, r_lo, nr, upe;
-  __host__ __device__ Range(int upe_, int n_routed, int G, int b, int wsh) {
-    upe = upe_;
-    s_lo = (int)((long long)b * upe / G);
-    ns = (int)((long long)(b + 1) * upe / G) - s_lo;
-    const long long M = (long long)(n_routed + wsh) * upe;
-    const long long t_lo = b * M / G, t_hi = (b + 1) * M / G;
-    r_lo = (int)(t_lo - (long long)wsh * s_lo);
-    nr = (int)(t_hi - t_lo) - wsh * ns;
-  }
-  __host__ __device__ int units() const { return ns + nr; }
-};
 
 // The bounded grid barrier (see g_grid_bar); false if the wait ran out.  ok_s: a word of
 // shared memory that carries thread 0's result to the CTA.  The CTA barrier orders the
@@ -431,67 +412,9 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
   // ---------------------------------------------------------------- routing / plan
   if (warp == 0) {
     if (MODE == kModeForward) {
-      // top-k of the E scores (each lane holds experts lane + 32 i): k rounds of a warp
-      // arg-max on (value desc, index asc), as a max of order-preserving integer keys and
-      // then a min of the indices holding it (two warp reductions a round); then
-      // w_j = sigmoid(s_j) / sum over the k
-      float v[PL];
-#pragma unroll
-      for (int i = 0; i < PL; ++i) {
-        const int e = lane + 32 * i;
-        v[i] = e < E ? __ldg(p.scores + e) : -INFINITY;
-      }
-      // keys: a larger score has a larger key (sign-magnitude to offset order); NaN and
-      // padding get 0, below every number, so they are taken only after all numbers
-      uint32_t key[PL];
-#pragma unroll
-      for (int i = 0; i < PL; ++i) {
-        const uint32_t u = __float_as_uint(v[i] == 0.f ? 0.f : v[i]);  // -0 ties +0
-        key[i] = (v[i] != v[i] || lane + 32 * i >= E) ? 0u : ((u & 0x80000000u) ? ~u : (u | 0x80000000u));
-      }
-      unsigned taken = 0;
-      float sel_v = 0.f;
-      int sel_i = 0;
-      for (int j = 0; j < k; ++j) {
-        uint32_t bk = 0u, bidx = 0xFFFFFFFFu;
-#pragma unroll
-        for (int i = 0; i < PL; ++i) {
-          if (!((taken >> i) & 1u) && (key[i] > bk || bidx == 0xFFFFFFFFu)) {
-            bk = key[i];
-            bidx = (uint32_t)(lane + 32 * i);
-          }
-        }
-        const uint32_t kmax = __reduce_max_sync(0xffffffffu, bk);
-        const uint32_t imin = __reduce_min_sync(0xffffffffu, bk == kmax ? bidx : 0xFFFFFFFFu);
-        if ((int)(imin & 31u) == lane) taken |= 1u << (imin >> 5);
-        if (lane == j) {
-          sel_v = __uint_as_float((kmax & 0x80000000u) ? (kmax ^ 0x80000000u) : ~kmax);
-          sel_i = (int)imin;
-        }
-      }
-      const float sig = lane < k ? 1.0f / (1.0f + expf(-sel_v)) : 0.0f;
-      float sum = sig;
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-      // slot (= sorted position) of pair j: the number of selected experts below it
-      int rank = 0;
-      for (int j = 0; j < k; ++j) {
-        const int ej = __shfl_sync(0xffffffffu, sel_i, j);
-        rank += (lane < k && ej < sel_i) ? 1 : 0;
-      }
-      if (lane < k) {
-        slot_e[rank] = sel_i;
-        slot_row[rank] = rank;
-        slot_n[rank] = 1;
-        pair_w[lane] = sig / sum;
-        pair_pos[lane] = rank;
-        if (b == 0) {
-          p.idx[lane] = sel_i;
-          p.w[lane] = sig / sum;
-          p.perm[rank] = lane;
-          p.pos[lane] = rank;
-        }
-      }
+      // top-k of the E scores and the gate weights; CTA 0 stores them with the dispatch
+      route_token_warp<PL>(p.scores, E, k, lane, slot_e, slot_row, slot_n, pair_w, pair_pos,
+                           b == 0 ? p.idx : nullptr, p.w, p.perm, p.pos);
       if (lane == 0) *n_active = k;
     } else {
       // active experts from the dispatch offsets, ascending: (expert, first row, rows)
@@ -919,6 +842,8 @@ bool decode_fits(int k, int d, int f, int ctas, bool q2) {
 }
 
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t s, int num_sms) {
+  if (a.forward && a.q2_gate_codes == nullptr && a.tc_ws != nullptr)
+    return launch_decode_tc(a, s, num_sms);
   DecodeParams p;
   memset(&p, 0, sizeof(p));
   const int maps_e = a.maps_E >= 0 ? a.maps_E : a.E;  // experts of the FP4 maps, shared last

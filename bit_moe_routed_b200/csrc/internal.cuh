@@ -42,7 +42,7 @@ constexpr int kBgMaxT = 64;
 constexpr int kBgSlotTokens = 8;  // tokens per slot of the batched GEMV (the MMA's N)
 
 struct WorkspaceLayout {
-  size_t plan, qx, sx, qh, sh, counters, partials, hbuf, done2, dispatch, total;
+  size_t plan, qx, sx, qh, sh, counters, partials, hbuf, done2, dtc, dispatch, total;
   size_t n_counters;
 };
 WorkspaceLayout workspace_layout(int T, int k, int E, int d, int f);
@@ -195,8 +195,18 @@ struct DecodeLaunch {
   // routed expert e's weights are in slot slot_of[e].  maps_E < 0: the plain layout.
   const int32_t* slot_of = nullptr;
   int maps_E = -1;
+  // forward, FP4: the tensor-core form of the kernel (decode_tc.cu) runs with this
+  // workspace region (decode_tc_ws_bytes); NULL: the CUDA-core form (decode.cu)
+  uint8_t* tc_ws = nullptr;
 };
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t s, int num_sms);
+cudaError_t launch_decode_tc(const DecodeLaunch& a, cudaStream_t s, int num_sms);
+// whether the tensor-core single-token kernel takes (k, d, f) on `ctas` CTAs, its shared
+// memory and its workspace region
+bool decode_tc_fits(int k, int d, int f, int ctas);
+size_t decode_tc_smem_bytes(int d, int f);
+size_t decode_tc_ws_bytes(int k, int d, int f);
+cudaError_t reset_tc_barrier();
 size_t decode_smem_bytes(int d, int f, bool q2 = false);
 // whether the single-token kernel's per-CTA limits hold for (k, d, f) on `ctas` CTAs
 // (q2: with 2-bit routed experts)

@@ -369,6 +369,20 @@ int moe_set_wait_limit_ns(long long n);
  * Applies to calls made after it. */
 int moe_set_gemv_max_tokens(int t);
 
+/* Which form of the single-token layer kernel moe_forward (T = 1) and
+ * moe_forward_streamed run; the pages have no counterpart (tcti.cn post, "DeepSeek-V4-
+ * Flash的可能性": decode is bound by reading the selected experts' weights; both forms
+ * read each weight byte once and compute the same layer).  0 (the default): on the CUDA
+ * cores (e2m1 decoded to f16 in registers, mma.sync), the faster form on a B200 at the
+ * decode sizes.  1: on the tensor cores (tcgen05.mma kind::mxf8f6f4.block_scale on the
+ * FP4 codes, unpacked by TMA) where the shapes allow it: d and f multiples of 256 and at
+ * most 4096, f such that three experts' h tiles fit in shared memory, k <= 32; other
+ * shapes stay on the CUDA cores.  Results of the two forms agree within the
+ * floating-point bounds of the parity rules, not bit for bit (their fp32 sums run in
+ * different orders); each form is deterministic.  Returns MOE_ERR_INVALID_ARG for other
+ * values.  Applies to calls made after it. */
+int moe_set_decode_engine(int engine);
+
 /* Testing knob; the pages have no counterpart.  While on, every launch of the
  * single-token FFN kernels makes warp 0 of CTA 0 wait, before its first weight stage, on
  * a shared-memory barrier that nothing completes, so that the wait's time limit
@@ -387,6 +401,12 @@ int moe_set_test_stall(int on);
 #define MOE_PATH_SINGLE 1
 #define MOE_PATH_BATCHED 2
 int moe_ffn_path(int T, int k, const moe_weights_t* w);
+
+/* The same for moe_forward, under the current moe_set_decode_engine as well: as
+ * moe_ffn_path, except MOE_PATH_SINGLE_TC where the single-token layer kernel runs on the
+ * tensor cores. */
+#define MOE_PATH_SINGLE_TC 3
+int moe_forward_path(int T, int k, const moe_weights_t* w);
 
 /* Synchronise `stream`, then return MOE_ERR_CUDA for a pending CUDA error,
  * MOE_ERR_TIMEOUT if a device-side wait expired since the last call (clearing the

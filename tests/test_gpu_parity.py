@@ -239,12 +239,15 @@ def test_gemv_single_token_shapes(E, k, d, f, calls):
 
 
 def test_single_token_paths_agree_bit_for_bit():
-    """One token through moe_forward (one kernel), the four calls (the FFN as one kernel),
-    and the three exposed FFN stages (two GEMV kernels): identical results."""
+    """One token through moe_forward (one kernel, its CUDA-core form), the four calls (the
+    FFN as one kernel), and the three exposed FFN stages (two GEMV kernels): identical
+    results.  (The tensor-core form of moe_forward sums in another order: its own tests
+    are in test_gpu_decode_tc.py.)"""
     E, k, d, f = 256, 6, 4096, 2048
     x = synth.gen_x(1, d, seed=61)
     s = synth.gen_scores_uniform(1, E, seed=62)
     W = device_weights(63, 0, E, d, f)
+    bm.set_decode_engine(0)  # the default
     a = gpu_layer(x, s, k, W)
     b = gpu_layer(x, s, k, W, calls=True)
     xd, sd = x.cuda(), s.cuda()

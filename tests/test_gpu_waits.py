@@ -66,11 +66,14 @@ def test_gemv_tiny_wait_limit_reports_or_completes():
     check_layer(g, x, s, k, E, d, f, 513, 0, [0], "after the tiny limit")
 
 
-def test_single_token_stall_times_out_and_recovers():
+@pytest.mark.parametrize("engine", [0, 1], ids=["cuda_cores", "tensor_cores"])
+def test_single_token_stall_times_out_and_recovers(engine):
     """The test stall makes one warp's bounded wait run out on every call: the status must
-    report MOE_ERR_TIMEOUT each time, and the next normal call must be correct."""
+    report MOE_ERR_TIMEOUT each time, and the next normal call must be correct (both forms
+    of the single-token kernel)."""
     if not torch.cuda.is_available():
         pytest.skip("no GPU")
+    bm.set_decode_engine(engine)
     T, E, k, d, f = 1, 64, 6, 4096, 2048
     x = synth.gen_x(T, d, seed=521)
     s = synth.gen_scores_uniform(T, E, seed=522)
@@ -88,5 +91,8 @@ def test_single_token_stall_times_out_and_recovers():
         bm.set_test_stall(False)
         bm.set_wait_limit_ns(0)
     bm.sync_status()
-    g = gpu_layer(x, s, k, W)
+    try:
+        g = gpu_layer(x, s, k, W)
+    finally:
+        bm.set_decode_engine(0)  # the default
     check_layer(g, x, s, k, E, d, f, 523, 0, [0], "after the stall")
