@@ -280,7 +280,7 @@ int moe_sync_status(void* stream) {
     if (host & kStatusTimeout) {
       // a CTA that gave up may have left the single-token kernel's grid barrier mid-count
       e = reset_grid_barrier();
-      if (e == cudaSuccess) e = reset_tc_barrier();
+      if (e == cudaSuccess) e = reset_tc_barrier(di.sms < kMaxCtas ? di.sms : kMaxCtas);
       if (e != cudaSuccess) return cuda_fail(e, "reset grid barrier");
       return fail(MOE_ERR_TIMEOUT, "a device-side wait exceeded its limit (status 0x%x)", host);
     }

@@ -61,11 +61,11 @@
 namespace bitmoe {
 
 // Grid barrier of the single-token kernel, one per device (zero when the module loads):
-// high word = generation, low word = CTAs arrived in the current generation.  The last
-// CTA to arrive adds 2^32 - G, which clears the count and opens the next generation.  It
-// serves one launch at a time: a launch holds every SM (one CTA per SM, by its shared
-// memory) until all its CTAs have passed the barrier, so a later launch's CTAs cannot
-// arrive before the barrier has opened.
+// the count of CTA arrivals, a multiple of G between barriers.  A CTA that adds 1 to n
+// waits until the count reaches the next multiple of G above n, so the last arrival's own
+// add opens the barrier (one atomic round trip).  It serves one launch at a time: a launch
+// holds every SM (one CTA per SM, by its shared memory) until all its CTAs have passed the
+// barrier, so a later launch's CTAs cannot arrive before the barrier has opened.
 __device__ unsigned long long g_grid_bar;
 
 namespace {
@@ -200,21 +200,18 @@ __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long
 // The bounded grid barrier (see g_grid_bar); false if the wait ran out.  ok_s: a word of
 // shared memory that carries thread 0's result to the CTA.  The CTA barrier orders the
 // CTA's writes before thread 0's arrival, an acq_rel atomic that releases them at GPU
-// scope; the last arrival (acq_rel: it has acquired every other arrival) opens the next
-// generation, and the waiters' acquire loads of it order their later reads after all
-// arrivals.
+// scope; the arrivals form one release sequence, so a waiter's acquire load that sees the
+// last arrival's count orders its later reads after every arrival.
 __device__ bool grid_barrier(long long limit, int* status, volatile int* ok_s) {
   __syncthreads();
   if (threadIdx.x == 0) {
     int ok = 1;
     const unsigned long long G = gridDim.x;
     const unsigned long long old = atom_add_acq_rel_u64(&g_grid_bar, 1ull);
-    const unsigned long long gen = old >> 32;
-    if ((old & 0xffffffffull) + 1 == G) {
-      atom_add_acq_rel_u64(&g_grid_bar, (1ull << 32) - G);
-    } else {
+    const unsigned long long target = (old / G + 1) * G;
+    if (old + 1 != target) {
       const uint64_t t0 = ptx::globaltimer();
-      while ((ld_acquire_u64(&g_grid_bar) >> 32) == gen) {
+      while (ld_acquire_u64(&g_grid_bar) < target) {
         if ((long long)(ptx::globaltimer() - t0) > limit) {
           atomicOr(status, kStatusTimeout);
           ok = 0;

@@ -69,13 +69,13 @@
 
 namespace bitmoe {
 
-// Grid barrier of this kernel, one per device (zero when the module loads): high word =
-// generation, low word = CTAs arrived.  As in decode.cu, it serves one launch at a time
-// (every CTA holds a whole SM until all have passed it); a launch passes it twice.  Its
-// generation also tags the workspace's piece flags: every launch reads it at entry (all
-// CTAs read the same value, as the previous launch on the stream has ended and this one's
-// barrier cannot open before every CTA has arrived), so a flag an earlier launch left
-// behind does not match.
+// Grid barrier of this kernel, one per device (zero when the module loads): the count of
+// CTA arrivals, a multiple of G between barriers, as in decode.cu (the last arrival's add
+// opens the barrier); it serves one launch at a time (every CTA holds a whole SM until all
+// have passed it), and a launch passes it twice.  The count at entry also tags the
+// workspace's piece flags: all CTAs read the same value (the previous launch on the stream
+// has ended and this one's first barrier cannot open before every CTA has arrived), and it
+// grows with every launch, so a flag an earlier launch left behind does not match.
 __device__ unsigned long long g_tc_bar;
 
 namespace {
@@ -270,20 +270,19 @@ __device__ __forceinline__ void reg_fence(float (&v)[N]) {
 
 // The bounded grid barrier, run by the 128 epilogue threads (et: 0..127); the other warps
 // keep streaming.  The named barrier orders the group's writes before thread 0's
-// acq_rel arrival, which releases them at GPU scope; the last arrival opens the next
-// generation, and the waiters' acquire loads order their later reads after all arrivals.
+// acq_rel arrival, which releases them at GPU scope; the arrivals form one release
+// sequence, so a waiter's acquire load that sees the last arrival's count orders its later
+// reads after every arrival.
 __device__ bool tc_grid_barrier(long long limit, int* status, volatile int* ok_s, int et) {
   bar_sync(1, 128);
   if (et == 0) {
     int ok = 1;
     const unsigned long long G = gridDim.x;
     const unsigned long long old = atom_add_acq_rel_u64(&g_tc_bar, 1ull);
-    const unsigned long long gen = old >> 32;
-    if ((old & 0xffffffffull) + 1 == G) {
-      atom_add_acq_rel_u64(&g_tc_bar, (1ull << 32) - G);
-    } else {
+    const unsigned long long target = (old / G + 1) * G;
+    if (old + 1 != target) {
       const uint64_t t0 = ptx::globaltimer();
-      while ((ld_acquire_u64(&g_tc_bar) >> 32) == gen) {
+      while (ld_acquire_u64(&g_tc_bar) < target) {
         if ((long long)(ptx::globaltimer() - t0) > limit) {
           atomicOr(status, kStatusTimeout);
           ok = 0;
@@ -356,7 +355,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
     for (int i = 0; i < kTcIssuers; ++i) ptx::mbar_init(drain(i), 1);
     ptx::mbar_init(stall_bar, 1);  // never arrived on: only the test stall waits on it
     *abort_flag = 0;
-    *epoch_s = (uint32_t)(ld_acquire_u64(&g_tc_bar) >> 32);
+    *epoch_s = (uint32_t)ld_acquire_u64(&g_tc_bar);
     ptx::fence_mbar_init();
   }
   if (warp == 2) {
@@ -995,13 +994,15 @@ cudaError_t launch_decode_tc(const DecodeLaunch& a, cudaStream_t s, int num_sms)
   return launch_tc<32>(p, s, grid);
 }
 
-// After a timeout a CTA may have left the barrier mid-count: open a fresh generation with
-// no arrivals.  The generation only grows, so the epoch tags of the counters stay unique.
-cudaError_t reset_tc_barrier() {
+// After a timeout a CTA may have left the barrier mid-count: move the count to a multiple
+// of the grid size (ctas) above it, with no arrival pending.  The count only grows, so the
+// epoch tags of the piece flags stay unique.
+cudaError_t reset_tc_barrier(int ctas) {
   unsigned long long v = 0;
   cudaError_t e = cudaMemcpyFromSymbol(&v, g_tc_bar, sizeof(v));
   if (e != cudaSuccess) return e;
-  v = ((v >> 32) + 1) << 32;
+  const unsigned long long G = ctas > 0 ? (unsigned long long)ctas : 1ull;
+  v = (v / G + 2) * G;
   return cudaMemcpyToSymbol(g_tc_bar, &v, sizeof(v));
 }
 

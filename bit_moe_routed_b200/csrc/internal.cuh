@@ -206,7 +206,7 @@ cudaError_t launch_decode_tc(const DecodeLaunch& a, cudaStream_t s, int num_sms)
 bool decode_tc_fits(int k, int d, int f, int ctas);
 size_t decode_tc_smem_bytes(int d, int f);
 size_t decode_tc_ws_bytes(int k, int d, int f);
-cudaError_t reset_tc_barrier();
+cudaError_t reset_tc_barrier(int ctas);
 size_t decode_smem_bytes(int d, int f, bool q2 = false);
 // whether the single-token kernel's per-CTA limits hold for (k, d, f) on `ctas` CTAs
 // (q2: with 2-bit routed experts)
