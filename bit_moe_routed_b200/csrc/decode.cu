@@ -115,6 +115,9 @@ struct DecodeParams {
   // at sh_e (E, or the cache's slot count)
   const int32_t* slot_of;
   int sh_e;
+  // the work split's divisors: stages per shared / routed unit in each phase, units per
+  // expert in each phase
+  FastDiv fd_s1, fd_s1q, fd_s2, fd_s2q, fd_u1, fd_u2;
 };
 
 // Shared memory: rings (codes, then scales), the phase-dependent area (phase 1: token as
@@ -227,15 +230,17 @@ __device__ bool grid_barrier(long long limit, int* status, volatile int* ok_s) {
 
 // Unit ul / chunk c of task `task` in a CTA range whose first ns units have S stages each
 // (the shared expert's) and the rest Sq (the routed experts'); true for a routed unit.
-__device__ __forceinline__ bool locate(int task, int ns, int S, int Sq, int& ul, int& c) {
-  if (task < ns * S) {
-    ul = task / S;
-    c = task % S;
+__device__ __forceinline__ bool locate(int task, int ns, const FastDiv& S, const FastDiv& Sq,
+                                       int& ul, int& c) {
+  if (task < ns * (int)S.d) {
+    ul = S.div(task);
+    c = task - ul * (int)S.d;
     return false;
   }
-  const int r = task - ns * S;
-  ul = ns + r / Sq;
-  c = r % Sq;
+  const int r = task - ns * (int)S.d;
+  const int u = Sq.div(r);
+  ul = ns + u;
+  c = r - u * (int)Sq.d;
   return true;
 }
 
@@ -346,16 +351,17 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
     ptx::mbar_arrive_expect_tx(full(st), kDcStageBytes);
     if (q < q1) {
       int ul, c;
-      const bool routed = locate(warp + q * kDcWarps, r1.ns, S1, S1q, ul, c);
+      const bool routed = locate(warp + q * kDcWarps, r1.ns, p.fd_s1, p.fd_s1q, ul, c);
       int e, uin;
       if (!routed) {
         e = p.sh_e;
         uin = r1.s_lo + ul;
       } else {
         const int ru = r1.r_lo + ul - r1.ns;
-        e = slot_e[ru / upe1];
+        const int sl = p.fd_u1.div(ru);
+        e = slot_e[sl];
         if (p.slot_of) e = p.slot_of[e];
-        uin = ru % upe1;
+        uin = ru - sl * upe1;
       }
       if (RQ && routed) {
         // 2-bit stage: 2 x 128 code bytes (1024 elements) per row; the 16-byte scale box
@@ -374,16 +380,17 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
       }
     } else {
       int ul, c;
-      const bool routed = locate(warp + (q - q1) * kDcWarps, r2.ns, S2, S2q, ul, c);
+      const bool routed = locate(warp + (q - q1) * kDcWarps, r2.ns, p.fd_s2, p.fd_s2q, ul, c);
       int e, uin;
       if (!routed) {
         e = p.sh_e;
         uin = r2.s_lo + ul;
       } else {
         const int ru = r2.r_lo + ul - r2.ns;
-        e = slot_e[ru / upe2];
+        const int sl = p.fd_u2.div(ru);
+        e = slot_e[sl];
         if (p.slot_of) e = p.slot_of[e];
-        uin = ru % upe2;
+        uin = ru - sl * upe2;
       }
       const int row = e * d + uin * 16;
       if (RQ && routed) {
@@ -533,9 +540,9 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
       slot = n_act;
     } else {
       const int ru = r2.r_lo + ul - r2.ns;
-      slot = ru / upe2;
+      slot = p.fd_u2.div(ru);
       e = slot_e[slot];
-      uin = ru % upe2;
+      uin = ru - slot * upe2;
       ls = 1 + slot - r2_slot0;
     }
   };
@@ -570,8 +577,8 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
           uin = r1.s_lo + ul;
         } else {
           const int ru = r1.r_lo + ul - r1.ns;
-          slot = ru / upe1;
-          uin = ru % upe1;
+          slot = p.fd_u1.div(ru);
+          uin = ru - slot * upe1;
         }
         const float h = __fdividef(gg, 1.0f + expf(-gg)) * uu;
         p.hbuf[(size_t)slot * f + uin * 8 + r] = h;
@@ -654,8 +661,8 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
       const uint8_t* sst = scales_at(st);
       const int task = warp + (PH == 1 ? q : q - q1) * kDcWarps;
       int ul, c;
-      const bool routed = PH == 1 ? locate(task, r1.ns, S1, S1q, ul, c)
-                                  : locate(task, r2.ns, S2, S2q, ul, c);
+      const bool routed = PH == 1 ? locate(task, r1.ns, p.fd_s1, p.fd_s1q, ul, c)
+                                  : locate(task, r2.ns, p.fd_s2, p.fd_s2q, ul, c);
       const uint16_t* xb = bx;
       const uint8_t* xq = bxq;
       const float* sxb = bs1;
@@ -890,6 +897,13 @@ cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t s, int num_sms) {
   p.stall = a.stall;
   p.slot_of = a.slot_of;
   p.sh_e = maps_e;
+  // the kernel's S1, S1q, S2, S2q, upe1, upe2 (2-bit routed stages hold 1024 elements)
+  p.fd_s1 = FastDiv((uint32_t)(a.d / 512));
+  p.fd_s1q = FastDiv((uint32_t)(q2 ? a.d / 1024 : a.d / 512));
+  p.fd_s2 = FastDiv((uint32_t)(a.f / 512));
+  p.fd_s2q = FastDiv((uint32_t)(q2 ? a.f / 1024 : a.f / 512));
+  p.fd_u1 = FastDiv((uint32_t)(a.f / 8));
+  p.fd_u2 = FastDiv((uint32_t)(a.d / 16));
   const int grid = num_sms < kMaxCtas ? num_sms : kMaxCtas;
   if (q2) {  // forward only
     if (!a.forward) return cudaErrorInvalidValue;

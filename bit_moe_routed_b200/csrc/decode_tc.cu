@@ -157,13 +157,17 @@ struct TcSmem {
   __host__ __device__ int bytes() const { return red() + 16 + 1024; }  // + alignment slack
 };
 
-// One CTA's work: its units in both phases (Range, wsh = 1) and their coordinates.
+// One CTA's work: its units in both phases (Range, wsh = 1) and their coordinates, with
+// the divisors of the per-stage arithmetic (units per expert, K chunks per row block).
 struct TcPlan {
   Range r1, r2;
   int NK1, NK2, RB1, n1, n2;
+  FastDiv fu1, fu2, fk1, fk2;
   __host__ __device__ TcPlan(int n_routed, int d, int f, int G, int b)
       : r1((f / 128) * (d / kTcKs), n_routed, G, b, 1),
-        r2((d / 128) * (f / kTcKs), n_routed, G, b, 1) {
+        r2((d / 128) * (f / kTcKs), n_routed, G, b, 1),
+        fu1((uint32_t)((f / 128) * (d / kTcKs))), fu2((uint32_t)((d / 128) * (f / kTcKs))),
+        fk1((uint32_t)(d / kTcKs)), fk2((uint32_t)(f / kTcKs)) {
     NK1 = d / kTcKs;
     NK2 = f / kTcKs;
     RB1 = f / 128;
@@ -172,14 +176,17 @@ struct TcPlan {
   }
 };
 
-// Unit ul of a phase's range: slot (-1 = the shared expert), 128-row block, K chunk, and
-// the first and last unit of its segment (the run of units of one expert and row block).
+// Unit ul of a phase's range (units per expert fu, K chunks per row block fk): slot (-1 =
+// the shared expert), 128-row block, K chunk, and the first and last unit of its segment
+// (the run of units of one expert and row block).
 struct TcUnit {
   int slot, rb, kc, ua, ub;
 };
-__host__ __device__ inline TcUnit tc_unit(const Range& r, int NK, int ul) {
+__host__ __device__ inline TcUnit tc_unit(const Range& r, const FastDiv& fu, const FastDiv& fk,
+                                          int ul) {
   TcUnit t;
   int u, lo, hi;
+  const int NK = (int)fk.d;
   if (ul < r.ns) {
     t.slot = -1;
     u = r.s_lo + ul;
@@ -187,28 +194,28 @@ __host__ __device__ inline TcUnit tc_unit(const Range& r, int NK, int ul) {
     hi = r.ns - 1;
   } else {
     const int ru = r.r_lo + ul - r.ns;
-    t.slot = ru / r.upe;
-    u = ru % r.upe;
+    t.slot = fu.div(ru);
+    u = ru - t.slot * (int)fu.d;
     lo = r.ns;
     hi = r.units() - 1;
   }
-  t.rb = u / NK;
-  t.kc = u % NK;
+  t.rb = fk.div(u);
+  t.kc = u - t.rb * NK;
   t.ua = ul - t.kc > lo ? ul - t.kc : lo;
   t.ub = ul + (NK - 1 - t.kc) < hi ? ul + (NK - 1 - t.kc) : hi;
   return t;
 }
 // Segments of a phase's range (shared ones first).
-__host__ __device__ inline int tc_segments(const Range& r, int NK) {
-  const int a = r.ns > 0 ? (r.s_lo + r.ns - 1) / NK - r.s_lo / NK + 1 : 0;
-  const int b = r.nr > 0 ? (r.r_lo + r.nr - 1) / NK - r.r_lo / NK + 1 : 0;
+__host__ __device__ inline int tc_segments(const Range& r, const FastDiv& fk) {
+  const int a = r.ns > 0 ? fk.div(r.s_lo + r.ns - 1) - fk.div(r.s_lo) + 1 : 0;
+  const int b = r.nr > 0 ? fk.div(r.r_lo + r.nr - 1) - fk.div(r.r_lo) + 1 : 0;
   return a + b;
 }
 // Index of unit ul's segment within its phase.
-__host__ __device__ inline int tc_segment_of(const Range& r, int NK, int ul) {
-  if (ul < r.ns) return (r.s_lo + ul) / NK - r.s_lo / NK;
-  const int a = r.ns > 0 ? (r.s_lo + r.ns - 1) / NK - r.s_lo / NK + 1 : 0;
-  return a + (r.r_lo + ul - r.ns) / NK - r.r_lo / NK;
+__host__ __device__ inline int tc_segment_of(const Range& r, const FastDiv& fk, int ul) {
+  if (ul < r.ns) return fk.div(r.s_lo + ul) - fk.div(r.s_lo);
+  const int a = r.ns > 0 ? fk.div(r.s_lo + r.ns - 1) - fk.div(r.s_lo) + 1 : 0;
+  return a + fk.div(r.r_lo + ul - r.ns) - fk.div(r.r_lo);
 }
 
 // Stage q of the CTA (phase 1: q < n1, unit q / 2, matrix q % 2; phase 2: unit q - n1):
@@ -222,15 +229,15 @@ __host__ __device__ inline TcStageInfo tc_stage(const TcPlan& P, int q) {
   if (q < P.n1) {
     s.ph = 1;
     s.mat = q & 1;
-    s.u = tc_unit(P.r1, P.NK1, q >> 1);
-    s.seg = tc_segment_of(P.r1, P.NK1, q >> 1);
+    s.u = tc_unit(P.r1, P.fu1, P.fk1, q >> 1);
+    s.seg = tc_segment_of(P.r1, P.fk1, q >> 1);
     s.qa = 2 * s.u.ua;
     s.qb = 2 * s.u.ub + 1;
   } else {
     s.ph = 2;
     s.mat = 0;
-    s.u = tc_unit(P.r2, P.NK2, q - P.n1);
-    s.seg = tc_segments(P.r1, P.NK1) + tc_segment_of(P.r2, P.NK2, q - P.n1);
+    s.u = tc_unit(P.r2, P.fu2, P.fk2, q - P.n1);
+    s.seg = tc_segments(P.r1, P.fk1) + tc_segment_of(P.r2, P.fk2, q - P.n1);
     s.qa = P.n1 + s.u.ua;
     s.qb = P.n1 + s.u.ub;
   }
@@ -306,7 +313,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
   const int b = blockIdx.x;
   const TcPlan P(k, d, f, (int)gridDim.x, b);
   const int nq = P.n1 + P.n2;
-  const int nseg1 = tc_segments(P.r1, P.NK1);
+  const int nseg1 = tc_segments(P.r1, P.fk1);
   const int nb1 = d / 128, nb2 = f / 128;  // 128-element K blocks of each phase
   const int RB2 = d / 128;
   const int r2s0 = P.r2.r_lo / P.r2.upe;   // first routed slot of phase 2
@@ -722,8 +729,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
     // ---- phase 1: each segment's partial sums go out with their length and, last, a flag
     // (release); the CTA holding a row block's first K chunk finishes its h
     for (int ul = 0; ok && ul < P.r1.units();) {
-      const TcUnit u = tc_unit(P.r1, P.NK1, ul);
-      const int seg = tc_segment_of(P.r1, P.NK1, ul);
+      const TcUnit u = tc_unit(P.r1, P.fu1, P.fk1, ul);
+      const int seg = tc_segment_of(P.r1, P.fk1, ul);
       const int len = u.ub - u.ua + 1;
       float acc[2];
       if (!segment_sums(seg, u.kc, u.kc + len - 1, 2, sxs, nb1, acc)) {
@@ -790,8 +797,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
 
     // ---- phase 2: each segment's partial sums and length
     for (int ul = 0; ok && ul < P.r2.units();) {
-      const TcUnit u = tc_unit(P.r2, P.NK2, ul);
-      const int seg = nseg1 + tc_segment_of(P.r2, P.NK2, ul);
+      const TcUnit u = tc_unit(P.r2, P.fu2, P.fk2, ul);
+      const int seg = nseg1 + tc_segment_of(P.r2, P.fk2, ul);
       const int ls = u.slot < 0 ? 0 : 1 + u.slot - r2s0;
       const int len = u.ub - u.ua + 1;
       float acc[2];
