@@ -272,12 +272,14 @@ __device__ __forceinline__ void q2_chunk_dot(uint2 wa, uint2 wb, uint4 x01, uint
                          x23.z, x23.w);
 }
 
-template <int MODE, int PL, bool RQ>
+// DK, FK: 0 for the sizes of the launch, or d and f fixed at compile time (the decode
+// sizes' instantiation, whose work-split and layout arithmetic folds to constants).
+template <int MODE, int PL, bool RQ, int DK = 0, int FK = 0>
 __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (ptx::smem_u32(smem_raw) & 1023)) & 1023);
-  const DcSmem L{p.d, p.f, RQ};
-  const int d = p.d, f = p.f, E = p.E, k = p.k;
+  const int d = DK ? DK : p.d, f = FK ? FK : p.f, E = p.E, k = p.k;
+  const DcSmem L{d, f, RQ};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int G = gridDim.x, b = blockIdx.x;
@@ -337,6 +339,12 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
   const int S1q = RQ ? d / 1024 : S1, S2q = RQ ? f / 1024 : S2;
   const int wsh = RQ ? 2 : 1;
   const int upe1 = f / 8, upe2 = d / 16;
+  const FastDiv fd_s1 = DK ? FastDiv(DK / 512) : p.fd_s1;
+  const FastDiv fd_s1q = DK ? FastDiv(RQ ? DK / 1024 : DK / 512) : p.fd_s1q;
+  const FastDiv fd_s2 = FK ? FastDiv(FK / 512) : p.fd_s2;
+  const FastDiv fd_s2q = FK ? FastDiv(RQ ? FK / 1024 : FK / 512) : p.fd_s2q;
+  const FastDiv fd_u1 = FK ? FastDiv(FK / 8) : p.fd_u1;
+  const FastDiv fd_u2 = DK ? FastDiv(DK / 16) : p.fd_u2;
   const uint64_t pol = ptx::make_policy_evict_first();
 
   // n_act routed experts (known after routing); ranges and task counts follow from it
@@ -351,14 +359,14 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
     ptx::mbar_arrive_expect_tx(full(st), kDcStageBytes);
     if (q < q1) {
       int ul, c;
-      const bool routed = locate(warp + q * kDcWarps, r1.ns, p.fd_s1, p.fd_s1q, ul, c);
+      const bool routed = locate(warp + q * kDcWarps, r1.ns, fd_s1, fd_s1q, ul, c);
       int e, uin;
       if (!routed) {
         e = p.sh_e;
         uin = r1.s_lo + ul;
       } else {
         const int ru = r1.r_lo + ul - r1.ns;
-        const int sl = p.fd_u1.div(ru);
+        const int sl = fd_u1.div(ru);
         e = slot_e[sl];
         if (p.slot_of) e = p.slot_of[e];
         uin = ru - sl * upe1;
@@ -380,14 +388,14 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
       }
     } else {
       int ul, c;
-      const bool routed = locate(warp + (q - q1) * kDcWarps, r2.ns, p.fd_s2, p.fd_s2q, ul, c);
+      const bool routed = locate(warp + (q - q1) * kDcWarps, r2.ns, fd_s2, fd_s2q, ul, c);
       int e, uin;
       if (!routed) {
         e = p.sh_e;
         uin = r2.s_lo + ul;
       } else {
         const int ru = r2.r_lo + ul - r2.ns;
-        const int sl = p.fd_u2.div(ru);
+        const int sl = fd_u2.div(ru);
         e = slot_e[sl];
         if (p.slot_of) e = p.slot_of[e];
         uin = ru - sl * upe2;
@@ -540,7 +548,7 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
       slot = n_act;
     } else {
       const int ru = r2.r_lo + ul - r2.ns;
-      slot = p.fd_u2.div(ru);
+      slot = fd_u2.div(ru);
       e = slot_e[slot];
       uin = ru - slot * upe2;
       ls = 1 + slot - r2_slot0;
@@ -577,7 +585,7 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
           uin = r1.s_lo + ul;
         } else {
           const int ru = r1.r_lo + ul - r1.ns;
-          slot = p.fd_u1.div(ru);
+          slot = fd_u1.div(ru);
           uin = ru - slot * upe1;
         }
         const float h = __fdividef(gg, 1.0f + expf(-gg)) * uu;
@@ -661,8 +669,8 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
       const uint8_t* sst = scales_at(st);
       const int task = warp + (PH == 1 ? q : q - q1) * kDcWarps;
       int ul, c;
-      const bool routed = PH == 1 ? locate(task, r1.ns, p.fd_s1, p.fd_s1q, ul, c)
-                                  : locate(task, r2.ns, p.fd_s2, p.fd_s2q, ul, c);
+      const bool routed = PH == 1 ? locate(task, r1.ns, fd_s1, fd_s1q, ul, c)
+                                  : locate(task, r2.ns, fd_s2, fd_s2q, ul, c);
       const uint16_t* xb = bx;
       const uint8_t* xq = bxq;
       const float* sxb = bs1;
@@ -803,11 +811,11 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
 }
 
 
-template <int MODE, int PL, bool RQ>
+template <int MODE, int PL, bool RQ, int DK = 0, int FK = 0>
 cudaError_t launch_one(const DecodeParams& prm, cudaStream_t s, int grid) {
   const DcSmem L{prm.d, prm.f, RQ};
   const size_t smem = (size_t)L.bytes();
-  auto kern = decode_kernel<MODE, PL, RQ>;
+  auto kern = decode_kernel<MODE, PL, RQ, DK, FK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -905,12 +913,15 @@ cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t s, int num_sms) {
   p.fd_u1 = FastDiv((uint32_t)(a.f / 8));
   p.fd_u2 = FastDiv((uint32_t)(a.d / 16));
   const int grid = num_sms < kMaxCtas ? num_sms : kMaxCtas;
+  const bool dec = a.d == 4096 && a.f == 2048;  // the decode sizes' instantiation
   if (q2) {  // forward only
     if (!a.forward) return cudaErrorInvalidValue;
+    if (a.E <= 256 && dec) return launch_one<kModeForward, 8, true, 4096, 2048>(p, s, grid);
     if (a.E <= 256) return launch_one<kModeForward, 8, true>(p, s, grid);
     return launch_one<kModeForward, 32, true>(p, s, grid);
   }
   if (a.forward) {
+    if (a.E <= 256 && dec) return launch_one<kModeForward, 8, false, 4096, 2048>(p, s, grid);
     if (a.E <= 256) return launch_one<kModeForward, 8, false>(p, s, grid);
     return launch_one<kModeForward, 32, false>(p, s, grid);
   }

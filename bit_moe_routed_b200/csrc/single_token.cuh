@@ -17,7 +17,7 @@ namespace {
 // division there costs tens of instructions on every warp's path.
 struct FastDiv {
   uint32_t d, m, s;
-  __host__ __device__ explicit FastDiv(uint32_t d_ = 1) : d(d_ < 1 ? 1 : d_), m(0), s(0) {
+  __host__ __device__ constexpr explicit FastDiv(uint32_t d_ = 1) : d(d_ < 1 ? 1 : d_), m(0), s(0) {
     while ((1ull << s) < d) ++s;
     m = (uint32_t)(((1ull << 32) * ((1ull << s) - d)) / d + 1);
   }
