@@ -63,6 +63,7 @@ struct BgParams {
   int E, K, rows_per_expert, P, R, d, f;
   long long wait_ns;
   int* status;
+  FastDiv fd_s, fd_upe;  // stages per unit (K / 512), units per expert
 };
 
 // Shared memory from a 1024-byte aligned base.
@@ -231,14 +232,16 @@ __global__ void __launch_bounds__(kBgThreads, 1) bgemv_kernel(const __grid_const
     return smem + L.off_rscale() + (warp * kBgStages + s) * kBgScaleBytes;
   };
   auto issue = [&](int i) {
-    const int u = u_lo + warp + (i / S) * kBgWarps, c = i % S;
-    const int sl = u / upe - first;
+    const int qi = p.fd_s.div(i);
+    const int u = u_lo + warp + qi * kBgWarps, c = i - qi * S;
+    const int ue = p.fd_upe.div(u);
+    const int sl = ue - first;
     const int e = slot_info[4 * sl];
     const uint64_t pol = slot_info[4 * sl + 3] ? pol_last : pol_first;
     const int st = i % kBgStages;
     const uint32_t dc = ptx::smem_u32(codes_at(st)), ds = ptx::smem_u32(scales_at(st));
     ptx::mbar_arrive_expect_tx(full(st), kBgStageBytes);
-    const int row = e * p.rows_per_expert + (u % upe) * rows_unit;
+    const int row = e * p.rows_per_expert + (u - ue * upe) * rows_unit;
     ptx::tma_load_3d_hint(dc, &p.tm_c0, 0, row, 2 * c, full(st), pol);
     ptx::tma_load_2d_hint(ds, &p.tm_s0, c * 16, row, full(st), pol);
     if (PHASE == 1) {
@@ -257,8 +260,9 @@ __global__ void __launch_bounds__(kBgThreads, 1) bgemv_kernel(const __grid_const
   int i = 0;
   for (int q = 0; q < my_units && ok; ++q) {
     const int u = u_lo + warp + q * kBgWarps;
-    const int sl = u / upe - first;
-    const int uin = u % upe;
+    const int ue = p.fd_upe.div(u);
+    const int sl = ue - first;
+    const int uin = u - ue * upe;
     for (; released < sl; ++released)
       if (lane == 0) ptx::mbar_arrive(act_empty(released % kBgBufs));
     if (!wait_warp(act_full(sl % kBgBufs), (uint32_t)(sl / kBgBufs) & 1u, p.wait_ns, abort_flag,
@@ -391,6 +395,8 @@ cudaError_t launch_bgemv(int phase, const BgLaunch& a, cudaStream_t s, int num_s
   p.f = a.f;
   p.wait_ns = a.wait_ns;
   p.status = a.status;
+  p.fd_s = FastDiv((uint32_t)(K / 512));
+  p.fd_upe = FastDiv((uint32_t)(rpe / (phase == 1 ? 8 : 16)));
   const int grid = num_sms < kMaxCtas ? num_sms : kMaxCtas;
   return phase == 1 ? launch_one<1>(p, s, grid, a.overlap) : launch_one<2>(p, s, grid, a.overlap);
 }

@@ -9,28 +9,6 @@
 namespace bitmoe {
 namespace {
 
-// Division by a divisor fixed for a launch, as a multiply-high, an add and a shift (the
-// round-up method of Granlund and Montgomery, "Division by invariant integers using
-// multiplication", 1994): with s = ceil(log2 d) and m = floor(2^32 (2^s - d) / d) + 1,
-// n / d = (umulhi(n, m) + n) >> s for 1 <= d < 2^31 and 0 <= n < 2^31 (the sum stays
-// below 2^32).  The per-stage work split divides by runtime sizes; a hardware-free integer
-// division there costs tens of instructions on every warp's path.
-struct FastDiv {
-  uint32_t d, m, s;
-  __host__ __device__ constexpr explicit FastDiv(uint32_t d_ = 1) : d(d_ < 1 ? 1 : d_), m(0), s(0) {
-    while ((1ull << s) < d) ++s;
-    m = (uint32_t)(((1ull << 32) * ((1ull << s) - d)) / d + 1);
-  }
-  __host__ __device__ __forceinline__ int div(int n) const {
-#ifdef __CUDA_ARCH__
-    const uint32_t hi = __umulhi((uint32_t)n, m);
-#else
-    const uint32_t hi = (uint32_t)(((uint64_t)(uint32_t)n * m) >> 32);
-#endif
-    return (int)((hi + (uint32_t)n) >> s);
-  }
-};
-
 // One CTA's share of a phase.  A shared unit weighs wsh (1; 2 in the Q2 form, where it
 // has twice the stages of a routed unit), a routed unit 1: M = (n_routed + wsh) * upe in
 // all, CTA b taking the weight range [b*M/G, (b+1)*M/G).  Its first ns units are the
