@@ -117,11 +117,14 @@ __device__ __forceinline__ uint32_t act_offset(int k, int g, int t) {
          8u * (uint32_t)(t & 1);
 }
 
-template <int PHASE>
+// KC, RPE: 0 for the sizes of the launch, or K and the rows per expert fixed at compile time
+// (the decode sizes' instantiations, whose work-split and layout arithmetic folds).
+template <int PHASE, int KC = 0, int RPE = 0>
 __global__ void __launch_bounds__(kBgThreads, 1) bgemv_kernel(const __grid_constant__ BgParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (ptx::smem_u32(smem_raw) & 1023)) & 1023);
-  const int K = p.K;
+  const int K = KC ? KC : p.K;
+  const int rpe = RPE ? RPE : p.rows_per_expert;
   const BgSmem L{K};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
@@ -161,7 +164,9 @@ __global__ void __launch_bounds__(kBgThreads, 1) bgemv_kernel(const __grid_const
 
   const int n_slots = __ldg(p.plan);
   const int rows_unit = PHASE == 1 ? 8 : 16;
-  const int upe = p.rows_per_expert / rows_unit;
+  const int upe = rpe / rows_unit;
+  const FastDiv fd_s = KC ? FastDiv(KC / 512) : p.fd_s;
+  const FastDiv fd_upe = RPE ? FastDiv(RPE / (PHASE == 1 ? 8 : 16)) : p.fd_upe;
   const long long U = (long long)n_slots * upe;
   const int u_lo = (int)(blockIdx.x * U / gridDim.x);
   const int u_hi = (int)((blockIdx.x + 1) * U / gridDim.x);
@@ -232,16 +237,16 @@ __global__ void __launch_bounds__(kBgThreads, 1) bgemv_kernel(const __grid_const
     return smem + L.off_rscale() + (warp * kBgStages + s) * kBgScaleBytes;
   };
   auto issue = [&](int i) {
-    const int qi = p.fd_s.div(i);
+    const int qi = fd_s.div(i);
     const int u = u_lo + warp + qi * kBgWarps, c = i - qi * S;
-    const int ue = p.fd_upe.div(u);
+    const int ue = fd_upe.div(u);
     const int sl = ue - first;
     const int e = slot_info[4 * sl];
     const uint64_t pol = slot_info[4 * sl + 3] ? pol_last : pol_first;
     const int st = i % kBgStages;
     const uint32_t dc = ptx::smem_u32(codes_at(st)), ds = ptx::smem_u32(scales_at(st));
     ptx::mbar_arrive_expect_tx(full(st), kBgStageBytes);
-    const int row = e * p.rows_per_expert + (u - ue * upe) * rows_unit;
+    const int row = e * rpe + (u - ue * upe) * rows_unit;
     ptx::tma_load_3d_hint(dc, &p.tm_c0, 0, row, 2 * c, full(st), pol);
     ptx::tma_load_2d_hint(ds, &p.tm_s0, c * 16, row, full(st), pol);
     if (PHASE == 1) {
@@ -260,7 +265,7 @@ __global__ void __launch_bounds__(kBgThreads, 1) bgemv_kernel(const __grid_const
   int i = 0;
   for (int q = 0; q < my_units && ok; ++q) {
     const int u = u_lo + warp + q * kBgWarps;
-    const int ue = p.fd_upe.div(u);
+    const int ue = fd_upe.div(u);
     const int sl = ue - first;
     const int uin = u - ue * upe;
     for (; released < sl; ++released)
@@ -353,10 +358,10 @@ __global__ void __launch_bounds__(kBgThreads, 1) bgemv_kernel(const __grid_const
   __syncwarp();
 }
 
-template <int PHASE>
+template <int PHASE, int KC = 0, int RPE = 0>
 cudaError_t launch_one(const BgParams& prm, cudaStream_t s, int grid, bool overlap) {
   const size_t smem = (size_t)BgSmem{prm.K}.bytes();
-  auto kern = bgemv_kernel<PHASE>;
+  auto kern = bgemv_kernel<PHASE, KC, RPE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3(grid), dim3(kBgThreads), smem, s, overlap, prm);
@@ -398,6 +403,9 @@ cudaError_t launch_bgemv(int phase, const BgLaunch& a, cudaStream_t s, int num_s
   p.fd_s = FastDiv((uint32_t)(K / 512));
   p.fd_upe = FastDiv((uint32_t)(rpe / (phase == 1 ? 8 : 16)));
   const int grid = num_sms < kMaxCtas ? num_sms : kMaxCtas;
+  if (a.d == 4096 && a.f == 2048)  // the decode sizes' instantiations
+    return phase == 1 ? launch_one<1, 4096, 2048>(p, s, grid, a.overlap)
+                      : launch_one<2, 2048, 4096>(p, s, grid, a.overlap);
   return phase == 1 ? launch_one<1>(p, s, grid, a.overlap) : launch_one<2>(p, s, grid, a.overlap);
 }
 

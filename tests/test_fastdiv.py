@@ -1,7 +1,8 @@
 """The single-token and batched GEMV kernels divide by runtime sizes in their per-stage
 work split with a multiply-high, an add and a shift (FastDiv in internal.cuh, the
-round-up method of Granlund and Montgomery): s = ceil(log2 d), m = floor(2^32 (2^s - d) / d) + 1, and
-n / d = (umulhi(n, m) + n) >> s for 1 <= d < 2^31, 0 <= n < 2^31.  This checks the
+round-up method of Granlund and Montgomery): s = ceil(log2 d),
+m = floor(2^32 (2^s - d) / d) + 1, and n / d = (umulhi(n, m) + n) >> s for
+1 <= d < 2^31, 0 <= n < 2^31.  This checks the
 formula, as the kernel evaluates it in 32-bit arithmetic, against Python's integer
 division: every n below 2^16 for every d up to 4096, and sampled n up to 2^31 - 1."""
 import random
