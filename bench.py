@@ -704,6 +704,7 @@ def e2e(bm, Ls, args, dev, stream, dist, world):
 
 def run_gpu(args, w):
     import bit_moe_routed_b200 as bm
+    bm.set_decode_engine(args.decode_engine)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -804,6 +805,9 @@ def main():
     ap.add_argument("--extra-cpu-seconds", type=float, default=4.0)
     ap.add_argument("--ref-seconds", type=float, default=None,
                     help="oracle seconds per step of the reference arm (default: fit ~1 min)")
+    ap.add_argument("--decode-engine", type=int, default=0, choices=[0, 1],
+                    help="single-token layer kernel of moe_forward: 0 CUDA cores (default), "
+                         "1 tensor cores")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
