@@ -505,7 +505,8 @@ def measure(bm, w, args, dev, stream, rank, dist, steps, warmup, peaks, cpu_seco
             kernel_name = ("decode_kernel, Q2 form: the whole layer in one cooperative kernel, "
                            "2-bit routed experts (byte-permute decode to e4m3, mma.sync e4m3) "
                            "and the FP4 shared expert")
-        traffic = kernel_traffic(kernel_file, "layer", w.name)
+        traffic = kernel_traffic(kernel_file, "layer_tc" if kernel_file.endswith("decode_tc.cu")
+                                 else "layer", w.name)
         io = 4 * E + 2 * d + 4 * d * (k + 2)  # scores, x; y_routed, y_shared and out
         work["gu_bytes"] = work["weight_bytes"] + io
     else:
