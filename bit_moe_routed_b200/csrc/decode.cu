@@ -788,22 +788,30 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
     }
   }
   if (MODE == kModeForward) {
-    // per 16-row output block, the last of the k + 1 experts to finish it sums out
+    // Per 16-row output block, the last of the k + 1 experts to finish it sums out.  The
+    // CTA barrier orders the CTA's y writes before each warp's acq_rel count (a release at
+    // GPU scope, as in grid_barrier); the count that finds n_act earlier arrivals acquires
+    // every other expert's rows.  The k routed rows are loaded together, then summed in
+    // j order.
     __syncthreads();
     for (int ul = warp; ul < r2.units(); ul += kDcWarps) {
       int e, uin, ls, slot;
       p2_local(ul, e, uin, ls, slot);
       int last = 0;
-      if (lane == 0) {
-        __threadfence();
-        last = atom_add_acq_rel(p.done2 + uin, 1) == n_act ? 1 : 0;
-      }
+      if (lane == 0) last = atom_add_acq_rel(p.done2 + uin, 1) == n_act ? 1 : 0;
       last = __shfl_sync(0xffffffffu, last, 0);
       if (last && lane < 16) {
         const size_t m = (size_t)uin * 16 + lane;
         float acc = __ldcg(p.y_shared + m);
-        for (int j = 0; j < k; ++j)
-          acc = fmaf(pair_w[j], __ldcg(p.y_routed + (size_t)pair_pos[j] * d + m), acc);
+        for (int j0 = 0; j0 < k; j0 += 8) {
+          float yv[8];
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj)
+            yv[jj] = j0 + jj < k ? __ldcg(p.y_routed + (size_t)pair_pos[j0 + jj] * d + m) : 0.f;
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj)
+            if (j0 + jj < k) acc = fmaf(pair_w[j0 + jj], yv[jj], acc);
+        }
         p.out[m] = acc;
       }
     }
