@@ -308,6 +308,15 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
     return smem + DcSmem::kOffScales + (warp * kDcStages + s) * kDcScaleBytes;
   };
 
+  // the token's scores (warp 0, for the routing) and its first 4096 values (warps 1-8, for
+  // the quantisation) are loaded first, so their latency overlaps the set-up below
+  float sc_v[PL];
+  uint4 xa = make_uint4(0, 0, 0, 0), xb = make_uint4(0, 0, 0, 0);
+  if (MODE == kModeForward && warp == 0) load_scores<PL>(p.scores, E, lane, sc_v);
+  if (warp >= 1 && warp <= 8 && (threadIdx.x - 32) * 16 < d) {
+    xa = *reinterpret_cast<const uint4*>(p.x + (threadIdx.x - 32) * 16);
+    xb = *reinterpret_cast<const uint4*>(p.x + (threadIdx.x - 32) * 16 + 8);
+  }
   if (threadIdx.x == 0) {
     ptx::prefetch_tmap(&p.tm_gc);
     ptx::prefetch_tmap(&p.tm_gs);
@@ -425,7 +434,7 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
   if (warp == 0) {
     if (MODE == kModeForward) {
       // top-k of the E scores and the gate weights; CTA 0 stores them with the dispatch
-      route_token_warp<PL>(p.scores, E, k, lane, slot_e, slot_row, slot_n, pair_w, pair_pos,
+      route_token_warp<PL>(sc_v, E, k, lane, slot_e, slot_row, slot_n, pair_w, pair_pos,
                            b == 0 ? p.idx : nullptr, p.w, p.perm, p.pos);
       if (lane == 0) *n_active = k;
     } else {
@@ -462,8 +471,8 @@ __global__ void __launch_bounds__(kDcThreads, 1) decode_kernel(const __grid_cons
     const int tid = threadIdx.x - 32;
     for (int c0 = tid * 16; c0 - (tid & 31) * 16 < d; c0 += 256 * 16) {
       const bool act = c0 < d;
-      uint4 a = make_uint4(0, 0, 0, 0), bb = make_uint4(0, 0, 0, 0);
-      if (act) {
+      uint4 a = xa, bb = xb;  // the first round's values were loaded at the start
+      if (act && c0 != tid * 16) {
         a = *reinterpret_cast<const uint4*>(p.x + c0);
         bb = *reinterpret_cast<const uint4*>(p.x + c0 + 8);
       }

@@ -36,18 +36,22 @@ struct Range {
 // the expert and, if non-NULL, slot_row[slot] = slot and slot_n[slot] = 1; for pair j (the
 // j-th largest score), pair_w[j] and pair_pos[j] = its slot.  If idx is non-NULL the
 // routing and dispatch results go to global memory too (idx, w, perm, pos).
+// The lane's scores (experts lane + 32 i), -inf past E: loaded on their own so that a
+// kernel can issue the loads first and route later.
 template <int PL>
-__device__ __forceinline__ void route_token_warp(const float* __restrict__ scores, int E, int k,
-                                                 int lane, int* slot_e, int* slot_row,
-                                                 int* slot_n, float* pair_w, int* pair_pos,
-                                                 int32_t* idx, float* w, int32_t* perm,
-                                                 int32_t* pos) {
-  float v[PL];
+__device__ __forceinline__ void load_scores(const float* __restrict__ scores, int E, int lane,
+                                            float (&v)[PL]) {
 #pragma unroll
   for (int i = 0; i < PL; ++i) {
     const int e = lane + 32 * i;
     v[i] = e < E ? __ldg(scores + e) : -INFINITY;
   }
+}
+template <int PL>
+__device__ __forceinline__ void route_token_warp(const float (&v)[PL], int E, int k, int lane,
+                                                 int* slot_e, int* slot_row, int* slot_n,
+                                                 float* pair_w, int* pair_pos, int32_t* idx,
+                                                 float* w, int32_t* perm, int32_t* pos) {
   // keys: a larger score has a larger key (sign-magnitude to offset order); NaN and
   // padding get 0, below every number, so they are taken only after all numbers
   uint32_t key[PL];
@@ -99,6 +103,17 @@ __device__ __forceinline__ void route_token_warp(const float* __restrict__ score
       pos[lane] = rank;
     }
   }
+}
+
+template <int PL>
+__device__ __forceinline__ void route_token_warp(const float* __restrict__ scores, int E, int k,
+                                                 int lane, int* slot_e, int* slot_row,
+                                                 int* slot_n, float* pair_w, int* pair_pos,
+                                                 int32_t* idx, float* w, int32_t* perm,
+                                                 int32_t* pos) {
+  float v[PL];
+  load_scores<PL>(scores, E, lane, v);
+  route_token_warp<PL>(v, E, k, lane, slot_e, slot_row, slot_n, pair_w, pair_pos, idx, w, perm, pos);
 }
 
 }  // namespace
