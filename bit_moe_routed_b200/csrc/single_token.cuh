@@ -29,13 +29,6 @@ struct Range {
   __host__ __device__ int units() const { return ns + nr; }
 };
 
-// Each lane holds experts lane + 32 i (i < PL, so E <= 32 PL).  k rounds of a warp arg-max
-// on (value desc, index asc), as a max of order-preserving integer keys and then a min of
-// the indices holding it (two warp reductions a round).  Outputs, in shared memory: for
-// slot = the expert's rank among the k selected ids (its sorted position), slot_e[slot] =
-// the expert and, if non-NULL, slot_row[slot] = slot and slot_n[slot] = 1; for pair j (the
-// j-th largest score), pair_w[j] and pair_pos[j] = its slot.  If idx is non-NULL the
-// routing and dispatch results go to global memory too (idx, w, perm, pos).
 // The lane's scores (experts lane + 32 i), -inf past E: loaded on their own so that a
 // kernel can issue the loads first and route later.
 template <int PL>
@@ -47,6 +40,13 @@ __device__ __forceinline__ void load_scores(const float* __restrict__ scores, in
     v[i] = e < E ? __ldg(scores + e) : -INFINITY;
   }
 }
+// Each lane holds experts lane + 32 i (i < PL, so E <= 32 PL).  k rounds of a warp arg-max
+// on (value desc, index asc), as a max of order-preserving integer keys and then a min of
+// the indices holding it (two warp reductions a round).  Outputs, in shared memory: for
+// slot = the expert's rank among the k selected ids (its sorted position), slot_e[slot] =
+// the expert and, if non-NULL, slot_row[slot] = slot and slot_n[slot] = 1; for pair j (the
+// j-th largest score), pair_w[j] and pair_pos[j] = its slot.  If idx is non-NULL the
+// routing and dispatch results go to global memory too (idx, w, perm, pos).
 template <int PL>
 __device__ __forceinline__ void route_token_warp(const float (&v)[PL], int E, int k, int lane,
                                                  int* slot_e, int* slot_row, int* slot_n,
@@ -105,6 +105,7 @@ __device__ __forceinline__ void route_token_warp(const float (&v)[PL], int E, in
   }
 }
 
+// The same, loading the scores itself.
 template <int PL>
 __device__ __forceinline__ void route_token_warp(const float* __restrict__ scores, int E, int k,
                                                  int lane, int* slot_e, int* slot_row,
