@@ -541,7 +541,12 @@ def measure(bm, w, args, dev, stream, rank, dist, steps, warmup, peaks, cpu_seco
     roof["avg_launch_us"] = gu_s * 1e6
     roof["algorithmic_per_launch"] = work["flops_gu"] if is_prefill else work["gu_bytes"]
     rec = {
-        "fused": fused, "launches_per_step": 1 if fused else (7 if batched else 6),
+        # route, gate/up, down, combine; the dispatch (two kernels from 8192 pairs); the
+        # prepare step (from 2048 pairs on the tile path two: the inverse permutation, the
+        # per-token quantisation) or, on the batched path, prepare and quant_h
+        "fused": fused,
+        "launches_per_step": 1 if fused else (4 + (2 if T * k >= 8192 else 1)
+                                              + (2 if batched or T * k >= 2048 else 1)),
         "value": world * T * steps / total_s, "unit": "tokens/s", "steps": steps,
         "ms_per_step": 1000.0 * layer_s,
         "ms_per_step_isolated": statistics.median(one_ms),

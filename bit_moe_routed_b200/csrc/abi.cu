@@ -206,6 +206,9 @@ WorkspaceLayout workspace_layout(int T, int k, int E, int d, int f) {
   // the multi-CTA dispatch's counts (moe_forward on large batches)
   L.dispatch = o;
   o = align256(o + dispatch_ws_bytes(T, k, E));
+  // the inverse of the dispatch permutation (the prepare step's row of each pair)
+  L.ipos = o;
+  o = align256(o + 4 * (size_t)T * k);
   L.total = o;
   return L;
 }
@@ -541,7 +544,7 @@ int moe_ffn_prepare(const uint16_t* x_bf16, int T, int k, const moe_weights_t* w
       x_bf16, T, k, w->d, perm, T * k, c.ws + c.L.qx, reinterpret_cast<float*>(c.ws + c.L.sx),
       offsets, w->E, c.nmax, reinterpret_cast<int32_t*>(c.ws + c.L.plan),
       reinterpret_cast<int*>(c.ws + c.L.counters), c.L.n_counters, c.di.status,
-      static_cast<cudaStream_t>(stream), 0, t_overlap);
+      static_cast<cudaStream_t>(stream), 0, t_overlap, reinterpret_cast<int32_t*>(c.ws + c.L.ipos));
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "ffn prepare launch");
 }
 

@@ -64,7 +64,7 @@ constexpr int kBgMaxT = 64;
 constexpr int kBgSlotTokens = 8;  // tokens per slot of the batched GEMV (the MMA's N)
 
 struct WorkspaceLayout {
-  size_t plan, qx, sx, qh, sh, counters, partials, hbuf, done2, dtc, dispatch, total;
+  size_t plan, qx, sx, qh, sh, counters, partials, hbuf, done2, dtc, dispatch, ipos, total;
   size_t n_counters;
 };
 WorkspaceLayout workspace_layout(int T, int k, int E, int d, int f);
@@ -87,13 +87,18 @@ cudaError_t launch_dispatch_multi(const int32_t* idx, int T, int k, int E, int32
                                   int* status, cudaStream_t s, bool overlap);
 // rows r < P = T*k take token perm[r]/k, rows P <= r < P+T take token r-P; perm may be
 // NULL with P = 0 for a plain quantisation of T rows.  If plan != NULL, one extra block
-// writes the token-tile plan (plan_mode 0) or the single-token path's list of active
-// experts (plan_mode 1).
+// writes the token-tile plan (plan_mode 0), the single-token path's list of active
+// experts (plan_mode 1) or the batched path's slot plan (plan_mode 2).  With perm and
+// ipos (T*k ints of scratch), from kQuantTokensMinPairs pairs, each token is quantised
+// once and its codes written to all its rows: a launch that inverts perm into ipos, then
+// one block per token (4096 tokens, top-6: 30 us against 85 us for one block per row; at
+// 64 tokens the second launch costs more than it saves).
+constexpr int kQuantTokensMinPairs = 2048;
 cudaError_t launch_quant_rows(const uint16_t* x, int T, int k, int d, const int32_t* perm,
                               int nrows_routed, uint8_t* q, float* s, const int32_t* offsets,
                               int E, int nmax, int32_t* plan, int* counters, size_t n_counters,
                               int* status, cudaStream_t st, int plan_mode = 0,
-                              bool overlap = false);
+                              bool overlap = false, int32_t* ipos = nullptr);
 // h [R][f] fp32 -> e4m3 codes [R][f] and scales [R][f/128] (batched GEMV path)
 cudaError_t launch_quant_h(const float* h, int R, int f, uint8_t* q, float* s, cudaStream_t st,
                            bool overlap);

@@ -181,6 +181,95 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(
   }
 }
 
+// The inverse of the dispatch's permutation: ipos[perm[r]] = r, the row of each (token,
+// choice) pair in expert-sorted order.  A value outside [0, P) is flagged and skipped.
+__global__ void __launch_bounds__(256) invperm_kernel(const int32_t* __restrict__ perm, int P,
+                                                      int32_t* __restrict__ ipos,
+                                                      int* __restrict__ status) {
+  ptx::griddep_launch_dependents();
+  ptx::griddep_wait();  // perm comes from the dispatch
+  for (int r = blockIdx.x * blockDim.x + threadIdx.x; r < P; r += gridDim.x * blockDim.x) {
+    const int p = perm[r];
+    if (p >= 0 && p < P) ipos[p] = r;
+    else atomicOr(status, kStatusBadIndex);
+  }
+}
+
+// The activation rows in expert-sorted order, one block per token: the token is quantised
+// once, as in quant_rows_kernel (s = amax / 448, IEEE divide, 1 if amax = 0; q = e4m3(x / s)
+// rounded to nearest even), and its codes and scales go to its k routed rows ipos[t*k + j]
+// and to its shared-expert row P + t.  The plan block and the counters as in
+// quant_rows_kernel.
+__global__ void __launch_bounds__(256) quant_tokens_kernel(
+    const uint16_t* __restrict__ x, int T, int k, int d, const int32_t* __restrict__ ipos,
+    uint8_t* __restrict__ q, float* __restrict__ s, const int32_t* __restrict__ offsets, int E,
+    int nmax, int32_t* __restrict__ plan, int* __restrict__ counters, size_t n_counters,
+    int* __restrict__ status, int plan_mode) {
+  ptx::griddep_launch_dependents();
+  ptx::griddep_wait();  // x, ipos, offsets, and the counters the previous FFN launch used
+  const int P = T * k;
+  const int t = blockIdx.x;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_counters;
+       i += (size_t)gridDim.x * blockDim.x)
+    counters[i] = 0;
+  if (t == T) {  // the plan block
+    if (threadIdx.x < 32) {
+      if (plan_mode == 2) write_slot_plan(offsets, E, T, P, plan);
+      else write_plan(offsets, E, T, P, nmax, plan);
+    }
+    return;
+  }
+  // the token's rows: k routed (from the inverse permutation), then its shared-expert row
+  __shared__ int rows[33];
+  if (threadIdx.x <= k) {
+    int r = threadIdx.x < k ? ipos[(size_t)t * k + threadIdx.x] : P + t;
+    if (r < 0 || r >= P + T) {
+      atomicOr(status, kStatusBadIndex);
+      r = -1;
+    }
+    rows[threadIdx.x] = r;
+  }
+  __syncthreads();
+  const uint16_t* xr = x + (size_t)t * d;
+  const int lane16 = (threadIdx.x & 31) * 16;
+  for (int c0 = threadIdx.x * 16; c0 - lane16 < d; c0 += blockDim.x * 16) {
+    const bool act = c0 < d;
+    uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
+    if (act) {
+      a = *reinterpret_cast<const uint4*>(xr + c0);
+      b = *reinterpret_cast<const uint4*>(xr + c0 + 8);
+    }
+    const float v[16] = {bf16_lo(a.x), bf16_hi(a.x), bf16_lo(a.y), bf16_hi(a.y),
+                         bf16_lo(a.z), bf16_hi(a.z), bf16_lo(a.w), bf16_hi(a.w),
+                         bf16_lo(b.x), bf16_hi(b.x), bf16_lo(b.y), bf16_hi(b.y),
+                         bf16_lo(b.z), bf16_hi(b.z), bf16_lo(b.w), bf16_hi(b.w)};
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+    const float sc = amax == 0.f ? 1.0f : __fdiv_rn(amax, 448.0f);
+    uint32_t packed[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint16_t lo = ptx::cvt_e4m3x2(__fdiv_rn(v[4 * i], sc), __fdiv_rn(v[4 * i + 1], sc));
+      const uint16_t hi =
+          ptx::cvt_e4m3x2(__fdiv_rn(v[4 * i + 2], sc), __fdiv_rn(v[4 * i + 3], sc));
+      packed[i] = (uint32_t)lo | ((uint32_t)hi << 16);
+    }
+    if (act) {
+      const uint4 code = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+      for (int j = 0; j <= k; ++j) {
+        const int r = rows[j];
+        if (r < 0) continue;
+        *reinterpret_cast<uint4*>(q + (size_t)r * d + c0) = code;
+        if ((threadIdx.x & 7) == 0) s[(size_t)r * (d / 128) + c0 / 128] = sc;
+      }
+    }
+  }
+}
+
 // The hidden state of the batched GEMV path, fp32 [R][f], re-quantised per row and
 // 128-block exactly as the activations: s = amax / 448 (IEEE divide; 1 if amax = 0),
 // q = e4m3(h / s) rounded to nearest even.  8 threads per block, 16 values each.
@@ -238,7 +327,23 @@ cudaError_t launch_quant_h(const float* h, int R, int f, uint8_t* q, float* s, c
 cudaError_t launch_quant_rows(const uint16_t* x, int T, int k, int d, const int32_t* perm,
                               int nrows_routed, uint8_t* q, float* s, const int32_t* offsets,
                               int E, int nmax, int32_t* plan, int* counters, size_t n_counters,
-                              int* status, cudaStream_t st, int plan_mode, bool overlap) {
+                              int* status, cudaStream_t st, int plan_mode, bool overlap,
+                              int32_t* ipos) {
+  if (perm != nullptr && ipos != nullptr && nrows_routed == T * k && k <= 32 && plan_mode != 1 &&
+      nrows_routed >= kQuantTokensMinPairs) {
+    // each token quantised once: the inverse permutation, then one block per token
+    const int P = T * k;
+    const unsigned ib = (unsigned)((P + 255) / 256 < 4 * 148 ? (P + 255) / 256 : 4 * 148);
+    cudaError_t e = launch_pdl(invperm_kernel, dim3(ib > 0 ? ib : 1), dim3(256), 0, st, overlap, perm,
+                               P, ipos, status);
+    if (e != cudaSuccess) return e;
+    int threads = (d / 16 + 31) / 32 * 32;
+    if (threads > 256) threads = 256;
+    if (threads < 64) threads = 64;  // the row list takes up to k + 1 = 33 threads
+    const unsigned blocks = (unsigned)(T + (plan != nullptr ? 1 : 0));
+    return launch_pdl(quant_tokens_kernel, dim3(blocks), dim3(threads), 0, st, true, x, T, k, d,
+                      ipos, q, s, offsets, E, nmax, plan, counters, n_counters, status, plan_mode);
+  }
   const int R = nrows_routed + T;
   const unsigned blocks = (unsigned)(R + (plan != nullptr ? 1 : 0));
   int threads = (d / 16 + 31) / 32 * 32;  // whole warps
