@@ -120,6 +120,36 @@ def test_act_quant_special_rows():
     assert np.array_equal(q.cpu().numpy(), q_o)
 
 
+def test_prepare_rows_for_any_permutation():
+    """The prepare step from 2048 pairs (the tile path's per-token form: the inverse of the
+    permutation, then each token quantised once) on a shuffled permutation, not the
+    dispatch's: row r holds token perm[r] // k's codes and scales, rows P.. the tokens in
+    order, bit for bit.  Then a permutation with an entry out of range is flagged."""
+    T, E, k, d, f = 512, 64, 6, 1024, 512
+    P = T * k
+    x = synth.gen_x(T, d, seed=515)
+    s = synth.gen_scores_uniform(T, E, 516)
+    W = device_weights(517, 0, E, d, f)
+    assert bm.ffn_path(T, k, W) == bm.PATH_TILES
+    idx, _ = bm.route_topk(s.cuda(), k)
+    _, offsets, _, _ = bm.dispatch(idx, E)
+    perm = torch.from_numpy(np.random.default_rng(518).permutation(P).astype(np.int32))
+    ws = bm.alloc_workspace(T, k, E, d, f)
+    bm.ffn_prepare(x.cuda(), k, W, offsets, perm.cuda(), ws)
+    bm.sync_status()
+    v = bm.workspace_views(ws, T, k, E, d, f)
+    q_o, s_o = oracle.act_quant(x)
+    src = np.concatenate([perm.numpy() // k, np.arange(T)])
+    assert np.array_equal(v["qx"].cpu().numpy(), q_o[src])
+    assert np.array_equal(v["sx"].cpu().numpy(), s_o[src])
+    bad = perm.clone()
+    bad[7] = P + 3
+    bm.ffn_prepare(x.cuda(), k, W, offsets, bad.cuda(), ws)
+    with pytest.raises(bm.MoeError):
+        bm.sync_status()
+    bm.sync_status()  # the status word is cleared once reported
+
+
 # ---------------------------------------------------------------- whole layer, small shapes
 def _small_layer(T, E, k, d, f, routing="uniform", seed=5, zero_rows=(), calls=False):
     x = synth.gen_x(T, d, seed=seed)
