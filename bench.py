@@ -377,6 +377,17 @@ class Layers:
                      "out": torch.empty((T, d), dtype=f32, device=dev)}
 
 
+def launches_per_step(T: int, k: int, fused: bool, batched: bool) -> int:
+    """This library's kernels in one layer step: one at T = 1 (the fused layer kernel);
+    otherwise route, gate/up, down and combine, the dispatch (two kernels from 8192 pairs),
+    and the prepare step (two kernels on the tile path from 2048 pairs: the inverse
+    permutation and the per-token quantisation) or, on the batched path, prepare and
+    quant_h."""
+    if fused:
+        return 1
+    return 4 + (2 if T * k >= 8192 else 1) + (2 if batched or T * k >= 2048 else 1)
+
+
 def resident_layers(w, max_layers):
     """Layers to rotate through so that a step's weights have been evicted from L2 by the
     other layers' since their last use (four times the L2 in between)."""
@@ -541,12 +552,7 @@ def measure(bm, w, args, dev, stream, rank, dist, steps, warmup, peaks, cpu_seco
     roof["avg_launch_us"] = gu_s * 1e6
     roof["algorithmic_per_launch"] = work["flops_gu"] if is_prefill else work["gu_bytes"]
     rec = {
-        # route, gate/up, down, combine; the dispatch (two kernels from 8192 pairs); the
-        # prepare step (from 2048 pairs on the tile path two: the inverse permutation, the
-        # per-token quantisation) or, on the batched path, prepare and quant_h
-        "fused": fused,
-        "launches_per_step": 1 if fused else (4 + (2 if T * k >= 8192 else 1)
-                                              + (2 if batched or T * k >= 2048 else 1)),
+        "fused": fused, "launches_per_step": launches_per_step(T, k, fused, batched),
         "value": world * T * steps / total_s, "unit": "tokens/s", "steps": steps,
         "ms_per_step": 1000.0 * layer_s,
         "ms_per_step_isolated": statistics.median(one_ms),

@@ -1,5 +1,5 @@
 """Host-side pieces of bench.py that need no GPU: the oracle timings of the
-cpu_baseline object and the DRAM-traffic lookup."""
+cpu_baseline object, the DRAM-traffic lookup and the launch count per step."""
 import os
 import sys
 
@@ -45,3 +45,16 @@ def test_fp8_peak_choice():
     assert bench.fp8_peak_of({"fp8_tensorwise_tflops": 4100.0}, 1600.0)[0] == 4100.0
     peak, src = bench.fp8_peak_of({}, 1600.0)
     assert peak == 3200.0 and "nominal" in src
+
+
+def test_launches_per_step():
+    # the layer kernels a step launches, as the library picks them by batch size
+    assert bench.launches_per_step(1, 6, fused=True, batched=False) == 1
+    # batched GEMV path: route, dispatch, prepare, gate/up, quant_h, down, combine
+    assert bench.launches_per_step(64, 6, fused=False, batched=True) == 7
+    assert bench.launches_per_step(32, 6, fused=False, batched=True) == 7
+    # tile path below 2048 pairs: route, dispatch, prepare, gate/up, down, combine
+    assert bench.launches_per_step(100, 8, fused=False, batched=False) == 6
+    # prefill: the dispatch and the prepare step are two kernels each
+    assert bench.launches_per_step(4096, 6, fused=False, batched=False) == 8
+    assert bench.launches_per_step(512, 6, fused=False, batched=False) == 7
